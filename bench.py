@@ -1,0 +1,449 @@
+#!/usr/bin/env python
+"""Benchmark: PKM layer forward tokens/s on B200, with the roofline fraction.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one pkm_forward over one batch of the 1024^2-slot workload (B = 16384
+tokens, d_model = 1024, H = 4, dq = 512, n = 1024, k = 32, v = 1024, bf16 inputs,
+fp32 scores and accumulation) with every input resident in HBM. L2 is flushed (a
+256 MiB write) before every timed step, outside the step's CUDA-event bracket.
+Under torchrun each rank runs the same workload on its own GPU with no collective
+on the data path (weak scaling); the reported time is the max over ranks.
+
+Rank 0 prints one JSON line. Besides the throughput it carries the roofline of the
+dominant kernel (stage times come from CUDA events the library records between its
+launches on the launching stream), the whole-step roofline, an end-to-end figure
+through the same call with host buffers, the value backward on the 512^2 layer, the
+oracle timed on this host's cores, and the SM clocks sampled during the timed loop.
+
+``--impl reference`` times the fp64 CPU oracle instead (a bounded sample of the
+same workload per step) and prints the same metric with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "PKM forward tokens/sec at 512² and 1024² slots (H=4,k=32); % of roofline"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FLUSH_BYTES = 256 << 20
+
+# DRAM bytes per launch of the dominant kernel from an ncu capture
+# (profiles/select_gather_c1024.md), keyed by the sha256 of the kernel's source at
+# capture time; reported as null once the source has changed.
+TRAFFIC = {}
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_desc(w) -> str:
+    return ("%s: B=%d tokens, d_model=%d, H=%d, dq=%d, n=%d (%d slots), k=%d, v=%d, %s"
+            % (w.name, w.B, w.d_model, w.H, w.dq, w.n, w.n * w.n, w.k, w.v, w.dtype))
+
+
+def per_token_bytes(w):
+    """Algorithmic HBM bytes per token of the select+gather kernel: the H*k gathered
+    value rows, the per-half lists read, the out row and idx/weight/score written."""
+    esz = 2 if w.dtype == "bf16" else 4
+    return w.H * w.k * w.v * esz + w.v * 4 + w.H * 2 * w.k * 8 + w.H * w.k * 12
+
+
+def gemm_flops_per_token(w):
+    """Query projection + per-half scoring, as the method defines them."""
+    return 2 * w.d_model * w.H * w.dq + 2 * w.H * 2 * w.n * (w.dq // 2)
+
+
+# --------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = None
+        try:
+            props = torch.cuda.get_device_properties(device_index)
+            uuid = str(getattr(props, "uuid", "") or "")
+            sel = ("GPU-" + uuid) if uuid and not uuid.startswith("GPU-") else uuid
+            if not sel:
+                vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+                sel = vis.split(",")[device_index] if vis else str(device_index)
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", sel, "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- CPU oracle
+def time_oracle(w, L, budget_s: float, max_tokens: int, chunk: int = 256):
+    """Oracle forward on consecutive chunks of the workload's tokens until the time
+    budget or max_tokens is reached. Returns (tokens/s, tokens, seconds, threads)."""
+    import oracle
+    threads = os.cpu_count() or 1
+    done, spent = 0, 0.0
+    while done < max_tokens and spent < budget_s:
+        m = min(chunk, max_tokens - done)
+        Ls = dict(L)
+        Ls["x"] = L["x"][done:done + m]
+        t0 = time.perf_counter()
+        oracle.forward(Ls, w.H, w.dq, w.n, w.k, threads=threads)
+        spent += time.perf_counter() - t0
+        done += m
+    return done / spent, done, spent, threads
+
+
+# ---------------------------------------------------------------- reference
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    import oracle  # noqa: F401  (builds the oracle library on first use)
+    w = synth.WORKLOADS[args.workload]
+    L = synth.make_layer(w)
+    # Size each step's sample so the whole run stays within about two minutes.
+    rate, _, _, threads = time_oracle(w, L, budget_s=2.0, max_tokens=min(w.B, 512), chunk=128)
+    per_step = max(64, min(w.B, int(rate * 120.0 / max(1, args.steps + args.warmup))))
+    per_step = (per_step // 64) * 64
+    times = []
+    for s in range(args.warmup + args.steps):
+        r, toks, sec, threads = time_oracle(w, L, budget_s=1e9, max_tokens=per_step,
+                                            chunk=per_step)
+        if s >= args.warmup:
+            times.append(sec)
+    mean = statistics.mean(times)
+    value = per_step / mean
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded, shapes of the pages' setups)",
+        "config": {"workload": workload_desc(w), "sample_tokens_per_step": per_step,
+                   "parallelism": "host cores, rank 0 only"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": "first %d of the %d tokens per step" % (per_step, w.B)},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------- our arm
+def kernel_sha() -> str:
+    h = hashlib.sha256()
+    with open(os.path.join(ROOT, "product_key_memory_b200", "csrc", "pkm_select_gather.cu"),
+              "rb") as f:
+        h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch.distributed as dist
+    import product_key_memory_b200 as P
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = synth.WORKLOADS[args.workload]
+    L = synth.make_layer(w)
+    d = {k: v.to(dev) for k, v in L.items()}
+    B = w.B
+    out = torch.empty(B, w.v, dtype=torch.float32, device=dev)
+    idx = torch.empty(B, w.H, w.k, dtype=torch.int32, device=dev)
+    wts = torch.empty(B, w.H, w.k, dtype=torch.float32, device=dev)
+    scs = torch.empty(B, w.H, w.k, dtype=torch.float32, device=dev)
+    shape = P.make_shape(B, w.d_model, w.H, w.dq, w.n, w.k, w.v, w.torch_dtype)
+    ws = P.alloc_workspace(shape, False, dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def fwd(x=None):
+        P.pkm_forward(d["x"] if x is None else x, d["W_q"], d["bn_mean"], d["bn_var"],
+                      d["bn_gamma"], d["bn_beta"], d["subkeys"], d["values"], k=w.k, out=out,
+                      indices=idx, weights=wts, scores=scs, workspace=ws)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for s in range(args.warmup):
+        flush.fill_(s & 0xff)
+        fwd()
+    if P.pkm_device_status(ws) != 0:
+        raise RuntimeError("device status after warm-up: %s" % P.pkm_status_string(-5))
+    P.pkm_trace_enable(True)
+    P.pkm_trace_read(0)
+    P.pkm_trace_read(1)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    barrier()
+    torch.cuda.synchronize(dev)
+    for s in range(args.steps):
+        flush.fill_((s + 1) & 0xff)
+        ev[s][0].record(stream)
+        fwd()
+        ev[s][1].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks = sampler.stop() if sampler else None
+    stage_ms, calls, launches = P.pkm_trace_read(0)
+    P.pkm_trace_enable(False)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    if P.pkm_device_status(ws) != 0:
+        raise RuntimeError("device status after timing: %s" % P.pkm_status_string(-5))
+    value = world * args.steps * B / (total_ms / 1e3)
+    ms_per_step = total_ms / args.steps
+
+    pk, pk_kind = peaks()
+    hbm = float(pk["hbm_gbs"])
+    bf16 = float(pk["bf16_tflops"])
+    stage_avg = [m / max(1, calls) for m in stage_ms[:3]]
+    names = ["query_network", "subkey_scores_topk", "select_softmax_gather"]
+    dom = max(range(3), key=lambda i: stage_avg[i])
+    F = w.H * w.dq
+    if dom == 2:
+        alg = per_token_bytes(w) * B
+        achieved = alg / (stage_avg[2] * 1e-3) / 1e9
+        sha = kernel_sha()
+        tr = TRAFFIC.get(sha)
+        roof = {"kernel": names[2], "bound": "hbm", "achieved": achieved, "peak": hbm,
+                "unit": "GB/s", "frac": achieved / hbm, "traffic": tr,
+                "algorithmic_bytes_per_launch": alg, "ms_per_launch": stage_avg[2],
+                "peak_kind": pk_kind}
+    else:
+        fl = (2 * B * w.d_model * F) if dom == 0 else (2 * B * w.H * 2 * w.n * (w.dq // 2))
+        achieved = fl / (stage_avg[dom] * 1e-3) / 1e12
+        roof = {"kernel": names[dom], "bound": "tensor", "achieved": achieved, "peak": bf16,
+                "unit": "TFLOP/s", "frac": achieved / bf16, "traffic": None,
+                "algorithmic_flops_per_launch": fl, "ms_per_launch": stage_avg[dom],
+                "peak_kind": pk_kind}
+    t_mem = w.H * w.k * w.v * (2 if w.dtype == "bf16" else 4) * B / (hbm * 1e9)
+    t_gemm = gemm_flops_per_token(w) * B / (bf16 * 1e12)
+    t_roof_ms = max(t_mem, t_gemm) * 1e3
+    step_roof = {"t_roof_ms": t_roof_ms, "t_step_ms": ms_per_step, "frac": t_roof_ms / ms_per_step,
+                 "bound": "hbm" if t_mem >= t_gemm else "tensor",
+                 "stage_ms": dict(zip(names, stage_avg)), "peak_kind": pk_kind}
+
+    # ---- end to end: host x -> device, forward, out/indices/weights -> host
+    x_h = L["x"].pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    idx_h = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
+    w_h = torch.empty(wts.shape, dtype=wts.dtype).pin_memory()
+    x_d = torch.empty_like(d["x"])
+
+    def e2e_step():
+        x_d.copy_(x_h, non_blocking=True)
+        fwd(x_d)
+        out_h.copy_(out, non_blocking=True)
+        idx_h.copy_(idx, non_blocking=True)
+        w_h.copy_(wts, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = {"value": world * args.steps * B / (e2e_ms / 1e3), "unit": UNIT,
+           "h2d_bytes_per_step": x_h.numel() * x_h.element_size(),
+           "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in (out_h, idx_h, w_h)),
+           "ms_per_step": e2e_ms / args.steps}
+    launches_e2e = P.pkm_trace_read(0)[2]
+
+    extra = {}
+    if not args.no_extras:
+        del d, x_d
+        torch.cuda.empty_cache()
+        extra = run_c512_and_backward(args, dev, P, hbm, bf16, stream, world, barrier)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic (seeded; shapes and distributions of the pages' 1024^2-slot setup)",
+        "config": {"workload": workload_desc(w), "global_batch": B * world,
+                   "seq_len": None, "parallelism": "dp%d (independent replicas)" % world,
+                   "l2": "flushed before every timed step (256 MiB write, outside the bracket)"},
+        "roofline": roof, "step_roofline": step_roof, "e2e": e2e,
+        "gpu_launches": launches, "gpu_launches_e2e": launches_e2e,
+        "clocks": clocks,
+    }
+    line.update(extra)
+    if rank == 0 and world == 1 and not args.no_extras:
+        budget = float(os.environ.get("PKM_CPU_BASELINE_S", "15"))
+        rate, toks, sec, threads = time_oracle(w, L, budget_s=budget, max_tokens=B)
+        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                "sample": "first %d of the %d tokens (%.1f s)" % (toks, B, sec)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_c512_and_backward(args, dev, P, hbm, bf16, stream, world, barrier):
+    """512^2-slot forward (the metric's other memory size) and the value backward on it."""
+    w = synth.WORKLOADS["c512"]
+    L = synth.make_layer(w)
+    d = {k: v.to(dev) for k, v in L.items()}
+    B = w.B
+    out = torch.empty(B, w.v, dtype=torch.float32, device=dev)
+    idx = torch.empty(B, w.H, w.k, dtype=torch.int32, device=dev)
+    wts = torch.empty(B, w.H, w.k, dtype=torch.float32, device=dev)
+    shape = P.make_shape(B, w.d_model, w.H, w.dq, w.n, w.k, w.v, w.torch_dtype)
+    ws = P.alloc_workspace(shape, False, dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def fwd():
+        P.pkm_forward(d["x"], d["W_q"], d["bn_mean"], d["bn_var"], d["bn_gamma"], d["bn_beta"],
+                      d["subkeys"], d["values"], k=w.k, out=out, indices=idx, weights=wts,
+                      want_scores=False, workspace=ws)
+
+    def timed(fn, steps):
+        ms = []
+        for s in range(steps):
+            flush.fill_(s & 0xff)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            ms.append((a, b))
+        torch.cuda.synchronize(dev)
+        return sum(a.elapsed_time(b) for a, b in ms) / steps
+
+    for _ in range(max(3, args.warmup)):
+        fwd()
+    barrier()
+    P.pkm_trace_read(0)
+    fwd_ms = timed(fwd, args.steps)
+    stage_ms, calls, _ = P.pkm_trace_read(0)
+    t_roof = max(w.H * w.k * w.v * 2 * B / (hbm * 1e9), gemm_flops_per_token(w) * B / (bf16 * 1e12))
+    res = {"c512": {"workload": workload_desc(w), "value": world * B / (fwd_ms / 1e3),
+                    "unit": UNIT, "ms_per_step": fwd_ms, "step_roofline_frac": t_roof * 1e3 / fwd_ms,
+                    "stage_ms": [m / max(1, calls) for m in stage_ms[:3]]}}
+
+    # Backward on the c512 picks: grad_out ~ N(0, 1) bf16 [4096][1024].
+    gout = synth.make_grad_out(w).to(dev)
+    gv = torch.zeros(w.n * w.n, w.v, dtype=torch.float32, device=dev)
+    gs = torch.empty(B, w.H, w.k, dtype=torch.float32, device=dev)
+    bshape = P.make_shape(B, 0, w.H, 0, w.n, w.k, w.v, w.torch_dtype)
+    bws = P.alloc_workspace(bshape, True, dev)
+
+    def bwd():
+        P.pkm_backward_values(d["values"], idx, wts, gout, gv, gs, w.n, workspace=bws)
+
+    for _ in range(max(3, args.warmup)):
+        bwd()
+    P.pkm_trace_read(1)
+    bwd_ms = timed(bwd, args.steps)
+    bstage, bcalls, _ = P.pkm_trace_read(1)
+    uniq = int(torch.unique(idx).numel())
+    picks = idx.numel()
+    bytes_alg = picks * w.v * 2 + B * w.v * 2 + picks * 8 + 2 * uniq * w.v * 4
+    res["backward"] = {
+        "workload": "bwd512: value backward on the c512 picks, grad_out bf16 [4096][1024]",
+        "value": world * B / (bwd_ms / 1e3), "unit": UNIT, "ms_per_step": bwd_ms,
+        "unique_rows": uniq, "picks": picks,
+        "algorithmic_bytes": bytes_alg, "achieved_gbs": bytes_alg / (bwd_ms * 1e-3) / 1e9,
+        "frac_of_hbm": bytes_alg / (bwd_ms * 1e-3) / 1e9 / hbm,
+        "stage_ms": [m / max(1, bcalls) for m in bstage[:2]]}
+    return res
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="c1024", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the c512 / backward / CPU-oracle measurements")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

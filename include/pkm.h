@@ -1,0 +1,158 @@
+/*
+ * pkm.h -- C ABI of the product-key memory (PKM) layer library for NVIDIA B200
+ * (sm_100a). Library file: libpkm.so (product_key_memory_b200/libpkm.so).
+ *
+ * The layer is the one of "Large Memory Layers with Product Keys" (Lample et al.,
+ * 2019). Per token and head (gptget.net summary of that paper, Methodology and the
+ * Deep Analysis / Methodology list; "Product Keys Give Transformers Million-Slot
+ * Memory Layers", sections "Why top-k of each half is enough" and "Implied keys
+ * vs stored sub-keys"):
+ *   q      = BN(x W_q^T)                query network: linear map + inference BatchNorm
+ *   q1, q2 = the two halves of q_h      (dq/2 each)
+ *   s1, s2 = q1 C_h^T, q2 C'_h^T        score every sub-key of each codebook
+ *   keep the top-k of s1 and of s2
+ *   score(i, j) = s1[i] + s2[j] over the k x k pairs; keep the exact top-k keys;
+ *   the key (i, j) has flat slot i*n + j
+ *   w      = softmax over the k kept scores
+ *   out[t] = sum over heads h, kept j of w[t,h,j] * V[slot[t,h,j]]
+ * Orders: every top-k is by score descending, ties to the lower id (sub-key id in
+ * the per-half lists, flat slot in the final list). Output lists are sorted in that
+ * order.
+ *
+ * Conventions for every entry point:
+ *   - Tensors are caller-owned DEVICE pointers, row-major and contiguous, 16-byte
+ *     aligned. The library keeps no device state between calls and allocates no
+ *     device memory: scratch is the caller's `workspace`.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     All work is enqueued asynchronously on it; no call synchronises.
+ *   - Arguments are validated before anything is launched: a call that returns an
+ *     error has launched nothing and written nothing.
+ *   - Kernels that wait on hardware barriers give up after a bounded number of
+ *     polls and record PKM_ERR_DEVICE in the workspace's status word; read it with
+ *     pkm_device_status() after the stream has finished.
+ */
+#ifndef PKM_H_
+#define PKM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element type of x, W_q, sub-keys, values and grad_out. BN vectors, scores,
+ * weights, out and gradients are always fp32. */
+typedef enum { PKM_F32 = 0, PKM_BF16 = 1 } pkm_dtype;
+
+/* Status codes. */
+enum {
+  PKM_OK = 0,
+  PKM_ERR_INVALID_ARG = -1, /* NULL pointer, size out of range, k > n, odd dq, n*n > 2^31-1 */
+  PKM_ERR_UNSUPPORTED = -2, /* valid layer this build does not run (k > 32, v not a multiple of
+                               16 bytes, misaligned pointer) */
+  PKM_ERR_WORKSPACE = -3,   /* workspace NULL or smaller than pkm_workspace_size() */
+  PKM_ERR_CUDA = -4,        /* a CUDA runtime call or kernel launch failed */
+  PKM_ERR_DEVICE = -5       /* a kernel recorded a device-side error (bounded wait ran out) */
+};
+
+/* Layer sizes. */
+typedef struct {
+  int64_t B;       /* tokens (rows of x); 0 is allowed and launches nothing */
+  int32_t d_model; /* input width of the query network */
+  int32_t H;       /* heads */
+  int32_t dq;      /* query size per head, even; each half is dq/2 */
+  int32_t n;       /* sub-keys per codebook; the memory has n*n slots */
+  int32_t k;       /* keys kept per half and per head, 1 <= k <= min(n, 32) */
+  int32_t v;       /* value width */
+  int32_t dtype;   /* pkm_dtype of x, W_q, sub-keys, values, grad_out */
+  float bn_eps;    /* BatchNorm epsilon (PyTorch's default is 1e-5) */
+} pkm_shape;
+
+/*
+ * Bytes of workspace pkm_forward (for_backward = 0) or pkm_backward_values
+ * (for_backward = 1) needs for this shape; 0 if the shape is invalid.
+ */
+size_t pkm_workspace_size(const pkm_shape* s, int for_backward);
+
+/*
+ * Forward pass of the PKM layer (the steps listed at the top of this file).
+ *
+ *   x        [B][d_model]            dtype
+ *   W_q      [H*dq][d_model]         dtype   (q = x W_q^T; no bias)
+ *   bn_mean, bn_var, bn_gamma, bn_beta  [H*dq] fp32 running statistics and affine
+ *            q = (acc - mean) / sqrt(var + bn_eps) * gamma + beta
+ *   subkeys  [H][2][n][dq/2]         dtype   ([h][0] = C scores q1, [h][1] = C' scores q2)
+ *   values   [n*n][v]                dtype   (one table shared by all heads)
+ * Outputs (overwritten):
+ *   out      [B][v]     fp32   sum over heads of the weighted value rows
+ *   indices  [B][H][k]  int32  flat slots i*n + j, best first
+ *   weights  [B][H][k]  fp32   softmax of the kept scores
+ *   scores   [B][H][k]  fp32   kept key scores s1[i] + s2[j]; may be NULL
+ * workspace: device scratch of at least pkm_workspace_size(s, 0) bytes, 256-byte
+ *   aligned; its contents on entry do not matter.
+ * Returns PKM_OK or a status code above.
+ */
+int pkm_forward(const pkm_shape* s, const void* x, const void* W_q, const float* bn_mean,
+                const float* bn_var, const float* bn_gamma, const float* bn_beta,
+                const void* subkeys, const void* values, float* out, int32_t* indices,
+                float* weights, float* scores, void* workspace, size_t workspace_bytes,
+                void* stream);
+
+/*
+ * Sparse value backward ("trained end-to-end with sparse updates"; only the kept
+ * slots receive gradient). With L = <grad_out, out>:
+ *   grad_scores[t,h,j] = w_j * (g_j - sum_l w_l g_l),  g_j = <grad_out[t], V[slot_j]>
+ *   grad_values[slot] += sum over picks (t,h,j) of that slot of w[t,h,j] * grad_out[t]
+ *
+ *   values      [n*n][v]   dtype
+ *   indices     [B][H][k]  int32  (as written by pkm_forward; each in [0, n*n))
+ *   weights     [B][H][k]  fp32
+ *   grad_out    [B][v]     dtype
+ *   grad_values [n*n][v]   fp32   ACCUMULATED into (the caller zeroes it once)
+ *   grad_scores [B][H][k]  fp32   overwritten; may be NULL
+ * Picks are grouped by slot with a counting sort, so each touched row is read and
+ * written once per group rather than once per pick. Slot ids outside [0, n*n) are
+ * skipped and counted in the status word (PKM_ERR_DEVICE).
+ * Only B, H, n, k, v and dtype of the shape are read; d_model, dq and bn_eps are
+ * ignored.
+ * workspace: at least pkm_workspace_size(s, 1) bytes, 256-byte aligned.
+ */
+int pkm_backward_values(const pkm_shape* s, const void* values, const int32_t* indices,
+                        const float* weights, const void* grad_out, float* grad_values,
+                        float* grad_scores, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
+/*
+ * Synchronises `stream`, reads the status word that the kernels of the last call
+ * on this workspace wrote (each call clears it when it starts), clears it and
+ * returns PKM_OK, PKM_ERR_DEVICE or PKM_ERR_CUDA. This is the only entry point
+ * that blocks the host.
+ */
+int pkm_device_status(void* workspace, void* stream);
+
+/*
+ * Stage timing (a measurement aid; the pages have no counterpart). While enabled,
+ * each pkm_forward call records a CUDA event on its stream before and after each of
+ * its 3 stages (0 query network, 1 per-half scores and top-k, 2 candidate top-k,
+ * softmax and value gather) and each pkm_backward_values call around its 2 stages
+ * (0 grad wrt kept scores, 1 slot grouping and row sums). The events are owned by
+ * the library (host-side handles only; no device memory).
+ * pkm_trace_read waits for the recorded events of `pass` (0 forward, 1 backward),
+ * writes the summed milliseconds per stage into stage_ms[0..max_stages), the number
+ * of traced calls into *calls, and the number of kernels the library launched since
+ * the last read (all passes, traced or not) into *launches; then forgets them.
+ * Returns PKM_OK, PKM_ERR_INVALID_ARG or PKM_ERR_CUDA.
+ */
+int pkm_trace_enable(int on);
+int pkm_trace_read(int pass, double* stage_ms, int max_stages, int64_t* calls,
+                   int64_t* launches);
+
+/* Static string for a status code. */
+const char* pkm_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PKM_H_ */

@@ -1,0 +1,54 @@
+// pkm_kernels.h -- internal launcher interface between the C ABI (pkm_api.cu) and
+// the kernels. Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <functional>
+
+namespace pkm {
+
+struct LayerArgs {
+  int64_t B;
+  int d_model, H, dq, n, k, v, dtype;
+  float bn_eps;
+  const void* x;
+  const void* W_q;
+  const float* bn_mean;
+  const float* bn_var;
+  const float* bn_gamma;
+  const float* bn_beta;
+  const void* subkeys;
+  const void* values;
+  int* status;  // device status word
+};
+
+// SIMT query network + per-half search (pkm_simt.cu).
+cudaError_t launch_query_bn_simt(const LayerArgs& a, float* q, cudaStream_t st);
+size_t subkey_topk_simt_smem(int dq);
+cudaError_t launch_subkey_topk_simt(const LayerArgs& a, const float* q, float* list_s,
+                                    int* list_i, cudaStream_t st);
+
+// Candidate top-k + softmax + value gather (pkm_select_gather.cu).
+bool select_gather_supported(int H, int k, int v, int dtype);
+cudaError_t launch_select_gather(const LayerArgs& a, const float* list_s, const int* list_i,
+                                 float* out, int* indices, float* weights, float* scores,
+                                 cudaStream_t st);
+
+// Value backward (pkm_backward.cu).
+struct BackwardWs {
+  int* counts;    // [slots]
+  int* offsets;   // [slots + 1]
+  int* partials;  // [scan blocks + 1]
+  int* order;     // [B*H*k] pick ids grouped by slot
+};
+size_t backward_ws_bytes(int64_t B, int H, int k, int64_t slots, BackwardWs* carve, char* base);
+cudaError_t launch_backward_values(int64_t B, int H, int k, int v, int dtype, int64_t slots,
+                                   const void* values, const int* indices, const float* weights,
+                                   const void* grad_out, float* grad_values, float* grad_scores,
+                                   const BackwardWs& ws, int* status, cudaStream_t st,
+                                   const std::function<void()>& between_stages);
+
+}  // namespace pkm

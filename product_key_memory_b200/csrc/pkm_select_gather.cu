@@ -1,0 +1,194 @@
+// pkm_select_gather.cu -- exact top-k over the k x k product candidates, softmax,
+// and the weighted value read summed over heads. One warp per token.
+//
+// "Large Memory Layers with Product Keys" (gptget.net summary, Methodology and the
+// Deep Analysis / Methodology list): the per-half sub-key sets are combined into
+// candidate keys, the k keys with the largest inner product are kept, and the
+// output is the weighted sum of their value vectors, over the heads. A key's score
+// is its left score plus its right score ("Product Keys Give Transformers
+// Million-Slot Memory Layers", "Why top-k of each half is enough"); key (i, j) is
+// left sub-key i joined with right sub-key j, flat slot i*n + j ("Implied keys vs
+// stored sub-keys").
+//
+// Candidate pruning: with both per-half lists sorted best first, the pair at list
+// positions (a, b) is beaten by every pair (a', b') with a' <= a and b' <= b, so it can
+// only be among the best k if (a + 1)(b + 1) <= k. That is the same argument the
+// pages give for keeping k per half, applied inside the k x k grid; it leaves
+// sum_a floor(k / (a + 1)) candidates (119 for k = 32) instead of k^2. In fp32 the
+// sums keep that order except where two sums round to the same value, which is a
+// tie at fp32 resolution.
+#include "pkm_common.cuh"
+#include "pkm_kernels.h"
+
+namespace pkm {
+
+constexpr int kSgWarps = 4;
+
+template <typename T, int MAXV>
+__global__ void __launch_bounds__(kSgWarps * 32) select_gather_kernel(
+    const float* __restrict__ list_s, const int* __restrict__ list_i,
+    const T* __restrict__ values, int64_t B, int H, int n, int k, int v,
+    float* __restrict__ out, int* __restrict__ indices, float* __restrict__ weights,
+    float* __restrict__ scores, int* status) {
+  constexpr int VPER = Vec<T>::kPer;
+  constexpr int U = MAXV >= 8 ? 2 : 4;  // rows in flight per lane step
+  extern __shared__ int sg_smem[];
+  int* pairs = sg_smem;                                  // [k*k] (a | b << 8)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int HK = H * k;
+  int* rows = sg_smem + kMaxK * kMaxK + warp * 2 * HK;   // [HK]
+  float* wts = reinterpret_cast<float*>(rows + HK);      // [HK]
+  __shared__ int npairs_s;
+
+  if (threadIdx.x == 0) {
+    int p = 0;
+    for (int a = 0; a < k; ++a)
+      for (int b = 0; (a + 1) * (b + 1) <= k; ++b) pairs[p++] = a | (b << 8);
+    npairs_s = p;
+  }
+  __syncthreads();
+  const int npairs = npairs_s;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * kSgWarps + warp;
+  if (t >= B) return;
+
+  for (int h = 0; h < H; ++h) {
+    const int64_t base = (t * H + h) * 2 * static_cast<int64_t>(k);
+    const float s1 = lane < k ? list_s[base + lane] : -INFINITY;
+    const int i1 = lane < k ? list_i[base + lane] : 0;
+    const float s2 = lane < k ? list_s[base + k + lane] : -INFINITY;
+    const int i2 = lane < k ? list_i[base + k + lane] : 0;
+    float bs = -INFINITY;
+    int bi = kIdPad;
+    for (int c0 = 0; c0 < npairs; c0 += 32) {
+      const int p = c0 + lane;
+      const int ab = p < npairs ? pairs[p] : 0;
+      const int a = ab & 0xff, b = ab >> 8;
+      const float sa = __shfl_sync(0xffffffffu, s1, a);
+      const int ia = __shfl_sync(0xffffffffu, i1, a);
+      const float sb = __shfl_sync(0xffffffffu, s2, b);
+      const int ib = __shfl_sync(0xffffffffu, i2, b);
+      // Padding ids can only surface when scores are NaN; they never form a slot.
+      const bool real = p < npairs && ia >= 0 && ia < n && ib >= 0 && ib < n;
+      float cs = real ? sa + sb : -INFINITY;
+      int ci = real ? ia * n + ib : kIdPad;
+      warp_sort32(cs, ci);
+      warp_merge32(bs, bi, cs, ci);
+    }
+    // Softmax over the k kept scores (lanes 0..k-1 hold them, best first).
+    const float mx = __shfl_sync(0xffffffffu, bs, 0);
+    const float e = lane < k ? expf(bs - mx) : 0.f;
+    const float den = warp_sum(e);
+    const float w = e / den;
+    if (lane < k) {
+      const int64_t o = (t * H + h) * static_cast<int64_t>(k) + lane;
+      indices[o] = bi;
+      weights[o] = w;
+      if (scores) scores[o] = bs;
+      rows[h * k + lane] = bi;
+      wts[h * k + lane] = w;
+    }
+  }
+  __syncwarp();
+
+  // Weighted value rows: lane covers 16-byte vectors lane, lane+32, ... of each row.
+  const int nvec = v / VPER;
+  float acc[MAXV][VPER];
+#pragma unroll
+  for (int m = 0; m < MAXV; ++m)
+#pragma unroll
+    for (int e = 0; e < VPER; ++e) acc[m][e] = 0.f;
+
+  for (int r0 = 0; r0 < HK; r0 += U) {
+    uint4 raw[U][MAXV];
+    float wr[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      bool live = r0 + u < HK;
+      int row = live ? rows[r0 + u] : 0;
+      if (live && (row < 0 || row >= n * n)) {  // only reachable with NaN scores
+        if (lane == 0) record_status(status, kDevBadSlot);
+        live = false;
+        row = 0;
+      }
+      wr[u] = live ? wts[r0 + u] : 0.f;
+      const T* rp = values + static_cast<int64_t>(row) * v;
+#pragma unroll
+      for (int m = 0; m < MAXV; ++m) {
+        const int vec = lane + 32 * m;
+        raw[u][m] = (live && vec < nvec) ? ld_stream_v4(rp + vec * VPER) : make_uint4(0, 0, 0, 0);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int m = 0; m < MAXV; ++m) {
+        float f[VPER];
+        Vec<T>::widen(raw[u][m], f);
+#pragma unroll
+        for (int e = 0; e < VPER; ++e) acc[m][e] = fmaf(wr[u], f[e], acc[m][e]);
+      }
+  }
+  float* orow = out + t * v;
+#pragma unroll
+  for (int m = 0; m < MAXV; ++m) {
+    const int vec = lane + 32 * m;
+    if (vec < nvec) {
+#pragma unroll
+      for (int e = 0; e < VPER; e += 4)
+        *reinterpret_cast<float4*>(orow + vec * VPER + e) =
+            make_float4(acc[m][e], acc[m][e + 1], acc[m][e + 2], acc[m][e + 3]);
+    }
+  }
+}
+
+static int maxv_for(int v, int dtype) {
+  const int per = dtype == 0 ? 4 : 8;
+  const int nvec = v / per;
+  const int m = (nvec + 31) / 32;
+  if (m <= 1) return 1;
+  if (m <= 2) return 2;
+  if (m <= 4) return 4;
+  if (m <= 8) return 8;
+  return 0;
+}
+
+bool select_gather_supported(int H, int k, int v, int dtype) {
+  return k >= 1 && k <= kMaxK && H >= 1 && H * k <= 2048 && maxv_for(v, dtype) > 0;
+}
+
+template <typename T, int MAXV>
+static cudaError_t launch_sg(const LayerArgs& a, const float* ls, const int* li, float* out,
+                             int* idx, float* w, float* sc, cudaStream_t st) {
+  const size_t smem = sizeof(int) * (kMaxK * kMaxK + kSgWarps * 2 * a.H * a.k);
+  cudaError_t e = cudaFuncSetAttribute(select_gather_kernel<T, MAXV>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = static_cast<unsigned>((a.B + kSgWarps - 1) / kSgWarps);
+  select_gather_kernel<T, MAXV><<<grid, kSgWarps * 32, smem, st>>>(
+      ls, li, static_cast<const T*>(a.values), a.B, a.H, a.n, a.k, a.v, out, idx, w, sc,
+      a.status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_gather(const LayerArgs& a, const float* ls, const int* li, float* out,
+                                 int* idx, float* w, float* sc, cudaStream_t st) {
+  const int m = maxv_for(a.v, a.dtype);
+  if (a.dtype == 0) {
+    switch (m) {
+      case 1: return launch_sg<float, 1>(a, ls, li, out, idx, w, sc, st);
+      case 2: return launch_sg<float, 2>(a, ls, li, out, idx, w, sc, st);
+      case 4: return launch_sg<float, 4>(a, ls, li, out, idx, w, sc, st);
+      case 8: return launch_sg<float, 8>(a, ls, li, out, idx, w, sc, st);
+    }
+  } else {
+    switch (m) {
+      case 1: return launch_sg<uint16_t, 1>(a, ls, li, out, idx, w, sc, st);
+      case 2: return launch_sg<uint16_t, 2>(a, ls, li, out, idx, w, sc, st);
+      case 4: return launch_sg<uint16_t, 4>(a, ls, li, out, idx, w, sc, st);
+      case 8: return launch_sg<uint16_t, 8>(a, ls, li, out, idx, w, sc, st);
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace pkm

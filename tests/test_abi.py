@@ -1,0 +1,84 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry point that
+include/pkm.h declares, sizes workspaces, and rejects bad arguments before any
+CUDA call (so these run without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import product_key_memory_b200 as P
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "pkm.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(pkm_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = _declared()
+    assert "pkm_forward" in names and "pkm_backward_values" in names
+    lib = ctypes.CDLL(P.LIB_PATH)
+    for name in names:
+        assert hasattr(lib, name), name
+    assert set(P.EXPORTED) <= set(names)
+
+
+def test_status_strings():
+    for c in (0, -1, -2, -3, -4, -5):
+        assert P.pkm_status_string(c)
+    assert P.pkm_status_string(7) == "unknown status"
+
+
+def _shape(**kw):
+    base = dict(B=16384, d_model=1024, H=4, dq=512, n=1024, k=32, v=1024, dtype=1, bn_eps=1e-5)
+    base.update(kw)
+    return P.make_shape(**base)
+
+
+def test_workspace_sizes():
+    s = _shape()
+    fw = P.pkm_workspace_size(s)
+    # status + 6 bytes per q element + 8 bytes per per-half list entry
+    assert fw >= 256 + 16384 * 2048 * 6 + 16384 * 4 * 2 * 32 * 8
+    bw = P.pkm_workspace_size(s, True)
+    assert bw >= 256 + 4 * (2 * 1024 * 1024 + 16384 * 4 * 32)
+    assert P.pkm_workspace_size(_shape(B=0)) > 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(k=0), -1), (dict(k=33, n=64), -2), (dict(k=8, n=4), -1), (dict(dq=7), -1),
+    (dict(H=0), -1), (dict(v=0), -1), (dict(dtype=3), -1), (dict(n=46341), -1),
+    (dict(v=1001), -2), (dict(bn_eps=-1.0), -1), (dict(B=-1), -1),
+])
+def test_invalid_shapes_rejected_without_launch(kw, code):
+    s = _shape(**kw)
+    assert P.pkm_workspace_size(s) == 0
+    fake = ctypes.c_void_p(1 << 20)
+    rc = P.lib().pkm_forward(ctypes.byref(s), *([fake] * 12), fake, 1 << 40, None)
+    assert rc == code
+
+
+def test_null_and_misaligned_pointers_rejected():
+    s = _shape(B=4)
+    ok = ctypes.c_void_p(1 << 20)
+    args = [ok] * 12
+    args[3] = None                                 # bn_var
+    assert P.lib().pkm_forward(ctypes.byref(s), *args, ok, 1 << 40, None) == -1
+    args = [ok] * 12
+    args[7] = ctypes.c_void_p((1 << 20) + 8)       # values not 16-byte aligned
+    assert P.lib().pkm_forward(ctypes.byref(s), *args, ok, 1 << 40, None) == -2
+    args = [ok] * 12
+    assert P.lib().pkm_forward(ctypes.byref(s), *args, ok, 100, None) == -3          # small
+    assert P.lib().pkm_forward(ctypes.byref(s), *args, ctypes.c_void_p((1 << 20) + 16),
+                               1 << 40, None) == -3                                     # unaligned
+    assert P.lib().pkm_backward_values(ctypes.byref(s), *([ok] * 6), ok, 10, None) == -3
+
+
+def test_null_shape_rejected():
+    assert P.lib().pkm_workspace_size(None, 0) == 0
+    ok = ctypes.c_void_p(1 << 20)
+    assert P.lib().pkm_forward(None, *([ok] * 13), 1 << 40, None) == -1
