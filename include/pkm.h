@@ -58,7 +58,9 @@ enum {
 
 /* Layer sizes. */
 typedef struct {
-  int64_t B;       /* tokens (rows of x); 0 is allowed and launches nothing */
+  int64_t B;       /* tokens (rows of x); 0 is allowed, launches nothing, and then the
+                      per-token pointers (x, out, indices, weights, scores, grad_out,
+                      grad_scores) may be NULL */
   int32_t d_model; /* input width of the query network */
   int32_t H;       /* heads */
   int32_t dq;      /* query size per head, even; each half is dq/2 */

@@ -200,8 +200,10 @@ int pkm_forward(const pkm_shape* s, const void* x, const void* W_q, const float*
                 void* stream) {
   int rc = validate_shape(s);
   if (rc != PKM_OK) return rc;
-  if (!x || !W_q || !bn_mean || !bn_var || !bn_gamma || !bn_beta || !subkeys || !values ||
-      !out || !indices || !weights)
+  // Per-token tensors may be NULL when there are no tokens.
+  const bool tok = s->B > 0;
+  if (!W_q || !bn_mean || !bn_var || !bn_gamma || !bn_beta || !subkeys || !values ||
+      (tok && (!x || !out || !indices || !weights)))
     return PKM_ERR_INVALID_ARG;
   const void* ptrs[] = {x, W_q, bn_mean, bn_var, bn_gamma, bn_beta, subkeys, values, out,
                         indices, weights, scores};
@@ -246,7 +248,8 @@ int pkm_backward_values(const pkm_shape* s, const void* values, const int32_t* i
                         void* stream) {
   int rc = validate_common(s);
   if (rc != PKM_OK) return rc;
-  if (!values || !indices || !weights || !grad_out || !grad_values) return PKM_ERR_INVALID_ARG;
+  if (!values || !grad_values || (s->B > 0 && (!indices || !weights || !grad_out)))
+    return PKM_ERR_INVALID_ARG;
   const void* ptrs[] = {values, indices, weights, grad_out, grad_values, grad_scores};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return PKM_ERR_UNSUPPORTED;

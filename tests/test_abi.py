@@ -82,3 +82,14 @@ def test_null_shape_rejected():
     assert P.lib().pkm_workspace_size(None, 0) == 0
     ok = ctypes.c_void_p(1 << 20)
     assert P.lib().pkm_forward(None, *([ok] * 13), 1 << 40, None) == -1
+
+
+def test_zero_tokens_accepts_null_per_token_pointers():
+    s = _shape(B=0)
+    ok = ctypes.c_void_p(1 << 20)
+    args = [None, ok, ok, ok, ok, ok, ok, ok, None, None, None, None]   # x, out, idx, w, scores NULL
+    assert P.lib().pkm_forward(ctypes.byref(s), *args, ok, 1 << 40, None) == 0
+    bargs = [ok, None, None, None, ok, None]     # values, indices, weights, grad_out, grad_values, grad_scores
+    assert P.lib().pkm_backward_values(ctypes.byref(s), *bargs, ok, 1 << 40, None) == 0
+    s4 = _shape(B=4)
+    assert P.lib().pkm_forward(ctypes.byref(s4), *args, ok, 1 << 40, None) == -1
