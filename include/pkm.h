@@ -126,6 +126,29 @@ int pkm_backward_values(const pkm_shape* s, const void* values, const int32_t* i
                         void* stream);
 
 /*
+ * pkm_backward_values without a workspace. The pages have no counterpart: this is
+ * a convenience of this library. It is for callers that cannot allocate device
+ * memory where they run the backward (a runtime that hands out all device memory
+ * from its own pool and forbids other allocations while it executes, or a plugin
+ * host that passes device pointers but no allocator). Arguments and results are
+ * those of pkm_backward_values; the caller still passes inputs and outputs.
+ *
+ * Scratch: one fixed 16 MiB device array inside libpkm.so, held on every GPU that
+ * loads the library until the process exits. Limits: n*n <= 1,048,576 slots and
+ * B*H*k <= 2,097,152 picks; larger shapes return PKM_ERR_UNSUPPORTED before any
+ * launch. The call allocates nothing (no cudaMalloc, no library allocator).
+ * The first call on a device looks up the array's device address with that device
+ * current; make that first call before any stream capture. All calls share the
+ * one array (each call clears what must start at zero), so calls that overlap on
+ * the GPU -- on different streams, or from different threads -- race and must
+ * not be issued. Slot ids outside [0, n*n) are skipped as in pkm_backward_values,
+ * but the status word is not readable through pkm_device_status.
+ */
+int pkm_backward_values_noalloc(const pkm_shape* s, const void* values, const int32_t* indices,
+                                const float* weights, const void* grad_out, float* grad_values,
+                                float* grad_scores, void* stream);
+
+/*
  * Synchronises `stream`, reads the status word that the kernels of the last call
  * on this workspace wrote (each call clears it when it starts), clears it and
  * returns PKM_OK, PKM_ERR_DEVICE or PKM_ERR_CUDA. This is the only entry point

@@ -24,7 +24,8 @@ _STATUS = {0: "PKM_OK", -1: "PKM_ERR_INVALID_ARG", -2: "PKM_ERR_UNSUPPORTED",
            -3: "PKM_ERR_WORKSPACE", -4: "PKM_ERR_CUDA", -5: "PKM_ERR_DEVICE"}
 
 EXPORTED = ("pkm_workspace_size", "pkm_forward", "pkm_backward_values", "pkm_device_status",
-            "pkm_trace_enable", "pkm_trace_read", "pkm_status_string")
+            "pkm_trace_enable", "pkm_trace_read", "pkm_status_string",
+            "pkm_backward_values_noalloc")
 
 
 class PKMError(RuntimeError):
@@ -58,6 +59,8 @@ def lib() -> ctypes.CDLL:
         L.pkm_forward.restype = ctypes.c_int
         L.pkm_backward_values.argtypes = [S] + [P] * 7 + [ctypes.c_size_t, P]
         L.pkm_backward_values.restype = ctypes.c_int
+        L.pkm_backward_values_noalloc.argtypes = [S] + [P] * 6 + [P]
+        L.pkm_backward_values_noalloc.restype = ctypes.c_int
         L.pkm_device_status.argtypes = [P, P]
         L.pkm_device_status.restype = ctypes.c_int
         L.pkm_trace_enable.argtypes = [ctypes.c_int]
@@ -169,6 +172,23 @@ def pkm_backward_values(values: torch.Tensor, indices: torch.Tensor, weights: to
                                    _stream(stream))
     if rc != PKM_OK:
         raise PKMError("pkm_backward_values", rc)
+    return grad_values, grad_scores
+
+
+def pkm_backward_values_noalloc(values: torch.Tensor, indices: torch.Tensor,
+                                weights: torch.Tensor, grad_out: torch.Tensor,
+                                grad_values: torch.Tensor, grad_scores: Optional[torch.Tensor],
+                                n: int, stream=None):
+    """pkm_backward_values with the library's fixed device scratch instead of a
+    workspace (for callers that cannot allocate; limits in include/pkm.h)."""
+    B, H, k = indices.shape
+    v = values.shape[1]
+    shape = make_shape(B, 0, H, 0, n, k, v, values.dtype)
+    rc = lib().pkm_backward_values_noalloc(ctypes.byref(shape), _ptr(values), _ptr(indices),
+                                           _ptr(weights), _ptr(grad_out), _ptr(grad_values),
+                                           _ptr(grad_scores), _stream(stream))
+    if rc != PKM_OK:
+        raise PKMError("pkm_backward_values_noalloc", rc)
     return grad_values, grad_scores
 
 
