@@ -58,13 +58,13 @@ struct ForwardWs {
   int* status;
   float* q;         // SIMT path: fp32 q [B][H*dq]
   void* planes;     // tensor path: bf16 q planes [3][B][H*dq]
-  float* list_s;    // [B][H][2][k]
-  int* list_i;      // [B][H][2][k]
+  float* list_s;    // [B][H][2][32] best 32 per half (any order)
+  int* list_i;      // [B][H][2][32]
 };
 
 size_t forward_ws(const pkm_shape* s, ForwardWs* w, char* base) {
   const int64_t F = static_cast<int64_t>(s->H) * s->dq;
-  const int64_t L = s->B * s->H * 2 * static_cast<int64_t>(s->k);
+  const int64_t L = s->B * s->H * 2 * static_cast<int64_t>(pkm::kMaxK);
   size_t off = pkm::kStatusBytes;
   const size_t o_q = off;  off += align256(static_cast<size_t>(s->B) * F * 6);  // fp32 q or 3 bf16 planes
   const size_t o_ls = off; off += align256(sizeof(float) * L);

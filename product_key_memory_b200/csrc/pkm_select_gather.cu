@@ -52,11 +52,15 @@ __global__ void __launch_bounds__(kSgWarps * 32) select_gather_kernel(
   if (t >= B) return;
 
   for (int h = 0; h < H; ++h) {
-    const int64_t base = (t * H + h) * 2 * static_cast<int64_t>(k);
-    const float s1 = lane < k ? list_s[base + lane] : -INFINITY;
-    const int i1 = lane < k ? list_i[base + lane] : 0;
-    const float s2 = lane < k ? list_s[base + k + lane] : -INFINITY;
-    const int i2 = lane < k ? list_i[base + k + lane] : 0;
+    // Per-half lists hold the best 32 sub-keys of each half (in any order; padding has
+    // id kIdPad and score -inf). Sorting them puts the best k first.
+    const int64_t base = (t * H + h) * 2 * static_cast<int64_t>(kMaxK);
+    float s1 = list_s[base + lane];
+    int i1 = list_i[base + lane];
+    float s2 = list_s[base + kMaxK + lane];
+    int i2 = list_i[base + kMaxK + lane];
+    warp_sort32(s1, i1);
+    warp_sort32(s2, i2);
     float bs = -INFINITY;
     int bi = kIdPad;
     for (int c0 = 0; c0 < npairs; c0 += 32) {

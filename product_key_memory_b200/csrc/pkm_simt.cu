@@ -75,7 +75,8 @@ __global__ void __launch_bounds__(256) query_bn_simt_kernel(
 // 8 warps x 4 tokens. Sub-keys are staged 32 rows at a time in shared memory;
 // lane i scores sub-key (chunk + i) for each of the warp's tokens, and the warp
 // keeps a sorted best-32 list per token (one entry per lane) with sort + merge.
-// Output: list_s / list_i [B][H][2][k], best first.
+// Output: list_s / list_i [B][H][2][32]: the best 32 of each half (best first here;
+// padding entries have score -inf and id kIdPad when n < 32).
 // ---------------------------------------------------------------------------
 constexpr int kSimtTokPerWarp = 4;
 constexpr int kSimtWarps = 8;
@@ -135,8 +136,8 @@ __global__ void __launch_bounds__(kSimtWarps * 32) subkey_topk_simt_kernel(
 #pragma unroll
   for (int u = 0; u < kSimtTokPerWarp; ++u) {
     const int64_t t = t0 + warp * kSimtTokPerWarp + u;
-    if (t < B && lane < k) {
-      const int64_t o = ((t * H + h) * 2 + side) * k + lane;
+    if (t < B) {
+      const int64_t o = ((t * H + h) * 2 + side) * kMaxK + lane;
       list_s[o] = best_s[u];
       list_i[o] = best_i[u];
     }

@@ -2,8 +2,8 @@
 //
 //   query_tc_kernel        q = BN(x W_q^T), written as three bf16 planes hi/mid/lo
 //   score_topk_tc_kernel   s = q_half C^T per (128-token tile, head, half), scored in
-//                          256-sub-key chunks into TMEM, with the per-row top-k kept
-//                          in registers: the scores never reach HBM
+//                          256-sub-key chunks into TMEM; one epilogue thread per row
+//                          keeps the row's best 32 sub-keys: the scores never reach HBM
 //
 // "Large Memory Layers with Product Keys" (gptget.net summary, Methodology and the
 // Deep Analysis / Methodology list): the query network q(x) is a linear map with
@@ -11,10 +11,11 @@
 // each half runs an inner-product search against its own sub-key set and keeps its
 // top-k sub-keys.
 //
-// Both kernels are persistent (one CTA per SM) and warp-specialised, 192 threads:
+// Both kernels are persistent (one CTA per SM) and warp-specialised, 320 threads:
 //   warp 0      TMA producer (one elected lane)
 //   warp 1      TMEM allocator and MMA issuer (one elected lane)
-//   warps 2..5  epilogue, one thread per accumulator row (TMEM lane)
+//   warps 2..9  epilogue: two warps per TMEM lane quadrant, one thread per
+//               accumulator row; each of the two takes half of every chunk's columns
 // Operands are staged by TMA with the 128-byte swizzle; the accumulator is double
 // buffered in TMEM (2 x 256 fp32 columns) so the epilogue of one tile overlaps the
 // MMAs of the next. Every barrier wait is bounded (pkm_tcgen05.cuh); on a timeout
@@ -36,7 +37,8 @@ namespace pkm {
 
 using namespace tc;
 
-constexpr int kTcThreads = 192;
+constexpr int kEpiWarps = 8;
+constexpr int kTcThreads = 64 + 32 * kEpiWarps;
 constexpr int kRowsPerTile = 128;  // MMA M (one TMEM lane per row)
 constexpr int kColsPerMma = 256;   // MMA N
 constexpr int kKBlock = 64;        // bf16 elements per 128-byte swizzled row
@@ -94,7 +96,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) query_tc_kernel(
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4);
+      mbar_init(&tempty[b], kEpiWarps);
     }
     mbar_init(drain, 1);
     *abort = 0;
@@ -181,8 +183,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) query_tc_kernel(
   } else {
     // ---------------- epilogue: BN affine + 3-plane split, one thread per row
     const int quad = warp & 3;
+    const int cset = (warp - 2) >> 2;  // which half of the 256 columns this warp converts
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
     const size_t plane_stride = static_cast<size_t>(B) * F;
+    constexpr int kGroups = kColsPerMma / 32 / 2;  // 32-column groups per warp
     int it = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
       const int buf = it & 1;
@@ -192,10 +196,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) query_tc_kernel(
       const int m = t / nt, nn = t - m * nt;
       const int64_t row = static_cast<int64_t>(m) * kRowsPerTile + quad * 32 + lane;
 #pragma unroll 1
-      for (int g = 0; g < kColsPerMma / 32; ++g) {
+      for (int gg = 0; gg < kGroups; ++gg) {
+        const int g = cset * kGroups + gg;
         float v[32];
         tmem_ld32(tmem_base + lane_addr + buf * kColsPerMma + g * 32, v);
-        if (g == kColsPerMma / 32 - 1) {
+        if (gg == kGroups - 1) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&tempty[buf]);
@@ -238,19 +243,25 @@ __global__ void __launch_bounds__(kTcThreads, 1) query_tc_kernel(
 // ===========================================================================
 // Per-half scores and top-k
 // ===========================================================================
+constexpr int kSEpiWarps = 4;  // one epilogue warp per TMEM lane quadrant
+constexpr int kSThreads = 64 + 32 * kSEpiWarps;
 constexpr int kSStages = 2;
 constexpr uint32_t kSPlaneBytes = kRowsPerTile * kKBlock * 2;      // 16 KiB
 constexpr uint32_t kSABytes = 3 * kSPlaneBytes;                     // 48 KiB
 constexpr uint32_t kSBBytes = kColsPerMma * kKBlock * 2;            // 32 KiB
 constexpr uint32_t kSStageBytes = kSABytes + kSBBytes;              // 80 KiB
-constexpr int kSCap = 64;  // survivors buffered per row before they are merged
+constexpr int kList = kMaxK;          // entries per per-half list (the best 32, unsorted)
+constexpr int kSStep = 8;             // columns read from TMEM per step
+constexpr int kSNewCap = 24;          // survivors logged between two merges
+constexpr int kSLogCap = kList + kSNewCap;
 
 size_t score_tc_smem_bytes() {
-  return 1024 + kSStages * kSStageBytes + 2 * kSCap * kRowsPerTile * sizeof(float) + 256;
+  // stages + per-row log of (score, id) + barriers and flags
+  return 1024 + kSStages * kSStageBytes + kSLogCap * kRowsPerTile * 8 + 256;
 }
 
-// Sort 32 (score, id) pairs held by one thread, best first (bitonic network).
-__device__ __forceinline__ void thread_sort32(float (&s)[32], int (&id)[32]) {
+// Sort 32 floats held by one thread, largest first (bitonic network of min/max).
+__device__ __forceinline__ void thread_sort32f(float (&x)[32]) {
 #pragma unroll
   for (int size = 2; size <= 32; size <<= 1)
 #pragma unroll
@@ -260,74 +271,37 @@ __device__ __forceinline__ void thread_sort32(float (&s)[32], int (&id)[32]) {
         const int j = i ^ stride;
         if (j > i) {
           const bool desc = (i & size) == 0 || size == 32;
-          const bool jb = better(s[j], id[j], s[i], id[i]);
-          const bool sw = desc ? jb : better(s[i], id[i], s[j], id[j]);
-          const float ts = sw ? s[j] : s[i];
-          const int ti = sw ? id[j] : id[i];
-          s[j] = sw ? s[i] : s[j];
-          id[j] = sw ? id[i] : id[j];
-          s[i] = ts;
-          id[i] = ti;
+          const float a = x[i], b = x[j];
+          x[i] = desc ? fmaxf(a, b) : fminf(a, b);
+          x[j] = desc ? fminf(a, b) : fmaxf(a, b);
         }
       }
 }
 
-// Keep the best 32 of the sorted list L and the sorted batch b; L stays sorted.
-__device__ __forceinline__ void thread_merge32(float (&Ls)[32], int (&Li)[32],
-                                               const float (&bs)[32], const int (&bi)[32]) {
+// 32nd largest of 64 floats: sort both halves, then the elementwise max of one half
+// and the other reversed is the best 32 (as a set); its minimum is the answer.
+__device__ __forceinline__ float kth32_of_64(float (&x)[64]) {
+  float a[32], b[32];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const bool take = better(bs[31 - i], bi[31 - i], Ls[i], Li[i]);
-    Ls[i] = take ? bs[31 - i] : Ls[i];
-    Li[i] = take ? bi[31 - i] : Li[i];
-  }
+  for (int i = 0; i < 32; ++i) { a[i] = x[i]; b[i] = x[32 + i]; }
+  thread_sort32f(a);
+  thread_sort32f(b);
+  float t = INFINITY;
 #pragma unroll
-  for (int stride = 16; stride > 0; stride >>= 1)
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const int j = i ^ stride;
-      if (j > i) {
-        const bool sw = better(Ls[j], Li[j], Ls[i], Li[i]);
-        const float ts = sw ? Ls[j] : Ls[i];
-        const int ti = sw ? Li[j] : Li[i];
-        Ls[j] = sw ? Ls[i] : Ls[j];
-        Li[j] = sw ? Li[i] : Li[j];
-        Ls[i] = ts;
-        Li[i] = ti;
-      }
-    }
+  for (int i = 0; i < 32; ++i) t = fminf(t, fmaxf(a[i], b[31 - i]));
+  return t;
 }
 
-// Merge this thread's buffered survivors (cnt of them) into L, 32 at a time. Called by
-// all lanes of the warp together.
-__device__ __forceinline__ void absorb_survivors(float (&Ls)[32], int (&Li)[32],
-                                                 const float* sv_s, const int* sv_i, int cnt,
-                                                 int r) {
-#pragma unroll 1
-  for (int b0 = 0; b0 < kSCap; b0 += 32) {
-    if (!__any_sync(0xffffffffu, cnt > b0)) break;
-    float bs[32];
-    int bi[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const bool ok = b0 + j < cnt;
-      bs[j] = ok ? sv_s[(b0 + j) * kRowsPerTile + r] : -INFINITY;
-      bi[j] = ok ? sv_i[(b0 + j) * kRowsPerTile + r] : kIdPad;
-    }
-    thread_sort32(bs, bi);
-    thread_merge32(Ls, Li, bs, bi);
-  }
-}
-
-__global__ void __launch_bounds__(kTcThreads, 1) score_topk_tc_kernel(
+__global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
     const __grid_constant__ CUtensorMap tm_planes, const __grid_constant__ CUtensorMap tm_keys,
-    int B, int H, int dq, int n, int k, float* __restrict__ list_s, int* __restrict__ list_i,
+    int B, int H, int dq, int n, float* __restrict__ list_s, int* __restrict__ list_i,
     int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* stages = align1024(smem_raw);
-  float* sv_s = reinterpret_cast<float*>(stages + kSStages * kSStageBytes);  // [kSCap][128]
-  int* sv_i = reinterpret_cast<int*>(sv_s + kSCap * kRowsPerTile);           // [kSCap][128]
-  uint64_t* full = reinterpret_cast<uint64_t*>(sv_i + kSCap * kRowsPerTile);
+  // per-row log: [kSLogCap][128] scores, then the same for ids
+  float* lg_s = reinterpret_cast<float*>(stages + kSStages * kSStageBytes);
+  int* lg_i = reinterpret_cast<int*>(lg_s + kSLogCap * kRowsPerTile);
+  uint64_t* full = reinterpret_cast<uint64_t*>(lg_i + kSLogCap * kRowsPerTile);
   uint64_t* empty = full + kSStages;
   uint64_t* tfull = empty + kSStages;
   uint64_t* tempty = tfull + 2;
@@ -350,7 +324,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) score_topk_tc_kernel(
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4);
+      mbar_init(&tempty[b], kSEpiWarps);
     }
     mbar_init(drain, 1);
     *abort = 0;
@@ -442,63 +416,138 @@ __global__ void __launch_bounds__(kTcThreads, 1) score_topk_tc_kernel(
       }
     }
   } else {
-    // ---------------- epilogue: running top-k per row (= TMEM lane)
+    // ---------------- epilogue: the best 32 of each row (= TMEM lane)
+    // Ls holds the 32 largest scores seen so far (values only, sorted); the log in
+    // shared memory holds (score, id) of every element that can still be among the
+    // best 32. Columns arrive in increasing sub-key id, so the log is in id order.
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
+    constexpr int kStepsPerChunk = kColsPerMma / kSStep;
     int ci = 0;
-    bool ok = true;
-    for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
+    for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
       const int m = u / HS, hs = u - m * HS;
       float Ls[32];
-      int Li[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) { Ls[i] = -INFINITY; Li[i] = kIdPad; }
-      float tau = -INFINITY;  // score of the current 32nd best: anything not above it loses
-      int cnt = 0;
-      for (int c = 0; c < nchunks; ++c, ++ci) {
-        const int buf = ci & 1;
-        const uint32_t tph = (ci >> 1) & 1;
-        if (!warp_wait(&tfull[buf], tph, status, abort)) { ok = false; break; }
-        tc_fence_after();
+      for (int i = 0; i < 32; ++i) Ls[i] = -INFINITY;
+      // A score can still be among the best 32 only if it is >= tau0 (a lower bound of
+      // the 32nd best of the first chunk, hence of the row) and > tau_run (the current
+      // 32nd best: an equal score comes later in id order and loses the tie).
+      float tau0 = -INFINITY, tau_run = -INFINITY;
+      int cnt = 0, fresh = 0;  // log entries; entries logged since the last merge
+      bool ok = true;
+      const int nsteps = nchunks * kStepsPerChunk;
 #pragma unroll 1
-        for (int g = 0; g < kColsPerMma / 32; ++g) {
-          float v[32];
-          tmem_ld32(tmem_base + lane_addr + buf * kColsPerMma + g * 32, v);
-          if (g == kColsPerMma / 32 - 1) {
+      for (int st = 0; st <= nsteps; ++st) {
+        const bool flush = st == nsteps;
+        const int c = st / kStepsPerChunk, sc = st - c * kStepsPerChunk;
+        const int buf = (ci + c) & 1;
+        const uint32_t col0 = tmem_base + lane_addr + buf * kColsPerMma;
+        float v[kSStep];
+        if (!flush) {
+          if (sc == 0) {
+            const uint32_t tph = ((ci + c) >> 1) & 1;
+            if (!warp_wait(&tfull[buf], tph, status, abort)) { ok = false; break; }
+            tc_fence_after();
+            if (c == 0) {
+              // The maxima of the 64 groups of 4 columns are 64 different scores of the
+              // chunk, so its 32nd best (and the row's) is at least the 32nd largest.
+              float mx[64];
+#pragma unroll
+              for (int g = 0; g < 8; ++g) {
+                float w[32];
+                tmem_ld32(col0 + g * 32, w);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                  mx[g * 8 + i] = fmaxf(fmaxf(w[4 * i], w[4 * i + 1]),
+                                        fmaxf(w[4 * i + 2], w[4 * i + 3]));
+              }
+              tau0 = kth32_of_64(mx);
+            }
+          }
+          tmem_ld8(col0 + sc * kSStep, v);
+          if (sc == kStepsPerChunk - 1) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[buf]);
           }
-          // Columns arrive in increasing sub-key id, so a score equal to tau has a larger
-          // id than the 32nd best and loses: strict comparison is exact.
-          const int id0 = c * kColsPerMma + g * 32;
+        }
+        // Merge when the next step could overflow the log, and once at the end.
+        if (__any_sync(0xffffffffu, flush ? fresh > 0 : fresh > kSNewCap - kSStep)) {
+          float b[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            if (v[i] > tau) {
-              sv_s[cnt * kRowsPerTile + r] = v[i];
-              sv_i[cnt * kRowsPerTile + r] = id0 + i;
-              ++cnt;
+          for (int j = 0; j < 32; ++j) {
+            const int e = cnt - fresh + j;
+            b[j] = j < fresh ? lg_s[e * kRowsPerTile + r] : -INFINITY;
+          }
+          thread_sort32f(b);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) Ls[i] = fmaxf(Ls[i], b[31 - i]);
+#pragma unroll
+          for (int stride = 16; stride > 0; stride >>= 1)
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int j = i ^ stride;
+              if (j > i) {
+                const float a = Ls[i], bb = Ls[j];
+                Ls[i] = fmaxf(a, bb);
+                Ls[j] = fminf(a, bb);
+              }
+            }
+          tau_run = Ls[31];
+          // Keep every entry above tau_run and, of those equal to it, the first `eq`
+          // in id order (eq = how many of the best 32 scores equal tau_run): the log is
+          // then exactly the current best 32 by (score desc, id asc).
+          int eq = 0;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) eq += Ls[i] == tau_run ? 1 : 0;
+          int w = 0;
+#pragma unroll 4
+          for (int e = 0; e < kSLogCap; ++e) {
+            if (e < cnt) {
+              const float sv = lg_s[e * kRowsPerTile + r];
+              const int iv = lg_i[e * kRowsPerTile + r];
+              bool keep = sv > tau_run;
+              if (sv == tau_run && eq > 0) {
+                keep = true;
+                --eq;
+              }
+              if (keep) {
+                lg_s[w * kRowsPerTile + r] = sv;
+                lg_i[w * kRowsPerTile + r] = iv;
+                ++w;
+              }
             }
           }
-          if (__any_sync(0xffffffffu, cnt >= 32)) {
-            absorb_survivors(Ls, Li, sv_s, sv_i, cnt, r);
-            cnt = 0;
-            tau = Ls[31];
+          cnt = w;
+          fresh = 0;
+        }
+        if (!flush) {
+          const int id0 = c * kColsPerMma + sc * kSStep;
+#pragma unroll
+          for (int i = 0; i < kSStep; ++i) {
+            if (v[i] >= tau0 && v[i] > tau_run) {
+              lg_s[cnt * kRowsPerTile + r] = v[i];
+              lg_i[cnt * kRowsPerTile + r] = id0 + i;
+              ++cnt;
+              ++fresh;
+            }
           }
         }
       }
+      ci += nchunks;
       if (!ok) break;
-      absorb_survivors(Ls, Li, sv_s, sv_i, cnt, r);
       const int64_t row = static_cast<int64_t>(m) * kRowsPerTile + r;
       if (row < B) {
-        const int64_t o = (row * HS + hs) * static_cast<int64_t>(k);
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (j < k) {
-            list_s[o + j] = Ls[j];
-            list_i[o + j] = Li[j];
-          }
+        // The log now holds exactly the best 32 (in id order); the candidate kernel
+        // sorts them.
+        const int64_t o = (row * HS + hs) * static_cast<int64_t>(kList);
+#pragma unroll 4
+        for (int j = 0; j < kList; ++j) {
+          const bool have = j < cnt;
+          list_s[o + j] = have ? lg_s[j * kRowsPerTile + r] : -INFINITY;
+          list_i[o + j] = have ? lg_i[j * kRowsPerTile + r] : kIdPad;
+        }
       }
     }
   }
@@ -612,8 +661,8 @@ cudaError_t launch_score_topk_tc(const LayerArgs& a, const void* planes, float* 
   if (e != cudaSuccess) return e;
   const int64_t units = ((a.B + kRowsPerTile - 1) / kRowsPerTile) * 2 * a.H;
   const int grid = static_cast<int>(units < sm_count() ? units : sm_count());
-  score_topk_tc_kernel<<<grid, kTcThreads, smem, st>>>(tm_p, tm_k, static_cast<int>(a.B), a.H,
-                                                       a.dq, a.n, a.k, list_s, list_i, a.status);
+  score_topk_tc_kernel<<<grid, kSThreads, smem, st>>>(tm_p, tm_k, static_cast<int>(a.B), a.H,
+                                                      a.dq, a.n, list_s, list_i, a.status);
   return cudaGetLastError();
 }
 

@@ -14,7 +14,7 @@ bool tc_supported(int dtype, int d_model, int H, int dq, int n, int k);
 cudaError_t launch_query_tc(const LayerArgs& a, void* planes, cudaStream_t st);
 
 // Per-half scores of the three q planes against the sub-keys, accumulated in TMEM,
-// and the per-half top-k lists [B][H][2][k].
+// and the best 32 sub-keys of each half, [B][H][2][32] (in id order, not by score).
 cudaError_t launch_score_topk_tc(const LayerArgs& a, const void* planes, float* list_s,
                                  int* list_i, cudaStream_t st);
 
