@@ -255,6 +255,7 @@ def run_ours(args, rank, world, local_rank):
     hbm = float(pk["hbm_gbs"])
     bf16 = float(pk["bf16_tflops"])
     stage_avg = [m / max(1, calls) for m in stage_ms[:3]]
+    call_avg = stage_ms[3] / max(1, calls)
     names = ["query_network", "subkey_scores_topk", "select_softmax_gather"]
     dom = max(range(3), key=lambda i: stage_avg[i])
     F = w.H * w.dq
@@ -279,7 +280,8 @@ def run_ours(args, rank, world, local_rank):
     t_roof_ms = max(t_mem, t_gemm) * 1e3
     step_roof = {"t_roof_ms": t_roof_ms, "t_step_ms": ms_per_step, "frac": t_roof_ms / ms_per_step,
                  "bound": "hbm" if t_mem >= t_gemm else "tensor",
-                 "stage_ms": dict(zip(names, stage_avg)), "peak_kind": pk_kind}
+                 "stage_ms": dict(zip(names, stage_avg)), "call_ms": call_avg,
+                 "peak_kind": pk_kind}
 
     # ---- end to end: host x -> device, forward, out/indices/weights -> host
     x_h = L["x"].pin_memory()

@@ -24,7 +24,7 @@
  *     aligned. The library keeps no device state between calls and allocates no
  *     device memory: scratch is the caller's `workspace`.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
- *     All work is enqueued asynchronously on it; no call synchronises.
+ *     All work is enqueued asynchronously and ordered on it; no call synchronises.
  *   - Arguments are validated before anything is launched: a call that returns an
  *     error has launched nothing and written nothing.
  *   - Kernels that wait on hardware barriers give up after a bounded number of
@@ -93,6 +93,10 @@ size_t pkm_workspace_size(const pkm_shape* s, int for_backward);
  *   scores   [B][H][k]  fp32   kept key scores s1[i] + s2[j]; may be NULL
  * workspace: device scratch of at least pkm_workspace_size(s, 0) bytes, 256-byte
  *   aligned; its contents on entry do not matter.
+ * Large batches are processed in up to 4 sub-batches; the value gather of one
+ * sub-batch runs on a second stream owned by the library (one per device) while the
+ * next sub-batch is scored on `stream`. Event waits order both ways, so all of the
+ * call's work is complete when `stream` reaches the point after the call.
  * Returns PKM_OK or a status code above.
  */
 int pkm_forward(const pkm_shape* s, const void* x, const void* W_q, const float* bn_mean,
@@ -158,16 +162,17 @@ int pkm_device_status(void* workspace, void* stream);
 
 /*
  * Stage timing (a measurement aid; the pages have no counterpart). While enabled,
- * each pkm_forward call records a CUDA event on its stream before and after each of
- * its 3 stages (0 query network, 1 per-half scores and top-k, 2 candidate top-k,
- * softmax and value gather) and each pkm_backward_values call around its 2 stages
- * (0 grad wrt kept scores, 1 slot grouping and row sums). The events are owned by
- * the library (host-side handles only; no device memory).
+ * every kernel a call launches is bracketed by two CUDA events recorded on the stream
+ * it runs on, and so is the whole call (on `stream`). Forward stages: 0 query network,
+ * 1 per-half scores and best 32, 2 candidate top-k + softmax + value gather, 3 the
+ * whole call. Backward stages: 0 grad wrt kept scores, 1 slot grouping and row sums,
+ * 3 the whole call. The events are owned by the library (host-side handles only).
  * pkm_trace_read waits for the recorded events of `pass` (0 forward, 1 backward),
- * writes the summed milliseconds per stage into stage_ms[0..max_stages), the number
- * of traced calls into *calls, and the number of kernels the library launched since
- * the last read (all passes, traced or not) into *launches; then forgets them.
- * Returns PKM_OK, PKM_ERR_INVALID_ARG or PKM_ERR_CUDA.
+ * writes the summed milliseconds per stage into stage_ms[0..max_stages) (a stage that
+ * runs several launches per call, or overlaps another stage, sums their own
+ * durations), the number of traced calls into *calls, and the number of kernels the
+ * library launched since the last read (all passes, traced or not) into *launches;
+ * then forgets them. Returns PKM_OK, PKM_ERR_INVALID_ARG or PKM_ERR_CUDA.
  */
 int pkm_trace_enable(int on);
 int pkm_trace_read(int pass, double* stage_ms, int max_stages, int64_t* calls,

@@ -57,16 +57,34 @@ int validate_shape(const pkm_shape* s) {
 struct ForwardWs {
   int* status;
   float* q;         // SIMT path: fp32 q [B][H*dq]
-  void* planes;     // tensor path: bf16 q planes [3][B][H*dq]
+  void* planes;     // tensor path: bf16 q planes [3][sub][H*dq] of one sub-batch
   float* list_s;    // [B][H][2][32] best 32 per half (any order)
   int* list_i;      // [B][H][2][32]
 };
 
+// Tokens per pipelined sub-batch of the tensor-core path: PKM_SUBBATCHES (1..4,
+// default 1) sub-batches of at least 2048 tokens, a multiple of the 128-token tile.
+int64_t sub_batch_tokens(int64_t B) {
+  const char* env = getenv("PKM_SUBBATCHES");
+  int64_t want = env ? atoi(env) : 1;
+  if (want < 1) want = 1;
+  if (want > 4) want = 4;
+  int64_t S = B / 2048;
+  if (S > want) S = want;
+  if (S < 1) S = 1;
+  int64_t sub = (B + S - 1) / S;
+  sub = (sub + 127) / 128 * 128;
+  return sub < B ? sub : B;
+}
+
 size_t forward_ws(const pkm_shape* s, ForwardWs* w, char* base) {
   const int64_t F = static_cast<int64_t>(s->H) * s->dq;
   const int64_t L = s->B * s->H * 2 * static_cast<int64_t>(pkm::kMaxK);
+  const size_t qbytes = choose_path(s) == Path::kTensor
+                            ? static_cast<size_t>(sub_batch_tokens(s->B)) * F * 6
+                            : static_cast<size_t>(s->B) * F * 4;
   size_t off = pkm::kStatusBytes;
-  const size_t o_q = off;  off += align256(static_cast<size_t>(s->B) * F * 6);  // fp32 q or 3 bf16 planes
+  const size_t o_q = off;  off += align256(qbytes);
   const size_t o_ls = off; off += align256(sizeof(float) * L);
   const size_t o_li = off; off += align256(sizeof(int) * L);
   if (w && base) {
@@ -84,25 +102,28 @@ size_t backward_ws(const pkm_shape* s, pkm::BackwardWs* w, char* base) {
 }
 
 // ---------------------------------------------------------------------------
-// Stage tracing: when enabled, every call records a CUDA event on its stream at
-// each stage boundary; pkm_trace_read() waits for them and sums the durations.
+// Stage tracing: when enabled, every kernel a call launches is bracketed by two CUDA
+// events on the stream it runs on; pkm_trace_read() waits for them and sums the
+// durations per stage.
 // ---------------------------------------------------------------------------
-constexpr int kMaxStages = 4;
 constexpr int kPasses = 2;
 
-struct TraceSet {
+struct TraceSpan {
+  int stage;
+  cudaEvent_t start, stop;
+};
+struct TraceCall {
   int pass;
-  int nstages;
-  cudaEvent_t ev[kMaxStages + 1];
+  std::vector<TraceSpan> spans;
 };
 
 std::mutex g_trace_mu;
 bool g_trace_on = false;
-std::vector<TraceSet> g_trace_pending;
-std::vector<cudaEvent_t> g_event_pool;
+std::vector<TraceCall> g_trace_pending;
+std::vector<cudaEvent_t> g_event_pool;  // timing events, reused
 int64_t g_launches = 0;
 
-cudaEvent_t take_event() {
+cudaEvent_t take_timing_event() {
   if (!g_event_pool.empty()) {
     cudaEvent_t e = g_event_pool.back();
     g_event_pool.pop_back();
@@ -113,38 +134,82 @@ cudaEvent_t take_event() {
   return e;
 }
 
-// Records stage boundaries for one call (no-op when tracing is off).
-struct Tracer {
-  bool on = false;
-  TraceSet set{};
-  int next = 0;
-  cudaStream_t st;
-  Tracer(int pass, int nstages, cudaStream_t s) : st(s) {
+class Tracer {
+ public:
+  Tracer(int pass) {
     std::lock_guard<std::mutex> lk(g_trace_mu);
-    on = g_trace_on;
-    if (!on) return;
-    set.pass = pass;
-    set.nstages = nstages;
-    for (int i = 0; i <= nstages; ++i) {
-      set.ev[i] = take_event();
-      if (!set.ev[i]) on = false;
-    }
+    on_ = g_trace_on;
+    call_.pass = pass;
   }
-  void mark() {
-    if (on && next <= set.nstages) cudaEventRecord(set.ev[next++], st);
+  // Spans nest: end() closes the most recently begun span that is still open.
+  void begin(int stage, cudaStream_t st) {
+    if (!on_) return;
+    std::lock_guard<std::mutex> lk(g_trace_mu);
+    TraceSpan sp{stage, take_timing_event(), take_timing_event()};
+    if (!sp.start || !sp.stop) {
+      if (sp.start) g_event_pool.push_back(sp.start);
+      if (sp.stop) g_event_pool.push_back(sp.stop);
+      on_ = false;
+      return;
+    }
+    cudaEventRecord(sp.start, st);
+    open_.push_back(call_.spans.size());
+    call_.spans.push_back(sp);
+  }
+  void end(cudaStream_t st) {
+    if (!on_ || open_.empty()) return;
+    cudaEventRecord(call_.spans[open_.back()].stop, st);
+    open_.pop_back();
   }
   void finish(bool ok, int launches) {
     std::lock_guard<std::mutex> lk(g_trace_mu);
     if (ok) g_launches += launches;
-    if (!on) return;
-    if (ok && next == set.nstages + 1) {
-      g_trace_pending.push_back(set);
+    if (!on_) return;
+    if (ok && open_.empty()) {
+      g_trace_pending.push_back(call_);
     } else {
-      for (int i = 0; i <= set.nstages; ++i)
-        if (set.ev[i]) g_event_pool.push_back(set.ev[i]);
+      for (const TraceSpan& sp : call_.spans) {
+        g_event_pool.push_back(sp.start);
+        g_event_pool.push_back(sp.stop);
+      }
     }
   }
+
+ private:
+  bool on_ = false;
+  TraceCall call_;
+  std::vector<size_t> open_;
 };
+
+// ---------------------------------------------------------------------------
+// Second stream per device for the pipelined forward, plus ordering events.
+// ---------------------------------------------------------------------------
+constexpr int kMaxDevices = 64;
+std::mutex g_aux_mu;
+cudaStream_t g_aux_stream[kMaxDevices] = {};
+std::vector<cudaEvent_t> g_sync_events[kMaxDevices];
+size_t g_sync_next[kMaxDevices] = {};
+
+// The calling thread's device's helper stream and `n` ordering events (created on
+// first use, then reused round robin).
+int aux_resources(int n, cudaStream_t* aux, cudaEvent_t* evs) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PKM_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_aux_mu);
+  if (!g_aux_stream[dev]) {
+    if (cudaStreamCreateWithFlags(&g_aux_stream[dev], cudaStreamNonBlocking) != cudaSuccess)
+      return PKM_ERR_CUDA;
+    for (int i = 0; i < 64; ++i) {
+      cudaEvent_t e;
+      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return PKM_ERR_CUDA;
+      g_sync_events[dev].push_back(e);
+    }
+  }
+  *aux = g_aux_stream[dev];
+  std::vector<cudaEvent_t>& pool = g_sync_events[dev];
+  for (int i = 0; i < n; ++i) evs[i] = pool[(g_sync_next[dev]++) % pool.size()];
+  return PKM_OK;
+}
 
 }  // namespace
 
@@ -163,20 +228,21 @@ int pkm_trace_read(int pass, double* stage_ms, int max_stages, int64_t* calls,
   std::lock_guard<std::mutex> lk(g_trace_mu);
   for (int i = 0; i < max_stages; ++i) stage_ms[i] = 0.0;
   int64_t n = 0;
-  std::vector<TraceSet> keep;
+  std::vector<TraceCall> keep;
   int rc = PKM_OK;
-  for (const TraceSet& t : g_trace_pending) {
-    if (t.pass != pass) {
-      keep.push_back(t);
+  for (const TraceCall& c : g_trace_pending) {
+    if (c.pass != pass) {
+      keep.push_back(c);
       continue;
     }
-    if (cudaEventSynchronize(t.ev[t.nstages]) != cudaSuccess) rc = PKM_ERR_CUDA;
-    for (int i = 0; i < t.nstages && i < max_stages; ++i) {
+    for (const TraceSpan& sp : c.spans) {
+      if (cudaEventSynchronize(sp.stop) != cudaSuccess) rc = PKM_ERR_CUDA;
       float ms = 0.f;
-      if (cudaEventElapsedTime(&ms, t.ev[i], t.ev[i + 1]) != cudaSuccess) rc = PKM_ERR_CUDA;
-      stage_ms[i] += ms;
+      if (cudaEventElapsedTime(&ms, sp.start, sp.stop) != cudaSuccess) rc = PKM_ERR_CUDA;
+      if (sp.stage < max_stages) stage_ms[sp.stage] += ms;
+      g_event_pool.push_back(sp.start);
+      g_event_pool.push_back(sp.stop);
     }
-    for (int i = 0; i <= t.nstages; ++i) g_event_pool.push_back(t.ev[i]);
     ++n;
   }
   g_trace_pending.swap(keep);
@@ -221,24 +287,69 @@ int pkm_forward(const pkm_shape* s, const void* x, const void* W_q, const float*
   LayerArgs a{s->B, s->d_model, s->H, s->dq, s->n, s->k, s->v, s->dtype, s->bn_eps,
               x, W_q, bn_mean, bn_var, bn_gamma, bn_beta, subkeys, values, w.status};
   if (cudaMemsetAsync(w.status, 0, sizeof(int), st) != cudaSuccess) return PKM_ERR_CUDA;
-  // Stages: 0 query network, 1 per-half scores + top-k, 2 candidate top-k + softmax + gather.
-  Tracer tr(0, 3, st);
-  cudaError_t e;
-  tr.mark();
-  if (choose_path(s) == Path::kTensor) {
-    e = pkm::launch_query_tc(a, w.planes, st);
-    tr.mark();
-    if (e == cudaSuccess) e = pkm::launch_score_topk_tc(a, w.planes, w.list_s, w.list_i, st);
-  } else {
+  // Stages: 0 query network, 1 per-half scores + best 32, 2 candidate top-k + softmax +
+  // gather, 3 the whole call.
+  Tracer tr(0);
+  cudaError_t e = cudaSuccess;
+  int launches = 0;
+  tr.begin(3, st);
+  if (choose_path(s) == Path::kSimt) {
+    tr.begin(0, st);
     e = pkm::launch_query_bn_simt(a, w.q, st);
-    tr.mark();
+    tr.end(st);
+    tr.begin(1, st);
     if (e == cudaSuccess) e = pkm::launch_subkey_topk_simt(a, w.q, w.list_s, w.list_i, st);
+    tr.end(st);
+    tr.begin(2, st);
+    if (e == cudaSuccess)
+      e = pkm::launch_select_gather(a, w.list_s, w.list_i, out, indices, weights, scores, st);
+    tr.end(st);
+    launches = 3;
+  } else {
+    // Pipelined over sub-batches: the query network and per-half search of sub-batch
+    // i+1 run on the caller's stream while the gather of sub-batch i runs on a second
+    // stream (it is bound by HBM, the others by the tensor cores and ALUs). The second
+    // stream waits for each sub-batch's lists and the caller's stream waits for the
+    // last gather, so the call stays ordered on `stream`.
+    const int64_t sub = sub_batch_tokens(s->B);
+    const int nsub = static_cast<int>((s->B + sub - 1) / sub);
+    cudaStream_t aux;
+    cudaEvent_t ev[5];
+    if (aux_resources(nsub + 1, &aux, ev) != PKM_OK) return PKM_ERR_CUDA;
+    const size_t xsz = s->dtype == PKM_F32 ? 4 : 2;
+    const int64_t per_tok = static_cast<int64_t>(s->H) * 2 * pkm::kMaxK;
+    for (int i = 0; i < nsub && e == cudaSuccess; ++i) {
+      const int64_t t0 = i * sub;
+      const int64_t bs = (s->B - t0 < sub) ? s->B - t0 : sub;
+      LayerArgs ai = a;
+      ai.B = bs;
+      ai.x = static_cast<const char*>(x) + t0 * s->d_model * xsz;
+      float* ls = w.list_s + t0 * per_tok;
+      int* li = w.list_i + t0 * per_tok;
+      tr.begin(0, st);
+      e = pkm::launch_query_tc(ai, w.planes, st);
+      tr.end(st);
+      tr.begin(1, st);
+      if (e == cudaSuccess) e = pkm::launch_score_topk_tc(ai, w.planes, ls, li, st);
+      tr.end(st);
+      if (e == cudaSuccess) e = cudaEventRecord(ev[i], st);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(aux, ev[i], 0);
+      tr.begin(2, aux);
+      const int64_t ok = t0 * s->H * static_cast<int64_t>(s->k);
+      if (e == cudaSuccess)
+        e = pkm::launch_select_gather(ai, ls, li, out + t0 * s->v, indices + ok, weights + ok,
+                                      scores ? scores + ok : nullptr, aux);
+      tr.end(aux);
+      launches += 3;
+    }
+    // Always join, even after an error, so the caller's stream never runs ahead of
+    // work already queued on the second stream.
+    cudaError_t e2 = cudaEventRecord(ev[nsub], aux);
+    if (e2 == cudaSuccess) e2 = cudaStreamWaitEvent(st, ev[nsub], 0);
+    if (e == cudaSuccess) e = e2;
   }
-  tr.mark();
-  if (e == cudaSuccess)
-    e = pkm::launch_select_gather(a, w.list_s, w.list_i, out, indices, weights, scores, st);
-  tr.mark();
-  tr.finish(e == cudaSuccess, 3);
+  tr.end(st);
+  tr.finish(e == cudaSuccess, launches);
   return e == cudaSuccess ? PKM_OK : PKM_ERR_CUDA;
 }
 
@@ -263,13 +374,19 @@ int pkm_backward_values(const pkm_shape* s, const void* values, const int32_t* i
   backward_ws(s, &w, static_cast<char*>(workspace));
   int* status = static_cast<int*>(workspace);
   if (cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess) return PKM_ERR_CUDA;
-  // Stages: 0 grad wrt kept scores, 1 slot grouping + row sums into grad_values.
-  Tracer tr(1, 2, st);
-  tr.mark();
+  // Stages: 0 grad wrt kept scores, 1 slot grouping + row sums into grad_values,
+  // 3 the whole call.
+  Tracer tr(1);
+  tr.begin(3, st);
+  tr.begin(0, st);
   cudaError_t e = pkm::launch_backward_values(
       s->B, s->H, s->k, s->v, s->dtype, static_cast<int64_t>(s->n) * s->n, values, indices,
-      weights, grad_out, grad_values, grad_scores, w, status, st, [&] { tr.mark(); });
-  tr.mark();
+      weights, grad_out, grad_values, grad_scores, w, status, st, [&] {
+        tr.end(st);
+        tr.begin(1, st);
+      });
+  tr.end(st);
+  tr.end(st);
   tr.finish(e == cudaSuccess, grad_scores ? 7 : 6);
   return e == cudaSuccess ? PKM_OK : PKM_ERR_CUDA;
 }

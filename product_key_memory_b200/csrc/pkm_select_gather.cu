@@ -23,6 +23,8 @@
 namespace pkm {
 
 constexpr int kSgWarps = 4;
+// Candidate pairs (a, b) with (a+1)(b+1) <= k number sum_a floor(k/(a+1)) <= 119 for k <= 32.
+constexpr int kMaxPairs = 128;
 
 template <typename T, int MAXV>
 __global__ void __launch_bounds__(kSgWarps * 32) select_gather_kernel(
@@ -33,10 +35,10 @@ __global__ void __launch_bounds__(kSgWarps * 32) select_gather_kernel(
   constexpr int VPER = Vec<T>::kPer;
   constexpr int U = MAXV >= 8 ? 2 : 4;  // rows in flight per lane step
   extern __shared__ int sg_smem[];
-  int* pairs = sg_smem;                                  // [k*k] (a | b << 8)
+  int* pairs = sg_smem;                                  // [kMaxPairs] (a | b << 8)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int HK = H * k;
-  int* rows = sg_smem + kMaxK * kMaxK + warp * 2 * HK;   // [HK]
+  int* rows = sg_smem + kMaxPairs + warp * 2 * HK;       // [HK]
   float* wts = reinterpret_cast<float*>(rows + HK);      // [HK]
   __shared__ int npairs_s;
 
@@ -163,7 +165,7 @@ bool select_gather_supported(int H, int k, int v, int dtype) {
 template <typename T, int MAXV>
 static cudaError_t launch_sg(const LayerArgs& a, const float* ls, const int* li, float* out,
                              int* idx, float* w, float* sc, cudaStream_t st) {
-  const size_t smem = sizeof(int) * (kMaxK * kMaxK + kSgWarps * 2 * a.H * a.k);
+  const size_t smem = sizeof(int) * (kMaxPairs + kSgWarps * 2 * a.H * a.k);
   cudaError_t e = cudaFuncSetAttribute(select_gather_kernel<T, MAXV>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

@@ -241,23 +241,30 @@ __global__ void __launch_bounds__(kTcThreads, 1) query_tc_kernel(
 }
 
 // ===========================================================================
-// Per-half scores and top-k
+// Per-half scores and the best 32 per row
 // ===========================================================================
-constexpr int kSEpiWarps = 4;  // one epilogue warp per TMEM lane quadrant
+// Two epilogue warp sets work on alternate units of the CTA, each with its own TMEM
+// accumulator (256 columns) and its own survivor log, so two warps share each SM
+// sub-partition. The MMA issuer interleaves the two sets' chunks.
+constexpr int kSSets = 2;
+constexpr int kSEpiWarps = 4 * kSSets;
 constexpr int kSThreads = 64 + 32 * kSEpiWarps;
-constexpr int kSStages = 2;
-constexpr uint32_t kSPlaneBytes = kRowsPerTile * kKBlock * 2;      // 16 KiB
-constexpr uint32_t kSABytes = 3 * kSPlaneBytes;                     // 48 KiB
-constexpr uint32_t kSBBytes = kColsPerMma * kKBlock * 2;            // 32 KiB
-constexpr uint32_t kSStageBytes = kSABytes + kSBBytes;              // 80 KiB
-constexpr int kList = kMaxK;          // entries per per-half list (the best 32, unsorted)
+constexpr int kSK = 32;                                             // K per stage
+constexpr int kSStages = 3;
+constexpr uint32_t kSPlaneBytes = kRowsPerTile * kSK * 2;           // 8 KiB
+constexpr uint32_t kSABytes = 3 * kSPlaneBytes;                     // 24 KiB
+constexpr uint32_t kSBBytes = kColsPerMma * kSK * 2;                // 16 KiB
+constexpr uint32_t kSStageBytes = kSABytes + kSBBytes;              // 40 KiB
+constexpr int kList = kMaxK;          // entries per per-half list (the best 32, any order)
 constexpr int kSStep = 8;             // columns read from TMEM per step
-constexpr int kSNewCap = 24;          // survivors logged between two merges
+constexpr int kSNewCap = 32;          // survivors logged between two merges
 constexpr int kSLogCap = kList + kSNewCap;
+constexpr int kSTrash = kSLogCap;     // log slot that absorbs the stores of rejected scores
+constexpr int kSLogRows = kSLogCap + 1;
 
 size_t score_tc_smem_bytes() {
-  // stages + per-row log of (score, id) + barriers and flags
-  return 1024 + kSStages * kSStageBytes + kSLogCap * kRowsPerTile * 8 + 256;
+  // stages + per-set log: fp32 scores and 16-bit ids for 128 rows + barriers
+  return 1024 + kSStages * kSStageBytes + kSSets * kSLogRows * kRowsPerTile * (4 + 2) + 256;
 }
 
 // Sort 32 floats held by one thread, largest first (bitonic network of min/max).
@@ -298,14 +305,14 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
     int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* stages = align1024(smem_raw);
-  // per-row log: [kSLogCap][128] scores, then the same for ids
-  float* lg_s = reinterpret_cast<float*>(stages + kSStages * kSStageBytes);
-  int* lg_i = reinterpret_cast<int*>(lg_s + kSLogCap * kRowsPerTile);
-  uint64_t* full = reinterpret_cast<uint64_t*>(lg_i + kSLogCap * kRowsPerTile);
+  // per set: log scores [kSLogRows][128], then (after both sets) log ids [kSLogRows][128]
+  float* lg_s_all = reinterpret_cast<float*>(stages + kSStages * kSStageBytes);
+  uint16_t* lg_i_all = reinterpret_cast<uint16_t*>(lg_s_all + kSSets * kSLogRows * kRowsPerTile);
+  uint64_t* full = reinterpret_cast<uint64_t*>(lg_i_all + kSSets * kSLogRows * kRowsPerTile);
   uint64_t* empty = full + kSStages;
-  uint64_t* tfull = empty + kSStages;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* drain = tempty + 2;
+  uint64_t* tfull = empty + kSStages;   // [kSSets]
+  uint64_t* tempty = tfull + kSSets;    // [kSSets]
+  uint64_t* drain = tempty + kSSets;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -315,16 +322,20 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
   const int HS = 2 * H;
   const int nunits = mt * HS;
   const int nchunks = n / kColsPerMma;
-  const int kiters = half / kKBlock;
+  const int kiters = half / kSK;
+  // This CTA's units are blockIdx.x + j * gridDim.x; set s takes the j with j % 2 == s.
+  const int myunits = nunits > static_cast<int>(blockIdx.x)
+                          ? (nunits - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1
+                          : 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kSStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kSSets; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], kSEpiWarps);
+      mbar_init(&tempty[b], 4);
     }
     mbar_init(drain, 1);
     *abort = 0;
@@ -345,31 +356,35 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- TMA producer: per K step three q planes + one sub-key tile
+      // ---------------- TMA producer: per K step three q planes + one sub-key tile, in
+      // the order the MMA issuer consumes them (chunks of the two sets interleaved)
       uint32_t s = 0, ph = 0;
       uint32_t issued_phase[kSStages];
       bool issued[kSStages];
       for (int i = 0; i < kSStages; ++i) issued[i] = false;
       bool ok = true;
-      for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
-        const int m = u / HS, hs = u - m * HS;
-        const int h = hs >> 1, side = hs & 1;
-        const int xq = h * dq + side * half;
+      for (int j0 = 0; j0 < myunits && ok; j0 += kSSets)
         for (int c = 0; c < nchunks && ok; ++c)
-          for (int kb = 0; kb < kiters; ++kb) {
-            if (!mbar_wait(&empty[s], ph ^ 1, status, abort)) { ok = false; break; }
-            uint8_t* a = stages + s * kSStageBytes;
-            mbar_arrive_expect_tx(&full[s], kSStageBytes);
+          for (int set = 0; set < kSSets && ok; ++set) {
+            const int j = j0 + set;
+            if (j >= myunits) break;
+            const int u = blockIdx.x + j * gridDim.x;
+            const int m = u / HS, hs = u - m * HS;
+            const int xq = (hs >> 1) * dq + (hs & 1) * half;
+            for (int kb = 0; kb < kiters; ++kb) {
+              if (!mbar_wait(&empty[s], ph ^ 1, status, abort)) { ok = false; break; }
+              uint8_t* a = stages + s * kSStageBytes;
+              mbar_arrive_expect_tx(&full[s], kSStageBytes);
 #pragma unroll
-            for (int p = 0; p < 3; ++p)
-              tma_load_3d(a + p * kSPlaneBytes, &tm_planes, &full[s], xq + kb * kKBlock,
-                          m * kRowsPerTile, p);
-            tma_load_2d(a + kSABytes, &tm_keys, &full[s], kb * kKBlock, hs * n + c * kColsPerMma);
-            issued[s] = true;
-            issued_phase[s] = ph;
-            if (++s == kSStages) { s = 0; ph ^= 1; }
+              for (int p = 0; p < 3; ++p)
+                tma_load_3d(a + p * kSPlaneBytes, &tm_planes, &full[s], xq + kb * kSK,
+                            m * kRowsPerTile, p);
+              tma_load_2d(a + kSABytes, &tm_keys, &full[s], kb * kSK, hs * n + c * kColsPerMma);
+              issued[s] = true;
+              issued_phase[s] = ph;
+              if (++s == kSStages) { s = 0; ph ^= 1; }
+            }
           }
-      }
       if (!ok) {
         for (int i = 0; i < kSStages; ++i)
           if (issued[i]) {
@@ -382,34 +397,36 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      // ---------------- MMA issuer: chunk of 256 sub-keys = kiters x 3 planes x 4 MMAs
+      // ---------------- MMA issuer: chunk of 256 sub-keys = kiters x 3 planes x 2 MMAs
       const uint32_t idesc = idesc_bf16_f32(kRowsPerTile, kColsPerMma);
       uint32_t s = 0, ph = 0;
+      int uses[kSSets] = {0, 0};  // chunks written into each set's accumulator so far
       bool ok = true;
-      int ci = 0;
-      for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x)
-        for (int c = 0; c < nchunks && ok; ++c, ++ci) {
-          const int buf = ci & 1;
-          const uint32_t tph = (ci >> 1) & 1;
-          if (!mbar_wait(&tempty[buf], tph ^ 1, status, abort)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t d_tmem = tmem_base + buf * kColsPerMma;
-          for (int kb = 0; kb < kiters; ++kb) {
-            if (!mbar_wait(&full[s], ph, status, abort)) { ok = false; break; }
+      for (int j0 = 0; j0 < myunits && ok; j0 += kSSets)
+        for (int c = 0; c < nchunks && ok; ++c)
+          for (int set = 0; set < kSSets && ok; ++set) {
+            if (j0 + set >= myunits) break;
+            const uint32_t tph = uses[set] & 1;
+            if (!mbar_wait(&tempty[set], tph ^ 1, status, abort)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t a = smem_addr(stages + s * kSStageBytes);
-            const uint32_t b = a + kSABytes;
+            const uint32_t d_tmem = tmem_base + set * kColsPerMma;
+            for (int kb = 0; kb < kiters; ++kb) {
+              if (!mbar_wait(&full[s], ph, status, abort)) { ok = false; break; }
+              tc_fence_after();
+              const uint32_t a = smem_addr(stages + s * kSStageBytes);
+              const uint32_t b = a + kSABytes;
 #pragma unroll
-            for (int p = 0; p < 3; ++p)
+              for (int p = 0; p < 3; ++p)
 #pragma unroll
-              for (int j = 0; j < kKBlock / 16; ++j)
-                mma_bf16(d_tmem, sw128_desc(a + p * kSPlaneBytes, j * 32),
-                         sw128_desc(b, j * 32), idesc, (kb | p | j) != 0);
-            mma_commit(&empty[s]);
-            if (++s == kSStages) { s = 0; ph ^= 1; }
+                for (int jj = 0; jj < kSK / 16; ++jj)
+                  mma_bf16(d_tmem, sw64_desc(a + p * kSPlaneBytes, jj * 32),
+                           sw64_desc(b, jj * 32), idesc, (kb | p | jj) != 0);
+              mma_commit(&empty[s]);
+              if (++s == kSStages) { s = 0; ph ^= 1; }
+            }
+            if (ok) mma_commit(&tfull[set]);
+            ++uses[set];
           }
-          if (ok) mma_commit(&tfull[buf]);
-        }
       mma_commit(drain);
       const uint64_t t0 = global_timer_ns();
       while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
@@ -420,12 +437,16 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
     // Ls holds the 32 largest scores seen so far (values only, sorted); the log in
     // shared memory holds (score, id) of every element that can still be among the
     // best 32. Columns arrive in increasing sub-key id, so the log is in id order.
+    const int set = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
+    float* lg_s = lg_s_all + set * kSLogRows * kRowsPerTile;  // [kSLogRows][128]
+    uint16_t* lg_i = lg_i_all + set * kSLogRows * kRowsPerTile;
     constexpr int kStepsPerChunk = kColsPerMma / kSStep;
-    int ci = 0;
-    for (int u = blockIdx.x; u < nunits; u += gridDim.x) {
+    int uses = 0;
+    for (int j = set; j < myunits; j += kSSets) {
+      const int u = blockIdx.x + j * gridDim.x;
       const int m = u / HS, hs = u - m * HS;
       float Ls[32];
 #pragma unroll
@@ -434,20 +455,19 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
       // the 32nd best of the first chunk, hence of the row) and > tau_run (the current
       // 32nd best: an equal score comes later in id order and loses the tie).
       float tau0 = -INFINITY, tau_run = -INFINITY;
-      int cnt = 0, fresh = 0;  // log entries; entries logged since the last merge
+      float thr = -INFINITY;   // v > thr  <=>  v >= tau0 && v > tau_run
+      int cnt = 0, kept = 0;   // log entries; entries kept by the last merge
       bool ok = true;
       const int nsteps = nchunks * kStepsPerChunk;
+      const uint32_t col0 = tmem_base + lane_addr + set * kColsPerMma;
 #pragma unroll 1
       for (int st = 0; st <= nsteps; ++st) {
         const bool flush = st == nsteps;
         const int c = st / kStepsPerChunk, sc = st - c * kStepsPerChunk;
-        const int buf = (ci + c) & 1;
-        const uint32_t col0 = tmem_base + lane_addr + buf * kColsPerMma;
         float v[kSStep];
         if (!flush) {
           if (sc == 0) {
-            const uint32_t tph = ((ci + c) >> 1) & 1;
-            if (!warp_wait(&tfull[buf], tph, status, abort)) { ok = false; break; }
+            if (!warp_wait(&tfull[set], (uses + c) & 1, status, abort)) { ok = false; break; }
             tc_fence_after();
             if (c == 0) {
               // The maxima of the 64 groups of 4 columns are 64 different scores of the
@@ -463,22 +483,24 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
                                         fmaxf(w[4 * i + 2], w[4 * i + 3]));
               }
               tau0 = kth32_of_64(mx);
+              thr = fmaxf(nextafterf(tau0, -INFINITY), tau_run);
             }
           }
           tmem_ld8(col0 + sc * kSStep, v);
           if (sc == kStepsPerChunk - 1) {
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[buf]);
+            if (lane == 0) mbar_arrive(&tempty[set]);
           }
         }
         // Merge when the next step could overflow the log, and once at the end.
+        const int fresh = cnt - kept;
         if (__any_sync(0xffffffffu, flush ? fresh > 0 : fresh > kSNewCap - kSStep)) {
           float b[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int e = cnt - fresh + j;
-            b[j] = j < fresh ? lg_s[e * kRowsPerTile + r] : -INFINITY;
+          for (int q = 0; q < 32; ++q) {
+            const int e = kept + q;
+            b[q] = q < fresh ? lg_s[e * kRowsPerTile + r] : -INFINITY;
           }
           thread_sort32f(b);
 #pragma unroll
@@ -487,55 +509,71 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
           for (int stride = 16; stride > 0; stride >>= 1)
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-              const int j = i ^ stride;
-              if (j > i) {
-                const float a = Ls[i], bb = Ls[j];
+              const int jj = i ^ stride;
+              if (jj > i) {
+                const float a = Ls[i], bb = Ls[jj];
                 Ls[i] = fmaxf(a, bb);
-                Ls[j] = fminf(a, bb);
+                Ls[jj] = fminf(a, bb);
               }
             }
           tau_run = Ls[31];
-          // Keep every entry above tau_run and, of those equal to it, the first `eq`
-          // in id order (eq = how many of the best 32 scores equal tau_run): the log is
-          // then exactly the current best 32 by (score desc, id asc).
-          int eq = 0;
-#pragma unroll
-          for (int i = 0; i < 32; ++i) eq += Ls[i] == tau_run ? 1 : 0;
+          // Branch-free in-place compaction to the entries >= tau_run: each entry is
+          // rewritten either to slot w (w <= e, so nothing unread is overwritten) or to
+          // the trash slot. That keeps the current best 32 plus any later entry tied
+          // with the 32nd score.
           int w = 0;
+          const int cmax = __reduce_max_sync(0xffffffffu, cnt);
 #pragma unroll 4
-          for (int e = 0; e < kSLogCap; ++e) {
-            if (e < cnt) {
+          for (int e = 0; e < cmax; ++e) {
+            const float sv = lg_s[e * kRowsPerTile + r];
+            const uint16_t iv = lg_i[e * kRowsPerTile + r];
+            const bool keep = e < cnt && sv >= tau_run;
+            const int dst = keep ? w : kSTrash;
+            lg_s[dst * kRowsPerTile + r] = sv;
+            lg_i[dst * kRowsPerTile + r] = iv;
+            w += keep ? 1 : 0;
+          }
+          if (__any_sync(0xffffffffu, w > kList)) {
+            // Rare: ties at the 32nd score. Of the entries equal to tau_run keep the first
+            // `eq` in id order (eq = how many of the best 32 scores equal it), so the log
+            // is exactly the best 32 by (score desc, id asc).
+            int eq = 0;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) eq += Ls[i] == tau_run ? 1 : 0;
+            const int wmax = __reduce_max_sync(0xffffffffu, w);
+            int w2 = 0;
+            for (int e = 0; e < wmax; ++e) {
               const float sv = lg_s[e * kRowsPerTile + r];
-              const int iv = lg_i[e * kRowsPerTile + r];
-              bool keep = sv > tau_run;
-              if (sv == tau_run && eq > 0) {
-                keep = true;
-                --eq;
-              }
-              if (keep) {
-                lg_s[w * kRowsPerTile + r] = sv;
-                lg_i[w * kRowsPerTile + r] = iv;
-                ++w;
-              }
+              const uint16_t iv = lg_i[e * kRowsPerTile + r];
+              const bool tie = e < w && sv == tau_run && eq > 0;
+              const bool keep = e < w && (sv > tau_run || tie);
+              eq -= tie ? 1 : 0;
+              const int dst = keep ? w2 : kSTrash;
+              lg_s[dst * kRowsPerTile + r] = sv;
+              lg_i[dst * kRowsPerTile + r] = iv;
+              w2 += keep ? 1 : 0;
             }
+            w = w2;
           }
           cnt = w;
-          fresh = 0;
+          kept = w;
+          thr = fmaxf(nextafterf(tau0, -INFINITY), tau_run);
         }
         if (!flush) {
+          // Branch-free filter: a kept score goes to the next log slot, a rejected one
+          // to the trash slot.
           const int id0 = c * kColsPerMma + sc * kSStep;
 #pragma unroll
           for (int i = 0; i < kSStep; ++i) {
-            if (v[i] >= tau0 && v[i] > tau_run) {
-              lg_s[cnt * kRowsPerTile + r] = v[i];
-              lg_i[cnt * kRowsPerTile + r] = id0 + i;
-              ++cnt;
-              ++fresh;
-            }
+            const bool take = v[i] > thr;
+            const int dst = take ? cnt : kSTrash;
+            lg_s[dst * kRowsPerTile + r] = v[i];
+            lg_i[dst * kRowsPerTile + r] = static_cast<uint16_t>(id0 + i);
+            cnt += take ? 1 : 0;
           }
         }
       }
-      ci += nchunks;
+      uses += nchunks;
       if (!ok) break;
       const int64_t row = static_cast<int64_t>(m) * kRowsPerTile + r;
       if (row < B) {
@@ -543,10 +581,10 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
         // sorts them.
         const int64_t o = (row * HS + hs) * static_cast<int64_t>(kList);
 #pragma unroll 4
-        for (int j = 0; j < kList; ++j) {
-          const bool have = j < cnt;
-          list_s[o + j] = have ? lg_s[j * kRowsPerTile + r] : -INFINITY;
-          list_i[o + j] = have ? lg_i[j * kRowsPerTile + r] : kIdPad;
+        for (int q = 0; q < kList; ++q) {
+          const bool have = q < cnt;
+          list_s[o + q] = have ? lg_s[q * kRowsPerTile + r] : -INFINITY;
+          list_i[o + q] = have ? static_cast<int>(lg_i[q * kRowsPerTile + r]) : kIdPad;
         }
       }
     }
@@ -585,13 +623,14 @@ EncodeTiledFn encode_fn() {
 // bf16 tensor map with a {64 x rows} box and the 128-byte swizzle. dims/strides are
 // innermost first; strides are in bytes for dims 1.. (dim 0 is contiguous).
 bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
-              const cuuint64_t* strides, const cuuint32_t* box) {
+              const cuuint64_t* strides, const cuuint32_t* box,
+              CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides,
-            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 int sm_count() {
@@ -647,12 +686,13 @@ cudaError_t launch_score_topk_tc(const LayerArgs& a, const void* planes, float* 
   CUtensorMap tm_p, tm_k;
   const cuuint64_t pd[3] = {static_cast<cuuint64_t>(F), static_cast<cuuint64_t>(a.B), 3};
   const cuuint64_t ps[2] = {static_cast<cuuint64_t>(F) * 2, static_cast<cuuint64_t>(F) * 2 * a.B};
-  const cuuint32_t pb[3] = {kKBlock, kRowsPerTile, 1};
+  const cuuint32_t pb[3] = {kSK, kRowsPerTile, 1};
   const cuuint64_t kd[2] = {static_cast<cuuint64_t>(half),
                             static_cast<cuuint64_t>(a.H) * 2 * a.n};
   const cuuint64_t ks[1] = {static_cast<cuuint64_t>(half) * 2};
-  const cuuint32_t kbx[2] = {kKBlock, kColsPerMma};
-  if (!make_map(&tm_p, planes, 3, pd, ps, pb) || !make_map(&tm_k, a.subkeys, 2, kd, ks, kbx))
+  const cuuint32_t kbx[2] = {kSK, kColsPerMma};
+  if (!make_map(&tm_p, planes, 3, pd, ps, pb, CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map(&tm_k, a.subkeys, 2, kd, ks, kbx, CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
   const size_t smem = score_tc_smem_bytes();
   cudaError_t e = cudaFuncSetAttribute(score_topk_tc_kernel,

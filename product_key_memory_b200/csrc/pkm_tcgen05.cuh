@@ -48,14 +48,18 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
+// Suspend-time hint of one try_wait: the thread sleeps in hardware until the phase
+// completes or this many ns pass, instead of spinning on the issue slots.
+constexpr uint32_t kTryWaitHintNs = 20000;
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t done;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(done)
-      : "r"(smem_addr(bar)), "r"(parity)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(kTryWaitHintNs)
       : "memory");
   return done != 0;
 }
@@ -66,15 +70,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
                                           volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
+  for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (*abort) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
-        record_status(status, kDevTimeout);
-        *abort = 1;
-        return false;
-      }
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      record_status(status, kDevTimeout);
+      *abort = 1;
+      return false;
     }
   }
 }
@@ -215,6 +217,15 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t tile_smem_addr, uint32_t
   const uint64_t sbo = (1024ull >> 4);       // 8 rows x 128 bytes
   return start | (lbo << 16) | (sbo << 32) | (1ull << 46) /* sm100 version */ |
          (2ull << 61) /* 128-byte swizzle */;
+}
+
+// The same for rows of 32 bf16 (64 bytes) with the 64-byte swizzle: 8-row groups are
+// 512 bytes apart; the tile base must be 512-byte aligned.
+__device__ __forceinline__ uint64_t sw64_desc(uint32_t tile_smem_addr, uint32_t kbytes) {
+  const uint64_t start = ((tile_smem_addr + kbytes) >> 4) & 0x3fffull;
+  const uint64_t lbo = 1ull;
+  const uint64_t sbo = (512ull >> 4);
+  return start | (lbo << 16) | (sbo << 32) | (1ull << 46) | (4ull << 61) /* 64-byte swizzle */;
 }
 
 // Instruction descriptor: bf16 A and B (K-major), fp32 accumulator, M x N tile.

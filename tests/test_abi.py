@@ -39,11 +39,19 @@ def _shape(**kw):
     return P.make_shape(**base)
 
 
-def test_workspace_sizes():
+def test_workspace_sizes(monkeypatch):
     s = _shape()
+    lists = 16384 * 4 * 2 * 32 * 8            # best 32 per half: fp32 score + int32 id
     fw = P.pkm_workspace_size(s)
-    # status + 6 bytes per q element + 8 bytes per per-half list entry
-    assert fw >= 256 + 16384 * 2048 * 6 + 16384 * 4 * 2 * 32 * 8
+    # tensor-core path: status + three bf16 q planes per token of a sub-batch + lists
+    assert fw >= 256 + 16384 * 2048 * 6 + lists
+    monkeypatch.setenv("PKM_SUBBATCHES", "4")
+    assert 256 + 4096 * 2048 * 6 + lists <= P.pkm_workspace_size(s) < fw
+    monkeypatch.delenv("PKM_SUBBATCHES")
+    monkeypatch.setenv("PKM_PATH", "simt")
+    # CUDA-core path: fp32 q for every token
+    assert P.pkm_workspace_size(s) >= 256 + 16384 * 2048 * 4 + lists
+    monkeypatch.delenv("PKM_PATH")
     bw = P.pkm_workspace_size(s, True)
     assert bw >= 256 + 4 * (2 * 1024 * 1024 + 16384 * 4 * 32)
     assert P.pkm_workspace_size(_shape(B=0)) > 0
