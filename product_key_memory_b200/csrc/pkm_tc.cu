@@ -51,26 +51,32 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 // ===========================================================================
 // Query network: q = BN(x W_q^T) -> bf16 planes [3][B][F]
 // ===========================================================================
-constexpr int kQStages = 4;
+constexpr int kQStages = 3;
 constexpr uint32_t kQABytes = kRowsPerTile * kKBlock * 2;  // 16 KiB
 constexpr uint32_t kQBBytes = kColsPerMma * kKBlock * 2;   // 32 KiB
 constexpr uint32_t kQStageBytes = kQABytes + kQBBytes;
 constexpr int kQMaxF = 4096;  // BN scale/shift of every feature live in shared memory
+// Output staging: per epilogue warp, its 32 rows x 32 columns of each of the 3 planes
+// (64-byte rows, 64-byte swizzle), written to HBM by TMA tensor stores.
+constexpr uint32_t kQStagePlane = 32 * 32 * 2;             // 2 KiB
+constexpr uint32_t kQStageWarp = 3 * kQStagePlane;         // 6 KiB
 
 size_t query_tc_smem_bytes() {
-  return 1024 + kQStages * kQStageBytes + 2 * kQMaxF * sizeof(float) + 256;
+  return 1024 + kQStages * kQStageBytes + 2 * kQMaxF * sizeof(float) + kEpiWarps * kQStageWarp +
+         256;
 }
 
 __global__ void __launch_bounds__(kTcThreads, 1) query_tc_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
-    const float* __restrict__ mean, const float* __restrict__ var,
-    const float* __restrict__ gamma, const float* __restrict__ beta, float eps, int B, int d,
-    int F, uint16_t* __restrict__ planes, int* status) {
+    const __grid_constant__ CUtensorMap tm_out, const float* __restrict__ mean,
+    const float* __restrict__ var, const float* __restrict__ gamma,
+    const float* __restrict__ beta, float eps, int B, int d, int F, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* stages = align1024(smem_raw);
   float* scale_s = reinterpret_cast<float*>(stages + kQStages * kQStageBytes);
   float* shift_s = scale_s + kQMaxF;
-  uint64_t* full = reinterpret_cast<uint64_t*>(shift_s + kQMaxF);
+  uint8_t* staging = reinterpret_cast<uint8_t*>(shift_s + kQMaxF);  // [kEpiWarps][6 KiB]
+  uint64_t* full = reinterpret_cast<uint64_t*>(staging + kEpiWarps * kQStageWarp);
   uint64_t* empty = full + kQStages;
   uint64_t* tfull = empty + kQStages;
   uint64_t* tempty = tfull + 2;
@@ -105,6 +111,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) query_tc_kernel(
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tm_x);
     prefetch_tensormap(&tm_w);
+    prefetch_tensormap(&tm_out);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -185,8 +192,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) query_tc_kernel(
     const int quad = warp & 3;
     const int cset = (warp - 2) >> 2;  // which half of the 256 columns this warp converts
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
-    const size_t plane_stride = static_cast<size_t>(B) * F;
     constexpr int kGroups = kColsPerMma / 32 / 2;  // 32-column groups per warp
+    uint8_t* stg = staging + (warp - 2) * kQStageWarp;
+    // This lane's row inside the staging tile; chunk c (8 columns, 16 bytes) of it sits
+    // at position c ^ ((lane >> 1) & 3): the 64-byte swizzle the store map expects.
+    uint8_t* my_row = stg + lane * 64;
+    const int swz = (lane >> 1) & 3;
     int it = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
       const int buf = it & 1;
@@ -194,7 +205,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) query_tc_kernel(
       if (!warp_wait(&tfull[buf], tph, status, abort)) break;
       tc_fence_after();
       const int m = t / nt, nn = t - m * nt;
-      const int64_t row = static_cast<int64_t>(m) * kRowsPerTile + quad * 32 + lane;
 #pragma unroll 1
       for (int gg = 0; gg < kGroups; ++gg) {
         const int g = cset * kGroups + gg;
@@ -205,33 +215,46 @@ __global__ void __launch_bounds__(kTcThreads, 1) query_tc_kernel(
           __syncwarp();
           if (lane == 0) mbar_arrive(&tempty[buf]);
         }
-        if (row < B) {
-          const int f0 = nn * kColsPerMma + g * 32;
-          uint32_t ph_[16], pm[16], pl[16];
+        const int f0 = nn * kColsPerMma + g * 32;
+        uint32_t ph_[16], pm[16], pl[16];
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            const float q0 = fmaf(v[i], scale_s[f0 + i], shift_s[f0 + i]);
-            const float q1 = fmaf(v[i + 1], scale_s[f0 + i + 1], shift_s[f0 + i + 1]);
-            uint16_t h0, m0, l0, h1, m1, l1;
-            split3(q0, h0, m0, l0);
-            split3(q1, h1, m1, l1);
-            ph_[i / 2] = h0 | (static_cast<uint32_t>(h1) << 16);
-            pm[i / 2] = m0 | (static_cast<uint32_t>(m1) << 16);
-            pl[i / 2] = l0 | (static_cast<uint32_t>(l1) << 16);
-          }
-          uint16_t* dst = planes + row * F + f0;
+        for (int i = 0; i < 32; i += 2) {
+          const float q0 = fmaf(v[i], scale_s[f0 + i], shift_s[f0 + i]);
+          const float q1 = fmaf(v[i + 1], scale_s[f0 + i + 1], shift_s[f0 + i + 1]);
+          uint16_t h0, m0, l0, h1, m1, l1;
+          split3(q0, h0, m0, l0);
+          split3(q1, h1, m1, l1);
+          ph_[i / 2] = h0 | (static_cast<uint32_t>(h1) << 16);
+          pm[i / 2] = m0 | (static_cast<uint32_t>(m1) << 16);
+          pl[i / 2] = l0 | (static_cast<uint32_t>(l1) << 16);
+        }
+        // The previous group's stores must have read the staging tile before it is
+        // overwritten.
+        if (lane == 0) bulk_wait_read0();
+        __syncwarp();
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            reinterpret_cast<uint4*>(dst)[c] =
-                make_uint4(ph_[4 * c], ph_[4 * c + 1], ph_[4 * c + 2], ph_[4 * c + 3]);
-            reinterpret_cast<uint4*>(dst + plane_stride)[c] =
-                make_uint4(pm[4 * c], pm[4 * c + 1], pm[4 * c + 2], pm[4 * c + 3]);
-            reinterpret_cast<uint4*>(dst + 2 * plane_stride)[c] =
-                make_uint4(pl[4 * c], pl[4 * c + 1], pl[4 * c + 2], pl[4 * c + 3]);
-          }
+        for (int c = 0; c < 4; ++c) {
+          const int pos = (c ^ swz) * 16;
+          *reinterpret_cast<uint4*>(my_row + pos) =
+              make_uint4(ph_[4 * c], ph_[4 * c + 1], ph_[4 * c + 2], ph_[4 * c + 3]);
+          *reinterpret_cast<uint4*>(my_row + kQStagePlane + pos) =
+              make_uint4(pm[4 * c], pm[4 * c + 1], pm[4 * c + 2], pm[4 * c + 3]);
+          *reinterpret_cast<uint4*>(my_row + 2 * kQStagePlane + pos) =
+              make_uint4(pl[4 * c], pl[4 * c + 1], pl[4 * c + 2], pl[4 * c + 3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        const int row0 = m * kRowsPerTile + quad * 32;
+        if (lane == 0 && row0 < B) {
+          // Rows past B in a partly filled box lie outside the tensor map and are not
+          // written; a box that starts past B is not issued at all.
+#pragma unroll
+          for (int p = 0; p < 3; ++p) tma_store_3d(&tm_out, stg + p * kQStagePlane, f0, row0, p);
+          bulk_commit();
         }
       }
     }
+    if (lane == 0) bulk_wait0();
   }
   __syncthreads();
   if (warp == 1) {
@@ -664,7 +687,12 @@ cudaError_t launch_query_tc(const LayerArgs& a, void* planes, cudaStream_t st) {
   const cuuint32_t xb[2] = {kKBlock, kRowsPerTile};
   const cuuint64_t wd[2] = {static_cast<cuuint64_t>(a.d_model), static_cast<cuuint64_t>(F)};
   const cuuint32_t wb[2] = {kKBlock, kColsPerMma};
-  if (!make_map(&tm_x, a.x, 2, xd, xs, xb) || !make_map(&tm_w, a.W_q, 2, wd, xs, wb))
+  CUtensorMap tm_out;
+  const cuuint64_t od[3] = {static_cast<cuuint64_t>(F), static_cast<cuuint64_t>(a.B), 3};
+  const cuuint64_t os[2] = {static_cast<cuuint64_t>(F) * 2, static_cast<cuuint64_t>(F) * 2 * a.B};
+  const cuuint32_t ob[3] = {32, 32, 1};
+  if (!make_map(&tm_x, a.x, 2, xd, xs, xb) || !make_map(&tm_w, a.W_q, 2, wd, xs, wb) ||
+      !make_map(&tm_out, planes, 3, od, os, ob, CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
   const size_t smem = query_tc_smem_bytes();
   cudaError_t e = cudaFuncSetAttribute(query_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -672,10 +700,9 @@ cudaError_t launch_query_tc(const LayerArgs& a, void* planes, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   const int64_t tiles = ((a.B + kRowsPerTile - 1) / kRowsPerTile) * (F / kColsPerMma);
   const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
-  query_tc_kernel<<<grid, kTcThreads, smem, st>>>(tm_x, tm_w, a.bn_mean, a.bn_var, a.bn_gamma,
-                                                  a.bn_beta, a.bn_eps, static_cast<int>(a.B),
-                                                  a.d_model, F, static_cast<uint16_t*>(planes),
-                                                  a.status);
+  query_tc_kernel<<<grid, kTcThreads, smem, st>>>(tm_x, tm_w, tm_out, a.bn_mean, a.bn_var,
+                                                  a.bn_gamma, a.bn_beta, a.bn_eps,
+                                                  static_cast<int>(a.B), a.d_model, F, a.status);
   return cudaGetLastError();
 }
 
