@@ -46,7 +46,10 @@ FLUSH_BYTES = 256 << 20
 # DRAM bytes per launch of the dominant kernel from an ncu capture
 # (profiles/select_gather_c1024.md), keyed by the sha256 of the kernel's source at
 # capture time; reported as null once the source has changed.
-TRAFFIC = {}
+TRAFFIC = {
+    # c1024, 4096 tokens: dram read 971.2 MB + write 5.4 MB, scaled x4 to 16384 tokens.
+    ("004aa70f33fc1f1e", "c1024"): 3.906e9,
+}
 
 
 def peaks():
@@ -73,6 +76,16 @@ def per_token_bytes(w):
 def gemm_flops_per_token(w):
     """Query projection + per-half scoring, as the method defines them."""
     return 2 * w.d_model * w.H * w.dq + 2 * w.H * 2 * w.n * (w.dq // 2)
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """Largest value of x over all ranks (the slowest rank sets a step's time)."""
+    if world <= 1:
+        return float(x)
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 # --------------------------------------------------------------------- clocks
@@ -241,11 +254,7 @@ def run_ours(args, rank, world, local_rank):
     stage_ms, calls, launches = P.pkm_trace_read(0)
     P.pkm_trace_enable(False)
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
     if P.pkm_device_status(ws) != 0:
         raise RuntimeError("device status after timing: %s" % P.pkm_status_string(-5))
     value = world * args.steps * B / (total_ms / 1e3)
@@ -263,7 +272,7 @@ def run_ours(args, rank, world, local_rank):
         alg = per_token_bytes(w) * B
         achieved = alg / (stage_avg[2] * 1e-3) / 1e9
         sha = kernel_sha()
-        tr = TRAFFIC.get(sha)
+        tr = TRAFFIC.get((sha, w.name))
         roof = {"kernel": names[2], "bound": "hbm", "achieved": achieved, "peak": hbm,
                 "unit": "GB/s", "frac": achieved / hbm, "traffic": tr,
                 "algorithmic_bytes_per_launch": alg, "ms_per_launch": stage_avg[2],
@@ -307,11 +316,7 @@ def run_ours(args, rank, world, local_rank):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     e2e = {"value": world * args.steps * B / (e2e_ms / 1e3), "unit": UNIT,
            "h2d_bytes_per_step": x_h.numel() * x_h.element_size(),
            "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in (out_h, idx_h, w_h)),

@@ -269,11 +269,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) query_tc_kernel(
 // Two epilogue warp sets work on alternate units of the CTA, each with its own TMEM
 // accumulator (256 columns) and its own survivor log, so two warps share each SM
 // sub-partition. The MMA issuer interleaves the two sets' chunks.
-constexpr int kSSets = 2;
+#ifndef PKM_SCORE_SETS
+#define PKM_SCORE_SETS 2
+#endif
+constexpr int kSSets = PKM_SCORE_SETS;
+constexpr int kSBufPerSet = 2 / kSSets;  // TMEM accumulators (256 columns) per set
 constexpr int kSEpiWarps = 4 * kSSets;
 constexpr int kSThreads = 64 + 32 * kSEpiWarps;
-constexpr int kSK = 32;                                             // K per stage
-constexpr int kSStages = 3;
+constexpr int kSK = kSSets == 2 ? 32 : 64;                          // K per stage
+constexpr int kSStages = kSSets == 2 ? 3 : 2;
+constexpr CUtensorMapSwizzle kSSwizzle =
+    kSK == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
 constexpr uint32_t kSPlaneBytes = kRowsPerTile * kSK * 2;           // 8 KiB
 constexpr uint32_t kSABytes = 3 * kSPlaneBytes;                     // 24 KiB
 constexpr uint32_t kSBBytes = kColsPerMma * kSK * 2;                // 16 KiB
@@ -333,9 +339,9 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
   uint16_t* lg_i_all = reinterpret_cast<uint16_t*>(lg_s_all + kSSets * kSLogRows * kRowsPerTile);
   uint64_t* full = reinterpret_cast<uint64_t*>(lg_i_all + kSSets * kSLogRows * kRowsPerTile);
   uint64_t* empty = full + kSStages;
-  uint64_t* tfull = empty + kSStages;   // [kSSets]
-  uint64_t* tempty = tfull + kSSets;    // [kSSets]
-  uint64_t* drain = tempty + kSSets;
+  uint64_t* tfull = empty + kSStages;   // [2] one per TMEM accumulator
+  uint64_t* tempty = tfull + 2;         // [2]
+  uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -356,7 +362,7 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < kSSets; ++b) {
+    for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], 4);
     }
@@ -423,31 +429,36 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
       // ---------------- MMA issuer: chunk of 256 sub-keys = kiters x 3 planes x 2 MMAs
       const uint32_t idesc = idesc_bf16_f32(kRowsPerTile, kColsPerMma);
       uint32_t s = 0, ph = 0;
-      int uses[kSSets] = {0, 0};  // chunks written into each set's accumulator so far
+      int uses[kSSets] = {};  // chunks written into each set's accumulators so far
       bool ok = true;
       for (int j0 = 0; j0 < myunits && ok; j0 += kSSets)
         for (int c = 0; c < nchunks && ok; ++c)
           for (int set = 0; set < kSSets && ok; ++set) {
             if (j0 + set >= myunits) break;
-            const uint32_t tph = uses[set] & 1;
-            if (!mbar_wait(&tempty[set], tph ^ 1, status, abort)) { ok = false; break; }
+            // Accumulator b of this set; its uses alternate between the set's buffers.
+            const int b = set * kSBufPerSet + uses[set] % kSBufPerSet;
+            const uint32_t tph = (uses[set] / kSBufPerSet) & 1;
+            if (!mbar_wait(&tempty[b], tph ^ 1, status, abort)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t d_tmem = tmem_base + set * kColsPerMma;
+            const uint32_t d_tmem = tmem_base + b * kColsPerMma;
             for (int kb = 0; kb < kiters; ++kb) {
               if (!mbar_wait(&full[s], ph, status, abort)) { ok = false; break; }
               tc_fence_after();
               const uint32_t a = smem_addr(stages + s * kSStageBytes);
-              const uint32_t b = a + kSABytes;
+              const uint32_t bb = a + kSABytes;
 #pragma unroll
               for (int p = 0; p < 3; ++p)
 #pragma unroll
-                for (int jj = 0; jj < kSK / 16; ++jj)
-                  mma_bf16(d_tmem, sw64_desc(a + p * kSPlaneBytes, jj * 32),
-                           sw64_desc(b, jj * 32), idesc, (kb | p | jj) != 0);
+                for (int jj = 0; jj < kSK / 16; ++jj) {
+                  const uint64_t ad = kSK == 32 ? sw64_desc(a + p * kSPlaneBytes, jj * 32)
+                                                : sw128_desc(a + p * kSPlaneBytes, jj * 32);
+                  const uint64_t bd = kSK == 32 ? sw64_desc(bb, jj * 32) : sw128_desc(bb, jj * 32);
+                  mma_bf16(d_tmem, ad, bd, idesc, (kb | p | jj) != 0);
+                }
               mma_commit(&empty[s]);
               if (++s == kSStages) { s = 0; ph ^= 1; }
             }
-            if (ok) mma_commit(&tfull[set]);
+            if (ok) mma_commit(&tfull[b]);
             ++uses[set];
           }
       mma_commit(drain);
@@ -482,7 +493,8 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
       int cnt = 0, kept = 0;   // log entries; entries kept by the last merge
       bool ok = true;
       const int nsteps = nchunks * kStepsPerChunk;
-      const uint32_t col0 = tmem_base + lane_addr + set * kColsPerMma;
+      int bsel = set * kSBufPerSet;
+      uint32_t col0 = tmem_base + lane_addr + bsel * kColsPerMma;
 #pragma unroll 1
       for (int st = 0; st <= nsteps; ++st) {
         const bool flush = st == nsteps;
@@ -490,7 +502,13 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
         float v[kSStep];
         if (!flush) {
           if (sc == 0) {
-            if (!warp_wait(&tfull[set], (uses + c) & 1, status, abort)) { ok = false; break; }
+            const int uc = uses + c;
+            bsel = set * kSBufPerSet + uc % kSBufPerSet;
+            col0 = tmem_base + lane_addr + bsel * kColsPerMma;
+            if (!warp_wait(&tfull[bsel], (uc / kSBufPerSet) & 1, status, abort)) {
+              ok = false;
+              break;
+            }
             tc_fence_after();
             if (c == 0) {
               // The maxima of the 64 groups of 4 columns are 64 different scores of the
@@ -513,7 +531,7 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
           if (sc == kStepsPerChunk - 1) {
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[set]);
+            if (lane == 0) mbar_arrive(&tempty[bsel]);
           }
         }
         // Merge when the next step could overflow the log, and once at the end.
@@ -718,8 +736,8 @@ cudaError_t launch_score_topk_tc(const LayerArgs& a, const void* planes, float* 
                             static_cast<cuuint64_t>(a.H) * 2 * a.n};
   const cuuint64_t ks[1] = {static_cast<cuuint64_t>(half) * 2};
   const cuuint32_t kbx[2] = {kSK, kColsPerMma};
-  if (!make_map(&tm_p, planes, 3, pd, ps, pb, CU_TENSOR_MAP_SWIZZLE_64B) ||
-      !make_map(&tm_k, a.subkeys, 2, kd, ks, kbx, CU_TENSOR_MAP_SWIZZLE_64B))
+  if (!make_map(&tm_p, planes, 3, pd, ps, pb, kSSwizzle) ||
+      !make_map(&tm_k, a.subkeys, 2, kd, ks, kbx, kSSwizzle))
     return cudaErrorInvalidValue;
   const size_t smem = score_tc_smem_bytes();
   cudaError_t e = cudaFuncSetAttribute(score_topk_tc_kernel,
