@@ -288,7 +288,7 @@ constexpr int kList = kMaxK;          // entries per per-half list (the best 32,
 constexpr int kSStep = 8;             // columns read from TMEM per step
 constexpr int kSNewCap = 32;          // survivors logged between two merges
 constexpr int kSLogCap = kList + kSNewCap;
-constexpr int kSTrash = kSLogCap;     // log slot that absorbs the stores of rejected scores
+constexpr int kSTrash = kSLogCap;     // slot written (and dropped) past a full log
 constexpr int kSLogRows = kSLogCap + 1;
 
 size_t score_tc_smem_bytes() {
@@ -477,6 +477,10 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
     float* lg_s = lg_s_all + set * kSLogRows * kRowsPerTile;  // [kSLogRows][128]
     uint16_t* lg_i = lg_i_all + set * kSLogRows * kRowsPerTile;
+    // Shared-window addresses of this row's log column: entry e of the row is at
+    // s_row + e * kSStrideS (score) and i_row + e * kSStrideI (id).
+    constexpr uint32_t kSStrideS = kRowsPerTile * 4, kSStrideI = kRowsPerTile * 2;
+    const uint32_t s_row = smem_addr(lg_s + r), i_row = smem_addr(lg_i + r);
     constexpr int kStepsPerChunk = kColsPerMma / kSStep;
     int uses = 0;
     for (int j = set; j < myunits; j += kSSets) {
@@ -538,11 +542,10 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
         const int fresh = cnt - kept;
         if (__any_sync(0xffffffffu, flush ? fresh > 0 : fresh > kSNewCap - kSStep)) {
           float b[32];
+          const uint32_t fresh_at = s_row + kept * kSStrideS;
 #pragma unroll
-          for (int q = 0; q < 32; ++q) {
-            const int e = kept + q;
-            b[q] = q < fresh ? lg_s[e * kRowsPerTile + r] : -INFINITY;
-          }
+          for (int q = 0; q < 32; ++q)
+            b[q] = q < fresh ? lds_f32(fresh_at + q * kSStrideS) : -INFINITY;
           thread_sort32f(b);
 #pragma unroll
           for (int i = 0; i < 32; ++i) Ls[i] = fmaxf(Ls[i], b[31 - i]);
@@ -562,18 +565,22 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
           // rewritten either to slot w (w <= e, so nothing unread is overwritten) or to
           // the trash slot. That keeps the current best 32 plus any later entry tied
           // with the 32nd score.
-          int w = 0;
+          // Every entry is written to the current write slot, which only advances for a
+          // kept entry (w <= e, so nothing unread is overwritten).
           const int cmax = __reduce_max_sync(0xffffffffu, cnt);
+          uint32_t ws = s_row, wi = i_row;
 #pragma unroll 4
           for (int e = 0; e < cmax; ++e) {
-            const float sv = lg_s[e * kRowsPerTile + r];
-            const uint16_t iv = lg_i[e * kRowsPerTile + r];
-            const bool keep = e < cnt && sv >= tau_run;
-            const int dst = keep ? w : kSTrash;
-            lg_s[dst * kRowsPerTile + r] = sv;
-            lg_i[dst * kRowsPerTile + r] = iv;
-            w += keep ? 1 : 0;
+            const float sv = lds_f32(s_row + e * kSStrideS);
+            const uint16_t iv = lds_u16(i_row + e * kSStrideI);
+            sts_f32(ws, sv);
+            sts_u16(wi, iv);
+            if (e < cnt && sv >= tau_run) {
+              ws += kSStrideS;
+              wi += kSStrideI;
+            }
           }
+          int w = static_cast<int>((ws - s_row) / kSStrideS);
           if (__any_sync(0xffffffffu, w > kList)) {
             // Rare: ties at the 32nd score. Of the entries equal to tau_run keep the first
             // `eq` in id order (eq = how many of the best 32 scores equal it), so the log
@@ -601,17 +608,20 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
           thr = fmaxf(nextafterf(tau0, -INFINITY), tau_run);
         }
         if (!flush) {
-          // Branch-free filter: a kept score goes to the next log slot, a rejected one
-          // to the trash slot.
+          // Branch-free filter: every score is written to the next free log slot, which
+          // only advances when the score is kept (a rejected one is overwritten).
           const int id0 = c * kColsPerMma + sc * kSStep;
+          uint32_t as = s_row + cnt * kSStrideS, ai = i_row + cnt * kSStrideI;
 #pragma unroll
           for (int i = 0; i < kSStep; ++i) {
-            const bool take = v[i] > thr;
-            const int dst = take ? cnt : kSTrash;
-            lg_s[dst * kRowsPerTile + r] = v[i];
-            lg_i[dst * kRowsPerTile + r] = static_cast<uint16_t>(id0 + i);
-            cnt += take ? 1 : 0;
+            sts_f32(as, v[i]);
+            sts_u16(ai, static_cast<uint16_t>(id0 + i));
+            if (v[i] > thr) {
+              as += kSStrideS;
+              ai += kSStrideI;
+            }
           }
+          cnt = static_cast<int>((as - s_row) / kSStrideS);
         }
       }
       uses += nchunks;
