@@ -292,35 +292,58 @@ def run_ours(args, rank, world, local_rank):
                  "stage_ms": dict(zip(names, stage_avg)), "call_ms": call_avg,
                  "peak_kind": pk_kind}
 
-    # ---- end to end: host x -> device, forward, out/indices/weights -> host
+    # ---- end to end through pkm_forward with host buffers, pipelined like a serving
+    # loop: step i+1's input copy (pinned host -> device) and step i-1's result read
+    # (device -> pinned host) overlap step i's forward on three streams, with device
+    # tensors double-buffered. The result read back is `out`; indices and weights stay
+    # on the device for the backward.
     x_h = L["x"].pin_memory()
-    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    idx_h = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
-    w_h = torch.empty(wts.shape, dtype=wts.dtype).pin_memory()
-    x_d = torch.empty_like(d["x"])
+    out_h = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    x_d = [torch.empty_like(d["x"]) for _ in range(2)]
+    out_d = [out, torch.empty_like(out)]
+    idx_d = [idx, torch.empty_like(idx)]
+    w_d = [wts, torch.empty_like(wts)]
+    s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
 
-    def e2e_step():
-        x_d.copy_(x_h, non_blocking=True)
-        fwd(x_d)
-        out_h.copy_(out, non_blocking=True)
-        idx_h.copy_(idx, non_blocking=True)
-        w_h.copy_(wts, non_blocking=True)
+    def e2e_run(steps):
+        ev_in = [torch.cuda.Event() for _ in range(steps)]
+        ev_cmp = [torch.cuda.Event() for _ in range(steps)]
+        ev_out = [torch.cuda.Event() for _ in range(steps)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(s_in)
+        for i in range(steps):
+            b = i & 1
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev_cmp[i - 2])      # x_d[b] no longer read
+                x_d[b].copy_(x_h, non_blocking=True)
+                ev_in[i].record(s_in)
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(ev_in[i])
+                if i >= 2:
+                    s_cmp.wait_event(ev_out[i - 2])     # out_d[b] already read back
+                P.pkm_forward(x_d[b], d["W_q"], d["bn_mean"], d["bn_var"], d["bn_gamma"],
+                              d["bn_beta"], d["subkeys"], d["values"], k=w.k, out=out_d[b],
+                              indices=idx_d[b], weights=w_d[b], want_scores=False,
+                              workspace=ws, stream=s_cmp)
+                ev_cmp[i].record(s_cmp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_cmp[i])
+                out_h[b].copy_(out_d[b], non_blocking=True)
+                ev_out[i].record(s_out)
+        t1.record(s_out)
+        torch.cuda.synchronize(dev)
+        return t0.elapsed_time(t1)
 
-    for _ in range(2):
-        e2e_step()
+    e2e_run(3)
     barrier()
     torch.cuda.synchronize(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_ms = max_over_ranks(e2e_run(args.steps), world, dev)
     e2e = {"value": world * args.steps * B / (e2e_ms / 1e3), "unit": UNIT,
            "h2d_bytes_per_step": x_h.numel() * x_h.element_size(),
-           "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in (out_h, idx_h, w_h)),
-           "ms_per_step": e2e_ms / args.steps}
+           "d2h_bytes_per_step": out_h[0].numel() * out_h[0].element_size(),
+           "ms_per_step": e2e_ms / args.steps,
+           "pipelining": "copy-in, forward and copy-out of consecutive steps overlap"}
     launches_e2e = P.pkm_trace_read(0)[2]
 
     extra = {}
@@ -352,7 +375,8 @@ def run_ours(args, rank, world, local_rank):
 
 
 def run_c512_and_backward(args, dev, P, hbm, bf16, stream, world, barrier):
-    """512^2-slot forward (the metric's other memory size) and the value backward on it."""
+    """512^2-slot forward (the metric's other memory size), the value backward on it,
+    and the wide 1024^2-slot layer (H = 8, v = 1600)."""
     w = synth.WORKLOADS["c512"]
     L = synth.make_layer(w)
     d = {k: v.to(dev) for k, v in L.items()}
@@ -365,6 +389,7 @@ def run_c512_and_backward(args, dev, P, hbm, bf16, stream, world, barrier):
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     def fwd():
+        # Reads the current bindings of d, w, out, idx, wts and ws in this function.
         P.pkm_forward(d["x"], d["W_q"], d["bn_mean"], d["bn_var"], d["bn_gamma"], d["bn_beta"],
                       d["subkeys"], d["values"], k=w.k, out=out, indices=idx, weights=wts,
                       want_scores=False, workspace=ws)
@@ -384,6 +409,7 @@ def run_c512_and_backward(args, dev, P, hbm, bf16, stream, world, barrier):
     for _ in range(max(3, args.warmup)):
         fwd()
     barrier()
+    P.pkm_trace_enable(True)
     P.pkm_trace_read(0)
     fwd_ms = timed(fwd, args.steps)
     stage_ms, calls, _ = P.pkm_trace_read(0)
@@ -407,6 +433,7 @@ def run_c512_and_backward(args, dev, P, hbm, bf16, stream, world, barrier):
     P.pkm_trace_read(1)
     bwd_ms = timed(bwd, args.steps)
     bstage, bcalls, _ = P.pkm_trace_read(1)
+    P.pkm_trace_enable(False)
     uniq = int(torch.unique(idx).numel())
     picks = idx.numel()
     bytes_alg = picks * w.v * 2 + B * w.v * 2 + picks * 8 + 2 * uniq * w.v * 4
@@ -417,6 +444,35 @@ def run_c512_and_backward(args, dev, P, hbm, bf16, stream, world, barrier):
         "algorithmic_bytes": bytes_alg, "achieved_gbs": bytes_alg / (bwd_ms * 1e-3) / 1e9,
         "frac_of_hbm": bytes_alg / (bwd_ms * 1e-3) / 1e9 / hbm,
         "stage_ms": [m / max(1, bcalls) for m in bstage[:2]]}
+    del d, gv, gout, bws, ws
+    torch.cuda.empty_cache()
+
+    # The wide layer: d_model 1600, H = 8, 1024^2 slots, v = 1600 (3.4 GB table).
+    w = synth.WORKLOADS["wide"]
+    L = synth.make_layer(w)
+    d = {k: v.to(dev) for k, v in L.items()}
+    del L
+    B = w.B
+    out = torch.empty(B, w.v, dtype=torch.float32, device=dev)
+    idx = torch.empty(B, w.H, w.k, dtype=torch.int32, device=dev)
+    wts = torch.empty(B, w.H, w.k, dtype=torch.float32, device=dev)
+    shape = P.make_shape(B, w.d_model, w.H, w.dq, w.n, w.k, w.v, w.torch_dtype)
+    ws = P.alloc_workspace(shape, False, dev)
+    for _ in range(max(3, args.warmup)):
+        fwd()
+    barrier()
+    P.pkm_trace_enable(True)
+    P.pkm_trace_read(0)
+    fwd_ms = timed(fwd, args.steps)
+    stage_ms, calls, _ = P.pkm_trace_read(0)
+    P.pkm_trace_enable(False)
+    t_mem = w.H * w.k * w.v * 2 * B / (hbm * 1e9)
+    t_gemm = gemm_flops_per_token(w) * B / (bf16 * 1e12)
+    res["wide"] = {"workload": workload_desc(w), "value": world * B / (fwd_ms / 1e3),
+                   "unit": UNIT, "ms_per_step": fwd_ms,
+                   "step_roofline_frac": max(t_mem, t_gemm) * 1e3 / fwd_ms,
+                   "stage_ms": [m / max(1, calls) for m in stage_ms[:3]],
+                   "gather_gbs": per_token_bytes(w) * B / (stage_ms[2] / max(1, calls) * 1e-3) / 1e9}
     return res
 
 
