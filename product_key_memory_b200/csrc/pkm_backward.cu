@@ -247,28 +247,63 @@ __global__ void __launch_bounds__(128) segment_rows_kernel(
       const int r = __shfl_sync(0xffffffffu, r_l, i - w0);
       const int seg0 = offsets[r], seg1 = offsets[r + 1];
       const int end = min(seg1, w1);
+      const bool whole = seg0 >= w0 && seg1 <= w1;
+      float* grow = grad_values + static_cast<int64_t>(r) * v;
+      // A slot group that lies inside this window is owned by this warp: load its row
+      // now so the HBM read overlaps the sums below. A group that crosses a window edge
+      // is added with vector atomics instead.
+      float4 old[MAXV][VPER / 4];
       float acc[MAXV][VPER];
 #pragma unroll
-      for (int m = 0; m < MAXV; ++m)
+      for (int m = 0; m < MAXV; ++m) {
+        const int vec = lane + 32 * m;
 #pragma unroll
-        for (int e = 0; e < VPER; ++e) acc[m][e] = 0.f;
-      for (int j = i; j < end; ++j) {
-        const int e = __shfl_sync(0xffffffffu, e_l, j - w0);
-        const float wt = __shfl_sync(0xffffffffu, wt_l, j - w0);
-        const T* gp = grad_out + static_cast<int64_t>(e / HK) * v;
+        for (int q = 0; q < VPER; q += 4) {
+          old[m][q / 4] = (whole && vec < nvec)
+                              ? *reinterpret_cast<const float4*>(grow + vec * VPER + q)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+          acc[m][q] = acc[m][q + 1] = acc[m][q + 2] = acc[m][q + 3] = 0.f;
+        }
+      }
+      int j = i;
+      for (; j + 1 < end; j += 2) {  // two picks in flight
+        const int ea = __shfl_sync(0xffffffffu, e_l, j - w0);
+        const int eb = __shfl_sync(0xffffffffu, e_l, j + 1 - w0);
+        const float wa = __shfl_sync(0xffffffffu, wt_l, j - w0);
+        const float wb = __shfl_sync(0xffffffffu, wt_l, j + 1 - w0);
+        const T* ga = grad_out + static_cast<int64_t>(ea / HK) * v;
+        const T* gb = grad_out + static_cast<int64_t>(eb / HK) * v;
+        uint4 ra[MAXV], rb[MAXV];
+#pragma unroll
+        for (int m = 0; m < MAXV; ++m) {
+          const int vec = lane + 32 * m;
+          ra[m] = vec < nvec ? __ldg(reinterpret_cast<const uint4*>(ga + vec * VPER)) : make_uint4(0, 0, 0, 0);
+          rb[m] = vec < nvec ? __ldg(reinterpret_cast<const uint4*>(gb + vec * VPER)) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int m = 0; m < MAXV; ++m) {
+          float fa[VPER], fb[VPER];
+          Vec<T>::widen(ra[m], fa);
+          Vec<T>::widen(rb[m], fb);
+#pragma unroll
+          for (int q = 0; q < VPER; ++q) acc[m][q] = fmaf(wb, fb[q], fmaf(wa, fa[q], acc[m][q]));
+        }
+      }
+      if (j < end) {
+        const int ea = __shfl_sync(0xffffffffu, e_l, j - w0);
+        const float wa = __shfl_sync(0xffffffffu, wt_l, j - w0);
+        const T* ga = grad_out + static_cast<int64_t>(ea / HK) * v;
 #pragma unroll
         for (int m = 0; m < MAXV; ++m) {
           const int vec = lane + 32 * m;
           if (vec < nvec) {
-            float f[VPER];
-            Vec<T>::widen(__ldg(reinterpret_cast<const uint4*>(gp + vec * VPER)), f);
+            float fa[VPER];
+            Vec<T>::widen(__ldg(reinterpret_cast<const uint4*>(ga + vec * VPER)), fa);
 #pragma unroll
-            for (int q = 0; q < VPER; ++q) acc[m][q] = fmaf(wt, f[q], acc[m][q]);
+            for (int q = 0; q < VPER; ++q) acc[m][q] = fmaf(wa, fa[q], acc[m][q]);
           }
         }
       }
-      float* grow = grad_values + static_cast<int64_t>(r) * v;
-      const bool whole = seg0 >= w0 && seg1 <= w1;
 #pragma unroll
       for (int m = 0; m < MAXV; ++m) {
         const int vec = lane + 32 * m;
@@ -276,14 +311,12 @@ __global__ void __launch_bounds__(128) segment_rows_kernel(
 #pragma unroll
           for (int q = 0; q < VPER; q += 4) {
             float4* p = reinterpret_cast<float4*>(grow + vec * VPER + q);
-            const float4 add = make_float4(acc[m][q], acc[m][q + 1], acc[m][q + 2], acc[m][q + 3]);
-            if (whole) {
-              float4 cur = *p;
-              cur.x += add.x; cur.y += add.y; cur.z += add.z; cur.w += add.w;
-              *p = cur;
-            } else {
-              atomicAdd(p, add);
-            }
+            const float4 o = old[m][q / 4];
+            if (whole)
+              *p = make_float4(o.x + acc[m][q], o.y + acc[m][q + 1], o.z + acc[m][q + 2],
+                               o.w + acc[m][q + 3]);
+            else
+              atomicAdd(p, make_float4(acc[m][q], acc[m][q + 1], acc[m][q + 2], acc[m][q + 3]));
           }
         }
       }
