@@ -258,6 +258,9 @@ def run_ours(args, rank, world, local_rank):
     if P.pkm_device_status(ws) != 0:
         raise RuntimeError("device status after timing: %s" % P.pkm_status_string(-5))
     value = world * args.steps * B / (total_ms / 1e3)
+    distinct = int(P.pkm_slot_usage(idx, w.n).item())
+    usage = {"distinct_slots": distinct, "slots": w.n * w.n, "fraction": distinct / (w.n * w.n),
+             "picks": B * w.H * w.k}
     ms_per_step = total_ms / args.steps
 
     pk, pk_kind = peaks()
@@ -360,7 +363,7 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": workload_desc(w), "global_batch": B * world,
                    "seq_len": None, "parallelism": "dp%d (independent replicas)" % world,
                    "l2": "flushed before every timed step (256 MiB write, outside the bracket)"},
-        "roofline": roof, "step_roofline": step_roof, "e2e": e2e,
+        "roofline": roof, "step_roofline": step_roof, "e2e": e2e, "slot_usage": usage,
         "gpu_launches": launches, "gpu_launches_e2e": launches_e2e,
         "clocks": clocks,
     }

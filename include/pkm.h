@@ -72,8 +72,9 @@ typedef struct {
 } pkm_shape;
 
 /*
- * Bytes of workspace pkm_forward (for_backward = 0) or pkm_backward_values
- * (for_backward = 1) needs for this shape; 0 if the shape is invalid.
+ * Bytes of workspace pkm_forward (for_backward = 0), pkm_backward_values
+ * (for_backward = 1) or pkm_slot_usage (for_backward = 2) needs for this shape; 0 if
+ * the shape is invalid.
  */
 size_t pkm_workspace_size(const pkm_shape* s, int for_backward);
 
@@ -151,6 +152,19 @@ int pkm_backward_values(const pkm_shape* s, const void* values, const int32_t* i
 int pkm_backward_values_noalloc(const pkm_shape* s, const void* values, const int32_t* indices,
                                 const float* weights, const void* grad_out, float* grad_values,
                                 float* grad_scores, void* stream);
+
+/*
+ * Memory utilisation of one batch ("Large Memory Layers with Product Keys", gptget.net
+ * summary, Key Results: BatchNorm in the query network raises the share of memory
+ * slots in use above 80 %): the number of distinct slots among the B*H*k picks.
+ *   indices  [B][H][k] int32, as written by pkm_forward
+ *   hits     one device uint64, overwritten with the count
+ * Only B, H, n and k of the shape are read. Ids outside [0, n*n) are not counted and
+ * set the status word (PKM_ERR_DEVICE).
+ * workspace: at least pkm_workspace_size(s, 2) bytes (status word + one bit per slot).
+ */
+int pkm_slot_usage(const pkm_shape* s, const int32_t* indices, unsigned long long* hits,
+                   void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Synchronises `stream`, reads the status word that the kernels of the last call

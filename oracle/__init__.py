@@ -51,6 +51,8 @@ def lib():
         L.pkm_oracle_finish.restype = _I
         L.pkm_oracle_backward.argtypes = [_I64, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]
         L.pkm_oracle_backward.restype = _I
+        L.pkm_oracle_slot_usage.argtypes = [_I64, _P, _I64, _P]
+        L.pkm_oracle_slot_usage.restype = _I64
         _lib = L
     return _lib
 
@@ -165,3 +167,13 @@ def backward(values: torch.Tensor, grad_out: torch.Tensor, indices: np.ndarray,
     if rc != 0:
         raise ValueError("pkm_oracle_backward rejected the sizes")
     return gv, gs
+
+
+def slot_usage(indices: np.ndarray, slots: int):
+    """(distinct slots among the picks, number of picks outside [0, slots))."""
+    indices = np.ascontiguousarray(indices, dtype=np.int32)
+    bad = ctypes.c_int64(0)
+    n = lib().pkm_oracle_slot_usage(indices.size, _ptr(indices), int(slots), ctypes.byref(bad))
+    if n < 0:
+        raise ValueError("pkm_oracle_slot_usage rejected the sizes")
+    return int(n), int(bad.value)

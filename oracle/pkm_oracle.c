@@ -317,3 +317,32 @@ int pkm_oracle_backward(int64_t B, int H, int k, int v, int dtype, const void* v
   free(gw);
   return 0;
 }
+
+/*
+ * Memory utilisation of one batch: the number of distinct slots among the B*H*k picks
+ * (the pages report the share of memory slots a trained layer uses, with and without
+ * BatchNorm in the query network). indices [B][H][k]; slots = n*n. Ids outside
+ * [0, slots) are not counted; their number goes to *bad (if not NULL).
+ * Returns the count of distinct slots, or -1 on bad sizes / allocation failure.
+ */
+int64_t pkm_oracle_slot_usage(int64_t picks, const int32_t* indices, int64_t slots,
+                              int64_t* bad) {
+  if (picks < 0 || slots < 1) return -1;
+  unsigned char* seen = (unsigned char*)calloc((size_t)slots, 1);
+  if (!seen) return -1;
+  int64_t distinct = 0, nbad = 0;
+  for (int64_t e = 0; e < picks; ++e) {
+    const int64_t r = indices[e];
+    if (r < 0 || r >= slots) {
+      ++nbad;
+      continue;
+    }
+    if (!seen[r]) {
+      seen[r] = 1;
+      ++distinct;
+    }
+  }
+  free(seen);
+  if (bad) *bad = nbad;
+  return distinct;
+}

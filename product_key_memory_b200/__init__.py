@@ -25,7 +25,7 @@ _STATUS = {0: "PKM_OK", -1: "PKM_ERR_INVALID_ARG", -2: "PKM_ERR_UNSUPPORTED",
 
 EXPORTED = ("pkm_workspace_size", "pkm_forward", "pkm_backward_values", "pkm_device_status",
             "pkm_trace_enable", "pkm_trace_read", "pkm_status_string",
-            "pkm_backward_values_noalloc")
+            "pkm_backward_values_noalloc", "pkm_slot_usage")
 
 
 class PKMError(RuntimeError):
@@ -61,6 +61,8 @@ def lib() -> ctypes.CDLL:
         L.pkm_backward_values.restype = ctypes.c_int
         L.pkm_backward_values_noalloc.argtypes = [S] + [P] * 6 + [P]
         L.pkm_backward_values_noalloc.restype = ctypes.c_int
+        L.pkm_slot_usage.argtypes = [S, P, P, P, ctypes.c_size_t, P]
+        L.pkm_slot_usage.restype = ctypes.c_int
         L.pkm_device_status.argtypes = [P, P]
         L.pkm_device_status.restype = ctypes.c_int
         L.pkm_trace_enable.argtypes = [ctypes.c_int]
@@ -190,6 +192,25 @@ def pkm_backward_values_noalloc(values: torch.Tensor, indices: torch.Tensor,
     if rc != PKM_OK:
         raise PKMError("pkm_backward_values_noalloc", rc)
     return grad_values, grad_scores
+
+
+def pkm_slot_usage(indices: torch.Tensor, n: int, hits: Optional[torch.Tensor] = None,
+                   workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Distinct slots among indices [B][H][k] (device int64 tensor of one element)."""
+    B, H, k = indices.shape
+    shape = make_shape(B, 0, H, 0, n, k, 8, PKM_F32)
+    if hits is None:
+        hits = torch.empty(1, dtype=torch.int64, device=indices.device)
+    if workspace is None:
+        nb = int(lib().pkm_workspace_size(ctypes.byref(shape), 2))
+        if nb == 0:
+            raise PKMError("pkm_workspace_size", -1)
+        workspace = torch.empty(nb, dtype=torch.uint8, device=indices.device)
+    rc = lib().pkm_slot_usage(ctypes.byref(shape), _ptr(indices), _ptr(hits), _ptr(workspace),
+                              workspace.numel(), _stream(stream))
+    if rc != PKM_OK:
+        raise PKMError("pkm_slot_usage", rc)
+    return hits
 
 
 def pkm_device_status(workspace: torch.Tensor, stream=None) -> int:

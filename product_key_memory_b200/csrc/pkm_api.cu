@@ -43,6 +43,15 @@ int validate_common(const pkm_shape* s) {
   return PKM_OK;
 }
 
+// The slot-usage count reads B, H, n and k.
+int validate_usage(const pkm_shape* s) {
+  if (!s) return PKM_ERR_INVALID_ARG;
+  if (s->B < 0 || s->H < 1 || s->n < 1 || s->k < 1 || s->k > s->n) return PKM_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(s->n) * s->n > 0x7fffffffLL) return PKM_ERR_INVALID_ARG;
+  if (s->B * s->H * static_cast<int64_t>(s->k) > 0x7fffffffLL) return PKM_ERR_UNSUPPORTED;
+  return PKM_OK;
+}
+
 // The forward also needs d_model, dq and bn_eps.
 int validate_shape(const pkm_shape* s) {
   const int rc = validate_common(s);
@@ -255,8 +264,36 @@ int pkm_trace_read(int pass, double* stage_ms, int max_stages, int64_t* calls,
 }
 
 size_t pkm_workspace_size(const pkm_shape* s, int for_backward) {
+  if (for_backward == 2) {
+    if (validate_usage(s) != PKM_OK) return 0;
+    return pkm::kStatusBytes + align256(pkm::usage_bitmap_bytes(static_cast<int64_t>(s->n) * s->n));
+  }
   if ((for_backward ? validate_common(s) : validate_shape(s)) != PKM_OK) return 0;
   return for_backward ? backward_ws(s, nullptr, nullptr) : forward_ws(s, nullptr, nullptr);
+}
+
+int pkm_slot_usage(const pkm_shape* s, const int32_t* indices, unsigned long long* hits,
+                   void* workspace, size_t workspace_bytes, void* stream) {
+  const int rc = validate_usage(s);
+  if (rc != PKM_OK) return rc;
+  if (!hits || (s->B > 0 && !indices)) return PKM_ERR_INVALID_ARG;
+  if ((indices && !aligned16(indices)) || (reinterpret_cast<uintptr_t>(hits) & 7u))
+    return PKM_ERR_UNSUPPORTED;
+  const int64_t slots = static_cast<int64_t>(s->n) * s->n;
+  const size_t need = pkm::kStatusBytes + align256(pkm::usage_bitmap_bytes(slots));
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return PKM_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int* status = static_cast<int*>(workspace);
+  unsigned* bitmap = reinterpret_cast<unsigned*>(static_cast<char*>(workspace) + pkm::kStatusBytes);
+  if (cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess) return PKM_ERR_CUDA;
+  const cudaError_t e = pkm::launch_slot_usage(indices, s->B * s->H * static_cast<int64_t>(s->k),
+                                               slots, bitmap, hits, status, st);
+  {
+    std::lock_guard<std::mutex> lk(g_trace_mu);
+    if (e == cudaSuccess) g_launches += s->B > 0 ? 2 : 1;
+  }
+  return e == cudaSuccess ? PKM_OK : PKM_ERR_CUDA;
 }
 
 int pkm_forward(const pkm_shape* s, const void* x, const void* W_q, const float* bn_mean,

@@ -51,4 +51,9 @@ cudaError_t launch_backward_values(int64_t B, int H, int k, int v, int dtype, in
                                    const BackwardWs& ws, int* status, cudaStream_t st,
                                    const std::function<void()>& between_stages);
 
+// Memory utilisation (pkm_usage.cu).
+size_t usage_bitmap_bytes(int64_t slots);
+cudaError_t launch_slot_usage(const int* indices, int64_t E, int64_t slots, unsigned* bitmap,
+                              unsigned long long* hits, int* status, cudaStream_t st);
+
 }  // namespace pkm

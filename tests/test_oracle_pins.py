@@ -314,3 +314,21 @@ def test_backward_row_slot_compaction_matches_dense():
     np.testing.assert_array_equal(gs, gs2)
     untouched = np.setdiff1d(np.arange(w.n * w.n), rows)
     assert not dense[untouched].any()
+
+
+# ------------------------------------------------------- slot-usage pins
+
+
+def test_slot_usage_matches_numpy_unique():
+    g = torch.Generator().manual_seed(31)
+    for slots, picks in ((16, 5), (256, 1000), (262144, 200000)):
+        idx = torch.randint(0, slots, (picks,), generator=g).numpy().astype(np.int32)
+        n, bad = oracle.slot_usage(idx, slots)
+        assert n == np.unique(idx).size and bad == 0
+
+
+def test_slot_usage_closed_forms():
+    assert oracle.slot_usage(np.arange(100, dtype=np.int32), 100) == (100, 0)      # all slots once
+    assert oracle.slot_usage(np.full(50, 7, np.int32), 100) == (1, 0)               # one slot
+    assert oracle.slot_usage(np.array([3, -1, 100, 3, 99], np.int32), 100) == (2, 2)  # bad ids
+    assert oracle.slot_usage(np.zeros(0, np.int32), 10) == (0, 0)
