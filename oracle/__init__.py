@@ -51,6 +51,8 @@ def lib():
         L.pkm_oracle_finish.restype = _I
         L.pkm_oracle_backward.argtypes = [_I64, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]
         L.pkm_oracle_backward.restype = _I
+        L.pkm_oracle_backward_full.argtypes = [_I64, _I, _I, _I, _I, _I, _I, _I, _D] + [_P] * 17
+        L.pkm_oracle_backward_full.restype = _I
         L.pkm_oracle_slot_usage.argtypes = [_I64, _P, _I64, _P]
         L.pkm_oracle_slot_usage.restype = _I64
         _lib = L
@@ -177,3 +179,34 @@ def slot_usage(indices: np.ndarray, slots: int):
     if n < 0:
         raise ValueError("pkm_oracle_slot_usage rejected the sizes")
     return int(n), int(bad.value)
+
+
+def backward_full(layer: dict, indices: np.ndarray, weights: np.ndarray,
+                  grad_out: torch.Tensor, H: int, dq: int, n: int, k: int, eps: float = 1e-5):
+    """Gradients of L = <grad_out, out> with the picks held fixed. Returns a dict of
+    fp64 arrays: x [B][d], W_q [H*dq][d], gamma, beta [H*dq], subkeys [H][2][n][dq/2],
+    q [B][H*dq] (dL/dq)."""
+    x, dt = _raw(layer["x"])
+    W, _ = _raw(layer["W_q"])
+    C, _ = _raw(layer["subkeys"])
+    V, _ = _raw(layer["values"])
+    G, dtg = _raw(grad_out)
+    if dtg != dt:
+        raise TypeError("grad_out must have the layer's dtype")
+    B, d = x.shape
+    v = V.shape[1]
+    F = H * dq
+    mean, var = _f32(layer["bn_mean"]), _f32(layer["bn_var"])
+    gamma, beta = _f32(layer["bn_gamma"]), _f32(layer["bn_beta"])
+    indices = np.ascontiguousarray(indices, dtype=np.int32)
+    weights = np.ascontiguousarray(weights, dtype=np.float64)
+    out = dict(x=np.zeros((B, d)), W_q=np.zeros((F, d)), gamma=np.zeros(F), beta=np.zeros(F),
+               subkeys=np.zeros((H, 2, n, dq // 2)), q=np.zeros((B, F)))
+    rc = lib().pkm_oracle_backward_full(B, d, H, dq, n, k, v, dt, eps, _ptr(x), _ptr(W),
+                                        _ptr(mean), _ptr(var), _ptr(gamma), _ptr(beta), _ptr(C),
+                                        _ptr(V), _ptr(indices), _ptr(weights), _ptr(G),
+                                        _ptr(out["x"]), _ptr(out["W_q"]), _ptr(out["gamma"]),
+                                        _ptr(out["beta"]), _ptr(out["subkeys"]), _ptr(out["q"]))
+    if rc != 0:
+        raise ValueError("pkm_oracle_backward_full rejected the sizes")
+    return out

@@ -346,3 +346,96 @@ int64_t pkm_oracle_slot_usage(int64_t picks, const int32_t* indices, int64_t slo
   if (bad) *bad = nbad;
   return distinct;
 }
+
+/*
+ * Full backward of the layer with the selection held fixed (the top-k choice is
+ * piecewise constant, so no gradient flows through it). With L = <grad_out, out>,
+ * for token t, head h and kept key j = (i_j, i'_j) (slot = i_j*n + i'_j):
+ *   g_c[j]  = w_j (g_j - sum_l w_l g_l),  g_j = <grad_out[t], V[slot_j]>
+ *   dL/dq1  = sum_j g_c[j] C_h[i_j]          dL/dq2 = sum_j g_c[j] C'_h[i'_j]
+ *   dL/dC_h[i]   += sum over (t, j) with i_j = i  of g_c[t,j] q1[t]   (same for C')
+ *   q = (acc - mean) * s + beta,  s = gamma / sqrt(var + eps),  acc = x W^T:
+ *   dL/dacc = dL/dq * s;  dL/dgamma = sum_t dL/dq * (acc - mean) / sqrt(var + eps);
+ *   dL/dbeta = sum_t dL/dq;  dL/dW = dL/dacc^T x;  dL/dx = dL/dacc W.
+ * Outputs (fp64, overwritten; any may be NULL): grad_x [B][d], grad_W [H*dq][d],
+ * grad_gamma, grad_beta [H*dq], grad_subkeys [H][2][n][dq/2], grad_q [B][H*dq].
+ * indices / weights [B][H][k] are the forward's picks; grad_out [B][v] in dtype.
+ * Tokens run one after another (the parameter gradients are sums over tokens).
+ */
+int pkm_oracle_backward_full(int64_t B, int d, int H, int dq, int n, int k, int v, int dtype,
+                             double eps, const void* x, const void* Wq, const float* mean,
+                             const float* var, const float* gamma, const float* beta,
+                             const void* subkeys, const void* values, const int32_t* indices,
+                             const double* weights, const void* grad_out, double* grad_x,
+                             double* grad_W, double* grad_gamma, double* grad_beta,
+                             double* grad_subkeys, double* grad_q_out) {
+  if (B < 0 || d < 1 || H < 1 || dq < 2 || dq % 2 || n < 1 || k < 1 || k > n || v < 1) return -1;
+  const int F = H * dq, half = dq / 2;
+  double* q = (double*)malloc(sizeof(double) * F);
+  double* acc = (double*)malloc(sizeof(double) * F);
+  double* gq = (double*)malloc(sizeof(double) * F);
+  double* gw = (double*)malloc(sizeof(double) * k);
+  double* gc = (double*)malloc(sizeof(double) * k);
+  if (!q || !acc || !gq || !gw || !gc) {
+    free(q); free(acc); free(gq); free(gw); free(gc);
+    return -1;
+  }
+  if (grad_x) memset(grad_x, 0, sizeof(double) * (size_t)B * d);
+  if (grad_W) memset(grad_W, 0, sizeof(double) * (size_t)F * d);
+  if (grad_gamma) memset(grad_gamma, 0, sizeof(double) * F);
+  if (grad_beta) memset(grad_beta, 0, sizeof(double) * F);
+  if (grad_subkeys) memset(grad_subkeys, 0, sizeof(double) * (size_t)H * 2 * n * half);
+  for (int64_t t = 0; t < B; ++t) {
+    /* Recompute acc and q for this token (step 1 of the forward). */
+    for (int f = 0; f < F; ++f) {
+      double a = 0.0;
+      for (int c = 0; c < d; ++c)
+        a += widen(x, dtype, t * (int64_t)d + c) * widen(Wq, dtype, (int64_t)f * d + c);
+      acc[f] = a;
+      q[f] = (a - (double)mean[f]) / sqrt((double)var[f] + eps) * (double)gamma[f] +
+             (double)beta[f];
+      gq[f] = 0.0;
+    }
+    for (int h = 0; h < H; ++h) {
+      const int64_t base = (t * H + h) * (int64_t)k;
+      /* Gradient wrt the kept scores (softmax Jacobian). */
+      double wsum = 0.0;
+      for (int j = 0; j < k; ++j) {
+        double a = 0.0;
+        for (int c = 0; c < v; ++c)
+          a += widen(grad_out, dtype, t * (int64_t)v + c) *
+               widen(values, dtype, (int64_t)indices[base + j] * v + c);
+        gw[j] = a;
+        wsum += weights[base + j] * a;
+      }
+      for (int j = 0; j < k; ++j) gc[j] = weights[base + j] * (gw[j] - wsum);
+      /* A kept score is s1[i] + s2[i']: its gradient goes to both halves. */
+      for (int j = 0; j < k; ++j) {
+        const int64_t slot = indices[base + j];
+        const int64_t sub[2] = {slot / n, slot % n};
+        for (int side = 0; side < 2; ++side) {
+          const int64_t row = ((int64_t)(h * 2 + side) * n + sub[side]) * half;
+          for (int e = 0; e < half; ++e) {
+            const int f = h * dq + side * half + e;
+            gq[f] += gc[j] * widen(subkeys, dtype, row + e);
+            if (grad_subkeys) grad_subkeys[row + e] += gc[j] * q[f];
+          }
+        }
+      }
+    }
+    if (grad_q_out) memcpy(grad_q_out + t * F, gq, sizeof(double) * F);
+    /* Through BatchNorm (inference mode) and the linear map. */
+    for (int f = 0; f < F; ++f) {
+      const double rs = 1.0 / sqrt((double)var[f] + eps);
+      const double gacc = gq[f] * (double)gamma[f] * rs;
+      if (grad_gamma) grad_gamma[f] += gq[f] * (acc[f] - (double)mean[f]) * rs;
+      if (grad_beta) grad_beta[f] += gq[f];
+      for (int c = 0; c < d; ++c) {
+        if (grad_W) grad_W[(int64_t)f * d + c] += gacc * widen(x, dtype, t * (int64_t)d + c);
+        if (grad_x) grad_x[t * (int64_t)d + c] += gacc * widen(Wq, dtype, (int64_t)f * d + c);
+      }
+    }
+  }
+  free(q); free(acc); free(gq); free(gw); free(gc);
+  return 0;
+}

@@ -332,3 +332,75 @@ def test_slot_usage_closed_forms():
     assert oracle.slot_usage(np.full(50, 7, np.int32), 100) == (1, 0)               # one slot
     assert oracle.slot_usage(np.array([3, -1, 100, 3, 99], np.int32), 100) == (2, 2)  # bad ids
     assert oracle.slot_usage(np.zeros(0, np.int32), 10) == (0, 0)
+
+
+# ------------------------------------------------------- full backward pins
+
+
+def _loss_and_picks(L, w, G):
+    r = oracle.forward(L, w.H, w.dq, w.n, w.k)
+    return float((r["out"] * G).sum()), r["indices"]
+
+
+@pytest.mark.parametrize("param", ["x", "W_q", "bn_gamma", "bn_beta", "subkeys"])
+def test_backward_full_matches_finite_differences(param):
+    """dL/dparam of L = <grad_out, out> by central differences through the forward,
+    with the picks held fixed (perturbations that change the picks are skipped)."""
+    w = synth.WORKLOADS["tiny"].with_(B=6, H=2, dq=8, d_model=10, n=6, k=3, v=8,
+                                      bn_random=True)
+    L = synth.make_layer(w, seed=41)
+    L["bn_gamma"] = torch.rand(w.H * w.dq, generator=torch.Generator().manual_seed(1)) + 0.5
+    L["bn_beta"] = torch.randn(w.H * w.dq, generator=torch.Generator().manual_seed(2))
+    g = torch.randn(w.B, w.v, generator=torch.Generator().manual_seed(3))
+    G = g.double().numpy()
+    r = oracle.forward(L, w.H, w.dq, w.n, w.k)
+    grads = oracle.backward_full(L, r["indices"], r["weights"], g, w.H, w.dq, w.n, w.k)
+    key = {"x": "x", "W_q": "W_q", "bn_gamma": "gamma", "bn_beta": "beta",
+           "subkeys": "subkeys"}[param]
+    base = L[param].clone()
+    flat = base.view(-1)
+    fd = np.zeros(flat.numel())
+    skipped = 0
+    h = 2e-4
+    for i in range(flat.numel()):
+        up, dn = flat.clone(), flat.clone()
+        up[i] = flat[i] + h
+        dn[i] = flat[i] - h
+        du = float(up[i].double() - flat[i].double())     # exact fp32 steps
+        dd = float(flat[i].double() - dn[i].double())
+        L[param] = up.view_as(base)
+        lu, iu = _loss_and_picks(L, w, G)
+        L[param] = dn.view_as(base)
+        ld, idn = _loss_and_picks(L, w, G)
+        L[param] = base
+        if not (np.array_equal(iu, r["indices"]) and np.array_equal(idn, r["indices"])):
+            fd[i] = np.nan
+            skipped += 1
+            continue
+        fd[i] = (lu - ld) / (du + dd)
+    got = grads[key].reshape(-1)
+    ok = ~np.isnan(fd)
+    assert skipped <= max(2, 0.1 * flat.numel())
+    np.testing.assert_allclose(got[ok], fd[ok], rtol=2e-5, atol=1e-7)
+
+
+def test_backward_full_value_and_score_parts_match_backward():
+    """The shared parts: dL/dq summed over a head's sub-keys equals the scores' chain."""
+    w = synth.WORKLOADS["tiny"].with_(B=9, H=2, dq=8, d_model=10, n=6, k=3, v=8)
+    L = synth.make_layer(w, seed=42)
+    r = oracle.forward(L, w.H, w.dq, w.n, w.k, want_q=True)
+    g = torch.randn(w.B, w.v, generator=torch.Generator().manual_seed(4))
+    grads = oracle.backward_full(L, r["indices"], r["weights"], g, w.H, w.dq, w.n, w.k)
+    _, gs = oracle.backward(L["values"], g, r["indices"], r["weights"])
+    # dL/d(kept score) pushed into q1 through <q1, C[i]>: sum_e dL/dq1[e] * q1[e]
+    # equals sum_j g_s[j] * s1[i_j] (Euler: s1 is linear in q1); the same for q2.
+    q = r["q"].reshape(w.B, w.H, 2, w.dq // 2)
+    gq = grads["q"].reshape(w.B, w.H, 2, w.dq // 2)
+    C = L["subkeys"].double().numpy()
+    for t in range(w.B):
+        for hh in range(w.H):
+            for side in range(2):
+                sub = r["indices"][t, hh] // w.n if side == 0 else r["indices"][t, hh] % w.n
+                s_half = C[hh, side][sub] @ q[t, hh, side]
+                np.testing.assert_allclose((gq[t, hh, side] * q[t, hh, side]).sum(),
+                                           (gs[t, hh] * s_half).sum(), rtol=1e-10, atol=1e-12)
