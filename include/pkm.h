@@ -73,8 +73,8 @@ typedef struct {
 
 /*
  * Bytes of workspace pkm_forward (for_backward = 0), pkm_backward_values
- * (for_backward = 1) or pkm_slot_usage (for_backward = 2) needs for this shape; 0 if
- * the shape is invalid.
+ * (for_backward = 1), pkm_slot_usage (for_backward = 2) or pkm_backward
+ * (for_backward = 3) needs for this shape; 0 if the shape is invalid.
  */
 size_t pkm_workspace_size(const pkm_shape* s, int for_backward);
 
@@ -129,6 +129,39 @@ int pkm_backward_values(const pkm_shape* s, const void* values, const int32_t* i
                         const float* weights, const void* grad_out, float* grad_values,
                         float* grad_scores, void* workspace, size_t workspace_bytes,
                         void* stream);
+
+/*
+ * Full backward of the layer ("Large Memory Layers with Product Keys", Methodology:
+ * the memory is trained end-to-end with the rest of the network). The top-k choice
+ * is piecewise constant, so the picks of the forward are held fixed. With
+ * L = <grad_out, out>, g_c the kept-score gradients of pkm_backward_values, key
+ * (i, i') = slot i*n + i', acc = x W_q^T and s = gamma / sqrt(var + eps):
+ *   dL/dq1_h = sum_j g_c[j] C_h[i_j],  dL/dq2_h = sum_j g_c[j] C'_h[i'_j]
+ *   grad_subkeys[h][0][i] = sum over picks with left sub-key i of g_c q1_h (C' alike)
+ *   grad_bn_beta = sum_t dL/dq,  grad_bn_gamma = sum_t dL/dq (acc - mean) / sqrt(var + eps)
+ *   grad_W_q = (dL/dq s)^T x,    grad_x = (dL/dq s) W_q
+ * Inputs are those of pkm_forward plus the forward's indices and weights and
+ * grad_out [B][v] (dtype). Outputs, each fp32 and each may be NULL (not computed):
+ *   grad_x        [B][d_model]        overwritten
+ *   grad_W_q      [H*dq][d_model]     overwritten
+ *   grad_bn_gamma [H*dq], grad_bn_beta [H*dq]  overwritten (inference BatchNorm:
+ *                 the running statistics are constants and get no gradient)
+ *   grad_subkeys  [H][2][n][dq/2]     overwritten
+ *   grad_values   [n*n][v]            ACCUMULATED into, as in pkm_backward_values
+ *   grad_scores   [B][H][k]           overwritten
+ * acc is recomputed with the forward's query kernel (no BatchNorm), so the caller
+ * keeps nothing from the forward beyond indices and weights. Sums over tokens are
+ * in fp32 in a fixed order except sub-key rows shared by two 32-pick windows, which
+ * are added atomically. Slot ids outside [0, n*n) are skipped and counted in the
+ * status word. workspace: at least pkm_workspace_size(s, 3) bytes, 256-byte aligned.
+ */
+int pkm_backward(const pkm_shape* s, const void* x, const void* W_q, const float* bn_mean,
+                 const float* bn_var, const float* bn_gamma, const float* bn_beta,
+                 const void* subkeys, const void* values, const int32_t* indices,
+                 const float* weights, const void* grad_out, float* grad_x, float* grad_W_q,
+                 float* grad_bn_gamma, float* grad_bn_beta, float* grad_subkeys,
+                 float* grad_values, float* grad_scores, void* workspace, size_t workspace_bytes,
+                 void* stream);
 
 /*
  * pkm_backward_values without a workspace. The pages have no counterpart: this is

@@ -25,7 +25,7 @@ _STATUS = {0: "PKM_OK", -1: "PKM_ERR_INVALID_ARG", -2: "PKM_ERR_UNSUPPORTED",
 
 EXPORTED = ("pkm_workspace_size", "pkm_forward", "pkm_backward_values", "pkm_device_status",
             "pkm_trace_enable", "pkm_trace_read", "pkm_status_string",
-            "pkm_backward_values_noalloc", "pkm_slot_usage")
+            "pkm_backward_values_noalloc", "pkm_slot_usage", "pkm_backward")
 
 
 class PKMError(RuntimeError):
@@ -59,6 +59,8 @@ def lib() -> ctypes.CDLL:
         L.pkm_forward.restype = ctypes.c_int
         L.pkm_backward_values.argtypes = [S] + [P] * 7 + [ctypes.c_size_t, P]
         L.pkm_backward_values.restype = ctypes.c_int
+        L.pkm_backward.argtypes = [S] + [P] * 19 + [ctypes.c_size_t, P]
+        L.pkm_backward.restype = ctypes.c_int
         L.pkm_backward_values_noalloc.argtypes = [S] + [P] * 6 + [P]
         L.pkm_backward_values_noalloc.restype = ctypes.c_int
         L.pkm_slot_usage.argtypes = [S, P, P, P, ctypes.c_size_t, P]
@@ -175,6 +177,40 @@ def pkm_backward_values(values: torch.Tensor, indices: torch.Tensor, weights: to
     if rc != PKM_OK:
         raise PKMError("pkm_backward_values", rc)
     return grad_values, grad_scores
+
+
+def pkm_backward(x: torch.Tensor, W_q: torch.Tensor, bn_mean: torch.Tensor,
+                 bn_var: torch.Tensor, bn_gamma: torch.Tensor, bn_beta: torch.Tensor,
+                 subkeys: torch.Tensor, values: torch.Tensor, indices: torch.Tensor,
+                 weights: torch.Tensor, grad_out: torch.Tensor, grads: dict,
+                 bn_eps: float = 1e-5, workspace: Optional[torch.Tensor] = None, stream=None):
+    """Full backward of the layer with the forward's picks held fixed.
+
+    ``grads`` maps any of x [B][d], W_q [H*dq][d], bn_gamma, bn_beta [H*dq],
+    subkeys [H][2][n][dq/2], values [n*n][v], scores [B][H][k] to fp32 device
+    tensors; missing entries are not computed. values is accumulated into, the
+    others are overwritten."""
+    B, d = x.shape
+    H, _, n, half = subkeys.shape
+    k = indices.shape[2]
+    v = values.shape[1]
+    shape = make_shape(B, d, H, 2 * half, n, k, v, x.dtype, bn_eps)
+    if workspace is None:
+        nb = int(lib().pkm_workspace_size(ctypes.byref(shape), 3))
+        if nb == 0:
+            raise PKMError("pkm_workspace_size", -1)
+        workspace = torch.empty(nb, dtype=torch.uint8, device=x.device)
+    g = grads
+    rc = lib().pkm_backward(ctypes.byref(shape), _ptr(x), _ptr(W_q), _ptr(bn_mean),
+                            _ptr(bn_var), _ptr(bn_gamma), _ptr(bn_beta), _ptr(subkeys),
+                            _ptr(values), _ptr(indices), _ptr(weights), _ptr(grad_out),
+                            _ptr(g.get("x")), _ptr(g.get("W_q")), _ptr(g.get("bn_gamma")),
+                            _ptr(g.get("bn_beta")), _ptr(g.get("subkeys")), _ptr(g.get("values")),
+                            _ptr(g.get("scores")), _ptr(workspace), workspace.numel(),
+                            _stream(stream))
+    if rc != PKM_OK:
+        raise PKMError("pkm_backward", rc)
+    return grads
 
 
 def pkm_backward_values_noalloc(values: torch.Tensor, indices: torch.Tensor,

@@ -264,12 +264,70 @@ int pkm_trace_read(int pass, double* stage_ms, int max_stages, int64_t* calls,
 }
 
 size_t pkm_workspace_size(const pkm_shape* s, int for_backward) {
+  if (for_backward == 3) {
+    if (validate_shape(s) != PKM_OK) return 0;
+    LayerArgs a{};
+    a.B = s->B; a.H = s->H; a.dq = s->dq; a.n = s->n; a.k = s->k; a.v = s->v;
+    return pkm::backward_full_ws_bytes(a, choose_path(s) == Path::kTensor, nullptr, nullptr);
+  }
   if (for_backward == 2) {
     if (validate_usage(s) != PKM_OK) return 0;
     return pkm::kStatusBytes + align256(pkm::usage_bitmap_bytes(static_cast<int64_t>(s->n) * s->n));
   }
   if ((for_backward ? validate_common(s) : validate_shape(s)) != PKM_OK) return 0;
   return for_backward ? backward_ws(s, nullptr, nullptr) : forward_ws(s, nullptr, nullptr);
+}
+
+int pkm_backward(const pkm_shape* s, const void* x, const void* W_q, const float* bn_mean,
+                 const float* bn_var, const float* bn_gamma, const float* bn_beta,
+                 const void* subkeys, const void* values, const int32_t* indices,
+                 const float* weights, const void* grad_out, float* grad_x, float* grad_W_q,
+                 float* grad_bn_gamma, float* grad_bn_beta, float* grad_subkeys,
+                 float* grad_values, float* grad_scores, void* workspace, size_t workspace_bytes,
+                 void* stream) {
+  int rc = validate_shape(s);
+  if (rc != PKM_OK) return rc;
+  const bool tok = s->B > 0;
+  if (!W_q || !bn_mean || !bn_var || !bn_gamma || !bn_beta || !subkeys || !values ||
+      (tok && (!x || !indices || !weights || !grad_out)))
+    return PKM_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, W_q, bn_mean, bn_var, bn_gamma, bn_beta, subkeys, values, indices,
+                        weights, grad_out, grad_x, grad_W_q, grad_bn_gamma, grad_bn_beta,
+                        grad_subkeys, grad_values, grad_scores};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return PKM_ERR_UNSUPPORTED;
+  const bool tensor = choose_path(s) == Path::kTensor;
+  LayerArgs a{s->B, s->d_model, s->H, s->dq, s->n, s->k, s->v, s->dtype, s->bn_eps,
+              x, W_q, bn_mean, bn_var, bn_gamma, bn_beta, subkeys, values,
+              static_cast<int*>(workspace), 0};
+  const size_t need = pkm::backward_full_ws_bytes(a, tensor, nullptr, nullptr);
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return PKM_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!tok) {
+    // Sums over no tokens: the requested parameter gradients are zero.
+    const int64_t F = static_cast<int64_t>(s->H) * s->dq;
+    const struct { float* p; int64_t count; } zero[] = {
+        {grad_W_q, F * s->d_model}, {grad_bn_gamma, F}, {grad_bn_beta, F},
+        {grad_subkeys, F * s->n}};
+    for (const auto& z : zero)
+      if (z.p && cudaMemsetAsync(z.p, 0, sizeof(float) * z.count, st) != cudaSuccess)
+        return PKM_ERR_CUDA;
+    return PKM_OK;
+  }
+  pkm::FullBackwardWs w;
+  pkm::backward_full_ws_bytes(a, tensor, &w, static_cast<char*>(workspace));
+  if (cudaMemsetAsync(workspace, 0, sizeof(int), st) != cudaSuccess) return PKM_ERR_CUDA;
+  Tracer tr(1);
+  tr.begin(3, st);
+  int launches = 0;
+  const cudaError_t e = pkm::launch_backward_full(a, tensor, indices, weights, grad_out, grad_x,
+                                                  grad_W_q, grad_bn_gamma, grad_bn_beta,
+                                                  grad_subkeys, grad_values, grad_scores, w, st,
+                                                  &launches);
+  tr.end(st);
+  tr.finish(e == cudaSuccess, launches);
+  return e == cudaSuccess ? PKM_OK : PKM_ERR_CUDA;
 }
 
 int pkm_slot_usage(const pkm_shape* s, const int32_t* indices, unsigned long long* hits,
@@ -322,7 +380,7 @@ int pkm_forward(const pkm_shape* s, const void* x, const void* W_q, const float*
   ForwardWs w;
   forward_ws(s, &w, static_cast<char*>(workspace));
   LayerArgs a{s->B, s->d_model, s->H, s->dq, s->n, s->k, s->v, s->dtype, s->bn_eps,
-              x, W_q, bn_mean, bn_var, bn_gamma, bn_beta, subkeys, values, w.status};
+              x, W_q, bn_mean, bn_var, bn_gamma, bn_beta, subkeys, values, w.status, 0};
   if (cudaMemsetAsync(w.status, 0, sizeof(int), st) != cudaSuccess) return PKM_ERR_CUDA;
   // Stages: 0 query network, 1 per-half scores + best 32, 2 candidate top-k + softmax +
   // gather, 3 the whole call.

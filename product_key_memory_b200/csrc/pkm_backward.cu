@@ -326,6 +326,26 @@ __global__ void __launch_bounds__(128) segment_rows_kernel(
 }
 
 // ------------------------------------------------------------------- launcher
+// Stable-enough grouping of E keys in [0, slots): ws.order lists pick ids grouped by
+// key, ws.offsets[key] .. ws.offsets[key + 1] is the key's group, ws.offsets[slots]
+// the number of valid keys. Keys outside the range are skipped (status word set).
+cudaError_t launch_counting_sort(const int* keys, int64_t E, int64_t slots, const BackwardWs& ws,
+                                 int* status, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(ws.counts, 0, sizeof(int) * slots, st);
+  if (e != cudaSuccess) return e;
+  const int64_t eblocks = (E + 255) / 256;
+  const unsigned egrid = static_cast<unsigned>(eblocks < 1 ? 1 : (eblocks < 148 * 32 ? eblocks : 148 * 32));
+  slot_histogram_kernel<<<egrid, 256, 0, st>>>(keys, E, slots, ws.counts, status);
+  const int64_t nblk = scan_blocks(slots);
+  scan_local_kernel<<<static_cast<unsigned>(nblk), kScanThreads, 0, st>>>(ws.counts, slots,
+                                                                           ws.offsets, ws.partials);
+  scan_partials_kernel<<<1, 1024, 0, st>>>(ws.partials, nblk);
+  scan_add_kernel<<<static_cast<unsigned>(nblk), kScanThreads, 0, st>>>(ws.offsets, slots,
+                                                                         ws.partials, nblk);
+  slot_scatter_kernel<<<egrid, 256, 0, st>>>(keys, E, slots, ws.offsets, ws.counts, ws.order);
+  return cudaGetLastError();
+}
+
 static int maxv_bwd(int v, int dtype) {
   const int per = dtype == 0 ? 4 : 8;
   const int m = (v / per + 31) / 32;
@@ -352,18 +372,8 @@ static cudaError_t launch_bwd_t(int64_t B, int H, int k, int v, int64_t slots, c
   }
   between_stages();
   if (!grad_values) return cudaGetLastError();
-  cudaError_t e = cudaMemsetAsync(ws.counts, 0, sizeof(int) * slots, st);
+  cudaError_t e = launch_counting_sort(indices, E, slots, ws, status, st);
   if (e != cudaSuccess) return e;
-  const int64_t eblocks = (E + 255) / 256;
-  const unsigned egrid = static_cast<unsigned>(eblocks < 148 * 32 ? eblocks : 148 * 32);
-  slot_histogram_kernel<<<egrid, 256, 0, st>>>(indices, E, slots, ws.counts, status);
-  const int64_t nblk = scan_blocks(slots);
-  scan_local_kernel<<<static_cast<unsigned>(nblk), kScanThreads, 0, st>>>(ws.counts, slots,
-                                                                           ws.offsets, ws.partials);
-  scan_partials_kernel<<<1, 1024, 0, st>>>(ws.partials, nblk);
-  scan_add_kernel<<<static_cast<unsigned>(nblk), kScanThreads, 0, st>>>(ws.offsets, slots,
-                                                                         ws.partials, nblk);
-  slot_scatter_kernel<<<egrid, 256, 0, st>>>(indices, E, slots, ws.offsets, ws.counts, ws.order);
   const int64_t windows = (E + 31) / 32;
   const int64_t sblocks = (windows + 3) / 4;
   const unsigned sgrid = static_cast<unsigned>(sblocks < 148 * 64 ? sblocks : 148 * 64);

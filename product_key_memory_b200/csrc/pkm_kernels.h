@@ -22,7 +22,8 @@ struct LayerArgs {
   const float* bn_beta;
   const void* subkeys;
   const void* values;
-  int* status;  // device status word
+  int* status;   // device status word
+  int raw_acc;   // query kernels: write acc = x W_q^T without BatchNorm
 };
 
 // SIMT query network + per-half search (pkm_simt.cu).
@@ -50,6 +51,28 @@ cudaError_t launch_backward_values(int64_t B, int H, int k, int v, int dtype, in
                                    const void* grad_out, float* grad_values, float* grad_scores,
                                    const BackwardWs& ws, int* status, cudaStream_t st,
                                    const std::function<void()>& between_stages);
+
+cudaError_t launch_counting_sort(const int* keys, int64_t E, int64_t slots, const BackwardWs& ws,
+                                 int* status, cudaStream_t st);
+
+// Full backward (pkm_backward_full.cu).
+struct FullBackwardWs {
+  BackwardWs values;  // value-gradient grouping
+  float* g_s;         // [B][H][k] kept-score gradients
+  float* acc;         // [B][H*dq] x W_q^T
+  float* g_q;         // [B][H*dq] dL/dq
+  float* g_acc;       // [B][H*dq] dL/dacc
+  void* planes;       // tensor path: acc as three bf16 planes
+  int* targets;       // [2*B*H*k] sub-key of each pick's two halves
+  BackwardWs sub;     // sub-key grouping
+  float* bn_part;     // BatchNorm column-sum partials
+};
+size_t backward_full_ws_bytes(const LayerArgs& a, bool tensor_path, FullBackwardWs* w, char* base);
+cudaError_t launch_backward_full(const LayerArgs& a, bool tensor_path, const int* indices,
+                                 const float* weights, const void* grad_out, float* grad_x,
+                                 float* grad_W, float* grad_gamma, float* grad_beta,
+                                 float* grad_subkeys, float* grad_values, float* grad_scores,
+                                 const FullBackwardWs& w, cudaStream_t st, int* launches);
 
 // Memory utilisation (pkm_usage.cu).
 size_t usage_bitmap_bytes(int64_t slots);

@@ -20,7 +20,7 @@ __global__ void __launch_bounds__(256) query_bn_simt_kernel(
     const T* __restrict__ x, const T* __restrict__ W, const float* __restrict__ mean,
     const float* __restrict__ var, const float* __restrict__ gamma,
     const float* __restrict__ beta, float eps, int64_t B, int d, int F,
-    float* __restrict__ q) {
+    float* __restrict__ q, int raw_acc) {
   __shared__ float xs[16][64 + 4];
   __shared__ float ws[16][64 + 4];
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
@@ -60,8 +60,8 @@ __global__ void __launch_bounds__(256) query_bn_simt_kernel(
   for (int j = 0; j < 4; ++j) {
     const int f = n0 + tx * 4 + j;
     if (f >= F) continue;
-    const float scale = gamma[f] / sqrtf(var[f] + eps);
-    const float mu = mean[f], bt = beta[f];
+    const float scale = raw_acc ? 1.f : gamma[f] / sqrtf(var[f] + eps);
+    const float mu = raw_acc ? 0.f : mean[f], bt = raw_acc ? 0.f : beta[f];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int64_t m = m0 + ty * 4 + i;
@@ -153,11 +153,11 @@ cudaError_t launch_query_bn_simt(const LayerArgs& a, float* q, cudaStream_t st) 
   if (a.dtype == 0)
     query_bn_simt_kernel<float><<<grid, 256, 0, st>>>(
         static_cast<const float*>(a.x), static_cast<const float*>(a.W_q), a.bn_mean, a.bn_var,
-        a.bn_gamma, a.bn_beta, a.bn_eps, a.B, a.d_model, F, q);
+        a.bn_gamma, a.bn_beta, a.bn_eps, a.B, a.d_model, F, q, a.raw_acc);
   else
     query_bn_simt_kernel<uint16_t><<<grid, 256, 0, st>>>(
         static_cast<const uint16_t*>(a.x), static_cast<const uint16_t*>(a.W_q), a.bn_mean,
-        a.bn_var, a.bn_gamma, a.bn_beta, a.bn_eps, a.B, a.d_model, F, q);
+        a.bn_var, a.bn_gamma, a.bn_beta, a.bn_eps, a.B, a.d_model, F, q, a.raw_acc);
   return cudaGetLastError();
 }
 

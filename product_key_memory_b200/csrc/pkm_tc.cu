@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) query_tc_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
     const __grid_constant__ CUtensorMap tm_out, const float* __restrict__ mean,
     const float* __restrict__ var, const float* __restrict__ gamma,
-    const float* __restrict__ beta, float eps, int B, int d, int F, int* status) {
+    const float* __restrict__ beta, float eps, int B, int d, int F, int raw_acc, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* stages = align1024(smem_raw);
   float* scale_s = reinterpret_cast<float*>(stages + kQStages * kQStageBytes);
@@ -91,9 +91,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) query_tc_kernel(
   const int kiters = d / kKBlock;
 
   for (int f = threadIdx.x; f < F; f += blockDim.x) {
-    const float sc = gamma[f] / sqrtf(var[f] + eps);
+    const float sc = raw_acc ? 1.f : gamma[f] / sqrtf(var[f] + eps);
     scale_s[f] = sc;
-    shift_s[f] = beta[f] - mean[f] * sc;
+    shift_s[f] = raw_acc ? 0.f : beta[f] - mean[f] * sc;
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < kQStages; ++s) {
@@ -730,7 +730,8 @@ cudaError_t launch_query_tc(const LayerArgs& a, void* planes, cudaStream_t st) {
   const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
   query_tc_kernel<<<grid, kTcThreads, smem, st>>>(tm_x, tm_w, tm_out, a.bn_mean, a.bn_var,
                                                   a.bn_gamma, a.bn_beta, a.bn_eps,
-                                                  static_cast<int>(a.B), a.d_model, F, a.status);
+                                                  static_cast<int>(a.B), a.d_model, F, a.raw_acc,
+                                                  a.status);
   return cudaGetLastError();
 }
 

@@ -101,3 +101,24 @@ def test_zero_tokens_accepts_null_per_token_pointers():
     assert P.lib().pkm_backward_values(ctypes.byref(s), *bargs, ok, 1 << 40, None) == 0
     s4 = _shape(B=4)
     assert P.lib().pkm_forward(ctypes.byref(s4), *args, ok, 1 << 40, None) == -1
+
+
+def test_full_backward_workspace_and_argument_checks():
+    s = _shape(B=4096, n=512)
+    need = P.lib().pkm_workspace_size(ctypes.byref(s), 3)
+    E = 4096 * 4 * 32
+    # kept-score grads + acc, dL/dq, dL/dacc + q planes + sub-key targets and order
+    assert need >= 256 + 4 * E + 3 * 4 * 4096 * 2048 + 6 * 4096 * 2048 + 2 * 4 * 2 * E
+    assert P.lib().pkm_workspace_size(ctypes.byref(_shape(dq=7)), 3) == 0
+    ok = ctypes.c_void_p(1 << 20)
+    args = [ok] * 11 + [None] * 7                   # inputs, no gradients requested
+    bad = list(args)
+    bad[1] = None                                   # W_q
+    assert P.lib().pkm_backward(ctypes.byref(s), *bad, ok, 1 << 40, None) == -1
+    bad = list(args)
+    bad[6] = ctypes.c_void_p((1 << 20) + 4)         # sub-keys misaligned
+    assert P.lib().pkm_backward(ctypes.byref(s), *bad, ok, 1 << 40, None) == -2
+    assert P.lib().pkm_backward(ctypes.byref(s), *args, ok, 100, None) == -3
+    s0 = _shape(B=0)
+    zargs = [None, ok, ok, ok, ok, ok, ok, ok, None, None, None] + [None] * 7
+    assert P.lib().pkm_backward(ctypes.byref(s0), *zargs, ok, 1 << 40, None) == 0
