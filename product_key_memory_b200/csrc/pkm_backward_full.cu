@@ -10,61 +10,134 @@
 //   dL/dC_h[i] = sum over picks with i_j = i of g_c q1     (C' likewise with q2)
 //   dL/dacc = dL/dq * s,  dL/dgamma = sum_t dL/dq (acc - mean)/sqrt(var + eps),
 //   dL/dbeta = sum_t dL/dq,  dL/dW_q = dL/dacc^T x,  dL/dx = dL/dacc W_q.
+#include <cuda_bf16.h>
+
 #include "pkm_common.cuh"
 #include "pkm_kernels.h"
 #include "pkm_tc.h"
 
 namespace pkm {
 
-// acc = hi + mid + lo from the three bf16 planes the tensor-core query kernel writes.
-__global__ void planes_to_acc_kernel(const uint16_t* __restrict__ planes, int64_t count,
-                                     float* __restrict__ acc) {
+// acc = x W_q^T and q = (acc - mean) * s + beta. With planes, acc = hi + mid + lo from
+// the three bf16 planes of the tensor-core query kernel; without, acc is read as is.
+__global__ void acc_q_kernel(const uint16_t* __restrict__ planes, float* __restrict__ acc,
+                             float* __restrict__ q, const float* __restrict__ mean,
+                             const float* __restrict__ var, const float* __restrict__ gamma,
+                             const float* __restrict__ beta, float eps, int64_t count, int F) {
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < count;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const float hi = load_elem(planes, i), mid = load_elem(planes, count + i);
-    const float lo = load_elem(planes, 2 * count + i);
-    acc[i] = hi + mid + lo;
+    float a;
+    if (planes) {
+      a = load_elem(planes, i) + load_elem(planes, count + i) + load_elem(planes, 2 * count + i);
+      acc[i] = a;
+    } else {
+      a = acc[i];
+    }
+    const int f = static_cast<int>(i % F);
+    q[i] = (a - mean[f]) * (gamma[f] / sqrtf(var[f] + eps)) + beta[f];
   }
 }
 
-// dL/dq and dL/dacc for one token per warp. g_s [B][H][k] are the kept-score gradients.
-template <typename T>
-__global__ void __launch_bounds__(128) grad_q_kernel(
+// VW consecutive elements of row r (8 for the vector forms: one 16-byte load of bf16,
+// two of fp32).
+template <int VW>
+__device__ __forceinline__ void load_run(const uint16_t* p, float (&v)[VW]) {
+  if constexpr (VW == 8) {
+    Vec<uint16_t>::widen(*reinterpret_cast<const uint4*>(p), v);
+  } else {
+#pragma unroll
+    for (int i = 0; i < VW; ++i) v[i] = load_elem(p, i);
+  }
+}
+template <int VW>
+__device__ __forceinline__ void load_run(const float* p, float (&v)[VW]) {
+  if constexpr (VW == 8) {
+    const float4 x = reinterpret_cast<const float4*>(p)[0];
+    const float4 y = reinterpret_cast<const float4*>(p)[1];
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+    v[4] = y.x; v[5] = y.y; v[6] = y.z; v[7] = y.w;
+  } else {
+#pragma unroll
+    for (int i = 0; i < VW; ++i) v[i] = p[i];
+  }
+}
+
+// One warp per (token, head), lane j holding pick j. For each half the picks that
+// share a sub-key are merged: S = sum of their g_c (in pick order), carried by the
+// lowest such lane. Then
+//   dL/dq_half = sum over distinct sub-keys of S * C_half[sub-key]     (VW per lane)
+// and each distinct sub-key becomes one contribution to its gradient row: targets
+// [B][H][k][2] (-1 for merged-away picks) with coefficient coef = S.
+// dL/dacc = dL/dq * s goes to g_acc (fp32) and/or g_planes (bf16 hi/lo [2][B][F]).
+template <typename T, int VW>
+__global__ void __launch_bounds__(128) grad_q_targets_kernel(
     const float* __restrict__ g_s, const int* __restrict__ indices, const T* __restrict__ subkeys,
     const float* __restrict__ gamma, const float* __restrict__ var, float eps, int64_t B, int H,
-    int dq, int n, int k, float* __restrict__ g_q, float* __restrict__ g_acc) {
+    int dq, int n, int k, float* __restrict__ g_q, float* __restrict__ g_acc,
+    uint16_t* __restrict__ g_planes, int* __restrict__ targets, float* __restrict__ coef) {
   const int lane = threadIdx.x & 31;
-  const int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (t >= B) return;
+  const int64_t u = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (u >= B * H) return;
+  const int64_t t = u / H;
+  const int h = static_cast<int>(u - t * H);
   const int half = dq / 2, F = H * dq;
   const int64_t slots = static_cast<int64_t>(n) * n;
-  for (int h = 0; h < H; ++h) {
-    const int64_t base = (t * H + h) * static_cast<int64_t>(k);
-    for (int side = 0; side < 2; ++side) {
-      const int f0 = h * dq + side * half;
-      for (int e0 = 0; e0 < half; e0 += 32 * 8) {
-        float acc[8];
+  const int64_t pick = u * k + lane;
+  int slot = -1;
+  float g = 0.f;
+  if (lane < k) {
+    slot = indices[pick];
+    g = g_s[pick];
+  }
+  const bool valid = lane < k && slot >= 0 && slot < slots;
+  if (!valid) g = 0.f;
+  for (int side = 0; side < 2; ++side) {
+    // Invalid lanes get distinct negative ids, so they match nobody.
+    const int id = valid ? (side ? slot % n : slot / n) : -1 - lane;
+    float S = 0.f;
+    for (int src = 0; src < k; ++src) {
+      const float gs = __shfl_sync(0xffffffffu, g, src);
+      const int is = __shfl_sync(0xffffffffu, id, src);
+      if (is == id) S += gs;
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, id);
+    const bool leader = valid && (__ffs(peers) - 1 == lane);
+    if (lane < k) {
+      targets[2 * pick + side] = leader ? (h * 2 + side) * n + id : -1;
+      coef[2 * pick + side] = S;
+    }
+    const unsigned lead = __ballot_sync(0xffffffffu, leader);
+    const T* book = subkeys + static_cast<int64_t>(h * 2 + side) * n * half;
+    const int f0 = h * dq + side * half;
+    for (int e0 = 0; e0 < half; e0 += 32 * VW) {
+      const int e = e0 + lane * VW;
+      float acc[VW];
 #pragma unroll
-        for (int m = 0; m < 8; ++m) acc[m] = 0.f;
-        for (int j = 0; j < k; ++j) {
-          const int slot = indices[base + j];
-          if (slot < 0 || slot >= slots) continue;
-          const int sub = side ? slot % n : slot / n;
-          const float g = g_s[base + j];
-          const T* row = subkeys + (static_cast<int64_t>(h * 2 + side) * n + sub) * half;
+      for (int i = 0; i < VW; ++i) acc[i] = 0.f;
+      for (unsigned m = lead; m; m &= m - 1) {
+        const int src = __ffs(m) - 1;
+        const float Sl = __shfl_sync(0xffffffffu, S, src);
+        const int il = __shfl_sync(0xffffffffu, id, src);
+        if (e < half) {
+          float r[VW];
+          load_run<VW>(book + static_cast<int64_t>(il) * half + e, r);
 #pragma unroll
-          for (int m = 0; m < 8; ++m) {
-            const int e = e0 + lane + 32 * m;
-            if (e < half) acc[m] = fmaf(g, load_elem(row, e), acc[m]);
-          }
+          for (int i = 0; i < VW; ++i) acc[i] = fmaf(Sl, r[i], acc[i]);
         }
+      }
+      if (e < half) {
+        const int64_t o = t * F + f0 + e;
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          const int e = e0 + lane + 32 * m;
-          if (e < half) {
-            const int f = f0 + e;
-            g_q[t * F + f] = acc[m];
-            g_acc[t * F + f] = acc[m] * (gamma[f] / sqrtf(var[f] + eps));
+        for (int i = 0; i < VW; ++i) {
+          const int f = f0 + e + i;
+          g_q[o + i] = acc[i];
+          const float ga = acc[i] * (gamma[f] / sqrtf(var[f] + eps));
+          if (g_acc) g_acc[o + i] = ga;
+          if (g_planes) {  // hi + lo within 2^-18 relative of ga, for the bf16 GEMMs
+            const __nv_bfloat16 hi = __float2bfloat16_rn(ga);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(ga - __bfloat162float(hi));
+            g_planes[o + i] = __bfloat16_as_ushort(hi);
+            g_planes[B * F + o + i] = __bfloat16_as_ushort(lo);
           }
         }
       }
@@ -108,29 +181,15 @@ __global__ void bn_grad_final_kernel(const float* __restrict__ part, int F,
   if (grad_gamma) grad_gamma[f] = sg;
 }
 
-// Each pick feeds two sub-keys: target 2e = left (h, 0, i), 2e + 1 = right (h, 1, i').
-__global__ void subkey_targets_kernel(const int* __restrict__ indices, int64_t E, int H, int n,
-                                      int k, int* __restrict__ targets) {
-  const int64_t slots = static_cast<int64_t>(n) * n;
-  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < E;
-       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int slot = indices[e];
-    const int h = static_cast<int>((e / k) % H);
-    const bool ok = slot >= 0 && slot < slots;
-    targets[2 * e] = ok ? (h * 2) * n + slot / n : -1;
-    targets[2 * e + 1] = ok ? (h * 2 + 1) * n + slot % n : -1;
-  }
-}
-
-// Windows of 32 sorted contributions per warp; a contribution adds g_c * q_half[t] to
-// its sub-key's gradient row. Groups inside a window are written once (the table was
-// zeroed); groups crossing a window edge use atomics.
+// Sub-key gradient rows from the contributions grouped by target: one warp per window
+// of 32 sorted contributions, a contribution c adding coef[c] * q_half[token] to its
+// row (VW elements per lane, two contributions in flight). Groups inside a window are
+// written once (the table was zeroed); groups crossing a window edge add atomically.
+template <int VW>
 __global__ void __launch_bounds__(128) segment_subkeys_kernel(
     const int* __restrict__ order, const int* __restrict__ offsets,
     const int* __restrict__ total_ptr, const int* __restrict__ targets,
-    const float* __restrict__ g_s, const float* __restrict__ acc, const float* __restrict__ mean,
-    const float* __restrict__ var, const float* __restrict__ gamma,
-    const float* __restrict__ beta, float eps, int H, int dq, int n, int k,
+    const float* __restrict__ coef, const float* __restrict__ q, int H, int dq, int n, int k,
     float* __restrict__ grad_subkeys) {
   const int lane = threadIdx.x & 31;
   const int total = *total_ptr;
@@ -140,10 +199,13 @@ __global__ void __launch_bounds__(128) segment_subkeys_kernel(
        win * 32 < total; win += nwarps) {
     const int w0 = static_cast<int>(win * 32);
     const int w1 = min(w0 + 32, total);
-    int c_l = 0, tg_l = 0;
+    int tg_l = 0, t_l = 0;
+    float cf_l = 0.f;
     if (w0 + lane < w1) {
-      c_l = order[w0 + lane];
-      tg_l = targets[c_l];
+      const int c = order[w0 + lane];
+      tg_l = targets[c];
+      cf_l = coef[c];
+      t_l = (c >> 1) / HK;
     }
     int i = w0;
     while (i < w1) {
@@ -153,32 +215,45 @@ __global__ void __launch_bounds__(128) segment_subkeys_kernel(
       const bool whole = seg0 >= w0 && seg1 <= w1;
       const int side = (tg / n) & 1;
       const int h = tg / (2 * n);
+      const float* qbase = q + h * dq + side * half;
       float* grow = grad_subkeys + static_cast<int64_t>(tg) * half;
-      for (int e0 = 0; e0 < half; e0 += 32 * 8) {
-        float sum[8];
+      for (int e0 = 0; e0 < half; e0 += 32 * VW) {
+        const int e = e0 + lane * VW;
+        const bool in = e < half;
+        float sum[VW];
 #pragma unroll
-        for (int m = 0; m < 8; ++m) sum[m] = 0.f;
-        for (int j = i; j < end; ++j) {
-          const int c = __shfl_sync(0xffffffffu, c_l, j - w0);
-          const int e = c >> 1;
-          const int64_t t = e / HK;
-          const float g = g_s[e];
+        for (int m = 0; m < VW; ++m) sum[m] = 0.f;
+        int j = i;
+        for (; j + 1 < end; j += 2) {
+          const float ca = __shfl_sync(0xffffffffu, cf_l, j - w0);
+          const int ta = __shfl_sync(0xffffffffu, t_l, j - w0);
+          const float cb = __shfl_sync(0xffffffffu, cf_l, j + 1 - w0);
+          const int tb = __shfl_sync(0xffffffffu, t_l, j + 1 - w0);
+          if (in) {
+            float ra[VW], rb[VW];
+            load_run<VW>(qbase + static_cast<int64_t>(ta) * F + e, ra);
+            load_run<VW>(qbase + static_cast<int64_t>(tb) * F + e, rb);
 #pragma unroll
-          for (int m = 0; m < 8; ++m) {
-            const int ee = e0 + lane + 32 * m;
-            if (ee < half) {
-              const int f = h * dq + side * half + ee;
-              const float q = (acc[t * F + f] - mean[f]) * (gamma[f] / sqrtf(var[f] + eps)) + beta[f];
-              sum[m] = fmaf(g, q, sum[m]);
-            }
+            for (int m = 0; m < VW; ++m) sum[m] = fmaf(cb, rb[m], fmaf(ca, ra[m], sum[m]));
           }
         }
+        if (j < end) {
+          const float ca = __shfl_sync(0xffffffffu, cf_l, j - w0);
+          const int ta = __shfl_sync(0xffffffffu, t_l, j - w0);
+          if (in) {
+            float ra[VW];
+            load_run<VW>(qbase + static_cast<int64_t>(ta) * F + e, ra);
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          const int ee = e0 + lane + 32 * m;
-          if (ee < half) {
-            if (whole) grow[ee] += sum[m];
-            else atomicAdd(grow + ee, sum[m]);
+            for (int m = 0; m < VW; ++m) sum[m] = fmaf(ca, ra[m], sum[m]);
+          }
+        }
+        if (in) {
+          if (whole) {
+#pragma unroll
+            for (int m = 0; m < VW; ++m) grow[e + m] = sum[m];
+          } else {
+#pragma unroll
+            for (int m = 0; m < VW; ++m) atomicAdd(grow + e + m, sum[m]);
           }
         }
       }
@@ -249,28 +324,33 @@ static size_t al256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 size_t backward_full_ws_bytes(const LayerArgs& a, bool tensor_path, FullBackwardWs* w, char* base) {
   const int64_t F = static_cast<int64_t>(a.H) * a.dq;
   const int64_t E = a.B * a.H * static_cast<int64_t>(a.k);
+  const int64_t E2 = 2 * E > 0 ? 2 * E : 1;
   const int64_t tslots = 2LL * a.H * a.n;
   BackwardWs vws;
   size_t off = backward_ws_bytes(a.B, a.H, a.k, static_cast<int64_t>(a.n) * a.n, &vws, base);
   const size_t o_gs = off;      off += al256(sizeof(float) * (E > 0 ? E : 1));
   const size_t o_acc = off;     off += al256(sizeof(float) * a.B * F);
+  const size_t o_q = off;       off += al256(sizeof(float) * a.B * F);
   const size_t o_gq = off;      off += al256(sizeof(float) * a.B * F);
-  const size_t o_gacc = off;    off += al256(sizeof(float) * a.B * F);
+  const size_t o_gacc = off;    off += al256(tensor_path ? 0 : sizeof(float) * a.B * F);
   const size_t o_planes = off;  off += al256(tensor_path ? static_cast<size_t>(a.B) * F * 6 : 0);
-  const size_t o_tg = off;      off += al256(sizeof(int) * (2 * E > 0 ? 2 * E : 1));
+  const size_t o_tg = off;      off += al256(sizeof(int) * E2);
+  const size_t o_cf = off;      off += al256(sizeof(float) * E2);
   const size_t o_cnt = off;     off += al256(sizeof(int) * tslots);
   const size_t o_offs = off;    off += al256(sizeof(int) * (tslots + 1));
   const size_t o_part = off;    off += al256(sizeof(int) * (scan_blocks_of(tslots) + 1));
-  const size_t o_ord = off;     off += al256(sizeof(int) * (2 * E > 0 ? 2 * E : 1));
+  const size_t o_ord = off;     off += al256(sizeof(int) * E2);
   const size_t o_bn = off;      off += al256(sizeof(float) * 2 * kBnChunks * F);
   if (w && base) {
     w->values = vws;
     w->g_s = reinterpret_cast<float*>(base + o_gs);
     w->acc = reinterpret_cast<float*>(base + o_acc);
+    w->q = reinterpret_cast<float*>(base + o_q);
     w->g_q = reinterpret_cast<float*>(base + o_gq);
-    w->g_acc = reinterpret_cast<float*>(base + o_gacc);
-    w->planes = base + o_planes;
+    w->g_acc = tensor_path ? nullptr : reinterpret_cast<float*>(base + o_gacc);
+    w->planes = tensor_path ? base + o_planes : nullptr;
     w->targets = reinterpret_cast<int*>(base + o_tg);
+    w->coef = reinterpret_cast<float*>(base + o_cf);
     w->sub.counts = reinterpret_cast<int*>(base + o_cnt);
     w->sub.offsets = reinterpret_cast<int*>(base + o_offs);
     w->sub.partials = reinterpret_cast<int*>(base + o_part);
@@ -278,6 +358,28 @@ size_t backward_full_ws_bytes(const LayerArgs& a, bool tensor_path, FullBackward
     w->bn_part = reinterpret_cast<float*>(base + o_bn);
   }
   return off;
+}
+
+static unsigned grid_of(int64_t blocks, int64_t cap) {
+  return static_cast<unsigned>(blocks < 1 ? 1 : (blocks < cap ? blocks : cap));
+}
+
+template <typename T, int VW>
+static void launch_sub_kernels(const LayerArgs& a, const int* indices, uint16_t* g_planes,
+                               const FullBackwardWs& w, cudaStream_t st) {
+  const int64_t units = a.B * a.H;
+  grad_q_targets_kernel<T, VW><<<grid_of((units + 3) / 4, 1LL << 30), 128, 0, st>>>(
+      w.g_s, indices, static_cast<const T*>(a.subkeys), a.bn_gamma, a.bn_var, a.bn_eps, a.B, a.H,
+      a.dq, a.n, a.k, w.g_q, w.g_acc, g_planes, w.targets, w.coef);
+}
+
+template <int VW>
+static void launch_segment_subkeys(const LayerArgs& a, int64_t E2, int64_t tslots,
+                                   float* grad_subkeys, const FullBackwardWs& w, cudaStream_t st) {
+  const int64_t windows = (E2 + 31) / 32;
+  segment_subkeys_kernel<VW><<<grid_of((windows + 3) / 4, 148 * 32), 128, 0, st>>>(
+      w.sub.order, w.sub.offsets, w.sub.offsets + tslots, w.targets, w.coef, w.q, a.H, a.dq, a.n,
+      a.k, grad_subkeys);
 }
 
 template <typename T>
@@ -289,6 +391,8 @@ static cudaError_t launch_full_t(const LayerArgs& a, bool tensor_path, const int
   const int64_t F = static_cast<int64_t>(a.H) * a.dq;
   const int64_t E = a.B * a.H * static_cast<int64_t>(a.k);
   const int64_t slots = static_cast<int64_t>(a.n) * a.n;
+  const int half = a.dq / 2;
+  const bool vec = (half % 8) == 0;
   cudaError_t e;
   // 1. kept-score gradients (into the workspace) and, if asked, the value gradients.
   e = launch_backward_values(a.B, a.H, a.k, a.v, a.dtype, slots, a.values, indices, weights,
@@ -299,26 +403,29 @@ static cudaError_t launch_full_t(const LayerArgs& a, bool tensor_path, const int
     e = cudaMemcpyAsync(grad_scores, w.g_s, sizeof(float) * E, cudaMemcpyDeviceToDevice, st);
     if (e != cudaSuccess) return e;
   }
-  // 2. acc = x W_q^T (the forward's query network without BatchNorm).
+  // 2. acc = x W_q^T (the forward's query network without BatchNorm), q = BN(acc).
   LayerArgs raw = a;
   raw.raw_acc = 1;
   if (tensor_path) {
     e = launch_query_tc(raw, w.planes, st);
-    if (e != cudaSuccess) return e;
-    const int64_t cnt = a.B * F;
-    const int64_t blocks = (cnt + 255) / 256;
-    planes_to_acc_kernel<<<static_cast<unsigned>(blocks < 148 * 8 ? blocks : 148 * 8), 256, 0, st>>>(
-        static_cast<const uint16_t*>(w.planes), cnt, w.acc);
-    *launches += 2;
   } else {
     e = launch_query_bn_simt(raw, w.acc, st);
-    if (e != cudaSuccess) return e;
-    *launches += 1;
   }
-  // 3. dL/dq, dL/dacc.
-  grad_q_kernel<T><<<static_cast<unsigned>((a.B + 3) / 4), 128, 0, st>>>(
-      w.g_s, indices, static_cast<const T*>(a.subkeys), a.bn_gamma, a.bn_var, a.bn_eps, a.B, a.H,
-      a.dq, a.n, a.k, w.g_q, w.g_acc);
+  if (e != cudaSuccess) return e;
+  acc_q_kernel<<<grid_of((a.B * F + 255) / 256, 148 * 8), 256, 0, st>>>(
+      tensor_path ? static_cast<const uint16_t*>(w.planes) : nullptr, w.acc, w.q, a.bn_mean,
+      a.bn_var, a.bn_gamma, a.bn_beta, a.bn_eps, a.B * F, static_cast<int>(F));
+  *launches += 2;
+  // 3. dL/dq, dL/dacc (bf16 hi/lo planes for the tensor-core GEMMs), merged sub-key
+  //    contributions.
+  // The tensor-core layer shapes always suit the tensor-core GEMMs (the workspace holds
+  // fp32 dL/dacc only for the CUDA-core path).
+  const bool tc_gemm = tensor_path;
+  if (tc_gemm && !gemm_tc_supported(a.B, static_cast<int>(F), a.d_model))
+    return cudaErrorNotSupported;
+  uint16_t* g_planes = tc_gemm ? static_cast<uint16_t*>(w.planes) : nullptr;
+  if (vec) launch_sub_kernels<T, 8>(a, indices, g_planes, w, st);
+  else launch_sub_kernels<T, 1>(a, indices, g_planes, w, st);
   *launches += 1;
   // 4. BatchNorm affine gradients.
   if (grad_gamma || grad_beta) {
@@ -329,25 +436,35 @@ static cudaError_t launch_full_t(const LayerArgs& a, bool tensor_path, const int
         w.bn_part, static_cast<int>(F), grad_gamma, grad_beta);
     *launches += 2;
   }
-  // 5. Sub-key gradients: group the 2E contributions by sub-key, sum in windows.
+  // 5. Sub-key gradients: group the merged contributions by row, sum in windows.
   if (grad_subkeys) {
     const int64_t tslots = 2LL * a.H * a.n;
     const int64_t E2 = 2 * E;
-    e = cudaMemsetAsync(grad_subkeys, 0, sizeof(float) * tslots * (a.dq / 2), st);
+    e = cudaMemsetAsync(grad_subkeys, 0, sizeof(float) * tslots * half, st);
     if (e != cudaSuccess) return e;
-    const int64_t eb = (E + 255) / 256;
-    subkey_targets_kernel<<<static_cast<unsigned>(eb < 148 * 16 ? eb : 148 * 16), 256, 0, st>>>(
-        indices, E, a.H, a.n, a.k, w.targets);
-    e = launch_counting_sort(w.targets, E2, tslots, w.sub, a.status, st);
+    // Merged-away picks carry target -1 and are skipped without a status.
+    e = launch_counting_sort(w.targets, E2, tslots, w.sub, nullptr, st);
     if (e != cudaSuccess) return e;
-    const int64_t windows = (E2 + 31) / 32;
-    const int64_t sblocks = (windows + 3) / 4;
-    segment_subkeys_kernel<<<static_cast<unsigned>(sblocks < 148 * 32 ? (sblocks > 0 ? sblocks : 1) : 148 * 32), 128, 0, st>>>(
-        w.sub.order, w.sub.offsets, w.sub.offsets + tslots, w.targets, w.g_s, w.acc, a.bn_mean,
-        a.bn_var, a.bn_gamma, a.bn_beta, a.bn_eps, a.H, a.dq, a.n, a.k, grad_subkeys);
-    *launches += 7;
+    if (vec) launch_segment_subkeys<8>(a, E2, tslots, grad_subkeys, w, st);
+    else launch_segment_subkeys<1>(a, E2, tslots, grad_subkeys, w, st);
+    *launches += 6;
   }
   // 6. dL/dW_q = dL/dacc^T x  [F][d];  dL/dx = dL/dacc W_q  [B][d].
+  if (tc_gemm) {
+    if (grad_W) {
+      e = launch_grad_w_tc(g_planes, a.x, grad_W, a.B, static_cast<int>(F), a.d_model, a.status,
+                           st);
+      if (e != cudaSuccess) return e;
+      *launches += 1;
+    }
+    if (grad_x) {
+      e = launch_grad_x_tc(g_planes, a.W_q, grad_x, a.B, static_cast<int>(F), a.d_model,
+                           a.status, st);
+      if (e != cudaSuccess) return e;
+      *launches += 1;
+    }
+    return cudaGetLastError();
+  }
   if (grad_W) {
     dim3 g(static_cast<unsigned>((a.d_model + 63) / 64), static_cast<unsigned>((F + 63) / 64));
     gemm_simt_kernel<T><<<g, 256, 0, st>>>(w.g_acc, 1, F, static_cast<const T*>(a.x), a.d_model,

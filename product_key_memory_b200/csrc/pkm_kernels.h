@@ -60,10 +60,12 @@ struct FullBackwardWs {
   BackwardWs values;  // value-gradient grouping
   float* g_s;         // [B][H][k] kept-score gradients
   float* acc;         // [B][H*dq] x W_q^T
+  float* q;           // [B][H*dq] BatchNorm(acc)
   float* g_q;         // [B][H*dq] dL/dq
   float* g_acc;       // [B][H*dq] dL/dacc
   void* planes;       // tensor path: acc as three bf16 planes
-  int* targets;       // [2*B*H*k] sub-key of each pick's two halves
+  int* targets;       // [B*H*k][2] sub-key row of each pick's halves (-1: merged away)
+  float* coef;        // [B*H*k][2] summed kept-score gradient of that row
   BackwardWs sub;     // sub-key grouping
   float* bn_part;     // BatchNorm column-sum partials
 };

@@ -671,11 +671,12 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+}  // namespace
+
 // bf16 tensor map with a {64 x rows} box and the 128-byte swizzle. dims/strides are
 // innermost first; strides are in bytes for dims 1.. (dim 0 is contiguous).
 bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
-              const cuuint64_t* strides, const cuuint32_t* box,
-              CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
+              const cuuint64_t* strides, const cuuint32_t* box, CUtensorMapSwizzle swz) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint32_t estr[3] = {1, 1, 1};
@@ -695,8 +696,6 @@ int sm_count() {
   });
   return n;
 }
-
-}  // namespace
 
 bool tc_supported(int dtype, int d_model, int H, int dq, int n, int k) {
   if (dtype != 1) return false;

@@ -2,6 +2,8 @@
 // the per-half sub-key search. Internal interface.
 #pragma once
 
+#include <cuda.h>
+
 #include "pkm_kernels.h"
 
 namespace pkm {
@@ -17,5 +19,21 @@ cudaError_t launch_query_tc(const LayerArgs& a, void* planes, cudaStream_t st);
 // and the best 32 sub-keys of each half, [B][H][2][32] (in id order, not by score).
 cudaError_t launch_score_topk_tc(const LayerArgs& a, const void* planes, float* list_s,
                                  int* list_i, cudaStream_t st);
+
+// Streaming multiprocessors of the current device (cached).
+int sm_count();
+
+// bf16 tensor map; dims/strides innermost first, strides in bytes for dims 1..
+bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+              const cuuint64_t* strides, const cuuint32_t* box,
+              CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B);
+
+// Tensor-core GEMMs of the backward (pkm_gemm_tc.cu). g_planes holds dL/dacc as two
+// bf16 planes hi/lo [2][B][F]. grad_x [B][d] = dL/dacc W_q; grad_W [F][d] = dL/dacc^T x.
+bool gemm_tc_supported(int64_t B, int F, int d);
+cudaError_t launch_grad_x_tc(const void* g_planes, const void* W_q, float* grad_x, int64_t B,
+                             int F, int d, int* status, cudaStream_t st);
+cudaError_t launch_grad_w_tc(const void* g_planes, const void* x, float* grad_W, int64_t B,
+                             int F, int d, int* status, cudaStream_t st);
 
 }  // namespace pkm
