@@ -22,6 +22,7 @@ same workload per step) and prints the same metric with "impl": "reference".
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import os
@@ -377,9 +378,12 @@ def run_ours(args, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
-def run_c512_and_backward(args, dev, P, hbm, bf16, stream, world, barrier):
-    """512^2-slot forward (the metric's other memory size), the value backward on it,
-    and the wide 1024^2-slot layer (H = 8, v = 1600)."""
+def run_c512_and_backward(args, dev, P, hbm, bf16, stream, world, barrier,
+                          parts=("c512", "backward", "backward_full", "wide")):
+    """512^2-slot forward (the metric's other memory size), the value backward and the
+    full backward on its picks, and the wide 1024^2-slot layer (H = 8, v = 1600).
+    `parts` selects the measurements (the c512 forward always runs: it makes the
+    picks)."""
     w = synth.WORKLOADS["c512"]
     L = synth.make_layer(w)
     d = {k: v.to(dev) for k, v in L.items()}
@@ -417,9 +421,12 @@ def run_c512_and_backward(args, dev, P, hbm, bf16, stream, world, barrier):
     fwd_ms = timed(fwd, args.steps)
     stage_ms, calls, _ = P.pkm_trace_read(0)
     t_roof = max(w.H * w.k * w.v * 2 * B / (hbm * 1e9), gemm_flops_per_token(w) * B / (bf16 * 1e12))
-    res = {"c512": {"workload": workload_desc(w), "value": world * B / (fwd_ms / 1e3),
-                    "unit": UNIT, "ms_per_step": fwd_ms, "step_roofline_frac": t_roof * 1e3 / fwd_ms,
-                    "stage_ms": [m / max(1, calls) for m in stage_ms[:3]]}}
+    res = {}
+    if "c512" in parts:
+        res["c512"] = {"workload": workload_desc(w), "value": world * B / (fwd_ms / 1e3),
+                       "unit": UNIT, "ms_per_step": fwd_ms,
+                       "step_roofline_frac": t_roof * 1e3 / fwd_ms,
+                       "stage_ms": [m / max(1, calls) for m in stage_ms[:3]]}
 
     # Backward on the c512 picks: grad_out ~ N(0, 1) bf16 [4096][1024].
     gout = synth.make_grad_out(w).to(dev)
@@ -431,24 +438,54 @@ def run_c512_and_backward(args, dev, P, hbm, bf16, stream, world, barrier):
     def bwd():
         P.pkm_backward_values(d["values"], idx, wts, gout, gv, gs, w.n, workspace=bws)
 
-    for _ in range(max(3, args.warmup)):
-        bwd()
-    P.pkm_trace_read(1)
-    bwd_ms = timed(bwd, args.steps)
-    bstage, bcalls, _ = P.pkm_trace_read(1)
-    P.pkm_trace_enable(False)
     uniq = int(torch.unique(idx).numel())
     picks = idx.numel()
     bytes_alg = picks * w.v * 2 + B * w.v * 2 + picks * 8 + 2 * uniq * w.v * 4
-    res["backward"] = {
-        "workload": "bwd512: value backward on the c512 picks, grad_out bf16 [4096][1024]",
-        "value": world * B / (bwd_ms / 1e3), "unit": UNIT, "ms_per_step": bwd_ms,
-        "unique_rows": uniq, "picks": picks,
-        "algorithmic_bytes": bytes_alg, "achieved_gbs": bytes_alg / (bwd_ms * 1e-3) / 1e9,
-        "frac_of_hbm": bytes_alg / (bwd_ms * 1e-3) / 1e9 / hbm,
-        "stage_ms": [m / max(1, bcalls) for m in bstage[:2]]}
-    del d, gv, gout, bws, ws
+    if "backward" in parts:
+        for _ in range(max(3, args.warmup)):
+            bwd()
+        P.pkm_trace_read(1)
+        bwd_ms = timed(bwd, args.steps)
+        bstage, bcalls, _ = P.pkm_trace_read(1)
+        res["backward"] = {
+            "workload": "bwd512: value backward on the c512 picks, grad_out bf16 [4096][1024]",
+            "value": world * B / (bwd_ms / 1e3), "unit": UNIT, "ms_per_step": bwd_ms,
+            "unique_rows": uniq, "picks": picks,
+            "algorithmic_bytes": bytes_alg, "achieved_gbs": bytes_alg / (bwd_ms * 1e-3) / 1e9,
+            "frac_of_hbm": bytes_alg / (bwd_ms * 1e-3) / 1e9 / hbm,
+            "stage_ms": [m / max(1, bcalls) for m in bstage[:2]]}
+    P.pkm_trace_enable(False)
+
+    # Full backward on the same picks: every gradient of the layer (x, W_q, BatchNorm
+    # affine, sub-keys, values, kept scores).
+    F = w.H * w.dq
+    fws = torch.empty(int(P.lib().pkm_workspace_size(ctypes.byref(shape), 3)), dtype=torch.uint8,
+                      device=dev)
+    grads = {"x": torch.empty(B, w.d_model, device=dev), "W_q": torch.empty(F, w.d_model, device=dev),
+             "bn_gamma": torch.empty(F, device=dev), "bn_beta": torch.empty(F, device=dev),
+             "subkeys": torch.empty(w.H, 2, w.n, w.dq // 2, device=dev), "values": gv, "scores": gs}
+
+    def bwd_full():
+        P.pkm_backward(d["x"], d["W_q"], d["bn_mean"], d["bn_var"], d["bn_gamma"], d["bn_beta"],
+                       d["subkeys"], d["values"], idx, wts, gout, grads, workspace=fws)
+
+    if "backward_full" in parts:
+        for _ in range(max(3, args.warmup)):
+            bwd_full()
+        full_ms = timed(bwd_full, args.steps)
+        full_bytes = (bytes_alg + B * w.d_model * (2 + 4) + F * w.d_model * (2 + 4)
+                      + w.H * w.n * w.dq * (2 + 4))
+        full_flops = 3 * 2 * B * F * w.d_model     # x W_q^T again, dL/dx, dL/dW_q
+        t_mem, t_gemm = full_bytes / (hbm * 1e9), full_flops / (bf16 * 1e12)
+        res["backward_full"] = {
+            "workload": "bwd512 full: every gradient of the c512 layer on its picks",
+            "value": world * B / (full_ms / 1e3), "unit": UNIT, "ms_per_step": full_ms,
+            "algorithmic_bytes": full_bytes, "gemm_flops": full_flops,
+            "step_roofline_frac": max(t_mem, t_gemm) * 1e3 / full_ms}
+    del d, gv, gout, bws, ws, fws, grads
     torch.cuda.empty_cache()
+    if "wide" not in parts:
+        return res
 
     # The wide layer: d_model 1600, H = 8, 1024^2 slots, v = 1600 (3.4 GB table).
     w = synth.WORKLOADS["wide"]
@@ -488,6 +525,10 @@ def main():
     ap.add_argument("--workload", default="c1024", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the c512 / backward / CPU-oracle measurements")
+    ap.add_argument("--part", default=None,
+                    choices=["c512", "backward", "backward_full", "wide"],
+                    help="run only this sub-measurement and print its JSON object "
+                         "(for profiling one kernel family; not a bench line)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -496,6 +537,16 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.part is not None:
+        import product_key_memory_b200 as P
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        pk, _ = peaks()
+        res = run_c512_and_backward(args, dev, P, float(pk["hbm_gbs"]), float(pk["bf16_tflops"]),
+                                    torch.cuda.current_stream(dev), 1, lambda: None,
+                                    parts=(args.part,))
+        print(json.dumps(res), flush=True)
         return
     if world > 1:
         import datetime
