@@ -51,7 +51,10 @@ def lib():
         L.pkm_oracle_finish.restype = _I
         L.pkm_oracle_backward.argtypes = [_I64, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]
         L.pkm_oracle_backward.restype = _I
-        L.pkm_oracle_backward_full.argtypes = [_I64, _I, _I, _I, _I, _I, _I, _I, _D] + [_P] * 17
+        L.pkm_oracle_forward_train.argtypes = ([_I64, _I, _I, _I, _I, _I, _I, _I, _D, _D]
+                                               + [_P] * 18 + [_I])
+        L.pkm_oracle_forward_train.restype = _I
+        L.pkm_oracle_backward_full.argtypes = [_I64, _I, _I, _I, _I, _I, _I, _I, _D, _I] + [_P] * 17
         L.pkm_oracle_backward_full.restype = _I
         L.pkm_oracle_slot_usage.argtypes = [_I64, _P, _I64, _P]
         L.pkm_oracle_slot_usage.restype = _I64
@@ -109,6 +112,39 @@ def forward(layer: dict, H: int, dq: int, n: int, k: int, eps: float = 1e-5,
     if rc != 0:
         raise ValueError("pkm_oracle_forward rejected the sizes")
     return dict(out=out, indices=idx, weights=w, scores=s, q=q, half=half)
+
+
+def forward_train(layer: dict, H: int, dq: int, n: int, k: int, eps: float = 1e-5,
+                  momentum: float = 0.1, want_q: bool = False, want_half: bool = False,
+                  threads: int = 0) -> dict:
+    """Forward with BatchNorm in training mode: the batch's own statistics normalise
+    it and the running statistics (layer['bn_mean'], layer['bn_var']) move towards
+    them. Returns forward()'s arrays plus batch_mean, batch_var (biased) and
+    running_mean, running_var (the updated running statistics), all fp64."""
+    x, dt = _raw(layer["x"])
+    W, _ = _raw(layer["W_q"])
+    C, _ = _raw(layer["subkeys"])
+    V, _ = _raw(layer["values"])
+    B, d = x.shape
+    v = V.shape[1]
+    F = H * dq
+    rm, rv = _f32(layer["bn_mean"]), _f32(layer["bn_var"])
+    gamma, beta = _f32(layer["bn_gamma"]), _f32(layer["bn_beta"])
+    r = dict(out=np.zeros((B, v)), indices=np.zeros((B, H, k), np.int32),
+             weights=np.zeros((B, H, k)), scores=np.zeros((B, H, k)),
+             q=np.zeros((B, F)) if want_q else None,
+             half=np.zeros((B, H, 2, n)) if want_half else None,
+             batch_mean=np.zeros(F), batch_var=np.zeros(F), running_mean=np.zeros(F),
+             running_var=np.zeros(F))
+    rc = lib().pkm_oracle_forward_train(
+        B, d, H, dq, n, k, v, dt, eps, momentum, _ptr(x), _ptr(W), _ptr(rm), _ptr(rv),
+        _ptr(gamma), _ptr(beta), _ptr(C), _ptr(V), _ptr(r["out"]), _ptr(r["indices"]),
+        _ptr(r["weights"]), _ptr(r["scores"]), _ptr(r["q"]), _ptr(r["half"]),
+        _ptr(r["batch_mean"]), _ptr(r["batch_var"]), _ptr(r["running_mean"]),
+        _ptr(r["running_var"]), threads)
+    if rc != 0:
+        raise ValueError("pkm_oracle_forward_train rejected the sizes")
+    return r
 
 
 def flat_topk(q: np.ndarray, subkeys: torch.Tensor, H: int, dq: int, n: int, k: int,
@@ -182,10 +218,13 @@ def slot_usage(indices: np.ndarray, slots: int):
 
 
 def backward_full(layer: dict, indices: np.ndarray, weights: np.ndarray,
-                  grad_out: torch.Tensor, H: int, dq: int, n: int, k: int, eps: float = 1e-5):
+                  grad_out: torch.Tensor, H: int, dq: int, n: int, k: int, eps: float = 1e-5,
+                  bn_training: bool = False):
     """Gradients of L = <grad_out, out> with the picks held fixed. Returns a dict of
     fp64 arrays: x [B][d], W_q [H*dq][d], gamma, beta [H*dq], subkeys [H][2][n][dq/2],
-    q [B][H*dq] (dL/dq)."""
+    q [B][H*dq] (dL/dq). With bn_training the batch's own statistics (recomputed from
+    the batch) normalised the forward and the gradient flows through them too;
+    layer['bn_mean'] / ['bn_var'] are then not read."""
     x, dt = _raw(layer["x"])
     W, _ = _raw(layer["W_q"])
     C, _ = _raw(layer["subkeys"])
@@ -202,7 +241,8 @@ def backward_full(layer: dict, indices: np.ndarray, weights: np.ndarray,
     weights = np.ascontiguousarray(weights, dtype=np.float64)
     out = dict(x=np.zeros((B, d)), W_q=np.zeros((F, d)), gamma=np.zeros(F), beta=np.zeros(F),
                subkeys=np.zeros((H, 2, n, dq // 2)), q=np.zeros((B, F)))
-    rc = lib().pkm_oracle_backward_full(B, d, H, dq, n, k, v, dt, eps, _ptr(x), _ptr(W),
+    rc = lib().pkm_oracle_backward_full(B, d, H, dq, n, k, v, dt, eps, int(bool(bn_training)),
+                                        _ptr(x), _ptr(W),
                                         _ptr(mean), _ptr(var), _ptr(gamma), _ptr(beta), _ptr(C),
                                         _ptr(V), _ptr(indices), _ptr(weights), _ptr(G),
                                         _ptr(out["x"]), _ptr(out["W_q"]), _ptr(out["gamma"]),

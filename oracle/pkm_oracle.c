@@ -97,24 +97,19 @@ static void sort_best_first(scored_t* all, int64_t count) {
   qsort(all, (size_t)count, sizeof(scored_t), better_first);
 }
 
-/* One token, all heads: steps 1-7. Scratch is allocated per call. */
-static int forward_token(int64_t t, int d, int H, int dq, int n, int k, int v, int dtype,
-                         double eps, const void* x, const void* Wq, const float* mean,
-                         const float* var, const float* gamma, const float* beta,
-                         const void* subkeys, const void* values, double* out,
-                         int32_t* indices, double* weights, double* scores, double* q_out,
-                         double* half_out) {
-  const int F = H * dq, half = dq / 2;
-  double* q = (double*)malloc(sizeof(double) * F);
+/* One token, all heads, steps 2-7 from its query q [H*dq]. Scratch is allocated per
+ * call. */
+static int search_token(int64_t t, int H, int dq, int n, int k, int v, int dtype,
+                        const double* q, const void* subkeys, const void* values, double* out,
+                        int32_t* indices, double* weights, double* scores, double* half_out) {
+  const int half = dq / 2;
   double* s = (double*)malloc(sizeof(double) * 2 * n);
   scored_t* lists = (scored_t*)malloc(sizeof(scored_t) * 2 * (size_t)n);
   scored_t* cand = (scored_t*)malloc(sizeof(scored_t) * (size_t)k * k);
-  if (!q || !s || !lists || !cand) {
-    free(q); free(s); free(lists); free(cand);
+  if (!s || !lists || !cand) {
+    free(s); free(lists); free(cand);
     return -1;
   }
-  query_one(x, Wq, dtype, t, d, F, mean, var, gamma, beta, eps, q);
-  if (q_out) memcpy(q_out + t * F, q, sizeof(double) * F);
   if (out)
     for (int c = 0; c < v; ++c) out[t * (int64_t)v + c] = 0.0;
 
@@ -156,8 +151,56 @@ static int forward_token(int64_t t, int d, int H, int dq, int n, int k, int v, i
           out[t * (int64_t)v + c] += w * widen(values, dtype, cand[j].id * (int64_t)v + c);
     }
   }
-  free(q); free(s); free(lists); free(cand);
+  free(s); free(lists); free(cand);
   return 0;
+}
+
+/* One token, all heads: steps 1-7. */
+static int forward_token(int64_t t, int d, int H, int dq, int n, int k, int v, int dtype,
+                         double eps, const void* x, const void* Wq, const float* mean,
+                         const float* var, const float* gamma, const float* beta,
+                         const void* subkeys, const void* values, double* out,
+                         int32_t* indices, double* weights, double* scores, double* q_out,
+                         double* half_out) {
+  const int F = H * dq;
+  double* q = (double*)malloc(sizeof(double) * F);
+  if (!q) return -1;
+  query_one(x, Wq, dtype, t, d, F, mean, var, gamma, beta, eps, q);
+  if (q_out) memcpy(q_out + t * F, q, sizeof(double) * F);
+  const int rc = search_token(t, H, dq, n, k, v, dtype, q, subkeys, values, out, indices,
+                              weights, scores, half_out);
+  free(q);
+  return rc;
+}
+
+/* acc[t][f] = sum_c x[t][c] W[f][c] for every token (the linear map of step 1). */
+static void linear_all(int64_t B, int d, int F, int dtype, const void* x, const void* Wq,
+                       double* acc) {
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static)
+#endif
+  for (int64_t t = 0; t < B; ++t)
+    for (int f = 0; f < F; ++f) {
+      double a = 0.0;
+      for (int c = 0; c < d; ++c)
+        a += widen(x, dtype, t * (int64_t)d + c) * widen(Wq, dtype, (int64_t)f * d + c);
+      acc[t * F + f] = a;
+    }
+}
+
+/* BatchNorm training-mode statistics of acc over the batch, per feature:
+ * mean = (1/B) sum_t acc, var = (1/B) sum_t (acc - mean)^2 (the biased variance that
+ * normalises the batch). Two passes, tokens in order. */
+static void batch_stats(int64_t B, int F, const double* acc, double* mean, double* var) {
+  for (int f = 0; f < F; ++f) {
+    double s = 0.0;
+    for (int64_t t = 0; t < B; ++t) s += acc[t * F + f];
+    const double mu = s / (double)B;
+    double m2 = 0.0;
+    for (int64_t t = 0; t < B; ++t) m2 += (acc[t * F + f] - mu) * (acc[t * F + f] - mu);
+    mean[f] = mu;
+    var[f] = m2 / (double)B;
+  }
 }
 
 /*
@@ -185,6 +228,67 @@ int pkm_oracle_forward(int64_t B, int d, int H, int dq, int n, int k, int v, int
     err |= forward_token(t, d, H, dq, n, k, v, dtype, eps, x, Wq, mean, var, gamma, beta,
                          subkeys, values, out, indices, weights, scores, q_out, half_out)
                ? 1 : 0;
+  (void)nthreads;
+  return err ? -1 : 0;
+}
+
+/*
+ * Forward with BatchNorm in training mode (the query network's "batch
+ * normalization" while the model trains): the batch's own statistics normalise it,
+ *   q = (acc - mean_B) / sqrt(var_B + eps) * gamma + beta,
+ * mean_B, var_B from batch_stats, and the running statistics move towards them:
+ *   running_mean' = (1 - momentum) running_mean + momentum mean_B
+ *   running_var'  = (1 - momentum) running_var  + momentum var_B B / (B - 1)
+ * (the unbiased variance, as the common BatchNorm layers keep it). Steps 2-7 as in
+ * pkm_oracle_forward. Outputs as pkm_oracle_forward plus batch_mean, batch_var,
+ * new_running_mean, new_running_var [H*dq] (fp64; any may be NULL). B >= 2.
+ */
+int pkm_oracle_forward_train(int64_t B, int d, int H, int dq, int n, int k, int v, int dtype,
+                             double eps, double momentum, const void* x, const void* Wq,
+                             const float* running_mean, const float* running_var,
+                             const float* gamma, const float* beta, const void* subkeys,
+                             const void* values, double* out, int32_t* indices,
+                             double* weights, double* scores, double* q_out, double* half_out,
+                             double* batch_mean, double* batch_var, double* new_running_mean,
+                             double* new_running_var, int nthreads) {
+  if (B < 2 || d < 1 || H < 1 || dq < 2 || dq % 2 || n < 1 || k < 1 || k > n || v < 0)
+    return -1;
+  const int F = H * dq;
+  double* acc = (double*)malloc(sizeof(double) * (size_t)B * F);
+  double* mu = (double*)malloc(sizeof(double) * F);
+  double* var = (double*)malloc(sizeof(double) * F);
+  double* q = (double*)malloc(sizeof(double) * (size_t)B * F);
+  if (!acc || !mu || !var || !q) {
+    free(acc); free(mu); free(var); free(q);
+    return -1;
+  }
+#ifdef _OPENMP
+  if (nthreads > 0) omp_set_num_threads(nthreads);
+#endif
+  linear_all(B, d, F, dtype, x, Wq, acc);
+  batch_stats(B, F, acc, mu, var);
+  for (int64_t t = 0; t < B; ++t)
+    for (int f = 0; f < F; ++f)
+      q[t * F + f] = (acc[t * F + f] - mu[f]) / sqrt(var[f] + eps) * (double)gamma[f] +
+                     (double)beta[f];
+  int err = 0;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : err)
+#endif
+  for (int64_t t = 0; t < B; ++t)
+    err |= search_token(t, H, dq, n, k, v, dtype, q + t * F, subkeys, values, out, indices,
+                        weights, scores, half_out) ? 1 : 0;
+  if (q_out) memcpy(q_out, q, sizeof(double) * (size_t)B * F);
+  for (int f = 0; f < F; ++f) {
+    if (batch_mean) batch_mean[f] = mu[f];
+    if (batch_var) batch_var[f] = var[f];
+    if (new_running_mean)
+      new_running_mean[f] = (1.0 - momentum) * (double)running_mean[f] + momentum * mu[f];
+    if (new_running_var)
+      new_running_var[f] = (1.0 - momentum) * (double)running_var[f] +
+                           momentum * var[f] * (double)B / (double)(B - 1);
+  }
+  free(acc); free(mu); free(var); free(q);
   (void)nthreads;
   return err ? -1 : 0;
 }
@@ -354,48 +458,62 @@ int64_t pkm_oracle_slot_usage(int64_t picks, const int32_t* indices, int64_t slo
  *   g_c[j]  = w_j (g_j - sum_l w_l g_l),  g_j = <grad_out[t], V[slot_j]>
  *   dL/dq1  = sum_j g_c[j] C_h[i_j]          dL/dq2 = sum_j g_c[j] C'_h[i'_j]
  *   dL/dC_h[i]   += sum over (t, j) with i_j = i  of g_c[t,j] q1[t]   (same for C')
- *   q = (acc - mean) * s + beta,  s = gamma / sqrt(var + eps),  acc = x W^T:
- *   dL/dacc = dL/dq * s;  dL/dgamma = sum_t dL/dq * (acc - mean) / sqrt(var + eps);
- *   dL/dbeta = sum_t dL/dq;  dL/dW = dL/dacc^T x;  dL/dx = dL/dacc W.
+ *   q = (acc - mean) / sqrt(var + eps) * gamma + beta,  acc = x W^T,
+ *   xhat = (acc - mean) / sqrt(var + eps):
+ *   dL/dgamma = sum_t dL/dq xhat;  dL/dbeta = sum_t dL/dq;
+ *   dL/dW = dL/dacc^T x;  dL/dx = dL/dacc W, where
+ *     inference BatchNorm (bn_training = 0; mean, var are the running statistics,
+ *     constants):  dL/dacc = dL/dq gamma / sqrt(var + eps)
+ *     training BatchNorm (bn_training = 1; mean, var are the batch's own, recomputed
+ *     here from acc, and depend on every token -- the backward of batch
+ *     normalisation, Ioffe and Szegedy 2015):
+ *       dL/dacc = gamma / sqrt(var + eps) (dL/dq - (1/B) sum_t dL/dq
+ *                                          - xhat (1/B) sum_t dL/dq xhat)
  * Outputs (fp64, overwritten; any may be NULL): grad_x [B][d], grad_W [H*dq][d],
  * grad_gamma, grad_beta [H*dq], grad_subkeys [H][2][n][dq/2], grad_q [B][H*dq].
  * indices / weights [B][H][k] are the forward's picks; grad_out [B][v] in dtype.
- * Tokens run one after another (the parameter gradients are sums over tokens).
+ * Every sum over tokens runs in token order; independent outputs run in parallel.
  */
 int pkm_oracle_backward_full(int64_t B, int d, int H, int dq, int n, int k, int v, int dtype,
-                             double eps, const void* x, const void* Wq, const float* mean,
-                             const float* var, const float* gamma, const float* beta,
-                             const void* subkeys, const void* values, const int32_t* indices,
-                             const double* weights, const void* grad_out, double* grad_x,
-                             double* grad_W, double* grad_gamma, double* grad_beta,
-                             double* grad_subkeys, double* grad_q_out) {
+                             double eps, int bn_training, const void* x, const void* Wq,
+                             const float* mean, const float* var, const float* gamma,
+                             const float* beta, const void* subkeys, const void* values,
+                             const int32_t* indices, const double* weights,
+                             const void* grad_out, double* grad_x, double* grad_W,
+                             double* grad_gamma, double* grad_beta, double* grad_subkeys,
+                             double* grad_q_out) {
   if (B < 0 || d < 1 || H < 1 || dq < 2 || dq % 2 || n < 1 || k < 1 || k > n || v < 1) return -1;
+  if (bn_training && B < 2) return -1;
   const int F = H * dq, half = dq / 2;
+  const size_t BF = (size_t)B * F;
+  double* acc = (double*)malloc(sizeof(double) * (BF ? BF : 1));
+  double* gq = (double*)calloc(BF ? BF : 1, sizeof(double));
+  double* gacc = (double*)malloc(sizeof(double) * (BF ? BF : 1));
+  double* mu = (double*)malloc(sizeof(double) * F);
+  double* sd = (double*)malloc(sizeof(double) * F);   /* sqrt(var + eps) */
   double* q = (double*)malloc(sizeof(double) * F);
-  double* acc = (double*)malloc(sizeof(double) * F);
-  double* gq = (double*)malloc(sizeof(double) * F);
   double* gw = (double*)malloc(sizeof(double) * k);
   double* gc = (double*)malloc(sizeof(double) * k);
-  if (!q || !acc || !gq || !gw || !gc) {
-    free(q); free(acc); free(gq); free(gw); free(gc);
+  if (!acc || !gq || !gacc || !mu || !sd || !q || !gw || !gc) {
+    free(acc); free(gq); free(gacc); free(mu); free(sd); free(q); free(gw); free(gc);
     return -1;
   }
-  if (grad_x) memset(grad_x, 0, sizeof(double) * (size_t)B * d);
-  if (grad_W) memset(grad_W, 0, sizeof(double) * (size_t)F * d);
-  if (grad_gamma) memset(grad_gamma, 0, sizeof(double) * F);
-  if (grad_beta) memset(grad_beta, 0, sizeof(double) * F);
   if (grad_subkeys) memset(grad_subkeys, 0, sizeof(double) * (size_t)H * 2 * n * half);
-  for (int64_t t = 0; t < B; ++t) {
-    /* Recompute acc and q for this token (step 1 of the forward). */
+  /* Step 1 again (acc = x W^T), and the statistics BatchNorm used. */
+  linear_all(B, d, F, dtype, x, Wq, acc);
+  if (bn_training) {
+    batch_stats(B, F, acc, mu, sd);
+    for (int f = 0; f < F; ++f) sd[f] = sqrt(sd[f] + eps);
+  } else {
     for (int f = 0; f < F; ++f) {
-      double a = 0.0;
-      for (int c = 0; c < d; ++c)
-        a += widen(x, dtype, t * (int64_t)d + c) * widen(Wq, dtype, (int64_t)f * d + c);
-      acc[f] = a;
-      q[f] = (a - (double)mean[f]) / sqrt((double)var[f] + eps) * (double)gamma[f] +
-             (double)beta[f];
-      gq[f] = 0.0;
+      mu[f] = (double)mean[f];
+      sd[f] = sqrt((double)var[f] + eps);
     }
+  }
+  for (int64_t t = 0; t < B; ++t) {
+    for (int f = 0; f < F; ++f)
+      q[f] = (acc[t * F + f] - mu[f]) / sd[f] * (double)gamma[f] + (double)beta[f];
+    double* g = gq + t * F;
     for (int h = 0; h < H; ++h) {
       const int64_t base = (t * H + h) * (int64_t)k;
       /* Gradient wrt the kept scores (softmax Jacobian). */
@@ -417,25 +535,58 @@ int pkm_oracle_backward_full(int64_t B, int d, int H, int dq, int n, int k, int 
           const int64_t row = ((int64_t)(h * 2 + side) * n + sub[side]) * half;
           for (int e = 0; e < half; ++e) {
             const int f = h * dq + side * half + e;
-            gq[f] += gc[j] * widen(subkeys, dtype, row + e);
+            g[f] += gc[j] * widen(subkeys, dtype, row + e);
             if (grad_subkeys) grad_subkeys[row + e] += gc[j] * q[f];
           }
         }
       }
     }
-    if (grad_q_out) memcpy(grad_q_out + t * F, gq, sizeof(double) * F);
-    /* Through BatchNorm (inference mode) and the linear map. */
-    for (int f = 0; f < F; ++f) {
-      const double rs = 1.0 / sqrt((double)var[f] + eps);
-      const double gacc = gq[f] * (double)gamma[f] * rs;
-      if (grad_gamma) grad_gamma[f] += gq[f] * (acc[f] - (double)mean[f]) * rs;
-      if (grad_beta) grad_beta[f] += gq[f];
-      for (int c = 0; c < d; ++c) {
-        if (grad_W) grad_W[(int64_t)f * d + c] += gacc * widen(x, dtype, t * (int64_t)d + c);
-        if (grad_x) grad_x[t * (int64_t)d + c] += gacc * widen(Wq, dtype, (int64_t)f * d + c);
+  }
+  if (grad_q_out) memcpy(grad_q_out, gq, sizeof(double) * BF);
+  /* Through BatchNorm. */
+  for (int f = 0; f < F; ++f) {
+    double sb = 0.0, sg = 0.0;
+    for (int64_t t = 0; t < B; ++t) {
+      sb += gq[t * F + f];
+      sg += gq[t * F + f] * ((acc[t * F + f] - mu[f]) / sd[f]);
+    }
+    if (grad_beta) grad_beta[f] = sb;
+    if (grad_gamma) grad_gamma[f] = sg;
+    for (int64_t t = 0; t < B; ++t) {
+      const double gt = gq[t * F + f];
+      if (bn_training) {
+        const double xhat = (acc[t * F + f] - mu[f]) / sd[f];
+        gacc[t * F + f] = (double)gamma[f] / sd[f] *
+                          (gt - sb / (double)B - xhat * sg / (double)B);
+      } else {
+        gacc[t * F + f] = gt * (double)gamma[f] / sd[f];
       }
     }
   }
-  free(q); free(acc); free(gq); free(gw); free(gc);
+  /* Through the linear map. */
+  if (grad_W) {
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static)
+#endif
+    for (int f = 0; f < F; ++f)
+      for (int c = 0; c < d; ++c) {
+        double a = 0.0;
+        for (int64_t t = 0; t < B; ++t)
+          a += gacc[t * F + f] * widen(x, dtype, t * (int64_t)d + c);
+        grad_W[(int64_t)f * d + c] = a;
+      }
+  }
+  if (grad_x) {
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static)
+#endif
+    for (int64_t t = 0; t < B; ++t)
+      for (int c = 0; c < d; ++c) {
+        double a = 0.0;
+        for (int f = 0; f < F; ++f) a += gacc[t * F + f] * widen(Wq, dtype, (int64_t)f * d + c);
+        grad_x[t * (int64_t)d + c] = a;
+      }
+  }
+  free(acc); free(gq); free(gacc); free(mu); free(sd); free(q); free(gw); free(gc);
   return 0;
 }

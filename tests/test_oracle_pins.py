@@ -404,3 +404,103 @@ def test_backward_full_value_and_score_parts_match_backward():
                 s_half = C[hh, side][sub] @ q[t, hh, side]
                 np.testing.assert_allclose((gq[t, hh, side] * q[t, hh, side]).sum(),
                                            (gs[t, hh] * s_half).sum(), rtol=1e-10, atol=1e-12)
+
+
+# ------------------------------------------------------- BatchNorm training-mode pins
+
+
+def _train_layer(seed=51, **kw):
+    shape = dict(B=7, H=2, dq=8, d_model=10, n=6, k=3, v=8, bn_random=True)
+    shape.update(kw)
+    w = synth.WORKLOADS["tiny"].with_(**shape)
+    L = synth.make_layer(w, seed=seed)
+    L["bn_gamma"] = torch.rand(w.H * w.dq, generator=torch.Generator().manual_seed(seed + 1)) + 0.5
+    L["bn_beta"] = torch.randn(w.H * w.dq, generator=torch.Generator().manual_seed(seed + 2))
+    return w, L
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_forward_train_batchnorm_matches_torch(dtype):
+    """q, the batch statistics and the running-statistics update against
+    torch.nn.functional.batch_norm(training=True) on a library fp64 matmul."""
+    w, L = _train_layer(B=13, d_model=24)
+    for key in ("x", "W_q", "subkeys", "values"):
+        L[key] = L[key].to(dtype)
+    mom = 0.3
+    r = oracle.forward_train(L, w.H, w.dq, w.n, w.k, eps=1e-5, momentum=mom, want_q=True)
+    acc = L["x"].double() @ L["W_q"].double().T
+    rm, rv = L["bn_mean"].double().clone(), L["bn_var"].double().clone()
+    q = torch.nn.functional.batch_norm(acc, rm, rv, L["bn_gamma"].double(), L["bn_beta"].double(),
+                                       training=True, momentum=mom, eps=1e-5)
+    np.testing.assert_allclose(r["q"], q.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(r["batch_mean"], acc.mean(0).numpy(), rtol=1e-10, atol=1e-13)
+    np.testing.assert_allclose(r["batch_var"], acc.var(0, unbiased=False).numpy(), rtol=1e-10)
+    np.testing.assert_allclose(r["running_mean"], rm.numpy(), rtol=1e-10, atol=1e-13)
+    np.testing.assert_allclose(r["running_var"], rv.numpy(), rtol=1e-10)
+
+
+def test_forward_train_search_is_the_flat_top_k_of_its_query():
+    """Steps 2-7 on the training-mode query: the picks are the brute-force top-k over
+    all n^2 explicit keys of that query."""
+    w, L = _train_layer(B=11, n=7, k=4)
+    r = oracle.forward_train(L, w.H, w.dq, w.n, w.k, want_q=True)
+    idx, sc = oracle.flat_topk(r["q"], L["subkeys"], w.H, w.dq, w.n, w.k)
+    np.testing.assert_array_equal(r["indices"], idx)
+    np.testing.assert_allclose(r["scores"], sc, rtol=1e-12, atol=1e-12)
+
+
+def test_forward_train_rejects_one_token():
+    w, L = _train_layer(B=1)
+    with pytest.raises(ValueError):
+        oracle.forward_train(L, w.H, w.dq, w.n, w.k)
+
+
+@pytest.mark.parametrize("param", ["x", "W_q", "bn_gamma", "bn_beta", "subkeys"])
+def test_backward_full_training_bn_matches_finite_differences(param):
+    """dL/dparam with training-mode BatchNorm: every perturbation moves the batch
+    statistics too, so x and W_q see the mean and variance terms; picks held fixed."""
+    w, L = _train_layer(seed=61)
+    g = torch.randn(w.B, w.v, generator=torch.Generator().manual_seed(7))
+    G = g.double().numpy()
+    r = oracle.forward_train(L, w.H, w.dq, w.n, w.k)
+    grads = oracle.backward_full(L, r["indices"], r["weights"], g, w.H, w.dq, w.n, w.k,
+                                 bn_training=True)
+    key = {"x": "x", "W_q": "W_q", "bn_gamma": "gamma", "bn_beta": "beta",
+           "subkeys": "subkeys"}[param]
+    base = L[param].clone()
+    flat = base.view(-1)
+    fd = np.full(flat.numel(), np.nan)
+    h = 2e-4
+    for i in range(flat.numel()):
+        up, dn = flat.clone(), flat.clone()
+        up[i] = flat[i] + h
+        dn[i] = flat[i] - h
+        du = float(up[i].double() - flat[i].double())
+        dd = float(flat[i].double() - dn[i].double())
+        L[param] = up.view_as(base)
+        ru = oracle.forward_train(L, w.H, w.dq, w.n, w.k)
+        L[param] = dn.view_as(base)
+        rd = oracle.forward_train(L, w.H, w.dq, w.n, w.k)
+        L[param] = base
+        if np.array_equal(ru["indices"], r["indices"]) and np.array_equal(rd["indices"], r["indices"]):
+            fd[i] = ((ru["out"] * G).sum() - (rd["out"] * G).sum()) / (du + dd)
+    ok = ~np.isnan(fd)
+    assert (~ok).sum() <= max(2, 0.1 * flat.numel())
+    np.testing.assert_allclose(grads[key].reshape(-1)[ok], fd[ok], rtol=2e-5, atol=1e-7)
+
+
+def test_training_bn_gradient_sums_vanish_through_the_mean():
+    """With batch statistics, shifting acc[:, f] by one constant for every token leaves
+    q unchanged, so sum_t dL/dacc[t, f] = 0 for every feature. With a constant input
+    column x[:, 0] = 1 that sum is dL/dW_q[f][0], which must vanish (it does not in
+    inference mode, where the mean is a constant)."""
+    w, L = _train_layer(seed=71, d_model=10)
+    L["x"][:, 0] = 1.0
+    g = torch.randn(w.B, w.v, generator=torch.Generator().manual_seed(9))
+    r = oracle.forward_train(L, w.H, w.dq, w.n, w.k)
+    grads = oracle.backward_full(L, r["indices"], r["weights"], g, w.H, w.dq, w.n, w.k,
+                                 bn_training=True)
+    scale = np.abs(grads["W_q"]).max()
+    np.testing.assert_allclose(grads["W_q"][:, 0], 0.0, atol=1e-12 * max(1.0, scale))
+    inf = oracle.backward_full(L, r["indices"], r["weights"], g, w.H, w.dq, w.n, w.k)
+    assert np.abs(inf["W_q"][:, 0]).max() > 1e-6 * scale
