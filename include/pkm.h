@@ -73,8 +73,9 @@ typedef struct {
 
 /*
  * Bytes of workspace pkm_forward (for_backward = 0), pkm_backward_values
- * (for_backward = 1), pkm_slot_usage (for_backward = 2) or pkm_backward
- * (for_backward = 3) needs for this shape; 0 if the shape is invalid.
+ * (for_backward = 1), pkm_slot_usage (for_backward = 2), pkm_backward or
+ * pkm_backward_train (for_backward = 3) or pkm_forward_train (for_backward = 4) needs
+ * for this shape; 0 if the shape is invalid.
  */
 size_t pkm_workspace_size(const pkm_shape* s, int for_backward);
 
@@ -162,6 +163,48 @@ int pkm_backward(const pkm_shape* s, const void* x, const void* W_q, const float
                  float* grad_bn_gamma, float* grad_bn_beta, float* grad_subkeys,
                  float* grad_values, float* grad_scores, void* workspace, size_t workspace_bytes,
                  void* stream);
+
+/*
+ * Forward with BatchNorm in training mode ("Large Memory Layers with Product Keys",
+ * Methodology: batch normalization in the query network; while the model trains, the
+ * batch's own statistics normalise it, after Ioffe and Szegedy 2015):
+ *   acc = x W_q^T,  mean_B = (1/B) sum_t acc[t],  var_B = (1/B) sum_t (acc[t] - mean_B)^2
+ *   q = (acc - mean_B) / sqrt(var_B + eps) * gamma + beta, then as pkm_forward.
+ * The running statistics move towards the batch's (PyTorch's convention):
+ *   bn_running_mean <- (1 - momentum) bn_running_mean + momentum mean_B
+ *   bn_running_var  <- (1 - momentum) bn_running_var  + momentum var_B B / (B - 1)
+ * Arguments as pkm_forward, with bn_running_mean / bn_running_var [H*dq] fp32 updated
+ * in place, momentum in [0, 1], and batch_mean / batch_var [H*dq] fp32 written: the
+ * statistics that normalised the batch (biased variance), which pkm_backward_train
+ * takes. B = 1 is rejected (PKM_ERR_INVALID_ARG: one token has no variance); B = 0
+ * launches nothing and leaves every array as it was. Statistics are summed in fp64 in
+ * chunks of 128 tokens and merged in chunk order (deterministic).
+ * workspace: at least pkm_workspace_size(s, 4) bytes, 256-byte aligned.
+ */
+int pkm_forward_train(const pkm_shape* s, const void* x, const void* W_q,
+                      float* bn_running_mean, float* bn_running_var, const float* bn_gamma,
+                      const float* bn_beta, float momentum, const void* subkeys,
+                      const void* values, float* out, int32_t* indices, float* weights,
+                      float* scores, float* batch_mean, float* batch_var, void* workspace,
+                      size_t workspace_bytes, void* stream);
+
+/*
+ * pkm_backward for a forward run by pkm_forward_train: batch_mean / batch_var are the
+ * statistics it wrote, and the gradient also flows through them (the backward of
+ * batch normalisation):
+ *   dL/dacc = gamma / sqrt(var_B + eps) (dL/dq - (1/B) sum_t dL/dq
+ *                                        - xhat (1/B) sum_t dL/dq xhat),
+ *   xhat = (acc - mean_B) / sqrt(var_B + eps).
+ * dL/dgamma, dL/dbeta and everything else as in pkm_backward. B = 1 is rejected.
+ * workspace: at least pkm_workspace_size(s, 3) bytes, 256-byte aligned.
+ */
+int pkm_backward_train(const pkm_shape* s, const void* x, const void* W_q,
+                       const float* batch_mean, const float* batch_var, const float* bn_gamma,
+                       const float* bn_beta, const void* subkeys, const void* values,
+                       const int32_t* indices, const float* weights, const void* grad_out,
+                       float* grad_x, float* grad_W_q, float* grad_bn_gamma, float* grad_bn_beta,
+                       float* grad_subkeys, float* grad_values, float* grad_scores,
+                       void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * pkm_backward_values without a workspace. The pages have no counterpart: this is

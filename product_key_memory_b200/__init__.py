@@ -25,7 +25,8 @@ _STATUS = {0: "PKM_OK", -1: "PKM_ERR_INVALID_ARG", -2: "PKM_ERR_UNSUPPORTED",
 
 EXPORTED = ("pkm_workspace_size", "pkm_forward", "pkm_backward_values", "pkm_device_status",
             "pkm_trace_enable", "pkm_trace_read", "pkm_status_string",
-            "pkm_backward_values_noalloc", "pkm_slot_usage", "pkm_backward")
+            "pkm_backward_values_noalloc", "pkm_slot_usage", "pkm_backward",
+            "pkm_forward_train", "pkm_backward_train")
 
 
 class PKMError(RuntimeError):
@@ -61,6 +62,11 @@ def lib() -> ctypes.CDLL:
         L.pkm_backward_values.restype = ctypes.c_int
         L.pkm_backward.argtypes = [S] + [P] * 19 + [ctypes.c_size_t, P]
         L.pkm_backward.restype = ctypes.c_int
+        L.pkm_backward_train.argtypes = [S] + [P] * 19 + [ctypes.c_size_t, P]
+        L.pkm_backward_train.restype = ctypes.c_int
+        L.pkm_forward_train.argtypes = [S] + [P] * 6 + [ctypes.c_float] + [P] * 9 + [
+            ctypes.c_size_t, P]
+        L.pkm_forward_train.restype = ctypes.c_int
         L.pkm_backward_values_noalloc.argtypes = [S] + [P] * 6 + [P]
         L.pkm_backward_values_noalloc.restype = ctypes.c_int
         L.pkm_slot_usage.argtypes = [S, P, P, P, ctypes.c_size_t, P]
@@ -179,17 +185,53 @@ def pkm_backward_values(values: torch.Tensor, indices: torch.Tensor, weights: to
     return grad_values, grad_scores
 
 
+def pkm_forward_train(x: torch.Tensor, W_q: torch.Tensor, bn_running_mean: torch.Tensor,
+                      bn_running_var: torch.Tensor, bn_gamma: torch.Tensor,
+                      bn_beta: torch.Tensor, subkeys: torch.Tensor, values: torch.Tensor, k: int,
+                      momentum: float = 0.1, bn_eps: float = 1e-5,
+                      workspace: Optional[torch.Tensor] = None, stream=None):
+    """Forward with BatchNorm in training mode. Updates bn_running_mean/var in place;
+    returns (out, indices, weights, scores, batch_mean, batch_var)."""
+    B, d = x.shape
+    H, _, n, half = subkeys.shape
+    v = values.shape[1]
+    F = H * 2 * half
+    shape = make_shape(B, d, H, 2 * half, n, k, v, x.dtype, bn_eps)
+    dev = x.device
+    if workspace is None:
+        nb = int(lib().pkm_workspace_size(ctypes.byref(shape), 4))
+        if nb == 0:
+            raise PKMError("pkm_workspace_size", -1)
+        workspace = torch.empty(nb, dtype=torch.uint8, device=dev)
+    out = torch.empty(B, v, dtype=torch.float32, device=dev)
+    idx = torch.empty(B, H, k, dtype=torch.int32, device=dev)
+    wts = torch.empty(B, H, k, dtype=torch.float32, device=dev)
+    scs = torch.empty(B, H, k, dtype=torch.float32, device=dev)
+    bm = torch.empty(F, dtype=torch.float32, device=dev)
+    bv = torch.empty(F, dtype=torch.float32, device=dev)
+    rc = lib().pkm_forward_train(ctypes.byref(shape), _ptr(x), _ptr(W_q), _ptr(bn_running_mean),
+                                 _ptr(bn_running_var), _ptr(bn_gamma), _ptr(bn_beta),
+                                 ctypes.c_float(momentum), _ptr(subkeys), _ptr(values), _ptr(out),
+                                 _ptr(idx), _ptr(wts), _ptr(scs), _ptr(bm), _ptr(bv),
+                                 _ptr(workspace), workspace.numel(), _stream(stream))
+    if rc != PKM_OK:
+        raise PKMError("pkm_forward_train", rc)
+    return out, idx, wts, scs, bm, bv
+
+
 def pkm_backward(x: torch.Tensor, W_q: torch.Tensor, bn_mean: torch.Tensor,
                  bn_var: torch.Tensor, bn_gamma: torch.Tensor, bn_beta: torch.Tensor,
                  subkeys: torch.Tensor, values: torch.Tensor, indices: torch.Tensor,
                  weights: torch.Tensor, grad_out: torch.Tensor, grads: dict,
-                 bn_eps: float = 1e-5, workspace: Optional[torch.Tensor] = None, stream=None):
+                 bn_eps: float = 1e-5, workspace: Optional[torch.Tensor] = None, stream=None,
+                 bn_training: bool = False):
     """Full backward of the layer with the forward's picks held fixed.
 
     ``grads`` maps any of x [B][d], W_q [H*dq][d], bn_gamma, bn_beta [H*dq],
     subkeys [H][2][n][dq/2], values [n*n][v], scores [B][H][k] to fp32 device
     tensors; missing entries are not computed. values is accumulated into, the
-    others are overwritten."""
+    others are overwritten. With bn_training, bn_mean / bn_var are the batch
+    statistics pkm_forward_train returned (pkm_backward_train)."""
     B, d = x.shape
     H, _, n, half = subkeys.shape
     k = indices.shape[2]
@@ -201,15 +243,15 @@ def pkm_backward(x: torch.Tensor, W_q: torch.Tensor, bn_mean: torch.Tensor,
             raise PKMError("pkm_workspace_size", -1)
         workspace = torch.empty(nb, dtype=torch.uint8, device=x.device)
     g = grads
-    rc = lib().pkm_backward(ctypes.byref(shape), _ptr(x), _ptr(W_q), _ptr(bn_mean),
-                            _ptr(bn_var), _ptr(bn_gamma), _ptr(bn_beta), _ptr(subkeys),
-                            _ptr(values), _ptr(indices), _ptr(weights), _ptr(grad_out),
-                            _ptr(g.get("x")), _ptr(g.get("W_q")), _ptr(g.get("bn_gamma")),
-                            _ptr(g.get("bn_beta")), _ptr(g.get("subkeys")), _ptr(g.get("values")),
-                            _ptr(g.get("scores")), _ptr(workspace), workspace.numel(),
-                            _stream(stream))
+    fn = lib().pkm_backward_train if bn_training else lib().pkm_backward
+    rc = fn(ctypes.byref(shape), _ptr(x), _ptr(W_q), _ptr(bn_mean), _ptr(bn_var),
+            _ptr(bn_gamma), _ptr(bn_beta), _ptr(subkeys), _ptr(values), _ptr(indices),
+            _ptr(weights), _ptr(grad_out), _ptr(g.get("x")), _ptr(g.get("W_q")),
+            _ptr(g.get("bn_gamma")), _ptr(g.get("bn_beta")), _ptr(g.get("subkeys")),
+            _ptr(g.get("values")), _ptr(g.get("scores")), _ptr(workspace), workspace.numel(),
+            _stream(stream))
     if rc != PKM_OK:
-        raise PKMError("pkm_backward", rc)
+        raise PKMError("pkm_backward_train" if bn_training else "pkm_backward", rc)
     return grads
 
 

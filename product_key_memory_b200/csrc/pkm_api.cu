@@ -106,6 +106,27 @@ size_t forward_ws(const pkm_shape* s, ForwardWs* w, char* base) {
   return off;
 }
 
+// BatchNorm training mode: acc of the whole batch (three bf16 planes on the tensor
+// path, fp32 otherwise) and the per-chunk statistics, after the forward's workspace.
+struct TrainWs {
+  void* acc;
+  double* part;
+};
+
+size_t forward_train_ws(const pkm_shape* s, ForwardWs* fw, TrainWs* tw, char* base) {
+  const int64_t F = static_cast<int64_t>(s->H) * s->dq;
+  const size_t accb = static_cast<size_t>(s->B) * F * (choose_path(s) == Path::kTensor ? 6 : 4);
+  const int64_t chunks = (s->B + pkm::kStatChunk - 1) / pkm::kStatChunk;
+  size_t off = forward_ws(s, fw, base);
+  const size_t o_acc = off;  off += align256(accb);
+  const size_t o_part = off; off += align256(sizeof(double) * 2 * F * (chunks > 0 ? chunks : 1));
+  if (tw && base) {
+    tw->acc = base + o_acc;
+    tw->part = reinterpret_cast<double*>(base + o_part);
+  }
+  return off;
+}
+
 size_t backward_ws(const pkm_shape* s, pkm::BackwardWs* w, char* base) {
   return pkm::backward_ws_bytes(s->B, s->H, s->k, static_cast<int64_t>(s->n) * s->n, w, base);
 }
@@ -264,6 +285,10 @@ int pkm_trace_read(int pass, double* stage_ms, int max_stages, int64_t* calls,
 }
 
 size_t pkm_workspace_size(const pkm_shape* s, int for_backward) {
+  if (for_backward == 4) {
+    if (validate_shape(s) != PKM_OK || s->B < 2) return 0;
+    return forward_train_ws(s, nullptr, nullptr, nullptr);
+  }
   if (for_backward == 3) {
     if (validate_shape(s) != PKM_OK) return 0;
     LayerArgs a{};
@@ -278,15 +303,20 @@ size_t pkm_workspace_size(const pkm_shape* s, int for_backward) {
   return for_backward ? backward_ws(s, nullptr, nullptr) : forward_ws(s, nullptr, nullptr);
 }
 
-int pkm_backward(const pkm_shape* s, const void* x, const void* W_q, const float* bn_mean,
-                 const float* bn_var, const float* bn_gamma, const float* bn_beta,
-                 const void* subkeys, const void* values, const int32_t* indices,
-                 const float* weights, const void* grad_out, float* grad_x, float* grad_W_q,
-                 float* grad_bn_gamma, float* grad_bn_beta, float* grad_subkeys,
-                 float* grad_values, float* grad_scores, void* workspace, size_t workspace_bytes,
-                 void* stream) {
+}  // extern "C"
+
+namespace {
+
+int backward_full_impl(const pkm_shape* s, bool bn_training, const void* x, const void* W_q,
+                       const float* bn_mean, const float* bn_var, const float* bn_gamma,
+                       const float* bn_beta, const void* subkeys, const void* values,
+                       const int32_t* indices, const float* weights, const void* grad_out,
+                       float* grad_x, float* grad_W_q, float* grad_bn_gamma, float* grad_bn_beta,
+                       float* grad_subkeys, float* grad_values, float* grad_scores,
+                       void* workspace, size_t workspace_bytes, void* stream) {
   int rc = validate_shape(s);
   if (rc != PKM_OK) return rc;
+  if (bn_training && s->B == 1) return PKM_ERR_INVALID_ARG;
   const bool tok = s->B > 0;
   if (!W_q || !bn_mean || !bn_var || !bn_gamma || !bn_beta || !subkeys || !values ||
       (tok && (!x || !indices || !weights || !grad_out)))
@@ -321,13 +351,43 @@ int pkm_backward(const pkm_shape* s, const void* x, const void* W_q, const float
   Tracer tr(1);
   tr.begin(3, st);
   int launches = 0;
-  const cudaError_t e = pkm::launch_backward_full(a, tensor, indices, weights, grad_out, grad_x,
-                                                  grad_W_q, grad_bn_gamma, grad_bn_beta,
-                                                  grad_subkeys, grad_values, grad_scores, w, st,
-                                                  &launches);
+  const cudaError_t e = pkm::launch_backward_full(a, tensor, bn_training, indices, weights,
+                                                  grad_out, grad_x, grad_W_q, grad_bn_gamma,
+                                                  grad_bn_beta, grad_subkeys, grad_values,
+                                                  grad_scores, w, st, &launches);
   tr.end(st);
   tr.finish(e == cudaSuccess, launches);
   return e == cudaSuccess ? PKM_OK : PKM_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int pkm_backward(const pkm_shape* s, const void* x, const void* W_q, const float* bn_mean,
+                 const float* bn_var, const float* bn_gamma, const float* bn_beta,
+                 const void* subkeys, const void* values, const int32_t* indices,
+                 const float* weights, const void* grad_out, float* grad_x, float* grad_W_q,
+                 float* grad_bn_gamma, float* grad_bn_beta, float* grad_subkeys,
+                 float* grad_values, float* grad_scores, void* workspace, size_t workspace_bytes,
+                 void* stream) {
+  return backward_full_impl(s, false, x, W_q, bn_mean, bn_var, bn_gamma, bn_beta, subkeys,
+                            values, indices, weights, grad_out, grad_x, grad_W_q, grad_bn_gamma,
+                            grad_bn_beta, grad_subkeys, grad_values, grad_scores, workspace,
+                            workspace_bytes, stream);
+}
+
+int pkm_backward_train(const pkm_shape* s, const void* x, const void* W_q,
+                       const float* batch_mean, const float* batch_var, const float* bn_gamma,
+                       const float* bn_beta, const void* subkeys, const void* values,
+                       const int32_t* indices, const float* weights, const void* grad_out,
+                       float* grad_x, float* grad_W_q, float* grad_bn_gamma, float* grad_bn_beta,
+                       float* grad_subkeys, float* grad_values, float* grad_scores,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  return backward_full_impl(s, true, x, W_q, batch_mean, batch_var, bn_gamma, bn_beta, subkeys,
+                            values, indices, weights, grad_out, grad_x, grad_W_q, grad_bn_gamma,
+                            grad_bn_beta, grad_subkeys, grad_values, grad_scores, workspace,
+                            workspace_bytes, stream);
 }
 
 int pkm_slot_usage(const pkm_shape* s, const int32_t* indices, unsigned long long* hits,
@@ -354,14 +414,19 @@ int pkm_slot_usage(const pkm_shape* s, const int32_t* indices, unsigned long lon
   return e == cudaSuccess ? PKM_OK : PKM_ERR_CUDA;
 }
 
-int pkm_forward(const pkm_shape* s, const void* x, const void* W_q, const float* bn_mean,
-                const float* bn_var, const float* bn_gamma, const float* bn_beta,
-                const void* subkeys, const void* values, float* out, int32_t* indices,
-                float* weights, float* scores, void* workspace, size_t workspace_bytes,
-                void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Checks shared by pkm_forward and pkm_forward_train (per-token tensors may be NULL
+// when there are no tokens).
+int validate_forward_args(const pkm_shape* s, const void* x, const void* W_q,
+                          const float* bn_mean, const float* bn_var, const float* bn_gamma,
+                          const float* bn_beta, const void* subkeys, const void* values,
+                          const float* out, const int32_t* indices, const float* weights,
+                          const float* scores) {
   int rc = validate_shape(s);
   if (rc != PKM_OK) return rc;
-  // Per-token tensors may be NULL when there are no tokens.
   const bool tok = s->B > 0;
   if (!W_q || !bn_mean || !bn_var || !bn_gamma || !bn_beta || !subkeys || !values ||
       (tok && (!x || !out || !indices || !weights)))
@@ -370,24 +435,18 @@ int pkm_forward(const pkm_shape* s, const void* x, const void* W_q, const float*
                         indices, weights, scores};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return PKM_ERR_UNSUPPORTED;
-  const size_t need = forward_ws(s, nullptr, nullptr);
-  if (!workspace || workspace_bytes < need ||
-      (reinterpret_cast<uintptr_t>(workspace) & 255u))
-    return PKM_ERR_WORKSPACE;
-  if (s->B == 0) return PKM_OK;
+  return PKM_OK;
+}
 
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  ForwardWs w;
-  forward_ws(s, &w, static_cast<char*>(workspace));
-  LayerArgs a{s->B, s->d_model, s->H, s->dq, s->n, s->k, s->v, s->dtype, s->bn_eps,
-              x, W_q, bn_mean, bn_var, bn_gamma, bn_beta, subkeys, values, w.status, 0};
-  if (cudaMemsetAsync(w.status, 0, sizeof(int), st) != cudaSuccess) return PKM_ERR_CUDA;
-  // Stages: 0 query network, 1 per-half scores + best 32, 2 candidate top-k + softmax +
-  // gather, 3 the whole call.
-  Tracer tr(0);
+// The forward's launches for a validated call with B > 0 (status word already cleared).
+// Stages: 0 query network, 1 per-half scores + best 32, 2 candidate top-k + softmax +
+// gather; the caller brackets stage 3 (the whole call).
+cudaError_t run_forward(const pkm_shape* s, const LayerArgs& a, const ForwardWs& w, float* out,
+                        int32_t* indices, float* weights, float* scores, cudaStream_t st,
+                        Tracer& tr, int* nlaunch) {
+  const void* x = a.x;
   cudaError_t e = cudaSuccess;
   int launches = 0;
-  tr.begin(3, st);
   if (choose_path(s) == Path::kSimt) {
     tr.begin(0, st);
     e = pkm::launch_query_bn_simt(a, w.q, st);
@@ -410,7 +469,7 @@ int pkm_forward(const pkm_shape* s, const void* x, const void* W_q, const float*
     const int nsub = static_cast<int>((s->B + sub - 1) / sub);
     cudaStream_t aux;
     cudaEvent_t ev[5];
-    if (aux_resources(nsub + 1, &aux, ev) != PKM_OK) return PKM_ERR_CUDA;
+    if (aux_resources(nsub + 1, &aux, ev) != PKM_OK) return cudaErrorUnknown;
     const size_t xsz = s->dtype == PKM_F32 ? 4 : 2;
     const int64_t per_tok = static_cast<int64_t>(s->H) * 2 * pkm::kMaxK;
     for (int i = 0; i < nsub && e == cudaSuccess; ++i) {
@@ -443,6 +502,91 @@ int pkm_forward(const pkm_shape* s, const void* x, const void* W_q, const float*
     if (e2 == cudaSuccess) e2 = cudaStreamWaitEvent(st, ev[nsub], 0);
     if (e == cudaSuccess) e = e2;
   }
+  *nlaunch += launches;
+  return e;
+}
+
+}  // namespace
+
+extern "C" {
+
+int pkm_forward(const pkm_shape* s, const void* x, const void* W_q, const float* bn_mean,
+                const float* bn_var, const float* bn_gamma, const float* bn_beta,
+                const void* subkeys, const void* values, float* out, int32_t* indices,
+                float* weights, float* scores, void* workspace, size_t workspace_bytes,
+                void* stream) {
+  int rc = validate_forward_args(s, x, W_q, bn_mean, bn_var, bn_gamma, bn_beta, subkeys, values,
+                                 out, indices, weights, scores);
+  if (rc != PKM_OK) return rc;
+  const size_t need = forward_ws(s, nullptr, nullptr);
+  if (!workspace || workspace_bytes < need ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return PKM_ERR_WORKSPACE;
+  if (s->B == 0) return PKM_OK;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ForwardWs w;
+  forward_ws(s, &w, static_cast<char*>(workspace));
+  LayerArgs a{s->B, s->d_model, s->H, s->dq, s->n, s->k, s->v, s->dtype, s->bn_eps,
+              x, W_q, bn_mean, bn_var, bn_gamma, bn_beta, subkeys, values, w.status, 0};
+  if (cudaMemsetAsync(w.status, 0, sizeof(int), st) != cudaSuccess) return PKM_ERR_CUDA;
+  Tracer tr(0);
+  int launches = 0;
+  tr.begin(3, st);
+  const cudaError_t e = run_forward(s, a, w, out, indices, weights, scores, st, tr, &launches);
+  tr.end(st);
+  tr.finish(e == cudaSuccess, launches);
+  return e == cudaSuccess ? PKM_OK : PKM_ERR_CUDA;
+}
+
+int pkm_forward_train(const pkm_shape* s, const void* x, const void* W_q,
+                      float* bn_running_mean, float* bn_running_var, const float* bn_gamma,
+                      const float* bn_beta, float momentum, const void* subkeys,
+                      const void* values, float* out, int32_t* indices, float* weights,
+                      float* scores, float* batch_mean, float* batch_var, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  int rc = validate_forward_args(s, x, W_q, bn_running_mean, bn_running_var, bn_gamma, bn_beta,
+                                 subkeys, values, out, indices, weights, scores);
+  if (rc != PKM_OK) return rc;
+  if (s->B == 1 || !batch_mean || !batch_var || !(momentum >= 0.f && momentum <= 1.f))
+    return PKM_ERR_INVALID_ARG;
+  if (!aligned16(batch_mean) || !aligned16(batch_var)) return PKM_ERR_UNSUPPORTED;
+  const size_t need = forward_train_ws(s, nullptr, nullptr, nullptr);
+  if (!workspace || workspace_bytes < need ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return PKM_ERR_WORKSPACE;
+  if (s->B == 0) return PKM_OK;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ForwardWs w;
+  TrainWs tw;
+  forward_train_ws(s, &w, &tw, static_cast<char*>(workspace));
+  const int F = s->H * s->dq;
+  // acc = x W_q^T without BatchNorm, its batch statistics (and the running-statistics
+  // update), then the forward normalised by the batch statistics.
+  LayerArgs raw{s->B, s->d_model, s->H, s->dq, s->n, s->k, s->v, s->dtype, s->bn_eps,
+                x, W_q, bn_running_mean, bn_running_var, bn_gamma, bn_beta, subkeys, values,
+                w.status, 1};
+  LayerArgs a = raw;
+  a.bn_mean = batch_mean;
+  a.bn_var = batch_var;
+  a.raw_acc = 0;
+  if (cudaMemsetAsync(w.status, 0, sizeof(int), st) != cudaSuccess) return PKM_ERR_CUDA;
+  Tracer tr(0);
+  int launches = 0;
+  tr.begin(3, st);
+  tr.begin(0, st);
+  const bool tensor = choose_path(s) == Path::kTensor;
+  cudaError_t e = tensor ? pkm::launch_query_tc(raw, tw.acc, st)
+                         : pkm::launch_query_bn_simt(raw, static_cast<float*>(tw.acc), st);
+  if (e == cudaSuccess)
+    e = pkm::launch_bn_batch_stats(tensor ? static_cast<const uint16_t*>(tw.acc) : nullptr,
+                                   tensor ? nullptr : static_cast<const float*>(tw.acc), s->B, F,
+                                   momentum, tw.part, batch_mean, batch_var, bn_running_mean,
+                                   bn_running_var, st);
+  tr.end(st);
+  launches += 3;
+  if (e == cudaSuccess) e = run_forward(s, a, w, out, indices, weights, scores, st, tr, &launches);
   tr.end(st);
   tr.finish(e == cudaSuccess, launches);
   return e == cudaSuccess ? PKM_OK : PKM_ERR_CUDA;

@@ -18,14 +18,54 @@
 
 namespace pkm {
 
-// acc = x W_q^T and q = (acc - mean) * s + beta. With planes, acc = hi + mid + lo from
-// the three bf16 planes of the tensor-core query kernel; without, acc is read as is.
-__global__ void acc_q_kernel(const uint16_t* __restrict__ planes, float* __restrict__ acc,
-                             float* __restrict__ q, const float* __restrict__ mean,
-                             const float* __restrict__ var, const float* __restrict__ gamma,
-                             const float* __restrict__ beta, float eps, int64_t count, int F) {
+// acc = x W_q^T and q = acc * s + (beta - mean * s), s = gamma / sqrt(var + eps) (the
+// forward's query epilogue). With planes, acc = hi + mid + lo from the three bf16 planes
+// of the tensor-core query kernel; without, acc is read as is. Eight features per
+// thread when F allows it.
+__global__ void __launch_bounds__(256) acc_q_kernel(
+    const uint16_t* __restrict__ planes, float* __restrict__ acc, float* __restrict__ q,
+    const float* __restrict__ mean, const float* __restrict__ var,
+    const float* __restrict__ gamma, const float* __restrict__ beta, float eps, int B, int F) {
+  const int64_t count = static_cast<int64_t>(B) * F;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  if ((F & 7) == 0) {
+    const int per_row = F >> 3;
+    const int64_t units = static_cast<int64_t>(B) * per_row;
+    for (int64_t u = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; u < units;
+         u += stride) {
+      const int row = static_cast<int>(u / per_row);
+      const int f0 = static_cast<int>(u - static_cast<int64_t>(row) * per_row) * 8;
+      const int64_t i0 = static_cast<int64_t>(row) * F + f0;
+      float a[8];
+      if (planes) {
+        float h[8], m[8], l[8];
+        Vec<uint16_t>::widen(*reinterpret_cast<const uint4*>(planes + i0), h);
+        Vec<uint16_t>::widen(*reinterpret_cast<const uint4*>(planes + count + i0), m);
+        Vec<uint16_t>::widen(*reinterpret_cast<const uint4*>(planes + 2 * count + i0), l);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) a[j] = h[j] + m[j] + l[j];
+        reinterpret_cast<float4*>(acc + i0)[0] = make_float4(a[0], a[1], a[2], a[3]);
+        reinterpret_cast<float4*>(acc + i0)[1] = make_float4(a[4], a[5], a[6], a[7]);
+      } else {
+        const float4 x = reinterpret_cast<const float4*>(acc + i0)[0];
+        const float4 y = reinterpret_cast<const float4*>(acc + i0)[1];
+        a[0] = x.x; a[1] = x.y; a[2] = x.z; a[3] = x.w;
+        a[4] = y.x; a[5] = y.y; a[6] = y.z; a[7] = y.w;
+      }
+      float r[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int f = f0 + j;
+        const float sc = gamma[f] / sqrtf(var[f] + eps);
+        r[j] = fmaf(a[j], sc, beta[f] - mean[f] * sc);
+      }
+      reinterpret_cast<float4*>(q + i0)[0] = make_float4(r[0], r[1], r[2], r[3]);
+      reinterpret_cast<float4*>(q + i0)[1] = make_float4(r[4], r[5], r[6], r[7]);
+    }
+    return;
+  }
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < count;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+       i += stride) {
     float a;
     if (planes) {
       a = load_elem(planes, i) + load_elem(planes, count + i) + load_elem(planes, 2 * count + i);
@@ -34,7 +74,8 @@ __global__ void acc_q_kernel(const uint16_t* __restrict__ planes, float* __restr
       a = acc[i];
     }
     const int f = static_cast<int>(i % F);
-    q[i] = (a - mean[f]) * (gamma[f] / sqrtf(var[f] + eps)) + beta[f];
+    const float sc = gamma[f] / sqrtf(var[f] + eps);
+    q[i] = fmaf(a, sc, beta[f] - mean[f] * sc);
   }
 }
 
@@ -94,13 +135,11 @@ __global__ void __launch_bounds__(128) grad_q_targets_kernel(
   for (int side = 0; side < 2; ++side) {
     // Invalid lanes get distinct negative ids, so they match nobody.
     const int id = valid ? (side ? slot % n : slot / n) : -1 - lane;
-    float S = 0.f;
-    for (int src = 0; src < k; ++src) {
-      const float gs = __shfl_sync(0xffffffffu, g, src);
-      const int is = __shfl_sync(0xffffffffu, id, src);
-      if (is == id) S += gs;
-    }
     const unsigned peers = __match_any_sync(0xffffffffu, id);
+    // Every lane of a group runs the same iterations, so the group's mask names exactly
+    // the lanes that take part in each shuffle.
+    float S = 0.f;
+    for (unsigned m = peers; m; m &= m - 1) S += __shfl_sync(peers, g, __ffs(m) - 1);
     const bool leader = valid && (__ffs(peers) - 1 == lane);
     if (lane < k) {
       targets[2 * pick + side] = leader ? (h * 2 + side) * n + id : -1;
@@ -114,15 +153,23 @@ __global__ void __launch_bounds__(128) grad_q_targets_kernel(
       float acc[VW];
 #pragma unroll
       for (int i = 0; i < VW; ++i) acc[i] = 0.f;
-      for (unsigned m = lead; m; m &= m - 1) {
-        const int src = __ffs(m) - 1;
-        const float Sl = __shfl_sync(0xffffffffu, S, src);
-        const int il = __shfl_sync(0xffffffffu, id, src);
+      // Two distinct rows in flight per step.
+      for (unsigned m = lead; m;) {
+        const int s0 = __ffs(m) - 1;
+        m &= m - 1;
+        const int s1 = m ? __ffs(m) - 1 : s0;
+        const bool two = m != 0;
+        if (two) m &= m - 1;
+        const float S0 = __shfl_sync(0xffffffffu, S, s0);
+        const int i0 = __shfl_sync(0xffffffffu, id, s0);
+        const float S1 = two ? __shfl_sync(0xffffffffu, S, s1) : 0.f;
+        const int i1 = __shfl_sync(0xffffffffu, id, s1);
         if (e < half) {
-          float r[VW];
-          load_run<VW>(book + static_cast<int64_t>(il) * half + e, r);
+          float r0[VW], r1[VW];
+          load_run<VW>(book + static_cast<int64_t>(i0) * half + e, r0);
+          load_run<VW>(book + static_cast<int64_t>(i1) * half + e, r1);
 #pragma unroll
-          for (int i = 0; i < VW; ++i) acc[i] = fmaf(Sl, r[i], acc[i]);
+          for (int i = 0; i < VW; ++i) acc[i] = fmaf(S1, r1[i], fmaf(S0, r0[i], acc[i]));
         }
       }
       if (e < half) {
@@ -147,7 +194,7 @@ __global__ void __launch_bounds__(128) grad_q_targets_kernel(
 
 // Column sums over tokens, pass 1: block (feature group of 256, token chunk) writes its
 // partial dL/dbeta and dL/dgamma sums; pass 2 adds the chunks in a fixed order.
-constexpr int kBnChunks = 32;
+constexpr int kBnChunks = 128;
 
 __global__ void bn_grad_partial_kernel(const float* __restrict__ g_q, const float* __restrict__ acc,
                                        const float* __restrict__ mean,
@@ -159,6 +206,7 @@ __global__ void bn_grad_partial_kernel(const float* __restrict__ g_q, const floa
   const int64_t t0 = blockIdx.y * per, t1 = min(B, t0 + per);
   const float mu = mean[f], rs = 1.f / sqrtf(var[f] + eps);
   float sb = 0.f, sg = 0.f;
+#pragma unroll 4
   for (int64_t t = t0; t < t1; ++t) {
     const float g = g_q[t * F + f];
     sb += g;
@@ -169,7 +217,8 @@ __global__ void bn_grad_partial_kernel(const float* __restrict__ g_q, const floa
 }
 
 __global__ void bn_grad_final_kernel(const float* __restrict__ part, int F,
-                                     float* __restrict__ grad_gamma, float* __restrict__ grad_beta) {
+                                     float* __restrict__ grad_gamma, float* __restrict__ grad_beta,
+                                     float* __restrict__ sums) {
   const int f = blockIdx.x * blockDim.x + threadIdx.x;
   if (f >= F) return;
   float sb = 0.f, sg = 0.f;
@@ -179,6 +228,10 @@ __global__ void bn_grad_final_kernel(const float* __restrict__ part, int F,
   }
   if (grad_beta) grad_beta[f] = sb;
   if (grad_gamma) grad_gamma[f] = sg;
+  if (sums) {
+    sums[f] = sb;
+    sums[F + f] = sg;
+  }
 }
 
 // Sub-key gradient rows from the contributions grouped by target: one warp per window
@@ -341,6 +394,7 @@ size_t backward_full_ws_bytes(const LayerArgs& a, bool tensor_path, FullBackward
   const size_t o_part = off;    off += al256(sizeof(int) * (scan_blocks_of(tslots) + 1));
   const size_t o_ord = off;     off += al256(sizeof(int) * E2);
   const size_t o_bn = off;      off += al256(sizeof(float) * 2 * kBnChunks * F);
+  const size_t o_sums = off;    off += al256(sizeof(float) * 2 * F);
   if (w && base) {
     w->values = vws;
     w->g_s = reinterpret_cast<float*>(base + o_gs);
@@ -356,6 +410,7 @@ size_t backward_full_ws_bytes(const LayerArgs& a, bool tensor_path, FullBackward
     w->sub.partials = reinterpret_cast<int*>(base + o_part);
     w->sub.order = reinterpret_cast<int*>(base + o_ord);
     w->bn_part = reinterpret_cast<float*>(base + o_bn);
+    w->bn_sums = reinterpret_cast<float*>(base + o_sums);
   }
   return off;
 }
@@ -383,7 +438,8 @@ static void launch_segment_subkeys(const LayerArgs& a, int64_t E2, int64_t tslot
 }
 
 template <typename T>
-static cudaError_t launch_full_t(const LayerArgs& a, bool tensor_path, const int* indices,
+static cudaError_t launch_full_t(const LayerArgs& a, bool tensor_path, bool bn_training,
+                                 const int* indices,
                                  const float* weights, const void* grad_out, float* grad_x,
                                  float* grad_W, float* grad_gamma, float* grad_beta,
                                  float* grad_subkeys, float* grad_values, float* grad_scores,
@@ -412,9 +468,9 @@ static cudaError_t launch_full_t(const LayerArgs& a, bool tensor_path, const int
     e = launch_query_bn_simt(raw, w.acc, st);
   }
   if (e != cudaSuccess) return e;
-  acc_q_kernel<<<grid_of((a.B * F + 255) / 256, 148 * 8), 256, 0, st>>>(
+  acc_q_kernel<<<grid_of((a.B * F / 8 + 255) / 256, 148 * 8), 256, 0, st>>>(
       tensor_path ? static_cast<const uint16_t*>(w.planes) : nullptr, w.acc, w.q, a.bn_mean,
-      a.bn_var, a.bn_gamma, a.bn_beta, a.bn_eps, a.B * F, static_cast<int>(F));
+      a.bn_var, a.bn_gamma, a.bn_beta, a.bn_eps, static_cast<int>(a.B), static_cast<int>(F));
   *launches += 2;
   // 3. dL/dq, dL/dacc (bf16 hi/lo planes for the tensor-core GEMMs), merged sub-key
   //    contributions.
@@ -424,17 +480,27 @@ static cudaError_t launch_full_t(const LayerArgs& a, bool tensor_path, const int
   if (tc_gemm && !gemm_tc_supported(a.B, static_cast<int>(F), a.d_model))
     return cudaErrorNotSupported;
   uint16_t* g_planes = tc_gemm ? static_cast<uint16_t*>(w.planes) : nullptr;
-  if (vec) launch_sub_kernels<T, 8>(a, indices, g_planes, w, st);
-  else launch_sub_kernels<T, 1>(a, indices, g_planes, w, st);
+  // With batch statistics dL/dacc needs the column sums first; the kernel then
+  // writes dL/dq only.
+  FullBackwardWs wq = w;
+  if (bn_training) wq.g_acc = nullptr;
+  if (vec) launch_sub_kernels<T, 8>(a, indices, bn_training ? nullptr : g_planes, wq, st);
+  else launch_sub_kernels<T, 1>(a, indices, bn_training ? nullptr : g_planes, wq, st);
   *launches += 1;
-  // 4. BatchNorm affine gradients.
-  if (grad_gamma || grad_beta) {
+  // 4. BatchNorm: affine gradients (and, in training mode, dL/dacc).
+  if (grad_gamma || grad_beta || bn_training) {
     dim3 g1(static_cast<unsigned>((F + 255) / 256), kBnChunks);
     bn_grad_partial_kernel<<<g1, 256, 0, st>>>(w.g_q, w.acc, a.bn_mean, a.bn_var, a.bn_eps, a.B,
                                                static_cast<int>(F), w.bn_part);
     bn_grad_final_kernel<<<static_cast<unsigned>((F + 255) / 256), 256, 0, st>>>(
-        w.bn_part, static_cast<int>(F), grad_gamma, grad_beta);
+        w.bn_part, static_cast<int>(F), grad_gamma, grad_beta, bn_training ? w.bn_sums : nullptr);
     *launches += 2;
+  }
+  if (bn_training) {
+    e = launch_bn_train_dacc(w.g_q, w.acc, a.bn_mean, a.bn_var, a.bn_gamma, w.bn_sums, a.bn_eps,
+                             a.B, static_cast<int>(F), tc_gemm ? nullptr : w.g_acc, g_planes, st);
+    if (e != cudaSuccess) return e;
+    *launches += 1;
   }
   // 5. Sub-key gradients: group the merged contributions by row, sum in windows.
   if (grad_subkeys) {
@@ -480,16 +546,17 @@ static cudaError_t launch_full_t(const LayerArgs& a, bool tensor_path, const int
   return cudaGetLastError();
 }
 
-cudaError_t launch_backward_full(const LayerArgs& a, bool tensor_path, const int* indices,
+cudaError_t launch_backward_full(const LayerArgs& a, bool tensor_path, bool bn_training,
+                                 const int* indices,
                                  const float* weights, const void* grad_out, float* grad_x,
                                  float* grad_W, float* grad_gamma, float* grad_beta,
                                  float* grad_subkeys, float* grad_values, float* grad_scores,
                                  const FullBackwardWs& w, cudaStream_t st, int* launches) {
   if (a.dtype == 0)
-    return launch_full_t<float>(a, tensor_path, indices, weights, grad_out, grad_x, grad_W,
+    return launch_full_t<float>(a, tensor_path, bn_training, indices, weights, grad_out, grad_x, grad_W,
                                 grad_gamma, grad_beta, grad_subkeys, grad_values, grad_scores, w,
                                 st, launches);
-  return launch_full_t<uint16_t>(a, tensor_path, indices, weights, grad_out, grad_x, grad_W,
+  return launch_full_t<uint16_t>(a, tensor_path, bn_training, indices, weights, grad_out, grad_x, grad_W,
                                  grad_gamma, grad_beta, grad_subkeys, grad_values, grad_scores, w,
                                  st, launches);
 }

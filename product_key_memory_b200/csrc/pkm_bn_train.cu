@@ -1,0 +1,129 @@
+// pkm_bn_train.cu -- BatchNorm of the query network in training mode.
+//
+// "Large Memory Layers with Product Keys" (gptget.net summary, Methodology: the
+// query network has batch normalization). While the model trains, the batch's own
+// statistics normalise it (Ioffe and Szegedy 2015):
+//   mean_B = (1/B) sum_t acc[t],  var_B = (1/B) sum_t (acc[t] - mean_B)^2
+// and the running statistics move towards them with momentum m:
+//   running_mean <- (1 - m) running_mean + m mean_B
+//   running_var  <- (1 - m) running_var  + m var_B B / (B - 1)
+// In the backward the statistics depend on every token:
+//   dL/dacc = gamma / sqrt(var_B + eps) (g - (1/B) sum_t g - xhat (1/B) sum_t g xhat),
+//   g = dL/dq, xhat = (acc - mean_B) / sqrt(var_B + eps).
+#include <cuda_bf16.h>
+
+#include "pkm_common.cuh"
+#include "pkm_kernels.h"
+
+namespace pkm {
+
+// Pass 1: per (256 features, chunk of kStatChunk tokens), fp64 chunk mean and sum of
+// squared deviations from it (two passes over the chunk; the second one hits cache).
+// acc comes as three bf16 planes (hi + mid + lo) or as fp32.
+__global__ void __launch_bounds__(256) bn_stats_partial_kernel(
+    const uint16_t* __restrict__ planes, const float* __restrict__ acc, int B, int F,
+    double* __restrict__ part) {
+  const int f = blockIdx.x * blockDim.x + threadIdx.x;
+  if (f >= F) return;
+  const int t0 = blockIdx.y * kStatChunk, t1 = min(B, t0 + kStatChunk);
+  const int64_t count = static_cast<int64_t>(B) * F;
+  auto value = [&](int t) -> double {
+    const int64_t i = static_cast<int64_t>(t) * F + f;
+    if (planes)
+      return static_cast<double>(load_elem(planes, i) + load_elem(planes, count + i) +
+                                 load_elem(planes, 2 * count + i));
+    return static_cast<double>(acc[i]);
+  };
+  double s = 0.0;
+  for (int t = t0; t < t1; ++t) s += value(t);
+  const double mu = s / (t1 - t0);
+  double m2 = 0.0;
+  for (int t = t0; t < t1; ++t) {
+    const double dv = value(t) - mu;
+    m2 = fma(dv, dv, m2);
+  }
+  part[(static_cast<int64_t>(blockIdx.y) * 2) * F + f] = mu;
+  part[(static_cast<int64_t>(blockIdx.y) * 2 + 1) * F + f] = m2;
+}
+
+// Pass 2: merge the chunks in order (Chan, Golub and LeVeque's pairwise update of
+// count, mean and M2), write the batch statistics and move the running ones.
+__global__ void bn_stats_final_kernel(const double* __restrict__ part, int B, int F,
+                                      float momentum, float* __restrict__ batch_mean,
+                                      float* __restrict__ batch_var,
+                                      float* __restrict__ running_mean,
+                                      float* __restrict__ running_var) {
+  const int f = blockIdx.x * blockDim.x + threadIdx.x;
+  if (f >= F) return;
+  const int chunks = (B + kStatChunk - 1) / kStatChunk;
+  double n = 0.0, mean = 0.0, m2 = 0.0;
+  for (int c = 0; c < chunks; ++c) {
+    const double nb = static_cast<double>(min(B, (c + 1) * kStatChunk) - c * kStatChunk);
+    const double mb = part[(static_cast<int64_t>(c) * 2) * F + f];
+    const double m2b = part[(static_cast<int64_t>(c) * 2 + 1) * F + f];
+    const double tot = n + nb;
+    const double delta = mb - mean;
+    mean += delta * (nb / tot);
+    m2 += m2b + delta * delta * (n * nb / tot);
+    n = tot;
+  }
+  const double var = m2 / B;
+  batch_mean[f] = static_cast<float>(mean);
+  batch_var[f] = static_cast<float>(var);
+  const double m = momentum;
+  running_mean[f] = static_cast<float>((1.0 - m) * running_mean[f] + m * mean);
+  running_var[f] = static_cast<float>((1.0 - m) * running_var[f] + m * (m2 / (B - 1)));
+}
+
+cudaError_t launch_bn_batch_stats(const uint16_t* planes, const float* acc, int64_t B, int F,
+                                  float momentum, double* part, float* batch_mean,
+                                  float* batch_var, float* running_mean, float* running_var,
+                                  cudaStream_t st) {
+  const int chunks = static_cast<int>((B + kStatChunk - 1) / kStatChunk);
+  dim3 g1((F + 255) / 256, chunks);
+  bn_stats_partial_kernel<<<g1, 256, 0, st>>>(planes, acc, static_cast<int>(B), F, part);
+  bn_stats_final_kernel<<<(F + 255) / 256, 256, 0, st>>>(part, static_cast<int>(B), F, momentum,
+                                                          batch_mean, batch_var, running_mean,
+                                                          running_var);
+  return cudaGetLastError();
+}
+
+// dL/dacc with batch statistics, from g = dL/dq, acc and the column sums
+// sums[0][f] = sum_t g, sums[1][f] = sum_t g xhat. Written as fp32 (g_acc) and/or bf16
+// hi/lo planes [2][B][F] for the tensor-core GEMMs.
+__global__ void __launch_bounds__(256) bn_train_dacc_kernel(
+    const float* __restrict__ g_q, const float* __restrict__ acc,
+    const float* __restrict__ mean, const float* __restrict__ var,
+    const float* __restrict__ gamma, const float* __restrict__ sums, float eps, int B, int F,
+    float* __restrict__ g_acc, uint16_t* __restrict__ g_planes) {
+  const int64_t count = static_cast<int64_t>(B) * F;
+  const float inv_b = 1.f / static_cast<float>(B);
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < count;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int f = static_cast<int>(i % F);
+    const float rs = 1.f / sqrtf(var[f] + eps);
+    const float xhat = (acc[i] - mean[f]) * rs;
+    const float ga =
+        gamma[f] * rs * (g_q[i] - sums[f] * inv_b - xhat * (sums[F + f] * inv_b));
+    if (g_acc) g_acc[i] = ga;
+    if (g_planes) {
+      const __nv_bfloat16 hi = __float2bfloat16_rn(ga);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(ga - __bfloat162float(hi));
+      g_planes[i] = __bfloat16_as_ushort(hi);
+      g_planes[count + i] = __bfloat16_as_ushort(lo);
+    }
+  }
+}
+
+cudaError_t launch_bn_train_dacc(const float* g_q, const float* acc, const float* mean,
+                                 const float* var, const float* gamma, const float* sums,
+                                 float eps, int64_t B, int F, float* g_acc, uint16_t* g_planes,
+                                 cudaStream_t st) {
+  const int64_t blocks = (B * F + 255) / 256;
+  bn_train_dacc_kernel<<<static_cast<unsigned>(blocks < 148 * 8 ? blocks : 148 * 8), 256, 0,
+                         st>>>(g_q, acc, mean, var, gamma, sums, eps, static_cast<int>(B), F,
+                               g_acc, g_planes);
+  return cudaGetLastError();
+}
+
+}  // namespace pkm

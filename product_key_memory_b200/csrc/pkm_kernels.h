@@ -68,13 +68,28 @@ struct FullBackwardWs {
   float* coef;        // [B*H*k][2] summed kept-score gradient of that row
   BackwardWs sub;     // sub-key grouping
   float* bn_part;     // BatchNorm column-sum partials
+  float* bn_sums;     // [2][H*dq] sum_t dL/dq, sum_t dL/dq xhat
 };
 size_t backward_full_ws_bytes(const LayerArgs& a, bool tensor_path, FullBackwardWs* w, char* base);
-cudaError_t launch_backward_full(const LayerArgs& a, bool tensor_path, const int* indices,
+cudaError_t launch_backward_full(const LayerArgs& a, bool tensor_path, bool bn_training,
+                                 const int* indices,
                                  const float* weights, const void* grad_out, float* grad_x,
                                  float* grad_W, float* grad_gamma, float* grad_beta,
                                  float* grad_subkeys, float* grad_values, float* grad_scores,
                                  const FullBackwardWs& w, cudaStream_t st, int* launches);
+
+// BatchNorm in training mode (pkm_bn_train.cu). Batch statistics of acc (three bf16
+// planes, or fp32 when planes is null) in chunks of kStatChunk tokens; part holds
+// [chunks][2][F] doubles.
+constexpr int kStatChunk = 128;
+cudaError_t launch_bn_batch_stats(const uint16_t* planes, const float* acc, int64_t B, int F,
+                                  float momentum, double* part, float* batch_mean,
+                                  float* batch_var, float* running_mean, float* running_var,
+                                  cudaStream_t st);
+cudaError_t launch_bn_train_dacc(const float* g_q, const float* acc, const float* mean,
+                                 const float* var, const float* gamma, const float* sums,
+                                 float eps, int64_t B, int F, float* g_acc, uint16_t* g_planes,
+                                 cudaStream_t st);
 
 // Memory utilisation (pkm_usage.cu).
 size_t usage_bitmap_bytes(int64_t slots);

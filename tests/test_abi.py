@@ -122,3 +122,25 @@ def test_full_backward_workspace_and_argument_checks():
     s0 = _shape(B=0)
     zargs = [None, ok, ok, ok, ok, ok, ok, ok, None, None, None] + [None] * 7
     assert P.lib().pkm_backward(ctypes.byref(s0), *zargs, ok, 1 << 40, None) == 0
+
+
+def test_training_bn_entry_points_validate_before_launch():
+    s = _shape(B=4096, n=512)
+    fw = P.lib().pkm_workspace_size(ctypes.byref(s), 4)
+    # forward workspace + acc of the whole batch (three bf16 planes) + fp64 chunk stats
+    assert fw >= P.pkm_workspace_size(s) + 4096 * 2048 * 6 + 32 * 2 * 2048 * 8
+    assert P.lib().pkm_workspace_size(ctypes.byref(_shape(B=1)), 4) == 0
+    ok = ctypes.c_void_p(1 << 20)
+    f = P.lib().pkm_forward_train
+    args = [ok] * 6 + [ctypes.c_float(0.1)] + [ok] * 8   # through batch_var
+    assert f(ctypes.byref(_shape(B=1)), *args, ok, 1 << 40, None) == -1        # one token
+    bad = list(args)
+    bad[6] = ctypes.c_float(1.5)                                                 # momentum
+    assert f(ctypes.byref(s), *bad, ok, 1 << 40, None) == -1
+    bad = list(args)
+    bad[14] = None                                                               # batch_var
+    assert f(ctypes.byref(s), *bad, ok, 1 << 40, None) == -1
+    assert f(ctypes.byref(s), *args, ok, 100, None) == -3
+    bargs = [ok] * 11 + [None] * 7
+    assert P.lib().pkm_backward_train(ctypes.byref(_shape(B=1)), *bargs, ok, 1 << 40, None) == -1
+    assert P.lib().pkm_backward_train(ctypes.byref(s), *bargs, ok, 100, None) == -3
