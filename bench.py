@@ -379,7 +379,7 @@ def run_ours(args, rank, world, local_rank):
 
 
 def run_c512_and_backward(args, dev, P, hbm, bf16, stream, world, barrier,
-                          parts=("c512", "backward", "backward_full", "wide")):
+                          parts=("c512", "backward", "backward_full", "train", "wide")):
     """512^2-slot forward (the metric's other memory size), the value backward and the
     full backward on its picks, and the wide 1024^2-slot layer (H = 8, v = 1600).
     `parts` selects the measurements (the c512 forward always runs: it makes the
@@ -482,6 +482,45 @@ def run_c512_and_backward(args, dev, P, hbm, bf16, stream, world, barrier,
             "value": world * B / (full_ms / 1e3), "unit": UNIT, "ms_per_step": full_ms,
             "algorithmic_bytes": full_bytes, "gemm_flops": full_flops,
             "step_roofline_frac": max(t_mem, t_gemm) * 1e3 / full_ms}
+    if "train" in parts:
+        # One training step of the layer with BatchNorm in training mode: the forward
+        # on batch statistics (running statistics updated), then the full backward
+        # through them.
+        tws = torch.empty(int(P.lib().pkm_workspace_size(ctypes.byref(shape), 4)),
+                          dtype=torch.uint8, device=dev)
+        rm, rv = d["bn_mean"].clone(), d["bn_var"].clone()
+        bm = torch.empty(F, device=dev)
+        bv = torch.empty(F, device=dev)
+        scs = torch.empty(B, w.H, w.k, dtype=torch.float32, device=dev)
+
+        def fwd_train():
+            rc = P.lib().pkm_forward_train(
+                ctypes.byref(shape), P._ptr(d["x"]), P._ptr(d["W_q"]), P._ptr(rm), P._ptr(rv),
+                P._ptr(d["bn_gamma"]), P._ptr(d["bn_beta"]), ctypes.c_float(0.1),
+                P._ptr(d["subkeys"]), P._ptr(d["values"]), P._ptr(out), P._ptr(idx),
+                P._ptr(wts), P._ptr(scs), P._ptr(bm), P._ptr(bv), P._ptr(tws), tws.numel(),
+                P._stream(None))
+            if rc != 0:
+                raise RuntimeError("pkm_forward_train: %s" % P.pkm_status_string(rc))
+
+        def bwd_train():
+            P.pkm_backward(d["x"], d["W_q"], bm, bv, d["bn_gamma"], d["bn_beta"], d["subkeys"],
+                           d["values"], idx, wts, gout, grads, workspace=fws, bn_training=True)
+
+        def train_step():
+            fwd_train()
+            bwd_train()
+
+        for _ in range(max(3, args.warmup)):
+            train_step()
+        ftr_ms = timed(fwd_train, args.steps)
+        step_ms = timed(train_step, args.steps)
+        res["train"] = {
+            "workload": "c512 training step: forward on batch statistics + full backward "
+                        "through them, B=4096",
+            "value": world * B / (step_ms / 1e3), "unit": UNIT, "ms_per_step": step_ms,
+            "forward_train_ms": ftr_ms, "backward_train_ms": step_ms - ftr_ms}
+        del tws
     del d, gv, gout, bws, ws, fws, grads
     torch.cuda.empty_cache()
     if "wide" not in parts:
@@ -526,7 +565,7 @@ def main():
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the c512 / backward / CPU-oracle measurements")
     ap.add_argument("--part", default=None,
-                    choices=["c512", "backward", "backward_full", "wide"],
+                    choices=["c512", "backward", "backward_full", "train", "wide"],
                     help="run only this sub-measurement and print its JSON object "
                          "(for profiling one kernel family; not a bench line)")
     args = ap.parse_args()
