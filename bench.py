@@ -379,7 +379,8 @@ def run_ours(args, rank, world, local_rank):
 
 
 def run_c512_and_backward(args, dev, P, hbm, bf16, stream, world, barrier,
-                          parts=("c512", "backward", "backward_full", "train", "wide")):
+                          parts=("c512", "backward", "backward_full", "train", "latency",
+                                 "wide")):
     """512^2-slot forward (the metric's other memory size), the value backward and the
     full backward on its picks, and the wide 1024^2-slot layer (H = 8, v = 1600).
     `parts` selects the measurements (the c512 forward always runs: it makes the
@@ -482,6 +483,8 @@ def run_c512_and_backward(args, dev, P, hbm, bf16, stream, world, barrier,
             "value": world * B / (full_ms / 1e3), "unit": UNIT, "ms_per_step": full_ms,
             "algorithmic_bytes": full_bytes, "gemm_flops": full_flops,
             "step_roofline_frac": max(t_mem, t_gemm) * 1e3 / full_ms}
+    if "latency" in parts:
+        res["small_batch"] = run_latency(args, dev, P)
     if "train" in parts:
         # One training step of the layer with BatchNorm in training mode: the forward
         # on batch statistics (running statistics updated), then the full backward
@@ -555,6 +558,42 @@ def run_c512_and_backward(args, dev, P, hbm, bf16, stream, world, barrier,
     return res
 
 
+def run_latency(args, dev, P):
+    """Forward latency for a few tokens on the 1024^2-slot layer (the serving case):
+    calls issued back to back on one stream, device time per call from CUDA events
+    around 200 calls; caches warm (one token touches 128 value rows)."""
+    w0 = synth.WORKLOADS["c1024"]
+    L = synth.make_layer(w0.with_(B=64))
+    d = {k: v.to(dev) for k, v in L.items()}
+    res = {"workload": "c1024 layer (1024^2 slots, H=4, k=32, v=1024, bf16), B tokens per call",
+           "unit": "us per call"}
+    for B in (1, 16, 64):
+        x = d["x"][:B].contiguous()
+        out = torch.empty(B, w0.v, device=dev)
+        idx = torch.empty(B, w0.H, w0.k, dtype=torch.int32, device=dev)
+        wts = torch.empty(B, w0.H, w0.k, device=dev)
+        shape = P.make_shape(B, w0.d_model, w0.H, w0.dq, w0.n, w0.k, w0.v, w0.torch_dtype)
+        ws = P.alloc_workspace(shape, False, dev)
+
+        def call():
+            P.pkm_forward(x, d["W_q"], d["bn_mean"], d["bn_var"], d["bn_gamma"], d["bn_beta"],
+                          d["subkeys"], d["values"], k=w0.k, out=out, indices=idx,
+                          weights=wts, want_scores=False, workspace=ws)
+
+        for _ in range(max(3, args.warmup) * 4):
+            call()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n = 200
+        a.record()
+        for _ in range(n):
+            call()
+        b.record()
+        torch.cuda.synchronize(dev)
+        res["B=%d" % B] = a.elapsed_time(b) / n * 1e3
+    return res
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -565,7 +604,7 @@ def main():
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the c512 / backward / CPU-oracle measurements")
     ap.add_argument("--part", default=None,
-                    choices=["c512", "backward", "backward_full", "train", "wide"],
+                    choices=["c512", "backward", "backward_full", "train", "latency", "wide"],
                     help="run only this sub-measurement and print its JSON object "
                          "(for profiling one kernel family; not a bench line)")
     args = ap.parse_args()

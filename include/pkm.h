@@ -95,10 +95,14 @@ size_t pkm_workspace_size(const pkm_shape* s, int for_backward);
  *   scores   [B][H][k]  fp32   kept key scores s1[i] + s2[j]; may be NULL
  * workspace: device scratch of at least pkm_workspace_size(s, 0) bytes, 256-byte
  *   aligned; its contents on entry do not matter.
- * Large batches are processed in up to 4 sub-batches; the value gather of one
- * sub-batch runs on a second stream owned by the library (one per device) while the
- * next sub-batch is scored on `stream`. Event waits order both ways, so all of the
- * call's work is complete when `stream` reaches the point after the call.
+ * Batches of at most 64 tokens (H <= 8) take the small-batch kernels, which spread
+ * W_q, the sub-keys and the heads over all SMs for latency; their three launches
+ * overlap through programmatic dependent launch on `stream`. Large batches of
+ * tensor-core shapes can be processed in up to 4 sub-batches (PKM_SUBBATCHES); the
+ * value gather of one sub-batch then runs on a second stream owned by the library
+ * (one per device) while the next sub-batch is scored on `stream`. Event waits order
+ * both ways, so all of the call's work is complete when `stream` reaches the point
+ * after the call.
  * Returns PKM_OK or a status code above.
  */
 int pkm_forward(const pkm_shape* s, const void* x, const void* W_q, const float* bn_mean,

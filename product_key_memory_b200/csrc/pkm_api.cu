@@ -18,12 +18,19 @@ using pkm::LayerArgs;
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Which implementation of the query network and per-half search runs.
-enum class Path { kTensor, kSimt };
+// Which implementation of the forward runs: the small-batch kernels for a few
+// tokens, else the tensor-core kernels where the shape fits their tiles, else the
+// CUDA-core kernels. PKM_PATH=simt or =tc pins one of the large-batch paths (tests
+// compare the paths on the same inputs).
+enum class Path { kTensor, kSimt, kSmall };
 
 Path choose_path(const pkm_shape* s) {
   const char* env = getenv("PKM_PATH");
   if (env && strcmp(env, "simt") == 0) return Path::kSimt;
+  const bool pin_tc = env && strcmp(env, "tc") == 0;
+  if (!pin_tc &&
+      pkm::small_supported(s->B, s->d_model, s->H, s->dq, s->n, s->k, s->v, s->dtype))
+    return Path::kSmall;
   return pkm::tc_supported(s->dtype, s->d_model, s->H, s->dq, s->n, s->k) ? Path::kTensor
                                                                           : Path::kSimt;
 }
@@ -88,10 +95,14 @@ int64_t sub_batch_tokens(int64_t B) {
 
 size_t forward_ws(const pkm_shape* s, ForwardWs* w, char* base) {
   const int64_t F = static_cast<int64_t>(s->H) * s->dq;
-  const int64_t L = s->B * s->H * 2 * static_cast<int64_t>(pkm::kMaxK);
-  const size_t qbytes = choose_path(s) == Path::kTensor
+  const Path path = choose_path(s);
+  const size_t qbytes = path == Path::kTensor
                             ? static_cast<size_t>(sub_batch_tokens(s->B)) * F * 6
                             : static_cast<size_t>(s->B) * F * 4;
+  // The small-batch path keeps each chunk's best 32 before merging them.
+  const int64_t L = path == Path::kSmall
+                        ? static_cast<int64_t>(pkm::small_chunk_entries(s->B, s->H, s->n))
+                        : s->B * s->H * 2 * static_cast<int64_t>(pkm::kMaxK);
   size_t off = pkm::kStatusBytes;
   const size_t o_q = off;  off += align256(qbytes);
   const size_t o_ls = off; off += align256(sizeof(float) * L);
@@ -447,7 +458,13 @@ cudaError_t run_forward(const pkm_shape* s, const LayerArgs& a, const ForwardWs&
   const void* x = a.x;
   cudaError_t e = cudaSuccess;
   int launches = 0;
-  if (choose_path(s) == Path::kSimt) {
+  const Path path = choose_path(s);
+  if (path == Path::kSmall) {
+    tr.begin(2, st);
+    e = pkm::launch_forward_small(a, w.q, w.list_s, w.list_i, out, indices, weights, scores, st);
+    tr.end(st);
+    launches = 3;
+  } else if (path == Path::kSimt) {
     tr.begin(0, st);
     e = pkm::launch_query_bn_simt(a, w.q, st);
     tr.end(st);

@@ -262,9 +262,7 @@ cudaError_t launch_gemm(const CUtensorMap& tm_a, const CUtensorMap& tm_b, float*
     if (e != cudaSuccess) return e;
   }
   const size_t smem = gemm_tc_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<A_MN>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  cudaError_t e = set_max_smem(reinterpret_cast<const void*>(gemm_tc_kernel<A_MN>), smem);
   if (e != cudaSuccess) return e;
   const int units = tiles * ksplit;
   const int grid = units < sms ? units : sms;

@@ -91,6 +91,19 @@ cudaError_t launch_bn_train_dacc(const float* g_q, const float* acc, const float
                                  float eps, int64_t B, int F, float* g_acc, uint16_t* g_planes,
                                  cudaStream_t st);
 
+// Small-batch forward (pkm_small.cu): B <= kSmallMaxB tokens, three launches that
+// spread the parameters over every SM. Workspace: q fp32 [B][H*dq] and chunk lists of
+// small_chunk_entries() (score, id) entries.
+constexpr int kSmallMaxB = 64;
+bool small_supported(int64_t B, int d_model, int H, int dq, int n, int k, int v, int dtype);
+size_t small_chunk_entries(int64_t B, int H, int n);
+cudaError_t launch_forward_small(const LayerArgs& a, float* q, float* chunk_s, int* chunk_i,
+                                 float* out, int* idx, float* w, float* sc, cudaStream_t st);
+
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device, size)
+// (pkm_util.cu).
+cudaError_t set_max_smem(const void* func, size_t bytes);
+
 // Memory utilisation (pkm_usage.cu).
 size_t usage_bitmap_bytes(int64_t slots);
 cudaError_t launch_slot_usage(const int* indices, int64_t E, int64_t slots, unsigned* bitmap,

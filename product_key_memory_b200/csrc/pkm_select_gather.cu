@@ -10,21 +10,18 @@
 // left sub-key i joined with right sub-key j, flat slot i*n + j ("Implied keys vs
 // stored sub-keys").
 //
-// Candidate pruning: with both per-half lists sorted best first, the pair at list
-// positions (a, b) is beaten by every pair (a', b') with a' <= a and b' <= b, so it can
-// only be among the best k if (a + 1)(b + 1) <= k. That is the same argument the
-// pages give for keeping k per half, applied inside the k x k grid; it leaves
-// sum_a floor(k / (a + 1)) candidates (119 for k = 32) instead of k^2. In fp32 the
+// Candidate pruning (pkm_select.cuh): with both per-half lists sorted best first,
+// only pairs at list positions (a + 1)(b + 1) <= k can be among the best k -- the
+// pages' argument for keeping k per half, applied inside the k x k grid. In fp32 the
 // sums keep that order except where two sums round to the same value, which is a
 // tie at fp32 resolution.
 #include "pkm_common.cuh"
 #include "pkm_kernels.h"
+#include "pkm_select.cuh"
 
 namespace pkm {
 
 constexpr int kSgWarps = 4;
-// Candidate pairs (a, b) with (a+1)(b+1) <= k number sum_a floor(k/(a+1)) <= 119 for k <= 32.
-constexpr int kMaxPairs = 128;
 
 template <typename T, int MAXV>
 __global__ void __launch_bounds__(kSgWarps * 32) select_gather_kernel(
@@ -42,12 +39,7 @@ __global__ void __launch_bounds__(kSgWarps * 32) select_gather_kernel(
   float* wts = reinterpret_cast<float*>(rows + HK);      // [HK]
   __shared__ int npairs_s;
 
-  if (threadIdx.x == 0) {
-    int p = 0;
-    for (int a = 0; a < k; ++a)
-      for (int b = 0; (a + 1) * (b + 1) <= k; ++b) pairs[p++] = a | (b << 8);
-    npairs_s = p;
-  }
+  if (threadIdx.x == 0) npairs_s = build_pairs(k, pairs);
   __syncthreads();
   const int npairs = npairs_s;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * kSgWarps + warp;
@@ -63,23 +55,9 @@ __global__ void __launch_bounds__(kSgWarps * 32) select_gather_kernel(
     int i2 = list_i[base + kMaxK + lane];
     warp_sort32(s1, i1);
     warp_sort32(s2, i2);
-    float bs = -INFINITY;
-    int bi = kIdPad;
-    for (int c0 = 0; c0 < npairs; c0 += 32) {
-      const int p = c0 + lane;
-      const int ab = p < npairs ? pairs[p] : 0;
-      const int a = ab & 0xff, b = ab >> 8;
-      const float sa = __shfl_sync(0xffffffffu, s1, a);
-      const int ia = __shfl_sync(0xffffffffu, i1, a);
-      const float sb = __shfl_sync(0xffffffffu, s2, b);
-      const int ib = __shfl_sync(0xffffffffu, i2, b);
-      // Padding ids can only surface when scores are NaN; they never form a slot.
-      const bool real = p < npairs && ia >= 0 && ia < n && ib >= 0 && ib < n;
-      float cs = real ? sa + sb : -INFINITY;
-      int ci = real ? ia * n + ib : kIdPad;
-      warp_sort32(cs, ci);
-      warp_merge32(bs, bi, cs, ci);
-    }
+    float bs;
+    int bi;
+    select_candidates(s1, i1, s2, i2, pairs, npairs, n, bs, bi);
     // Softmax over the k kept scores (lanes 0..k-1 hold them, best first).
     const float mx = __shfl_sync(0xffffffffu, bs, 0);
     const float e = lane < k ? expf(bs - mx) : 0.f;
@@ -166,8 +144,7 @@ template <typename T, int MAXV>
 static cudaError_t launch_sg(const LayerArgs& a, const float* ls, const int* li, float* out,
                              int* idx, float* w, float* sc, cudaStream_t st) {
   const size_t smem = sizeof(int) * (kMaxPairs + kSgWarps * 2 * a.H * a.k);
-  cudaError_t e = cudaFuncSetAttribute(select_gather_kernel<T, MAXV>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = set_max_smem(reinterpret_cast<const void*>(select_gather_kernel<T, MAXV>), smem);
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>((a.B + kSgWarps - 1) / kSgWarps);
   select_gather_kernel<T, MAXV><<<grid, kSgWarps * 32, smem, st>>>(

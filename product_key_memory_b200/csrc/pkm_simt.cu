@@ -172,14 +172,12 @@ cudaError_t launch_subkey_topk_simt(const LayerArgs& a, const float* q, float* l
   dim3 grid(static_cast<unsigned>((a.B + kSimtTok - 1) / kSimtTok), a.H * 2);
   cudaError_t e;
   if (a.dtype == 0) {
-    e = cudaFuncSetAttribute(subkey_topk_simt_kernel<float>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = set_max_smem(reinterpret_cast<const void*>(subkey_topk_simt_kernel<float>), smem);
     if (e != cudaSuccess) return e;
     subkey_topk_simt_kernel<float><<<grid, kSimtWarps * 32, smem, st>>>(
         q, static_cast<const float*>(a.subkeys), a.B, a.H, a.dq, a.n, a.k, list_s, list_i);
   } else {
-    e = cudaFuncSetAttribute(subkey_topk_simt_kernel<uint16_t>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = set_max_smem(reinterpret_cast<const void*>(subkey_topk_simt_kernel<uint16_t>), smem);
     if (e != cudaSuccess) return e;
     subkey_topk_simt_kernel<uint16_t><<<grid, kSimtWarps * 32, smem, st>>>(
         q, static_cast<const uint16_t*>(a.subkeys), a.B, a.H, a.dq, a.n, a.k, list_s, list_i);

@@ -1,0 +1,562 @@
+// pkm_small.cu -- the forward for small batches (B <= kSmallMaxB tokens): the
+// serving case of one or a few sequences' tokens, where latency rather than HBM
+// bandwidth is the goal ("Large Memory Layers with Product Keys", gptget.net
+// summary: the memory layer makes inference faster than a larger dense model).
+//
+// The large-batch kernels tile 128 tokens per CTA, so a handful of tokens leaves
+// almost every SM idle and each stage is bound by one SM's bandwidth. Here every
+// stage spreads the layer's parameters over the whole GPU instead:
+//   query_small_kernel   q = BN(x W_q^T): CTA = 16 features x all tokens, its W_q rows
+//                        staged in shared memory, one warp per token (fp32 FMA)
+//   score_small_kernel   CTA = (64 sub-keys, head-half, 16 tokens): the chunk's scores
+//                        and its best 32 per token
+//   gather_small_kernel  CTA = (token, head), the H heads of a token one cluster:
+//                        merge the chunk lists of each half, exact top-k of the
+//                        pruned candidates, softmax, the head's k weighted value rows
+//                        over 8 warps, heads summed over distributed shared memory
+// Same arithmetic as the CUDA-core large-batch path (fp32 q, fp32 dot products, the
+// same selection order and candidate pruning).
+#include <cooperative_groups.h>
+
+#include <algorithm>
+
+#include "pkm_common.cuh"
+#include "pkm_kernels.h"
+#include "pkm_select.cuh"
+
+namespace pkm {
+
+constexpr int kQFeat = 16;        // features per query CTA
+constexpr int kSChunk = 64;       // sub-keys per scoring CTA
+constexpr int kSTok = 16;         // tokens per scoring CTA (2 per warp)
+constexpr int kSmallWarps = 8;
+constexpr int kQTok = kSmallWarps;  // tokens per query CTA (one per warp)
+
+// Programmatic dependent launch: the next kernel on the stream may start launching
+// once every CTA of this one has passed launch_dependents; its CTAs block in
+// wait_prior_grid until this grid has finished and its writes are visible.
+__device__ __forceinline__ void allow_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void wait_prior_grid() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Copy `words` 32-bit words from global to shared memory with every thread keeping
+// kCopyDepth loads in flight (the staging loops otherwise serialise on latency).
+// Row r of `rows` words lands at dst + r * dst_ld; rows at or past `valid_rows` are
+// zero-filled.
+constexpr int kCopyDepth = 8;
+
+__device__ __forceinline__ void stage_rows(const uint32_t* __restrict__ src, uint32_t* dst,
+                                           int nrows, int valid_rows, int row_words,
+                                           int dst_ld) {
+  if ((row_words & 3) == 0 && (reinterpret_cast<uintptr_t>(src) & 15) == 0) {
+    // 16-byte loads (four words of one row each), stored as words (rows may be padded).
+    const int row_vecs = row_words >> 2;
+    const int total = nrows * row_vecs;
+    const uint4* s4 = reinterpret_cast<const uint4*>(src);
+    for (int base = threadIdx.x; base < total; base += blockDim.x * kCopyDepth) {
+      uint4 v[kCopyDepth];
+#pragma unroll
+      for (int u = 0; u < kCopyDepth; ++u) {
+        const int i = base + u * blockDim.x;
+        const int r = i / row_vecs;
+        v[u] = (i < total && r < valid_rows) ? __ldg(s4 + i) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < kCopyDepth; ++u) {
+        const int i = base + u * blockDim.x;
+        if (i < total) {
+          const int r = i / row_vecs;
+          uint32_t* d = dst + r * dst_ld + ((i - r * row_vecs) << 2);
+          d[0] = v[u].x; d[1] = v[u].y; d[2] = v[u].z; d[3] = v[u].w;
+        }
+      }
+    }
+    return;
+  }
+  const int total = nrows * row_words;
+  for (int base = threadIdx.x; base < total; base += blockDim.x * kCopyDepth) {
+    uint32_t v[kCopyDepth];
+#pragma unroll
+    for (int u = 0; u < kCopyDepth; ++u) {
+      const int i = base + u * blockDim.x;
+      const int r = i / row_words;
+      v[u] = (i < total && r < valid_rows) ? __ldg(src + i) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < kCopyDepth; ++u) {
+      const int i = base + u * blockDim.x;
+      if (i < total) {
+        const int r = i / row_words;
+        dst[r * dst_ld + (i - r * row_words)] = v[u];
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// q[t][f] = (sum_c x[t][c] W[f][c]) * scale[f] + shift[f], scale = gamma / sqrt(var + eps),
+// shift = beta - mean * scale (the tensor-core epilogue's form). CTA = 16 features x 8
+// tokens: the 16 rows of W_q staged in shared memory, one warp per token reading x in
+// runs of 8 per lane; the 16 per-lane partial sums are reduced by a butterfly that
+// leaves feature j's total in lanes 2j and 2j + 1 (16 shuffles instead of 80).
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(kSmallWarps * 32) query_small_kernel(
+    const T* __restrict__ x, const T* __restrict__ W, const float* __restrict__ mean,
+    const float* __restrict__ var, const float* __restrict__ gamma,
+    const float* __restrict__ beta, float eps, int B, int d, int F, float* __restrict__ q) {
+  extern __shared__ __align__(16) unsigned char qs_raw[];
+  T* ws = reinterpret_cast<T*>(qs_raw);  // [kQFeat][d]
+  T* xs = ws + kQFeat * d;               // [kQTok][d]
+  allow_dependents();
+  const int f0 = blockIdx.x * kQFeat;
+  const int nf = min(kQFeat, F - f0);
+  const int t0 = blockIdx.y * kQTok;
+  // d * sizeof(T) is a multiple of 4 (checked on the host): whole rows are words.
+  const int row_words = d * static_cast<int>(sizeof(T)) / 4;
+  stage_rows(reinterpret_cast<const uint32_t*>(W + static_cast<int64_t>(f0) * d),
+             reinterpret_cast<uint32_t*>(ws), kQFeat, nf, row_words, row_words);
+  stage_rows(reinterpret_cast<const uint32_t*>(x + static_cast<int64_t>(t0) * d),
+             reinterpret_cast<uint32_t*>(xs), kQTok, min(kQTok, B - t0), row_words, row_words);
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = t0 + warp;
+  if (t < B) {
+    float acc[kQFeat];
+#pragma unroll
+    for (int j = 0; j < kQFeat; ++j) acc[j] = 0.f;
+    const T* xr = xs + warp * d;
+    for (int c0 = 0; c0 < d; c0 += 32 * 8) {
+      float xv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int c = c0 + lane + 32 * u;
+        xv[u] = c < d ? load_elem(xr, c) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int c = c0 + lane + 32 * u;
+        if (c < d) {
+#pragma unroll
+          for (int j = 0; j < kQFeat; ++j) acc[j] = fmaf(xv[u], load_elem(ws, j * d + c), acc[j]);
+        }
+      }
+    }
+    // Butterfly: at mask m each lane keeps half of its values (the upper half when
+    // its bit m is set) and adds the partner's copy of them.
+#pragma unroll
+    for (int m = 16, c = kQFeat / 2; c >= 1; m >>= 1, c >>= 1) {
+      const bool up = (lane & m) != 0;
+#pragma unroll
+      for (int i = 0; i < c; ++i) {
+        const float send = up ? acc[i] : acc[i + c];
+        const float keep = up ? acc[i + c] : acc[i];
+        acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+      }
+    }
+    const float a = acc[0] + __shfl_xor_sync(0xffffffffu, acc[0], 1);
+    const int j = lane >> 1;  // this lane's feature
+    if ((lane & 1) == 0 && j < nf) {
+      const int f = f0 + j;
+      const float sc = gamma[f] / sqrtf(var[f] + eps);
+      q[static_cast<int64_t>(t) * F + f] = fmaf(a, sc, beta[f] - mean[f] * sc);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Per-half scores of one chunk of kSChunk sub-keys for up to kSTok tokens, and each
+// token's best 32 of the chunk. Lane i scores sub-keys c0 + i and c0 + 32 + i; the two
+// sorted halves are merged (warp_sort32 / warp_merge32). Output chunk lists
+// [B][H][2][nchunks][32], best first (padding: -inf, kIdPad).
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(kSmallWarps * 32) score_small_kernel(
+    const float* __restrict__ q, const T* __restrict__ subkeys, int B, int H, int dq, int n,
+    float* __restrict__ chunk_s, int* __restrict__ chunk_i) {
+  extern __shared__ __align__(16) unsigned char ss_raw[];
+  const int half = dq >> 1;
+  const int ld = half + (sizeof(T) == 2 ? 2 : 1);  // padded row: lanes hit distinct banks
+  T* rows = reinterpret_cast<T*>(ss_raw);           // [kSChunk][ld]
+  float* qs = reinterpret_cast<float*>(ss_raw + ((sizeof(T) * kSChunk * ld + 15) & ~15));
+  const int chunk = blockIdx.x, hs = blockIdx.y;
+  const int h = hs >> 1, side = hs & 1;
+  const int c0 = chunk * kSChunk;
+  const int nchunks = (n + kSChunk - 1) / kSChunk;
+  const T* book = subkeys + (static_cast<int64_t>(hs) * n + c0) * half;
+  // half * sizeof(T) is a multiple of 4 (checked on the host); ld * sizeof(T) too.
+  const int row_words = half * static_cast<int>(sizeof(T)) / 4;
+  allow_dependents();
+  stage_rows(reinterpret_cast<const uint32_t*>(book), reinterpret_cast<uint32_t*>(rows),
+             kSChunk, min(kSChunk, n - c0), row_words, ld * static_cast<int>(sizeof(T)) / 4);
+  wait_prior_grid();  // q comes from the query kernel
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int F = H * dq;
+  // The warp's two tokens' query halves.
+  float* qw = qs + warp * 2 * half;
+  const int tb = blockIdx.z * kSTok + warp * 2;
+  for (int i0 = 0; i0 < 2 * half; i0 += 32 * 8) {
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + lane + 32 * u;
+      const int uu = i / half, e = i - uu * half;
+      const int t = tb + uu;
+      v[u] = (i < 2 * half && t < B) ? q[static_cast<int64_t>(t) * F + h * dq + side * half + e]
+                                     : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + lane + 32 * u;
+      if (i < 2 * half) qw[i] = v[u];
+    }
+  }
+  __syncthreads();
+  const bool v0 = c0 + lane < n, v1 = c0 + 32 + lane < n;
+  const T* r0 = rows + lane * ld;
+  const T* r1 = rows + (lane + 32) * ld;
+  for (int u = 0; u < 2; ++u) {
+    const int t = tb + u;
+    if (t >= B) break;  // warp-uniform
+    const float* qq = qw + u * half;
+    // Two chains per row (even and odd elements), added at the end.
+    float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+    int e = 0;
+    for (; e + 1 < half; e += 2) {
+      const float qv = qq[e], qv2 = qq[e + 1];
+      a0 = fmaf(qv, load_elem(r0, e), a0);
+      a1 = fmaf(qv, load_elem(r1, e), a1);
+      b0 = fmaf(qv2, load_elem(r0, e + 1), b0);
+      b1 = fmaf(qv2, load_elem(r1, e + 1), b1);
+    }
+    if (e < half) {
+      a0 = fmaf(qq[e], load_elem(r0, e), a0);
+      a1 = fmaf(qq[e], load_elem(r1, e), a1);
+    }
+    a0 += b0;
+    a1 += b1;
+    float s0 = v0 ? a0 : -INFINITY, s1 = v1 ? a1 : -INFINITY;
+    int i0 = v0 ? c0 + lane : kIdPad, i1 = v1 ? c0 + 32 + lane : kIdPad;
+    warp_sort32(s0, i0);
+    warp_sort32(s1, i1);
+    warp_merge32(s0, i0, s1, i1);
+    const int64_t o = ((((static_cast<int64_t>(t) * H + h) * 2 + side) * nchunks + chunk) << 5) + lane;
+    chunk_s[o] = s0;
+    chunk_i[o] = i0;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// One CTA per (token, head); the H CTAs of a token form a thread-block cluster.
+// (a) Warps 0 and 1 merge the chunk lists of the head's two halves into each half's
+// best 32. (b) Warp 0: exact top-k of the pruned product candidates, softmax,
+// indices / weights / scores. (c) The k weighted value rows, split over the 8 warps,
+// summed into the CTA's partial output in shared memory. (d) After a cluster
+// barrier, each CTA adds the H partial outputs of its slice of the columns in head
+// order through distributed shared memory and writes them to out[t]; a second
+// barrier keeps every CTA's shared memory alive until the others have read it.
+// ---------------------------------------------------------------------------
+template <typename T, int MAXV>
+__global__ void __launch_bounds__(kSmallWarps * 32) gather_small_kernel(
+    const float* __restrict__ chunk_s, const int* __restrict__ chunk_i,
+    const T* __restrict__ values, int H, int n, int k, int v, float* __restrict__ out,
+    int* __restrict__ indices, float* __restrict__ weights, float* __restrict__ scores,
+    int* status) {
+  namespace cg = cooperative_groups;
+  constexpr int VPER = Vec<T>::kPer;
+  extern __shared__ __align__(16) unsigned char gs_raw[];
+  const int nchunks = (n + kSChunk - 1) / kSChunk;
+  const int list_words = 2 * nchunks * kMaxK;                    // this head's two halves
+  float* part = reinterpret_cast<float*>(gs_raw);                 // [v] this head's output
+  float* red = part + v;                                          // [kSmallWarps][v]
+  float* cls = red;                                               // [2][nchunks][32] (phase a)
+  int* cli = reinterpret_cast<int*>(red + list_words);
+  const int scratch = max(kSmallWarps * v, 2 * list_words);
+  float* cand_s = red + scratch;                                  // [kMaxPairs]
+  int* cand_i = reinterpret_cast<int*>(cand_s + kMaxPairs);       // [kMaxPairs]
+  int* rows = cand_i + kMaxPairs;                                 // [k]
+  float* wts = reinterpret_cast<float*>(rows + kMaxK);            // [k]
+  int* pairs = reinterpret_cast<int*>(wts + kMaxK);               // [kMaxPairs]
+  __shared__ int npairs_s;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t t = blockIdx.x;
+  const int h = blockIdx.y;
+  if (threadIdx.x == 0) npairs_s = build_pairs(k, pairs);
+  wait_prior_grid();  // the chunk lists come from the scoring kernel
+  const int64_t src = (t * H + h) * list_words;
+  stage_rows(reinterpret_cast<const uint32_t*>(chunk_s + src), reinterpret_cast<uint32_t*>(cls),
+             1, 1, list_words, list_words);
+  stage_rows(reinterpret_cast<const uint32_t*>(chunk_i + src), reinterpret_cast<uint32_t*>(cli),
+             1, 1, list_words, list_words);
+  __syncthreads();
+
+  // (a) merge the chunk lists of each half, as a tree over the 8 warps: at stride st
+  // the list at 2 st i + st is merged into the list at 2 st i (each list is read and
+  // written by one warp per round).
+  for (int st = 1; st < nchunks; st <<= 1) {
+    const int per_side = (nchunks + 2 * st - 1) / (2 * st);
+    for (int item = warp; item < 2 * per_side; item += kSmallWarps) {
+      const int side = item / per_side, i = item - side * per_side;
+      const int a0 = 2 * st * i, b0 = a0 + st;
+      if (b0 >= nchunks) continue;  // warp-uniform
+      const int pa = ((side * nchunks + a0) << 5) + lane, pb = ((side * nchunks + b0) << 5) + lane;
+      float bs = cls[pa];
+      int bi = cli[pa];
+      const float cs = cls[pb];
+      const int ci = cli[pb];
+      // Merge only when the second list's best beats the first's 32nd.
+      const float ks = __shfl_sync(0xffffffffu, bs, 31);
+      const int ki = __shfl_sync(0xffffffffu, bi, 31);
+      const float c0s = __shfl_sync(0xffffffffu, cs, 0);
+      const int c0i = __shfl_sync(0xffffffffu, ci, 0);
+      if (better(c0s, c0i, ks, ki)) warp_merge32(bs, bi, cs, ci);
+      cls[pa] = bs;
+      cli[pa] = bi;
+    }
+    __syncthreads();
+  }
+  float* ls = cls;                          // half 0's best 32 at chunk 0, half 1's after
+  int* li = cli;
+  const int l1 = nchunks << 5;
+
+  // (b) the pruned candidates in chunks of 32, one chunk per warp, each sorted; then
+  // merged as a tree; warp 0 takes softmax and the head's picks.
+  const int npairs = npairs_s;
+  const int nc = (npairs + 31) / 32;
+  for (int c = warp; c < nc; c += kSmallWarps) {
+    const int p = c * 32 + lane;
+    const int ab = p < npairs ? pairs[p] : 0;
+    const int pa = ab & 0xff, pb = ab >> 8;
+    const float sa = ls[pa], sb = ls[l1 + pb];
+    const int ia = li[pa], ib = li[l1 + pb];
+    // Padding ids can only surface when scores are NaN; they never form a slot.
+    const bool real = p < npairs && ia >= 0 && ia < n && ib >= 0 && ib < n;
+    float cs = real ? sa + sb : -INFINITY;
+    int ci = real ? ia * n + ib : kIdPad;
+    warp_sort32(cs, ci);
+    cand_s[(c << 5) + lane] = cs;
+    cand_i[(c << 5) + lane] = ci;
+  }
+  __syncthreads();
+  for (int st = 1; st < nc; st <<= 1) {
+    for (int i = warp; 2 * st * i + st < nc; i += kSmallWarps) {
+      const int pa = ((2 * st * i) << 5) + lane, pb = ((2 * st * i + st) << 5) + lane;
+      float bs = cand_s[pa];
+      int bi = cand_i[pa];
+      warp_merge32(bs, bi, cand_s[pb], cand_i[pb]);
+      cand_s[pa] = bs;
+      cand_i[pa] = bi;
+    }
+    __syncthreads();
+  }
+  if (warp == 0) {
+    const float bs = cand_s[lane];
+    const int bi = cand_i[lane];
+    const float mx = __shfl_sync(0xffffffffu, bs, 0);
+    const float e = lane < k ? expf(bs - mx) : 0.f;
+    const float den = warp_sum(e);
+    const float w = e / den;
+    if (lane < k) {
+      const int64_t o = (t * H + h) * static_cast<int64_t>(k) + lane;
+      indices[o] = bi;
+      weights[o] = w;
+      if (scores) scores[o] = bs;
+      rows[lane] = bi;
+      wts[lane] = w;
+    }
+  }
+  __syncthreads();
+
+  // (c) weighted value rows r = warp, warp + 8, ... (all of a warp's rows in flight).
+  constexpr int U = 4;  // k <= 32 rows over 8 warps
+  const int nvec = v / VPER;
+  float acc[MAXV][VPER];
+#pragma unroll
+  for (int m = 0; m < MAXV; ++m)
+#pragma unroll
+    for (int e = 0; e < VPER; ++e) acc[m][e] = 0.f;
+  {
+    uint4 raw[U][MAXV];
+    float wr[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int r = warp + u * kSmallWarps;
+      bool live = r < k;
+      int row = live ? rows[r] : 0;
+      if (live && (row < 0 || row >= n * n)) {  // only reachable with NaN scores
+        if (lane == 0) record_status(status, kDevBadSlot);
+        live = false;
+        row = 0;
+      }
+      wr[u] = live ? wts[r] : 0.f;
+      const T* rp = values + static_cast<int64_t>(row) * v;
+#pragma unroll
+      for (int m = 0; m < MAXV; ++m) {
+        const int vec = lane + 32 * m;
+        raw[u][m] = (live && vec < nvec) ? ld_stream_v4(rp + vec * VPER) : make_uint4(0, 0, 0, 0);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int m = 0; m < MAXV; ++m) {
+        float f[VPER];
+        Vec<T>::widen(raw[u][m], f);
+#pragma unroll
+        for (int e = 0; e < VPER; ++e) acc[m][e] = fmaf(wr[u], f[e], acc[m][e]);
+      }
+  }
+  float* my = red + warp * v;
+#pragma unroll
+  for (int m = 0; m < MAXV; ++m) {
+    const int vec = lane + 32 * m;
+    if (vec < nvec) {
+#pragma unroll
+      for (int e = 0; e < VPER; ++e) my[vec * VPER + e] = acc[m][e];
+    }
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < v; c += blockDim.x) {
+    float sum = 0.f;
+#pragma unroll
+    for (int w = 0; w < kSmallWarps; ++w) sum += red[w * v + c];
+    part[c] = sum;
+  }
+
+  // (d) heads summed in head order, each CTA of the cluster taking one slice of the
+  // columns (all H partial rows of a column read together from the cluster's
+  // shared memory).
+  cg::cluster_group cluster = cg::this_cluster();
+  cluster.sync();
+  const int slice = (v + H - 1) / H;
+  const int c1 = min(v, (h + 1) * slice);
+  for (int c = h * slice + threadIdx.x; c < c1; c += blockDim.x) {
+    float pv[8];
+#pragma unroll
+    for (int hh = 0; hh < 8; ++hh)
+      pv[hh] = hh < H ? cluster.map_shared_rank(part, hh)[c] : 0.f;
+    float sum = pv[0];
+#pragma unroll
+    for (int hh = 1; hh < 8; ++hh)
+      if (hh < H) sum += pv[hh];
+    out[t * v + c] = sum;
+  }
+  cluster.sync();
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+static int maxv_small(int v, int dtype) {
+  const int per = dtype == 0 ? 4 : 8;
+  const int m = (v / per + 31) / 32;
+  if (m <= 1) return 1;
+  if (m <= 2) return 2;
+  if (m <= 4) return 4;
+  if (m <= 8) return 8;
+  return 0;
+}
+
+static size_t query_small_smem(int d, int dtype) {
+  return static_cast<size_t>(kQFeat + kQTok) * d * (dtype == 0 ? 4 : 2);
+}
+static size_t score_small_smem(int dq, int dtype) {
+  const int half = dq / 2;
+  const size_t esz = dtype == 0 ? 4 : 2;
+  const size_t rows = (esz * kSChunk * (half + (esz == 2 ? 2 : 1)) + 15) & ~static_cast<size_t>(15);
+  return rows + sizeof(float) * kSmallWarps * 2 * half;
+}
+static size_t gather_small_smem(int n, int v) {
+  const size_t list_words = static_cast<size_t>(2) * ((n + kSChunk - 1) / kSChunk) * kMaxK;
+  const size_t scratch = std::max(static_cast<size_t>(kSmallWarps) * v, 2 * list_words);
+  return sizeof(float) * (v + scratch) + kMaxPairs * 8 + kMaxK * 8 + sizeof(int) * kMaxPairs;
+}
+
+bool small_supported(int64_t B, int d_model, int H, int dq, int n, int k, int v, int dtype) {
+  constexpr size_t kLimit = 200 * 1024;
+  const int esz = dtype == 0 ? 4 : 2;
+  // Staging copies whole 32-bit words of W_q rows and sub-key rows.
+  if ((static_cast<int64_t>(d_model) * esz) % 4 || (static_cast<int64_t>(dq / 2) * esz) % 4)
+    return false;
+  return B >= 1 && B <= kSmallMaxB && k <= kMaxK && maxv_small(v, dtype) > 0 &&
+         query_small_smem(d_model, dtype) <= kLimit && score_small_smem(dq, dtype) <= kLimit &&
+         gather_small_smem(n, v) <= kLimit && n >= 1 && H <= 8;  // H CTAs per cluster
+}
+
+size_t small_chunk_entries(int64_t B, int H, int n) {
+  return static_cast<size_t>(B) * H * 2 * ((n + kSChunk - 1) / kSChunk) * kMaxK;
+}
+
+template <typename T, int MAXV>
+static cudaError_t launch_gather_small(const LayerArgs& a, const float* cs, const int* ci,
+                                       float* out, int* idx, float* w, float* sc,
+                                       cudaStream_t st) {
+  const size_t smem = gather_small_smem(a.n, a.v);
+  cudaError_t e = set_max_smem(reinterpret_cast<const void*>(gather_small_kernel<T, MAXV>), smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(a.B), a.H, 1);
+  cfg.blockDim = dim3(kSmallWarps * 32, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = a.H;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, gather_small_kernel<T, MAXV>, cs, ci,
+                            static_cast<const T*>(a.values), a.H, a.n, a.k, a.v, out, idx, w,
+                            sc, a.status);
+}
+
+template <typename T>
+static cudaError_t launch_small_t(const LayerArgs& a, float* q, float* cs, int* ci, float* out,
+                                  int* idx, float* w, float* sc, cudaStream_t st) {
+  const int F = a.H * a.dq;
+  const int B = static_cast<int>(a.B);
+  size_t smem = query_small_smem(a.d_model, a.dtype);
+  cudaError_t e = set_max_smem(reinterpret_cast<const void*>(query_small_kernel<T>), smem);
+  if (e != cudaSuccess) return e;
+  dim3 gq((F + kQFeat - 1) / kQFeat, (B + kQTok - 1) / kQTok);
+  query_small_kernel<T><<<gq, kSmallWarps * 32, smem, st>>>(
+      static_cast<const T*>(a.x), static_cast<const T*>(a.W_q), a.bn_mean, a.bn_var, a.bn_gamma,
+      a.bn_beta, a.bn_eps, B, a.d_model, F, q);
+  smem = score_small_smem(a.dq, a.dtype);
+  e = set_max_smem(reinterpret_cast<const void*>(score_small_kernel<T>), smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((a.n + kSChunk - 1) / kSChunk, a.H * 2, (B + kSTok - 1) / kSTok);
+  cfg.blockDim = dim3(kSmallWarps * 32, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, score_small_kernel<T>, static_cast<const float*>(q),
+                         static_cast<const T*>(a.subkeys), B, a.H, a.dq, a.n, cs, ci);
+  if (e != cudaSuccess) return e;
+  switch (maxv_small(a.v, a.dtype)) {
+    case 1: return launch_gather_small<T, 1>(a, cs, ci, out, idx, w, sc, st);
+    case 2: return launch_gather_small<T, 2>(a, cs, ci, out, idx, w, sc, st);
+    case 4: return launch_gather_small<T, 4>(a, cs, ci, out, idx, w, sc, st);
+    case 8: return launch_gather_small<T, 8>(a, cs, ci, out, idx, w, sc, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_forward_small(const LayerArgs& a, float* q, float* chunk_s, int* chunk_i,
+                                 float* out, int* idx, float* w, float* sc, cudaStream_t st) {
+  if (a.dtype == 0) return launch_small_t<float>(a, q, chunk_s, chunk_i, out, idx, w, sc, st);
+  return launch_small_t<uint16_t>(a, q, chunk_s, chunk_i, out, idx, w, sc, st);
+}
+
+}  // namespace pkm

@@ -722,8 +722,7 @@ cudaError_t launch_query_tc(const LayerArgs& a, void* planes, cudaStream_t st) {
       !make_map(&tm_out, planes, 3, od, os, ob, CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
   const size_t smem = query_tc_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(query_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  cudaError_t e = set_max_smem(reinterpret_cast<const void*>(query_tc_kernel), smem);
   if (e != cudaSuccess) return e;
   const int64_t tiles = ((a.B + kRowsPerTile - 1) / kRowsPerTile) * (F / kColsPerMma);
   const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
@@ -750,9 +749,7 @@ cudaError_t launch_score_topk_tc(const LayerArgs& a, const void* planes, float* 
       !make_map(&tm_k, a.subkeys, 2, kd, ks, kbx, kSSwizzle))
     return cudaErrorInvalidValue;
   const size_t smem = score_tc_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(score_topk_tc_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  cudaError_t e = set_max_smem(reinterpret_cast<const void*>(score_topk_tc_kernel), smem);
   if (e != cudaSuccess) return e;
   const int64_t units = ((a.B + kRowsPerTile - 1) / kRowsPerTile) * 2 * a.H;
   const int grid = static_cast<int>(units < sm_count() ? units : sm_count());

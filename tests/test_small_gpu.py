@@ -1,0 +1,111 @@
+"""GPU parity of the small-batch forward (B <= 64 tokens: pkm_forward picks the
+small-batch kernels by itself) against the fp64 oracle, through the C ABI.
+
+Same bar as tests/test_forward_gpu.py: indices bit-exact except fp64 near-ties
+within 1e-5 relative of the k-th score; weights, kept scores and out within
+1e-4 + 2e-3 |ref|.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from parity import compare_forward, to_numpy
+
+pytestmark = pytest.mark.gpu
+
+
+def _P():
+    import product_key_memory_b200 as mod
+    return mod
+
+
+def _forward(L, w, path=None):
+    old = os.environ.get("PKM_PATH")
+    if path is None:
+        os.environ.pop("PKM_PATH", None)
+    else:
+        os.environ["PKM_PATH"] = path
+    try:
+        d = {k: v.cuda() for k, v in L.items()}
+        out, idx, wt, sc = _P().pkm_forward(d["x"], d["W_q"], d["bn_mean"], d["bn_var"],
+                                            d["bn_gamma"], d["bn_beta"], d["subkeys"],
+                                            d["values"], k=w.k)
+        torch.cuda.synchronize()
+        return to_numpy(out, idx, wt, sc)
+    finally:
+        if old is None:
+            os.environ.pop("PKM_PATH", None)
+        else:
+            os.environ["PKM_PATH"] = old
+
+
+def _check(L, w):
+    g = _forward(L, w)
+    r = oracle.forward(L, w.H, w.dq, w.n, w.k, want_half=True)
+    stats = compare_forward(g, r, L["values"], w.n)
+    print(w.name, w.B, stats)
+    return g, r
+
+
+@pytest.mark.parametrize("B", [1, 7, 64])
+def test_c1024_small_batches(B):
+    w = synth.WORKLOADS["c1024"].with_(B=B)
+    _check(synth.make_layer(w), w)
+
+
+@pytest.mark.parametrize("name,B", [("c512", 33), ("wide", 16), ("tiny", 5)])
+def test_other_shapes(name, B):
+    w = synth.WORKLOADS[name].with_(B=B)
+    _check(synth.make_layer(w), w)
+
+
+@pytest.mark.parametrize("k,n", [(1, 256), (3, 256), (8, 8), (32, 32)])
+def test_k_and_small_codebooks(k, n):
+    w = synth.WORKLOADS["c512"].with_(B=9, n=n, k=k)
+    _check(synth.make_layer(w), w)
+
+
+def test_exact_ties_go_to_lower_slot():
+    w = synth.WORKLOADS["c512"].with_(B=12, n=256)
+    L = synth.make_layer(w)
+    L["subkeys"][:, 0] = L["subkeys"][:, 0, :1]
+    g = _forward(L, w)
+    r = oracle.forward(L, w.H, w.dq, w.n, w.k, want_half=True)
+    jstar = r["half"][:, :, 1].argmax(-1)
+    expect = np.arange(w.k)[None, None, :] * w.n + jstar[..., None]
+    np.testing.assert_array_equal(g["indices"], expect)
+    np.testing.assert_allclose(g["weights"], 1.0 / w.k, rtol=1e-6)
+
+
+def test_small_and_tensor_core_paths_agree():
+    """The same 48 tokens through the small-batch kernels and the large-batch
+    tensor-core kernels: identical picks except fp32 near-ties."""
+    w = synth.WORKLOADS["c1024"].with_(B=48)
+    L = synth.make_layer(w)
+    a = _forward(L, w)
+    b = _forward(L, w, "tc")
+    same = (a["indices"] == b["indices"]).all(-1)
+    assert same.mean() > 0.98
+    ok = same[..., None].repeat(w.k, -1)
+    np.testing.assert_allclose(a["weights"][ok], b["weights"][ok], rtol=2e-3, atol=1e-4)
+    np.testing.assert_allclose(a["out"][same.all(-1)], b["out"][same.all(-1)], rtol=2e-3, atol=1e-4)
+
+
+def test_forward_train_small_batch():
+    """BatchNorm training mode on 8 tokens runs the small-batch forward."""
+    w = synth.WORKLOADS["c512"].with_(B=8)
+    L = synth.make_layer(w)
+    d = {k: v.cuda() for k, v in L.items()}
+    rm, rv = d["bn_mean"].clone(), d["bn_var"].clone()
+    out, idx, wt, sc, bm, bv = _P().pkm_forward_train(d["x"], d["W_q"], rm, rv, d["bn_gamma"],
+                                                      d["bn_beta"], d["subkeys"], d["values"],
+                                                      k=w.k)
+    torch.cuda.synchronize()
+    r = oracle.forward_train(L, w.H, w.dq, w.n, w.k, want_half=True)
+    compare_forward(to_numpy(out, idx, wt, sc), r, L["values"], w.n)
+    np.testing.assert_allclose(bm.cpu().numpy(), r["batch_mean"], rtol=2e-3, atol=1e-4)
+    np.testing.assert_allclose(rv.cpu().numpy(), r["running_var"], rtol=2e-3, atol=1e-4)
