@@ -18,6 +18,8 @@
 
 namespace pkm {
 
+constexpr int kAccQSmemF = 4096;  // features whose BN scale/shift acc_q_kernel stages
+
 // acc = x W_q^T and q = acc * s + (beta - mean * s), s = gamma / sqrt(var + eps) (the
 // forward's query epilogue). With planes, acc = hi + mid + lo from the three bf16 planes
 // of the tensor-core query kernel; without, acc is read as is. Eight features per
@@ -28,6 +30,16 @@ __global__ void __launch_bounds__(256) acc_q_kernel(
     const float* __restrict__ gamma, const float* __restrict__ beta, float eps, int B, int F) {
   const int64_t count = static_cast<int64_t>(B) * F;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  extern __shared__ float aq_smem[];  // scale [F], shift [F] when F <= kAccQSmemF
+  const bool staged = F <= kAccQSmemF;
+  if (staged) {
+    for (int f = threadIdx.x; f < F; f += blockDim.x) {
+      const float sc = gamma[f] / sqrtf(var[f] + eps);
+      aq_smem[f] = sc;
+      aq_smem[F + f] = beta[f] - mean[f] * sc;
+    }
+    __syncthreads();
+  }
   if ((F & 7) == 0) {
     const int per_row = F >> 3;
     const int64_t units = static_cast<int64_t>(B) * per_row;
@@ -56,8 +68,12 @@ __global__ void __launch_bounds__(256) acc_q_kernel(
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const int f = f0 + j;
-        const float sc = gamma[f] / sqrtf(var[f] + eps);
-        r[j] = fmaf(a[j], sc, beta[f] - mean[f] * sc);
+        if (staged) {
+          r[j] = fmaf(a[j], aq_smem[f], aq_smem[F + f]);
+        } else {
+          const float sc = gamma[f] / sqrtf(var[f] + eps);
+          r[j] = fmaf(a[j], sc, beta[f] - mean[f] * sc);
+        }
       }
       reinterpret_cast<float4*>(q + i0)[0] = make_float4(r[0], r[1], r[2], r[3]);
       reinterpret_cast<float4*>(q + i0)[1] = make_float4(r[4], r[5], r[6], r[7]);
@@ -100,6 +116,28 @@ __device__ __forceinline__ void load_run(const float* p, float (&v)[VW]) {
   } else {
 #pragma unroll
     for (int i = 0; i < VW; ++i) v[i] = p[i];
+  }
+}
+
+// VW consecutive fp32 values to p (two 16-byte stores in the vector form; p is then
+// 32-byte aligned), optionally added atomically.
+template <int VW>
+__device__ __forceinline__ void store_run(float* p, const float (&v)[VW], bool atomic) {
+  if constexpr (VW == 8) {
+    const float4 a = make_float4(v[0], v[1], v[2], v[3]), b = make_float4(v[4], v[5], v[6], v[7]);
+    if (atomic) {
+      atomicAdd(reinterpret_cast<float4*>(p), a);
+      atomicAdd(reinterpret_cast<float4*>(p) + 1, b);
+    } else {
+      reinterpret_cast<float4*>(p)[0] = a;
+      reinterpret_cast<float4*>(p)[1] = b;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < VW; ++i) {
+      if (atomic) atomicAdd(p + i, v[i]);
+      else p[i] = v[i];
+    }
   }
 }
 
@@ -174,17 +212,36 @@ __global__ void __launch_bounds__(128) grad_q_targets_kernel(
       }
       if (e < half) {
         const int64_t o = t * F + f0 + e;
+        float ga[VW];
+        uint16_t ph[VW], pl[VW];
 #pragma unroll
         for (int i = 0; i < VW; ++i) {
           const int f = f0 + e + i;
-          g_q[o + i] = acc[i];
-          const float ga = acc[i] * (gamma[f] / sqrtf(var[f] + eps));
-          if (g_acc) g_acc[o + i] = ga;
-          if (g_planes) {  // hi + lo within 2^-18 relative of ga, for the bf16 GEMMs
-            const __nv_bfloat16 hi = __float2bfloat16_rn(ga);
-            const __nv_bfloat16 lo = __float2bfloat16_rn(ga - __bfloat162float(hi));
-            g_planes[o + i] = __bfloat16_as_ushort(hi);
-            g_planes[B * F + o + i] = __bfloat16_as_ushort(lo);
+          ga[i] = acc[i] * (gamma[f] / sqrtf(var[f] + eps));
+          // hi + lo within 2^-18 relative of ga, for the bf16 GEMMs
+          const __nv_bfloat16 hi = __float2bfloat16_rn(ga[i]);
+          const __nv_bfloat16 lo = __float2bfloat16_rn(ga[i] - __bfloat162float(hi));
+          ph[i] = __bfloat16_as_ushort(hi);
+          pl[i] = __bfloat16_as_ushort(lo);
+        }
+        store_run<VW>(g_q + o, acc, false);
+        if (g_acc) store_run<VW>(g_acc + o, ga, false);
+        if (g_planes) {
+          if constexpr (VW == 8) {
+            auto pack = [](const uint16_t (&u)[VW]) {
+              return make_uint4(u[0] | (static_cast<uint32_t>(u[1]) << 16),
+                                u[2] | (static_cast<uint32_t>(u[3]) << 16),
+                                u[4] | (static_cast<uint32_t>(u[5]) << 16),
+                                u[6] | (static_cast<uint32_t>(u[7]) << 16));
+            };
+            *reinterpret_cast<uint4*>(g_planes + o) = pack(ph);
+            *reinterpret_cast<uint4*>(g_planes + B * F + o) = pack(pl);
+          } else {
+#pragma unroll
+            for (int i = 0; i < VW; ++i) {
+              g_planes[o + i] = ph[i];
+              g_planes[B * F + o + i] = pl[i];
+            }
           }
         }
       }
@@ -216,15 +273,35 @@ __global__ void bn_grad_partial_kernel(const float* __restrict__ g_q, const floa
   part[static_cast<int64_t>(blockIdx.y) * 2 * F + F + f] = sg;
 }
 
-__global__ void bn_grad_final_kernel(const float* __restrict__ part, int F,
-                                     float* __restrict__ grad_gamma, float* __restrict__ grad_beta,
-                                     float* __restrict__ sums) {
-  const int f = blockIdx.x * blockDim.x + threadIdx.x;
-  if (f >= F) return;
+// Pass 2: block = 32 features x 8 warps; warp w adds chunks [16 w, 16 w + 16) in
+// order, then warp 0 adds the 8 warp sums in order (a fixed order: deterministic).
+constexpr int kBnFinalWarps = 8;
+static_assert(kBnChunks % kBnFinalWarps == 0, "chunks split evenly over the warps");
+
+__global__ void __launch_bounds__(kBnFinalWarps * 32) bn_grad_final_kernel(
+    const float* __restrict__ part, int F, float* __restrict__ grad_gamma,
+    float* __restrict__ grad_beta, float* __restrict__ sums) {
+  __shared__ float wb[kBnFinalWarps][32], wg[kBnFinalWarps][32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int f = blockIdx.x * 32 + lane;
+  constexpr int per = kBnChunks / kBnFinalWarps;
+  float pb = 0.f, pg = 0.f;
+  if (f < F) {
+#pragma unroll 4
+    for (int c = warp * per; c < (warp + 1) * per; ++c) {
+      pb += part[static_cast<int64_t>(c) * 2 * F + f];
+      pg += part[static_cast<int64_t>(c) * 2 * F + F + f];
+    }
+  }
+  wb[warp][lane] = pb;
+  wg[warp][lane] = pg;
+  __syncthreads();
+  if (warp != 0 || f >= F) return;
   float sb = 0.f, sg = 0.f;
-  for (int c = 0; c < kBnChunks; ++c) {
-    sb += part[static_cast<int64_t>(c) * 2 * F + f];
-    sg += part[static_cast<int64_t>(c) * 2 * F + F + f];
+#pragma unroll
+  for (int w = 0; w < kBnFinalWarps; ++w) {
+    sb += wb[w][lane];
+    sg += wg[w][lane];
   }
   if (grad_beta) grad_beta[f] = sb;
   if (grad_gamma) grad_gamma[f] = sg;
@@ -300,15 +377,7 @@ __global__ void __launch_bounds__(128) segment_subkeys_kernel(
             for (int m = 0; m < VW; ++m) sum[m] = fmaf(ca, ra[m], sum[m]);
           }
         }
-        if (in) {
-          if (whole) {
-#pragma unroll
-            for (int m = 0; m < VW; ++m) grow[e + m] = sum[m];
-          } else {
-#pragma unroll
-            for (int m = 0; m < VW; ++m) atomicAdd(grow + e + m, sum[m]);
-          }
-        }
+        if (in) store_run<VW>(grow + e, sum, !whole);
       }
       i = end;
     }
@@ -468,7 +537,8 @@ static cudaError_t launch_full_t(const LayerArgs& a, bool tensor_path, bool bn_t
     e = launch_query_bn_simt(raw, w.acc, st);
   }
   if (e != cudaSuccess) return e;
-  acc_q_kernel<<<grid_of((a.B * F / 8 + 255) / 256, 148 * 8), 256, 0, st>>>(
+  const size_t aq_smem = F <= kAccQSmemF ? sizeof(float) * 2 * F : 0;
+  acc_q_kernel<<<grid_of((a.B * F / 8 + 255) / 256, 148 * 8), 256, aq_smem, st>>>(
       tensor_path ? static_cast<const uint16_t*>(w.planes) : nullptr, w.acc, w.q, a.bn_mean,
       a.bn_var, a.bn_gamma, a.bn_beta, a.bn_eps, static_cast<int>(a.B), static_cast<int>(F));
   *launches += 2;
@@ -492,7 +562,7 @@ static cudaError_t launch_full_t(const LayerArgs& a, bool tensor_path, bool bn_t
     dim3 g1(static_cast<unsigned>((F + 255) / 256), kBnChunks);
     bn_grad_partial_kernel<<<g1, 256, 0, st>>>(w.g_q, w.acc, a.bn_mean, a.bn_var, a.bn_eps, a.B,
                                                static_cast<int>(F), w.bn_part);
-    bn_grad_final_kernel<<<static_cast<unsigned>((F + 255) / 256), 256, 0, st>>>(
+    bn_grad_final_kernel<<<static_cast<unsigned>((F + 31) / 32), kBnFinalWarps * 32, 0, st>>>(
         w.bn_part, static_cast<int>(F), grad_gamma, grad_beta, bn_training ? w.bn_sums : nullptr);
     *launches += 2;
   }
