@@ -47,9 +47,12 @@ FLUSH_BYTES = 256 << 20
 # DRAM bytes per launch of the dominant kernel from an ncu capture
 # (profiles/select_gather_c1024.md), keyed by the sha256 of the kernel's source at
 # capture time; reported as null once the source has changed.
+# DRAM bytes (read + write) of one select_gather launch, from an ncu capture, keyed by
+# (kernel_sha(), workload, tokens); None once the kernel source changes.
 TRAFFIC = {
-    # c1024, 4096 tokens: dram read 971.2 MB + write 5.4 MB, scaled x4 to 16384 tokens.
-    ("004aa70f33fc1f1e", "c1024"): 3.906e9,
+    # c1024 at 4096 tokens: dram read 961.1 MB + write 6.5 MB, scaled x4 to the
+    # 16384-token launch (the gather's traffic grows with the tokens).
+    ("54feafc4d4ae7967", "c1024", 16384): 3.870e9,
 }
 
 
@@ -196,10 +199,11 @@ def run_reference(args, rank, world):
 
 # ----------------------------------------------------------------- our arm
 def kernel_sha() -> str:
+    """Hash of the gather kernel's source (its file and the selection header)."""
     h = hashlib.sha256()
-    with open(os.path.join(ROOT, "product_key_memory_b200", "csrc", "pkm_select_gather.cu"),
-              "rb") as f:
-        h.update(f.read())
+    for name in ("pkm_select_gather.cu", "pkm_select.cuh"):
+        with open(os.path.join(ROOT, "product_key_memory_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
@@ -211,6 +215,11 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     w = synth.WORKLOADS[args.workload]
     L = synth.make_layer(w)
+    if args.tokens is not None:
+        if not 1 <= args.tokens <= w.B:
+            raise SystemExit("--tokens must be in [1, %d]" % w.B)
+        w = w.with_tokens(args.tokens)
+        L["x"] = L["x"][:args.tokens].contiguous()
     d = {k: v.to(dev) for k, v in L.items()}
     B = w.B
     out = torch.empty(B, w.v, dtype=torch.float32, device=dev)
@@ -276,7 +285,7 @@ def run_ours(args, rank, world, local_rank):
         alg = per_token_bytes(w) * B
         achieved = alg / (stage_avg[2] * 1e-3) / 1e9
         sha = kernel_sha()
-        tr = TRAFFIC.get((sha, w.name))
+        tr = TRAFFIC.get((sha, w.name, B))
         roof = {"kernel": names[2], "bound": "hbm", "achieved": achieved, "peak": hbm,
                 "unit": "GB/s", "frac": achieved / hbm, "traffic": tr,
                 "algorithmic_bytes_per_launch": alg, "ms_per_launch": stage_avg[2],
@@ -601,6 +610,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="c1024", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="tokens per step instead of the workload's (the first B rows of "
+                         "its seeded input; for profiling a smaller case of the same layer)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the c512 / backward / CPU-oracle measurements")
     ap.add_argument("--part", default=None,
