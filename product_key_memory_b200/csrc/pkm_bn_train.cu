@@ -90,21 +90,24 @@ cudaError_t launch_bn_batch_stats(const uint16_t* planes, const float* acc, int6
 
 // dL/dacc with batch statistics, from g = dL/dq, acc and the column sums
 // sums[0][f] = sum_t g, sums[1][f] = sum_t g xhat. Written as fp32 (g_acc) and/or bf16
-// hi/lo planes [2][B][F] for the tensor-core GEMMs.
+// hi/lo planes [2][B][F] for the tensor-core GEMMs. Thread = one feature (its BN
+// constants in registers), rows strided over grid.y.
 __global__ void __launch_bounds__(256) bn_train_dacc_kernel(
     const float* __restrict__ g_q, const float* __restrict__ acc,
     const float* __restrict__ mean, const float* __restrict__ var,
     const float* __restrict__ gamma, const float* __restrict__ sums, float eps, int B, int F,
     float* __restrict__ g_acc, uint16_t* __restrict__ g_planes) {
+  const int f = blockIdx.x * blockDim.x + threadIdx.x;
+  if (f >= F) return;
   const int64_t count = static_cast<int64_t>(B) * F;
   const float inv_b = 1.f / static_cast<float>(B);
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < count;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int f = static_cast<int>(i % F);
-    const float rs = 1.f / sqrtf(var[f] + eps);
-    const float xhat = (acc[i] - mean[f]) * rs;
-    const float ga =
-        gamma[f] * rs * (g_q[i] - sums[f] * inv_b - xhat * (sums[F + f] * inv_b));
+  const float rs = 1.f / sqrtf(var[f] + eps);
+  const float mu = mean[f], gs = gamma[f] * rs;
+  const float mb = sums[f] * inv_b, mg = sums[F + f] * inv_b;
+  for (int t = blockIdx.y; t < B; t += gridDim.y) {
+    const int64_t i = static_cast<int64_t>(t) * F + f;
+    const float xhat = (acc[i] - mu) * rs;
+    const float ga = gs * (g_q[i] - mb - xhat * mg);
     if (g_acc) g_acc[i] = ga;
     if (g_planes) {
       const __nv_bfloat16 hi = __float2bfloat16_rn(ga);
@@ -119,10 +122,10 @@ cudaError_t launch_bn_train_dacc(const float* g_q, const float* acc, const float
                                  const float* var, const float* gamma, const float* sums,
                                  float eps, int64_t B, int F, float* g_acc, uint16_t* g_planes,
                                  cudaStream_t st) {
-  const int64_t blocks = (B * F + 255) / 256;
-  bn_train_dacc_kernel<<<static_cast<unsigned>(blocks < 148 * 8 ? blocks : 148 * 8), 256, 0,
-                         st>>>(g_q, acc, mean, var, gamma, sums, eps, static_cast<int>(B), F,
-                               g_acc, g_planes);
+  const unsigned gx = static_cast<unsigned>((F + 255) / 256);
+  const unsigned gy = static_cast<unsigned>(B < 1024 ? B : 1024);
+  bn_train_dacc_kernel<<<dim3(gx, gy), 256, 0, st>>>(g_q, acc, mean, var, gamma, sums, eps,
+                                                     static_cast<int>(B), F, g_acc, g_planes);
   return cudaGetLastError();
 }
 

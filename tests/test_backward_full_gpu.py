@@ -214,3 +214,15 @@ def test_zero_tokens():
     torch.cuda.synchronize()
     # a sum over no tokens: the requested parameter gradients are zero
     assert torch.all(gW == 0.0)
+
+
+@pytest.mark.parametrize("path", ["auto", "simt"])
+def test_wide_layer_ragged_gemm_tiles(path):
+    """d_model 1600, H = 8, v = 1600: the GEMMs' N = 1600 leaves a ragged 256-column
+    tile, K = 200 tokens a ragged 64-row block, and the small output splits K."""
+    w = synth.WORKLOADS["wide"].with_(B=200, n=256)
+    L = synth.make_layer(w)
+    gout = synth.make_grad_out(w)
+    idx, wt, g = _device_forward_backward(L, w, gout, path=path,
+                                          want=("x", "W_q", "bn_gamma", "bn_beta", "subkeys"))
+    _compare_all(L, w, idx, wt, gout, g, _oracle_full(L, idx, wt, gout, w, chunks=4))
