@@ -49,7 +49,7 @@ typedef enum { PKM_F32 = 0, PKM_BF16 = 1 } pkm_dtype;
 enum {
   PKM_OK = 0,
   PKM_ERR_INVALID_ARG = -1, /* NULL pointer, size out of range, k > n, odd dq, n*n > 2^31-1 */
-  PKM_ERR_UNSUPPORTED = -2, /* valid layer this build does not run (k > 32, v not a multiple of
+  PKM_ERR_UNSUPPORTED = -2, /* valid layer this library does not run (k > 32, v not a multiple of
                                16 bytes, misaligned pointer) */
   PKM_ERR_WORKSPACE = -3,   /* workspace NULL or smaller than pkm_workspace_size() */
   PKM_ERR_CUDA = -4,        /* a CUDA runtime call or kernel launch failed */
