@@ -218,14 +218,15 @@ __global__ void slot_scatter_kernel(const int* __restrict__ indices, int64_t E, 
 }
 
 // ----------------------------------------------------------- segmented row sums
-// One warp per window of 32 sorted picks. offsets has slots + 1 entries; its last
-// entry is the number of valid picks.
+// One warp per window of 32 sorted picks; total_ptr points at the number of valid
+// picks (the last entry of the sort's offsets). Group bounds inside the window come from the
+// sorted keys themselves (a ballot on key changes); the keys just before and after
+// the window tell whether the first and last groups continue into a neighbour.
 template <typename T, int MAXV>
 __global__ void __launch_bounds__(128) segment_rows_kernel(
-    const int* __restrict__ order, const int* __restrict__ offsets,
-    const int* __restrict__ total_ptr, const int* __restrict__ indices,
-    const float* __restrict__ weights, const T* __restrict__ grad_out, int HK, int v,
-    float* __restrict__ grad_values) {
+    const int* __restrict__ order, const int* __restrict__ total_ptr,
+    const int* __restrict__ indices, const float* __restrict__ weights,
+    const T* __restrict__ grad_out, int HK, int v, float* __restrict__ grad_values) {
   constexpr int VPER = Vec<T>::kPer;
   const int lane = threadIdx.x & 31;
   const int total = *total_ptr;
@@ -235,19 +236,25 @@ __global__ void __launch_bounds__(128) segment_rows_kernel(
        win * 32 < total; win += nwarps) {
     const int w0 = static_cast<int>(win * 32);
     const int w1 = min(w0 + 32, total);
-    int e_l = 0, r_l = 0;
+    int e_l = 0, r_l = -1;
     float wt_l = 0.f;
     if (w0 + lane < w1) {
       e_l = order[w0 + lane];
       r_l = indices[e_l];
       wt_l = weights[e_l];
     }
+    // Keys of the picks just outside the window (-1: none).
+    int edge = -1;
+    if (lane == 0 && w0 > 0) edge = indices[order[w0 - 1]];
+    if (lane == 1 && w1 < total) edge = indices[order[w1]];
+    const int prev_r = __shfl_sync(0xffffffffu, edge, 0);
+    const int next_r = __shfl_sync(0xffffffffu, edge, 1);
     int i = w0;
     while (i < w1) {
       const int r = __shfl_sync(0xffffffffu, r_l, i - w0);
-      const int seg0 = offsets[r], seg1 = offsets[r + 1];
-      const int end = min(seg1, w1);
-      const bool whole = seg0 >= w0 && seg1 <= w1;
+      const unsigned change = __ballot_sync(0xffffffffu, lane > i - w0 && r_l != r);
+      const int end = change ? w0 + __ffs(change) - 1 : w1;
+      const bool whole = (i > w0 || prev_r != r) && (end < w1 || next_r != r);
       float* grow = grad_values + static_cast<int64_t>(r) * v;
       // A slot group that lies inside this window is owned by this warp: load its row
       // now so the HBM read overlaps the sums below. A group that crosses a window edge
@@ -378,7 +385,7 @@ static cudaError_t launch_bwd_t(int64_t B, int H, int k, int v, int64_t slots, c
   const int64_t sblocks = (windows + 3) / 4;
   const unsigned sgrid = static_cast<unsigned>(sblocks < 148 * 64 ? sblocks : 148 * 64);
   segment_rows_kernel<T, MAXV><<<sgrid > 0 ? sgrid : 1, 128, 0, st>>>(
-      ws.order, ws.offsets, ws.offsets + slots, indices, weights, G, H * k, v, grad_values);
+      ws.order, ws.offsets + slots, indices, weights, G, H * k, v, grad_values);
   return cudaGetLastError();
 }
 

@@ -317,9 +317,9 @@ __global__ void __launch_bounds__(kBnFinalWarps * 32) bn_grad_final_kernel(
 // written once (the table was zeroed); groups crossing a window edge add atomically.
 template <int VW>
 __global__ void __launch_bounds__(128) segment_subkeys_kernel(
-    const int* __restrict__ order, const int* __restrict__ offsets,
-    const int* __restrict__ total_ptr, const int* __restrict__ targets,
-    const float* __restrict__ coef, const float* __restrict__ q, int H, int dq, int n, int k,
+    const int* __restrict__ order, const int* __restrict__ total_ptr,
+    const int* __restrict__ targets, const float* __restrict__ coef,
+    const float* __restrict__ q, int H, int dq, int n, int k,
     float* __restrict__ grad_subkeys) {
   const int lane = threadIdx.x & 31;
   const int total = *total_ptr;
@@ -329,7 +329,7 @@ __global__ void __launch_bounds__(128) segment_subkeys_kernel(
        win * 32 < total; win += nwarps) {
     const int w0 = static_cast<int>(win * 32);
     const int w1 = min(w0 + 32, total);
-    int tg_l = 0, t_l = 0;
+    int tg_l = -1, t_l = 0;
     float cf_l = 0.f;
     if (w0 + lane < w1) {
       const int c = order[w0 + lane];
@@ -337,12 +337,19 @@ __global__ void __launch_bounds__(128) segment_subkeys_kernel(
       cf_l = coef[c];
       t_l = (c >> 1) / HK;
     }
+    // Group bounds from the sorted keys; the keys just outside the window tell
+    // whether the first and last groups continue into a neighbour (-1: none).
+    int edge = -1;
+    if (lane == 0 && w0 > 0) edge = targets[order[w0 - 1]];
+    if (lane == 1 && w1 < total) edge = targets[order[w1]];
+    const int prev_t = __shfl_sync(0xffffffffu, edge, 0);
+    const int next_t = __shfl_sync(0xffffffffu, edge, 1);
     int i = w0;
     while (i < w1) {
       const int tg = __shfl_sync(0xffffffffu, tg_l, i - w0);
-      const int seg0 = offsets[tg], seg1 = offsets[tg + 1];
-      const int end = min(seg1, w1);
-      const bool whole = seg0 >= w0 && seg1 <= w1;
+      const unsigned change = __ballot_sync(0xffffffffu, lane > i - w0 && tg_l != tg);
+      const int end = change ? w0 + __ffs(change) - 1 : w1;
+      const bool whole = (i > w0 || prev_t != tg) && (end < w1 || next_t != tg);
       const int side = (tg / n) & 1;
       const int h = tg / (2 * n);
       const float* qbase = q + h * dq + side * half;
@@ -502,8 +509,8 @@ static void launch_segment_subkeys(const LayerArgs& a, int64_t E2, int64_t tslot
                                    float* grad_subkeys, const FullBackwardWs& w, cudaStream_t st) {
   const int64_t windows = (E2 + 31) / 32;
   segment_subkeys_kernel<VW><<<grid_of((windows + 3) / 4, 148 * 32), 128, 0, st>>>(
-      w.sub.order, w.sub.offsets, w.sub.offsets + tslots, w.targets, w.coef, w.q, a.H, a.dq, a.n,
-      a.k, grad_subkeys);
+      w.sub.order, w.sub.offsets + tslots, w.targets, w.coef, w.q, a.H, a.dq, a.n, a.k,
+      grad_subkeys);
 }
 
 template <typename T>
