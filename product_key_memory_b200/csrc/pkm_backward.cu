@@ -63,14 +63,18 @@ __global__ void __launch_bounds__(128) grad_scores_kernel(
   }
   for (int h = 0; h < H; ++h) {
     const int64_t base = (t * H + h) * static_cast<int64_t>(k);
+    // The head's slot ids, one per lane, handed out by shuffles (no dependent load
+    // before each group of row reads).
+    const int row_l = lane < k ? indices[base + lane] : 0;
     float gj = 0.f;
     for (int j0 = 0; j0 < k; j0 += U) {
       float part[U];
+      uint4 raw[U][MAXV];
+      // All U rows' loads are issued before any of them is used.
 #pragma unroll
       for (int u = 0; u < U; ++u) {
-        part[u] = 0.f;
         const bool live = j0 + u < k;
-        int row = live ? indices[base + j0 + u] : 0;
+        int row = __shfl_sync(0xffffffffu, row_l, (j0 + u) & 31);
         const bool ok = live && row >= 0 && row < slots;
         if (live && !ok && lane == 0) record_status(status, kDevBadSlot);
         if (!ok) row = 0;
@@ -78,12 +82,18 @@ __global__ void __launch_bounds__(128) grad_scores_kernel(
 #pragma unroll
         for (int m = 0; m < MAXV; ++m) {
           const int vec = lane + 32 * m;
-          if (ok && vec < nvec) {
-            float f[VPER];
-            Vec<T>::widen(ld_stream_v4(rp + vec * VPER), f);
+          raw[u][m] = (ok && vec < nvec) ? ld_stream_v4(rp + vec * VPER) : make_uint4(0, 0, 0, 0);
+        }
+      }
 #pragma unroll
-            for (int e = 0; e < VPER; ++e) part[u] = fmaf(f[e], g[m][e], part[u]);
-          }
+      for (int u = 0; u < U; ++u) {
+        part[u] = 0.f;
+#pragma unroll
+        for (int m = 0; m < MAXV; ++m) {
+          float f[VPER];
+          Vec<T>::widen(raw[u][m], f);
+#pragma unroll
+          for (int e = 0; e < VPER; ++e) part[u] = fmaf(f[e], g[m][e], part[u]);
         }
       }
 #pragma unroll
