@@ -16,7 +16,8 @@ from typing import Optional, Tuple
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libpkm.so")
+# PKM_LIBRARY selects another build of the library (the timeout test build).
+LIB_PATH = os.environ.get("PKM_LIBRARY") or os.path.join(_HERE, "libpkm.so")
 
 PKM_F32, PKM_BF16 = 0, 1
 PKM_OK = 0
@@ -50,7 +51,8 @@ def lib() -> ctypes.CDLL:
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
-            raise ImportError("libpkm.so not built: run python product_key_memory_b200/build.py")
+            raise ImportError("%s not built: run python product_key_memory_b200/build.py"
+                              % os.path.basename(LIB_PATH))
         L = ctypes.CDLL(LIB_PATH)
         P = ctypes.c_void_p
         S = ctypes.POINTER(pkm_shape)

@@ -21,6 +21,11 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libpkm.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
+# Test build: every pipeline wait of the tensor-core kernels gives up after 2 us (the
+# drains keep their full second), so tests can run the timeout path; see
+# tests/test_timeout_gpu.py. Loaded only through PKM_LIBRARY.
+WAITTEST_LIB = os.path.join(HERE, "libpkm_waittest.so")
+WAITTEST_DEFINES = ("-DPKM_WAIT_LIMIT_NS=2000ull", "-DPKM_TRY_WAIT_HINT_NS=100")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
@@ -42,12 +47,13 @@ def _stale(obj: str, src: str) -> bool:
     return any(os.path.getmtime(d) > os.path.getmtime(obj) for d in deps)
 
 
-def build(verbose: bool = False, force: bool = False, extra=()) -> str:
-    os.makedirs(BUILD_DIR, exist_ok=True)
+def build(verbose: bool = False, force: bool = False, extra=(), lib: str = LIB,
+          build_dir: str = BUILD_DIR) -> str:
+    os.makedirs(build_dir, exist_ok=True)
     objs = []
     procs = []
     for src in sorted(glob.glob(os.path.join(CSRC, "*.cu"))):
-        obj = os.path.join(BUILD_DIR, os.path.basename(src) + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src) + ".o")
         objs.append(obj)
         if force or _stale(obj, src):
             cmd = [nvcc(), *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
@@ -65,15 +71,22 @@ def build(verbose: bool = False, force: bool = False, extra=()) -> str:
     if failed:
         msg = "\n".join("%s:\n%s" % (s, o) for s, o in failed)
         raise RuntimeError("nvcc failed:\n" + msg)
-    if force or procs or not os.path.exists(LIB):
-        tmp = LIB + ".tmp%d" % os.getpid()
+    if force or procs or not os.path.exists(lib):
+        tmp = lib + ".tmp%d" % os.getpid()
         cmd = [nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]
         subprocess.check_call(cmd)
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
+
+
+def build_waittest(verbose: bool = False, force: bool = False) -> str:
+    return build(verbose, force, extra=WAITTEST_DEFINES, lib=WAITTEST_LIB,
+                 build_dir=os.path.join(BUILD_DIR, "waittest"))
 
 
 if __name__ == "__main__":
     build(verbose=True, force="--force" in sys.argv,
           extra=("-Xptxas", "-v") if "--ptxas-v" in sys.argv else ())
     print(LIB)
+    if "--no-waittest" not in sys.argv:
+        print(build_waittest(verbose=False, force="--force" in sys.argv))

@@ -155,7 +155,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_tc_kernel(
           if (issued[i]) {
             const uint64_t t0 = global_timer_ns();
             while (!mbar_try_wait(&full[i], issued_phase[i]) &&
-                   global_timer_ns() - t0 < kWaitLimitNs) {
+                   global_timer_ns() - t0 < kDrainLimitNs) {
             }
           }
       }
@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gemm_tc_kernel(
       }
       mma_commit(drain);
       const uint64_t t0 = global_timer_ns();
-      while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
+      while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < kDrainLimitNs) {
       }
     }
   } else {

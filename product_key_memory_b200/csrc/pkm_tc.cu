@@ -148,7 +148,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) query_tc_kernel(
           if (issued[i]) {
             const uint64_t t0 = global_timer_ns();
             while (!mbar_try_wait(&full[i], issued_phase[i]) &&
-                   global_timer_ns() - t0 < kWaitLimitNs) {
+                   global_timer_ns() - t0 < kDrainLimitNs) {
             }
           }
       }
@@ -184,7 +184,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) query_tc_kernel(
       // and writing TMEM before the CTA tears down.
       mma_commit(drain);
       const uint64_t t0 = global_timer_ns();
-      while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
+      while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < kDrainLimitNs) {
       }
     }
   } else {
@@ -419,7 +419,7 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
           if (issued[i]) {
             const uint64_t t0 = global_timer_ns();
             while (!mbar_try_wait(&full[i], issued_phase[i]) &&
-                   global_timer_ns() - t0 < kWaitLimitNs) {
+                   global_timer_ns() - t0 < kDrainLimitNs) {
             }
           }
       }
@@ -463,7 +463,7 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
           }
       mma_commit(drain);
       const uint64_t t0 = global_timer_ns();
-      while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
+      while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < kDrainLimitNs) {
       }
     }
   } else {

@@ -13,10 +13,17 @@
 namespace pkm {
 namespace tc {
 
-// A wait on a hardware barrier gives up after this long (globaltimer ns), records
-// kDevTimeout in the status word and reports failure so the kernel can drain and
-// exit instead of hanging the GPU.
-constexpr uint64_t kWaitLimitNs = 1000000000ull;
+// A wait on a hardware barrier of the pipeline gives up after this long (globaltimer
+// ns), records kDevTimeout in the status word and reports failure so the kernel can
+// drain and exit instead of hanging the GPU. A test build lowers it (and the
+// try_wait hint below) so that the timeout path runs.
+#ifndef PKM_WAIT_LIMIT_NS
+#define PKM_WAIT_LIMIT_NS 1000000000ull
+#endif
+constexpr uint64_t kWaitLimitNs = PKM_WAIT_LIMIT_NS;
+// Waits for a kernel's own copies and MMAs already in flight, before it frees TMEM
+// and exits, keep the full second in every build.
+constexpr uint64_t kDrainLimitNs = 1000000000ull;
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -50,7 +57,10 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 
 // Suspend-time hint of one try_wait: the thread sleeps in hardware until the phase
 // completes or this many ns pass, instead of spinning on the issue slots.
-constexpr uint32_t kTryWaitHintNs = 20000;
+#ifndef PKM_TRY_WAIT_HINT_NS
+#define PKM_TRY_WAIT_HINT_NS 20000
+#endif
+constexpr uint32_t kTryWaitHintNs = PKM_TRY_WAIT_HINT_NS;
 
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t done;
