@@ -3,6 +3,8 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include <mutex>
 #include <vector>
 
@@ -175,6 +177,14 @@ cudaEvent_t take_timing_event() {
   return e;
 }
 
+// NVTX range names of the traced stages (pass 0 forward, pass 1 backward).
+const char* stage_name(int pass, int stage) {
+  static const char* const kNames[kPasses][4] = {
+      {"pkm.forward.query", "pkm.forward.scores", "pkm.forward.gather", "pkm.forward"},
+      {"pkm.backward.scores", "pkm.backward.values", "pkm.backward.stage2", "pkm.backward"}};
+  return kNames[pass][stage & 3];
+}
+
 class Tracer {
  public:
   Tracer(int pass) {
@@ -182,8 +192,17 @@ class Tracer {
     on_ = g_trace_on;
     call_.pass = pass;
   }
-  // Spans nest: end() closes the most recently begun span that is still open.
+  ~Tracer() {
+    while (nvtx_open_ > 0) {
+      nvtxRangePop();
+      --nvtx_open_;
+    }
+  }
+  // Spans nest: end() closes the most recently begun span that is still open. Every
+  // span is also an NVTX range (host side; profilers attach the launches inside it).
   void begin(int stage, cudaStream_t st) {
+    nvtxRangePushA(stage_name(call_.pass, stage));
+    ++nvtx_open_;
     if (!on_) return;
     std::lock_guard<std::mutex> lk(g_trace_mu);
     TraceSpan sp{stage, take_timing_event(), take_timing_event()};
@@ -198,6 +217,10 @@ class Tracer {
     call_.spans.push_back(sp);
   }
   void end(cudaStream_t st) {
+    if (nvtx_open_ > 0) {
+      nvtxRangePop();
+      --nvtx_open_;
+    }
     if (!on_ || open_.empty()) return;
     cudaEventRecord(call_.spans[open_.back()].stop, st);
     open_.pop_back();
@@ -218,6 +241,7 @@ class Tracer {
 
  private:
   bool on_ = false;
+  int nvtx_open_ = 0;
   TraceCall call_;
   std::vector<size_t> open_;
 };
