@@ -46,27 +46,48 @@ __global__ void __launch_bounds__(256) bn_stats_partial_kernel(
   part[(static_cast<int64_t>(blockIdx.y) * 2 + 1) * F + f] = m2;
 }
 
-// Pass 2: merge the chunks in order (Chan, Golub and LeVeque's pairwise update of
-// count, mean and M2), write the batch statistics and move the running ones.
-__global__ void bn_stats_final_kernel(const double* __restrict__ part, int B, int F,
-                                      float momentum, float* __restrict__ batch_mean,
-                                      float* __restrict__ batch_var,
-                                      float* __restrict__ running_mean,
-                                      float* __restrict__ running_var) {
-  const int f = blockIdx.x * blockDim.x + threadIdx.x;
-  if (f >= F) return;
+// Chan, Golub and LeVeque's pairwise update: (n, mean, m2) absorbs (nb, mb, m2b).
+__device__ __forceinline__ void chan_merge(double& n, double& mean, double& m2, double nb,
+                                           double mb, double m2b) {
+  if (nb == 0.0) return;
+  const double tot = n + nb;
+  const double delta = mb - mean;
+  mean += delta * (nb / tot);
+  m2 += m2b + delta * delta * (n * nb / tot);
+  n = tot;
+}
+
+// Pass 2: block = 32 features x 8 warps; warp w merges its share of the chunks in
+// order, then warp 0 merges the 8 warp results in order (a fixed order:
+// deterministic). Writes the batch statistics and moves the running ones.
+constexpr int kStatWarps = 8;
+
+__global__ void __launch_bounds__(kStatWarps * 32) bn_stats_final_kernel(
+    const double* __restrict__ part, int B, int F, float momentum,
+    float* __restrict__ batch_mean, float* __restrict__ batch_var,
+    float* __restrict__ running_mean, float* __restrict__ running_var) {
+  __shared__ double sn[kStatWarps][32], sm[kStatWarps][32], s2[kStatWarps][32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int f = blockIdx.x * 32 + lane;
   const int chunks = (B + kStatChunk - 1) / kStatChunk;
+  const int per = (chunks + kStatWarps - 1) / kStatWarps;
   double n = 0.0, mean = 0.0, m2 = 0.0;
-  for (int c = 0; c < chunks; ++c) {
-    const double nb = static_cast<double>(min(B, (c + 1) * kStatChunk) - c * kStatChunk);
-    const double mb = part[(static_cast<int64_t>(c) * 2) * F + f];
-    const double m2b = part[(static_cast<int64_t>(c) * 2 + 1) * F + f];
-    const double tot = n + nb;
-    const double delta = mb - mean;
-    mean += delta * (nb / tot);
-    m2 += m2b + delta * delta * (n * nb / tot);
-    n = tot;
+  if (f < F) {
+    for (int c = warp * per; c < min(chunks, (warp + 1) * per); ++c) {
+      const double nb = static_cast<double>(min(B, (c + 1) * kStatChunk) - c * kStatChunk);
+      chan_merge(n, mean, m2, nb, part[(static_cast<int64_t>(c) * 2) * F + f],
+                 part[(static_cast<int64_t>(c) * 2 + 1) * F + f]);
+    }
   }
+  sn[warp][lane] = n;
+  sm[warp][lane] = mean;
+  s2[warp][lane] = m2;
+  __syncthreads();
+  if (warp != 0 || f >= F) return;
+  n = 0.0;
+  mean = 0.0;
+  m2 = 0.0;
+  for (int w = 0; w < kStatWarps; ++w) chan_merge(n, mean, m2, sn[w][lane], sm[w][lane], s2[w][lane]);
   const double var = m2 / B;
   batch_mean[f] = static_cast<float>(mean);
   batch_var[f] = static_cast<float>(var);
@@ -82,9 +103,8 @@ cudaError_t launch_bn_batch_stats(const uint16_t* planes, const float* acc, int6
   const int chunks = static_cast<int>((B + kStatChunk - 1) / kStatChunk);
   dim3 g1((F + 255) / 256, chunks);
   bn_stats_partial_kernel<<<g1, 256, 0, st>>>(planes, acc, static_cast<int>(B), F, part);
-  bn_stats_final_kernel<<<(F + 255) / 256, 256, 0, st>>>(part, static_cast<int>(B), F, momentum,
-                                                          batch_mean, batch_var, running_mean,
-                                                          running_var);
+  bn_stats_final_kernel<<<(F + 31) / 32, kStatWarps * 32, 0, st>>>(
+      part, static_cast<int>(B), F, momentum, batch_mean, batch_var, running_mean, running_var);
   return cudaGetLastError();
 }
 
