@@ -221,12 +221,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) query_tc_kernel(
         for (int i = 0; i < 32; i += 2) {
           const float q0 = fmaf(v[i], scale_s[f0 + i], shift_s[f0 + i]);
           const float q1 = fmaf(v[i + 1], scale_s[f0 + i + 1], shift_s[f0 + i + 1]);
-          uint16_t h0, m0, l0, h1, m1, l1;
-          split3(q0, h0, m0, l0);
-          split3(q1, h1, m1, l1);
-          ph_[i / 2] = h0 | (static_cast<uint32_t>(h1) << 16);
-          pm[i / 2] = m0 | (static_cast<uint32_t>(m1) << 16);
-          pl[i / 2] = l0 | (static_cast<uint32_t>(l1) << 16);
+          split3_pair(q0, q1, ph_[i / 2], pm[i / 2], pl[i / 2]);
         }
         // The previous group's stores must have read the staging tile before it is
         // overwritten.

@@ -293,16 +293,20 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-// Split an fp32 value into three bf16 values whose sum equals it to ~2^-24 relative.
-__device__ __forceinline__ void split3(float q, uint16_t& hi, uint16_t& mid, uint16_t& lo) {
-  const __nv_bfloat16 h = __float2bfloat16_rn(q);
-  const float r1 = q - __bfloat162float(h);
-  const __nv_bfloat16 m = __float2bfloat16_rn(r1);
-  const float r2 = r1 - __bfloat162float(m);
-  const __nv_bfloat16 l = __float2bfloat16_rn(r2);
-  hi = __bfloat16_as_ushort(h);
-  mid = __bfloat16_as_ushort(m);
-  lo = __bfloat16_as_ushort(l);
+// Split two fp32 values into three bf16 planes each, hi + mid + lo equal to the value
+// to ~2^-24 relative (hi = RN(q), mid = RN(q - hi), lo = RN(q - hi - mid)), returned
+// packed as bf16 pairs (q0 in the low half): each rounding converts both values in
+// one instruction.
+__device__ __forceinline__ void split3_pair(float q0, float q1, uint32_t& hi, uint32_t& mid,
+                                            uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(q0, q1);
+  const float r0 = q0 - __low2float(h), r1 = q1 - __high2float(h);
+  const __nv_bfloat162 m = __floats2bfloat162_rn(r0, r1);
+  const float s0 = r0 - __low2float(m), s1 = r1 - __high2float(m);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(s0, s1);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  mid = *reinterpret_cast<const uint32_t*>(&m);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
 }  // namespace tc
