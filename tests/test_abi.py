@@ -144,3 +144,25 @@ def test_training_bn_entry_points_validate_before_launch():
     bargs = [ok] * 11 + [None] * 7
     assert P.lib().pkm_backward_train(ctypes.byref(_shape(B=1)), *bargs, ok, 1 << 40, None) == -1
     assert P.lib().pkm_backward_train(ctypes.byref(s), *bargs, ok, 100, None) == -3
+
+
+def test_no_cpu_fallback_host_tensors_are_refused():
+    """The binding hands only device pointers to the library: CPU tensors raise
+    instead of running anywhere else."""
+    import torch
+    x = torch.zeros(4, 32)
+    with pytest.raises(ValueError, match="device tensors"):
+        P.pkm_forward(x, torch.zeros(16, 32), torch.zeros(16), torch.ones(16), torch.ones(16),
+                      torch.zeros(16), torch.zeros(1, 2, 16, 8), torch.zeros(256, 32), k=4)
+
+
+def test_missing_library_fails_loudly():
+    import subprocess
+    import sys
+    # The package loads the library when it is imported.
+    code = ("try:\n    import product_key_memory_b200\n"
+            "except ImportError as e:\n    print('raised', e)\n")
+    env = dict(os.environ, PKM_LIBRARY=os.path.join(ROOT, "no_such_library.so"))
+    r = subprocess.run([sys.executable, "-c", code], env=env, cwd=ROOT, capture_output=True,
+                       text=True, timeout=120)
+    assert "raised" in r.stdout and "not built" in r.stdout, r.stdout + r.stderr
