@@ -363,16 +363,6 @@ cudaError_t launch_counting_sort(const int* keys, int64_t E, int64_t slots, cons
   return cudaGetLastError();
 }
 
-static int maxv_bwd(int v, int dtype) {
-  const int per = dtype == 0 ? 4 : 8;
-  const int m = (v / per + 31) / 32;
-  if (m <= 1) return 1;
-  if (m <= 2) return 2;
-  if (m <= 4) return 4;
-  if (m <= 8) return 8;
-  return 0;
-}
-
 template <typename T, int MAXV>
 static cudaError_t launch_bwd_t(int64_t B, int H, int k, int v, int64_t slots, const void* values,
                                 const int* indices, const float* weights, const void* grad_out,
@@ -404,7 +394,7 @@ cudaError_t launch_backward_values(int64_t B, int H, int k, int v, int dtype, in
                                    const void* grad_out, float* grad_values, float* grad_scores,
                                    const BackwardWs& ws, int* status, cudaStream_t st,
                                    const std::function<void()>& between_stages) {
-  const int m = maxv_bwd(v, dtype);
+  const int m = row_vecs_per_lane(v, dtype);
 #define PKM_BWD(T, M)                                                                        \
   return launch_bwd_t<T, M>(B, H, k, v, slots, values, indices, weights, grad_out, grad_values, \
                             grad_scores, ws, status, st, between_stages)

@@ -100,6 +100,18 @@ size_t small_chunk_entries(int64_t B, int H, int n);
 cudaError_t launch_forward_small(const LayerArgs& a, float* q, float* chunk_s, int* chunk_i,
                                  float* out, int* idx, float* w, float* sc, cudaStream_t st);
 
+// 16-byte vectors of a v-wide row each lane of a warp holds, rounded up to the kernel
+// instantiations (1, 2, 4 or 8); 0 when a row is wider than 8 vectors per lane.
+inline int row_vecs_per_lane(int v, int dtype) {
+  const int per = dtype == 0 ? 4 : 8;
+  const int m = (v / per + 31) / 32;
+  if (m <= 1) return 1;
+  if (m <= 2) return 2;
+  if (m <= 4) return 4;
+  if (m <= 8) return 8;
+  return 0;
+}
+
 // Raise a kernel's dynamic shared-memory limit once per (kernel, device, size)
 // (pkm_util.cu).
 cudaError_t set_max_smem(const void* func, size_t bytes);

@@ -125,19 +125,8 @@ __global__ void __launch_bounds__(kSgWarps * 32) select_gather_kernel(
   }
 }
 
-static int maxv_for(int v, int dtype) {
-  const int per = dtype == 0 ? 4 : 8;
-  const int nvec = v / per;
-  const int m = (nvec + 31) / 32;
-  if (m <= 1) return 1;
-  if (m <= 2) return 2;
-  if (m <= 4) return 4;
-  if (m <= 8) return 8;
-  return 0;
-}
-
 bool select_gather_supported(int H, int k, int v, int dtype) {
-  return k >= 1 && k <= kMaxK && H >= 1 && H * k <= 2048 && maxv_for(v, dtype) > 0;
+  return k >= 1 && k <= kMaxK && H >= 1 && H * k <= 2048 && row_vecs_per_lane(v, dtype) > 0;
 }
 
 template <typename T, int MAXV>
@@ -155,7 +144,7 @@ static cudaError_t launch_sg(const LayerArgs& a, const float* ls, const int* li,
 
 cudaError_t launch_select_gather(const LayerArgs& a, const float* ls, const int* li, float* out,
                                  int* idx, float* w, float* sc, cudaStream_t st) {
-  const int m = maxv_for(a.v, a.dtype);
+  const int m = row_vecs_per_lane(a.v, a.dtype);
   if (a.dtype == 0) {
     switch (m) {
       case 1: return launch_sg<float, 1>(a, ls, li, out, idx, w, sc, st);

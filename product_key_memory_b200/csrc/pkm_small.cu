@@ -450,16 +450,6 @@ __global__ void __launch_bounds__(kSmallWarps * 32) gather_small_kernel(
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-static int maxv_small(int v, int dtype) {
-  const int per = dtype == 0 ? 4 : 8;
-  const int m = (v / per + 31) / 32;
-  if (m <= 1) return 1;
-  if (m <= 2) return 2;
-  if (m <= 4) return 4;
-  if (m <= 8) return 8;
-  return 0;
-}
-
 static size_t query_small_smem(int d, int dtype) {
   return static_cast<size_t>(kQFeat + kQTok) * d * (dtype == 0 ? 4 : 2);
 }
@@ -481,7 +471,7 @@ bool small_supported(int64_t B, int d_model, int H, int dq, int n, int k, int v,
   // Staging copies whole 32-bit words of W_q rows and sub-key rows.
   if ((static_cast<int64_t>(d_model) * esz) % 4 || (static_cast<int64_t>(dq / 2) * esz) % 4)
     return false;
-  return B >= 1 && B <= kSmallMaxB && k <= kMaxK && maxv_small(v, dtype) > 0 &&
+  return B >= 1 && B <= kSmallMaxB && k <= kMaxK && row_vecs_per_lane(v, dtype) > 0 &&
          query_small_smem(d_model, dtype) <= kLimit && score_small_smem(dq, dtype) <= kLimit &&
          gather_small_smem(n, v) <= kLimit && n >= 1 && H <= 8;  // H CTAs per cluster
 }
@@ -544,7 +534,7 @@ static cudaError_t launch_small_t(const LayerArgs& a, float* q, float* cs, int* 
   e = cudaLaunchKernelEx(&cfg, score_small_kernel<T>, static_cast<const float*>(q),
                          static_cast<const T*>(a.subkeys), B, a.H, a.dq, a.n, cs, ci);
   if (e != cudaSuccess) return e;
-  switch (maxv_small(a.v, a.dtype)) {
+  switch (row_vecs_per_lane(a.v, a.dtype)) {
     case 1: return launch_gather_small<T, 1>(a, cs, ci, out, idx, w, sc, st);
     case 2: return launch_gather_small<T, 2>(a, cs, ci, out, idx, w, sc, st);
     case 4: return launch_gather_small<T, 4>(a, cs, ci, out, idx, w, sc, st);

@@ -259,11 +259,6 @@ __device__ __forceinline__ uint16_t lds_u16(uint32_t addr) {
   return v;
 }
 
-// Named barrier over `count` threads (ids 1..15; 0 is __syncthreads).
-__device__ __forceinline__ void named_barrier(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
 // ------------------------------------------------------------- descriptors
 // Shared-memory matrix descriptor of a K-major operand tile stored as rows of 64 bf16
 // (128 bytes) with the 128-byte swizzle, 8-row groups 1024 bytes apart. The tile
