@@ -13,8 +13,14 @@ on the data path (weak scaling); the reported time is the max over ranks.
 Rank 0 prints one JSON line. Besides the throughput it carries the roofline of the
 dominant kernel (stage times come from CUDA events the library records between its
 launches on the launching stream), the whole-step roofline, an end-to-end figure
-through the same call with host buffers, the value backward on the 512^2 layer, the
-oracle timed on this host's cores, and the SM clocks sampled during the timed loop.
+through the same call with host buffers, the oracle timed on this host's cores, the
+SM clocks sampled during the timed loop, and sub-objects for the 512^2 forward
+(c512), the value backward and the full backward on its picks (backward,
+backward_full), a training step with BatchNorm on batch statistics (train), the
+small-batch latency on the 1024^2 layer (small_batch) and the wide layer (wide).
+
+    python bench.py --part NAME          # one sub-object alone (for profiling)
+    python bench.py --tokens B           # the main workload on its first B tokens
 
 ``--impl reference`` times the fp64 CPU oracle instead (a bounded sample of the
 same workload per step) and prints the same metric with "impl": "reference".
