@@ -158,7 +158,9 @@ int pkm_backward_values(const pkm_shape* s, const void* values, const int32_t* i
  * keeps nothing from the forward beyond indices and weights. Sums over tokens are
  * in fp32 in a fixed order except sub-key rows shared by two 32-pick windows, which
  * are added atomically. Slot ids outside [0, n*n) are skipped and counted in the
- * status word. workspace: at least pkm_workspace_size(s, 3) bytes, 256-byte aligned.
+ * status word. 2*B*H*k must stay below 2^31 (PKM_ERR_UNSUPPORTED otherwise: the
+ * sub-key grouping sorts two contributions per pick with 32-bit positions).
+ * workspace: at least pkm_workspace_size(s, 3) bytes, 256-byte aligned.
  */
 int pkm_backward(const pkm_shape* s, const void* x, const void* W_q, const float* bn_mean,
                  const float* bn_var, const float* bn_gamma, const float* bn_beta,

@@ -325,7 +325,8 @@ size_t pkm_workspace_size(const pkm_shape* s, int for_backward) {
     return forward_train_ws(s, nullptr, nullptr, nullptr);
   }
   if (for_backward == 3) {
-    if (validate_shape(s) != PKM_OK) return 0;
+    if (validate_shape(s) != PKM_OK || 2 * s->B * s->H * static_cast<int64_t>(s->k) > 0x7fffffffLL)
+      return 0;
     LayerArgs a{};
     a.B = s->B; a.H = s->H; a.dq = s->dq; a.n = s->n; a.k = s->k; a.v = s->v;
     return pkm::backward_full_ws_bytes(a, choose_path(s) == Path::kTensor, nullptr, nullptr);
@@ -352,6 +353,8 @@ int backward_full_impl(const pkm_shape* s, bool bn_training, const void* x, cons
   int rc = validate_shape(s);
   if (rc != PKM_OK) return rc;
   if (bn_training && s->B == 1) return PKM_ERR_INVALID_ARG;
+  // The sub-key grouping sorts two contributions per pick with 32-bit positions.
+  if (2 * s->B * s->H * static_cast<int64_t>(s->k) > 0x7fffffffLL) return PKM_ERR_UNSUPPORTED;
   const bool tok = s->B > 0;
   if (!W_q || !bn_mean || !bn_var || !bn_gamma || !bn_beta || !subkeys || !values ||
       (tok && (!x || !indices || !weights || !grad_out)))

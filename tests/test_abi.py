@@ -166,3 +166,12 @@ def test_missing_library_fails_loudly():
     r = subprocess.run([sys.executable, "-c", code], env=env, cwd=ROOT, capture_output=True,
                        text=True, timeout=120)
     assert "raised" in r.stdout and "not built" in r.stdout, r.stdout + r.stderr
+
+
+def test_full_backward_rejects_more_picks_than_32_bit_positions():
+    # 2 * B * H * k contributions must fit the sort's 32-bit positions.
+    s = _shape(B=(1 << 30) // (4 * 32) + 1, n=512)
+    assert P.lib().pkm_workspace_size(ctypes.byref(s), 3) == 0
+    ok = ctypes.c_void_p(1 << 20)
+    assert P.lib().pkm_backward(ctypes.byref(s), *([ok] * 11), *([None] * 7), ok, 1 << 40,
+                                None) == -2
