@@ -21,15 +21,18 @@
  *
  * Conventions for every entry point:
  *   - Tensors are caller-owned DEVICE pointers, row-major and contiguous, 16-byte
- *     aligned. The library keeps no device state between calls and allocates no
- *     device memory: scratch is the caller's `workspace`.
+ *     aligned. The library allocates no device memory: scratch is the caller's
+ *     `workspace` (pkm_backward_values_noalloc alone uses a fixed array compiled
+ *     into the library). On first use per device it creates one helper stream and
+ *     a pool of ordering events for the pipelined forward.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *     All work is enqueued asynchronously and ordered on it; no call synchronises.
  *   - Arguments are validated before anything is launched: a call that returns an
  *     error has launched nothing and written nothing.
- *   - Kernels that wait on hardware barriers give up after a bounded number of
- *     polls and record PKM_ERR_DEVICE in the workspace's status word; read it with
- *     pkm_device_status() after the stream has finished.
+ *   - Kernels that wait on hardware barriers give up after a bounded time (1 s)
+ *     and record it in the workspace's status word, as do gathers that meet a slot
+ *     id outside [0, n*n) (skipped); pkm_device_status() waits for the stream and
+ *     returns PKM_ERR_DEVICE if either happened.
  */
 #ifndef PKM_H_
 #define PKM_H_
@@ -53,7 +56,8 @@ enum {
                                16 bytes, misaligned pointer) */
   PKM_ERR_WORKSPACE = -3,   /* workspace NULL or smaller than pkm_workspace_size() */
   PKM_ERR_CUDA = -4,        /* a CUDA runtime call or kernel launch failed */
-  PKM_ERR_DEVICE = -5       /* a kernel recorded a device-side error (bounded wait ran out) */
+  PKM_ERR_DEVICE = -5       /* a kernel recorded a device-side error: a bounded wait ran
+                               out, or a slot id outside [0, n*n) was read */
 };
 
 /* Layer sizes. */
