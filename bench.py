@@ -306,7 +306,14 @@ def run_ours(args, rank, world, local_rank):
     t_mem = w.H * w.k * w.v * (2 if w.dtype == "bf16" else 4) * B / (hbm * 1e9)
     t_gemm = gemm_flops_per_token(w) * B / (bf16 * 1e12)
     t_roof_ms = max(t_mem, t_gemm) * 1e3
+    # Compulsory I/O besides the gathered rows: x in, W_q and the sub-keys, out,
+    # indices and weights out.
+    esz = 2 if w.dtype == "bf16" else 4
+    secondary = (B * w.d_model * esz + F * w.d_model * esz + w.H * w.n * w.dq * esz
+                 + B * w.v * 4 + B * w.H * w.k * 8)
     step_roof = {"t_roof_ms": t_roof_ms, "t_step_ms": ms_per_step, "frac": t_roof_ms / ms_per_step,
+                 "secondary_io_bytes": secondary,
+                 "secondary_io_share": secondary / (w.H * w.k * w.v * esz * B),
                  "bound": "hbm" if t_mem >= t_gemm else "tensor",
                  "stage_ms": dict(zip(names, stage_avg)), "call_ms": call_avg,
                  "peak_kind": pk_kind}
@@ -380,6 +387,10 @@ def run_ours(args, rank, world, local_rank):
                    "seq_len": None, "parallelism": "dp%d (independent replicas)" % world,
                    "l2": "flushed before every timed step (256 MiB write, outside the bracket)"},
         "roofline": roof, "step_roofline": step_roof, "e2e": e2e, "slot_usage": usage,
+        # Keys scored per (token, head): the product search scores both codebooks
+        # (2n) and the pruned candidate pairs, the flat search every one of n^2 keys.
+        "search_cost": {"product": 2 * w.n + pruned_pairs(w.k), "flat": w.n * w.n,
+                        "flat_over_product": w.n * w.n / (2 * w.n + pruned_pairs(w.k))},
         "gpu_launches": launches, "gpu_launches_e2e": launches_e2e,
         "clocks": clocks,
     }
@@ -571,6 +582,11 @@ def run_c512_and_backward(args, dev, P, hbm, bf16, stream, world, barrier,
                    "stage_ms": [m / max(1, calls) for m in stage_ms[:3]],
                    "gather_gbs": per_token_bytes(w) * B / (stage_ms[2] / max(1, calls) * 1e-3) / 1e9}
     return res
+
+
+def pruned_pairs(k: int) -> int:
+    """Candidate pairs (a, b) of the two sorted per-half lists with (a+1)(b+1) <= k."""
+    return sum(k // (a + 1) for a in range(k))
 
 
 def run_latency(args, dev, P):
