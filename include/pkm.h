@@ -99,7 +99,7 @@ size_t pkm_workspace_size(const pkm_shape* s, int for_backward);
  *   scores   [B][H][k]  fp32   kept key scores s1[i] + s2[j]; may be NULL
  * workspace: device scratch of at least pkm_workspace_size(s, 0) bytes, 256-byte
  *   aligned; its contents on entry do not matter.
- * Batches of at most 96 tokens (H <= 8) take the small-batch kernels, which spread
+ * Batches of at most 128 tokens (H <= 8) take the small-batch kernels, which spread
  * W_q, the sub-keys and the heads over all SMs for latency; their three launches
  * overlap through programmatic dependent launch on `stream`. Large batches of
  * tensor-core shapes can be processed in up to 4 sub-batches (PKM_SUBBATCHES); the

@@ -94,7 +94,7 @@ cudaError_t launch_bn_train_dacc(const float* g_q, const float* acc, const float
 // Small-batch forward (pkm_small.cu): B <= kSmallMaxB tokens, three launches that
 // spread the parameters over every SM. Workspace: q fp32 [B][H*dq] and chunk lists of
 // small_chunk_entries() (score, id) entries.
-constexpr int kSmallMaxB = 96;  // measured crossover with the tensor-core path
+constexpr int kSmallMaxB = 128;  // measured crossover with the tensor-core path
 bool small_supported(int64_t B, int d_model, int H, int dq, int n, int k, int v, int dtype);
 size_t small_chunk_entries(int64_t B, int H, int n);
 cudaError_t launch_forward_small(const LayerArgs& a, float* q, float* chunk_s, int* chunk_i,

@@ -129,19 +129,46 @@ __global__ void __launch_bounds__(kSmallWarps * 32) query_small_kernel(
 #pragma unroll
     for (int j = 0; j < kQFeat; ++j) acc[j] = 0.f;
     const T* xr = xs + warp * d;
-    for (int c0 = 0; c0 < d; c0 += 32 * 8) {
-      float xv[8];
+    if constexpr (sizeof(T) == 2) {
+      // bf16: one 32-bit shared-memory word holds two consecutive columns (d is even).
+      const uint32_t* xw = reinterpret_cast<const uint32_t*>(xr);
+      const uint32_t* ww = reinterpret_cast<const uint32_t*>(ws);
+      const int dw = d >> 1;
+      for (int c0 = 0; c0 < dw; c0 += 32 * 4) {
+        uint32_t xv[4];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int c = c0 + lane + 32 * u;
-        xv[u] = c < d ? load_elem(xr, c) : 0.f;
+        for (int u = 0; u < 4; ++u) {
+          const int c = c0 + lane + 32 * u;
+          xv[u] = c < dw ? xw[c] : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int c = c0 + lane + 32 * u;
+          if (c < dw) {
+            const float xa = bf16_lo(xv[u]), xb = bf16_hi(xv[u]);
+#pragma unroll
+            for (int j = 0; j < kQFeat; ++j) {
+              const uint32_t wv = ww[j * dw + c];
+              acc[j] = fmaf(xb, bf16_hi(wv), fmaf(xa, bf16_lo(wv), acc[j]));
+            }
+          }
+        }
       }
+    } else {
+      for (int c0 = 0; c0 < d; c0 += 32 * 8) {
+        float xv[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int c = c0 + lane + 32 * u;
-        if (c < d) {
+        for (int u = 0; u < 8; ++u) {
+          const int c = c0 + lane + 32 * u;
+          xv[u] = c < d ? load_elem(xr, c) : 0.f;
+        }
 #pragma unroll
-          for (int j = 0; j < kQFeat; ++j) acc[j] = fmaf(xv[u], load_elem(ws, j * d + c), acc[j]);
+        for (int u = 0; u < 8; ++u) {
+          const int c = c0 + lane + 32 * u;
+          if (c < d) {
+#pragma unroll
+            for (int j = 0; j < kQFeat; ++j) acc[j] = fmaf(xv[u], load_elem(ws, j * d + c), acc[j]);
+          }
         }
       }
     }
@@ -222,19 +249,25 @@ __global__ void __launch_bounds__(kSmallWarps * 32) score_small_kernel(
     const int t = tb + u;
     if (t >= B) break;  // warp-uniform
     const float* qq = qw + u * half;
-    // Two chains per row (even and odd elements), added at the end.
+    // Two chains per row (even and odd elements), added at the end. half is even; a
+    // bf16 row is read a 32-bit word (two elements) at a time.
     float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
-    int e = 0;
-    for (; e + 1 < half; e += 2) {
-      const float qv = qq[e], qv2 = qq[e + 1];
-      a0 = fmaf(qv, load_elem(r0, e), a0);
-      a1 = fmaf(qv, load_elem(r1, e), a1);
-      b0 = fmaf(qv2, load_elem(r0, e + 1), b0);
-      b1 = fmaf(qv2, load_elem(r1, e + 1), b1);
-    }
-    if (e < half) {
-      a0 = fmaf(qq[e], load_elem(r0, e), a0);
-      a1 = fmaf(qq[e], load_elem(r1, e), a1);
+    for (int e = 0; e < half; e += 2) {
+      const float2 qv = *reinterpret_cast<const float2*>(qq + e);
+      float x0a, x0b, x1a, x1b;
+      if constexpr (sizeof(T) == 2) {
+        const uint32_t w0 = *reinterpret_cast<const uint32_t*>(r0 + e);
+        const uint32_t w1 = *reinterpret_cast<const uint32_t*>(r1 + e);
+        x0a = bf16_lo(w0); x0b = bf16_hi(w0);
+        x1a = bf16_lo(w1); x1b = bf16_hi(w1);
+      } else {
+        x0a = load_elem(r0, e); x0b = load_elem(r0, e + 1);
+        x1a = load_elem(r1, e); x1b = load_elem(r1, e + 1);
+      }
+      a0 = fmaf(qv.x, x0a, a0);
+      a1 = fmaf(qv.x, x1a, a1);
+      b0 = fmaf(qv.y, x0b, b0);
+      b1 = fmaf(qv.y, x1b, b1);
     }
     a0 += b0;
     a1 += b1;
@@ -471,6 +504,7 @@ bool small_supported(int64_t B, int d_model, int H, int dq, int n, int k, int v,
   // Staging copies whole 32-bit words of W_q rows and sub-key rows.
   if ((static_cast<int64_t>(d_model) * esz) % 4 || (static_cast<int64_t>(dq / 2) * esz) % 4)
     return false;
+  if ((dq / 2) % 2) return false;  // the scoring loop takes element pairs
   return B >= 1 && B <= kSmallMaxB && k <= kMaxK && row_vecs_per_lane(v, dtype) > 0 &&
          query_small_smem(d_model, dtype) <= kLimit && score_small_smem(dq, dtype) <= kLimit &&
          gather_small_smem(n, v) <= kLimit && n >= 1 && H <= 8;  // H CTAs per cluster

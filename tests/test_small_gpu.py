@@ -1,4 +1,4 @@
-"""GPU parity of the small-batch forward (B <= 96 tokens: pkm_forward picks the
+"""GPU parity of the small-batch forward (B <= 128 tokens: pkm_forward picks the
 small-batch kernels by itself) against the fp64 oracle, through the C ABI.
 
 Same bar as tests/test_forward_gpu.py: indices bit-exact except fp64 near-ties
@@ -51,7 +51,7 @@ def _check(L, w):
     return g, r
 
 
-@pytest.mark.parametrize("B", [1, 7, 64, 96])
+@pytest.mark.parametrize("B", [1, 7, 64, 96, 128])
 def test_c1024_small_batches(B):
     w = synth.WORKLOADS["c1024"].with_(B=B)
     _check(synth.make_layer(w), w)
