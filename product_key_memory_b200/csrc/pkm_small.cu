@@ -99,8 +99,9 @@ __device__ __forceinline__ void stage_rows(const uint32_t* __restrict__ src, uin
 // ---------------------------------------------------------------------------
 // q[t][f] = (sum_c x[t][c] W[f][c]) * scale[f] + shift[f], scale = gamma / sqrt(var + eps),
 // shift = beta - mean * scale (the tensor-core epilogue's form). CTA = 16 features x 8
-// tokens: the 16 rows of W_q staged in shared memory, one warp per token reading x in
-// runs of 8 per lane; the 16 per-lane partial sums are reduced by a butterfly that
+// tokens: the 16 rows of W_q and the 8 rows of x staged in shared memory, one warp
+// per token, each lane reading bf16 rows two elements (one 32-bit word) at a time,
+// 4 words in flight; the 16 per-lane partial sums are reduced by a butterfly that
 // leaves feature j's total in lanes 2j and 2j + 1 (16 shuffles instead of 80).
 // ---------------------------------------------------------------------------
 template <typename T>
@@ -196,7 +197,8 @@ __global__ void __launch_bounds__(kSmallWarps * 32) query_small_kernel(
 
 // ---------------------------------------------------------------------------
 // Per-half scores of one chunk of kSChunk sub-keys for up to kSTok tokens, and each
-// token's best 32 of the chunk. Lane i scores sub-keys c0 + i and c0 + 32 + i; the two
+// token's best 32 of the chunk. Lane i scores sub-keys c0 + i and c0 + 32 + i (a
+// 32-bit word, two elements, of each bf16 row per step); the two
 // sorted halves are merged (warp_sort32 / warp_merge32). Output chunk lists
 // [B][H][2][nchunks][32], best first (padding: -inf, kIdPad).
 // ---------------------------------------------------------------------------
