@@ -50,11 +50,9 @@ UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FLUSH_BYTES = 256 << 20
 
-# DRAM bytes per launch of the dominant kernel from an ncu capture
-# (profiles/select_gather_c1024.md), keyed by the sha256 of the kernel's source at
-# capture time; reported as null once the source has changed.
-# DRAM bytes (read + write) of one select_gather launch, from an ncu capture, keyed by
-# (kernel_sha(), workload, tokens); None once the kernel source changes.
+# DRAM bytes (read + write) of one launch of the dominant kernel, from an ncu capture,
+# keyed by (kernel_sha(), workload, tokens); reported as null once the kernel's source
+# has changed since the capture.
 TRAFFIC = {
     # c1024 at 4096 tokens: dram read 960.7 MB + write 4.7 MB, scaled x4 to the
     # 16384-token launch (the gather's traffic grows with the tokens).

@@ -23,8 +23,14 @@
  *   - Tensors are caller-owned DEVICE pointers, row-major and contiguous, 16-byte
  *     aligned. The library allocates no device memory: scratch is the caller's
  *     `workspace` (pkm_backward_values_noalloc alone uses a fixed array compiled
- *     into the library). On first use per device it creates one helper stream and
- *     a pool of ordering events for the pipelined forward.
+ *     into the library).
+ *   - Persistent state the library keeps: two process-wide option values
+ *     (pkm_set_option), the tensor-map encoder's address and the SM count (looked
+ *     up once), each kernel's raised shared-memory limit, and, only while tracing
+ *     is on, a pool of timing events. A forward pipelined over sub-batches
+ *     (PKM_OPT_SUBBATCHES > 1) also creates, on first use per device, one helper
+ *     stream and a pool of ordering events; the default forward (one batch) uses
+ *     neither and issues its three kernels on `stream` alone.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *     All work is enqueued asynchronously and ordered on it; no call synchronises.
  *   - Arguments are validated before anything is launched: a call that returns an
@@ -101,12 +107,14 @@ size_t pkm_workspace_size(const pkm_shape* s, int for_backward);
  *   aligned; its contents on entry do not matter.
  * Batches of at most 128 tokens (H <= 8) take the small-batch kernels, which spread
  * W_q, the sub-keys and the heads over all SMs for latency; their three launches
- * overlap through programmatic dependent launch on `stream`. Large batches of
- * tensor-core shapes can be processed in up to 4 sub-batches (PKM_SUBBATCHES); the
- * value gather of one sub-batch then runs on a second stream owned by the library
- * (one per device) while the next sub-batch is scored on `stream`. Event waits order
- * both ways, so all of the call's work is complete when `stream` reaches the point
- * after the call.
+ * overlap through programmatic dependent launch on `stream`. Larger batches run
+ * three kernels on `stream` (query network, per-half scores and top-k, candidate
+ * top-k + softmax + gather). With PKM_OPT_SUBBATCHES > 1, large batches of
+ * tensor-core shapes are processed in up to that many sub-batches; the value gather
+ * of one sub-batch then runs on a second stream owned by the library (one per
+ * device) while the next sub-batch is scored on `stream`. Event waits order both
+ * ways, so all of the call's work is complete when `stream` reaches the point after
+ * the call.
  * Returns PKM_OK or a status code above.
  */
 int pkm_forward(const pkm_shape* s, const void* x, const void* W_q, const float* bn_mean,
@@ -277,6 +285,28 @@ int pkm_device_status(void* workspace, void* stream);
 int pkm_trace_enable(int on);
 int pkm_trace_read(int pass, double* stage_ms, int max_stages, int64_t* calls,
                    int64_t* launches);
+
+/*
+ * Implementation switches (a convenience of this library; the pages have no
+ * counterpart). Process-wide, for every device; a change applies to calls made after
+ * it. The environment variables PKM_PATH (auto | tc | simt) and PKM_SUBBATCHES (1..4)
+ * give the initial values and are read once, at the first call that needs them.
+ *   PKM_OPT_PATH        PKM_PATH_AUTO (default): small-batch kernels for up to 128
+ *                       tokens, else the tensor-core kernels where the layer fits
+ *                       their tiles (bf16, d_model and dq/2 multiples of 64, n a
+ *                       multiple of 256, H*dq <= 4096), else the CUDA-core kernels;
+ *                       PKM_PATH_TC: never the small-batch kernels;
+ *                       PKM_PATH_SIMT: always the CUDA-core kernels.
+ *   PKM_OPT_SUBBATCHES  1 (default) to 4: sub-batches of the pipelined tensor-core
+ *                       forward (see pkm_forward). The forward's workspace size
+ *                       depends on it: query it after setting the option.
+ * pkm_set_option returns PKM_OK or PKM_ERR_INVALID_ARG (unknown option or value);
+ * pkm_get_option returns the current value or PKM_ERR_INVALID_ARG.
+ */
+enum { PKM_OPT_PATH = 0, PKM_OPT_SUBBATCHES = 1 };
+enum { PKM_PATH_AUTO = 0, PKM_PATH_TC = 1, PKM_PATH_SIMT = 2 };
+int pkm_set_option(int option, int value);
+int pkm_get_option(int option);
 
 /* Static string for a status code. */
 const char* pkm_status_string(int status);

@@ -21,13 +21,16 @@ LIB_PATH = os.environ.get("PKM_LIBRARY") or os.path.join(_HERE, "libpkm.so")
 
 PKM_F32, PKM_BF16 = 0, 1
 PKM_OK = 0
+PKM_OPT_PATH, PKM_OPT_SUBBATCHES = 0, 1
+PKM_PATH_AUTO, PKM_PATH_TC, PKM_PATH_SIMT = 0, 1, 2
+_PATHS = {"auto": PKM_PATH_AUTO, "tc": PKM_PATH_TC, "simt": PKM_PATH_SIMT}
 _STATUS = {0: "PKM_OK", -1: "PKM_ERR_INVALID_ARG", -2: "PKM_ERR_UNSUPPORTED",
            -3: "PKM_ERR_WORKSPACE", -4: "PKM_ERR_CUDA", -5: "PKM_ERR_DEVICE"}
 
 EXPORTED = ("pkm_workspace_size", "pkm_forward", "pkm_backward_values", "pkm_device_status",
             "pkm_trace_enable", "pkm_trace_read", "pkm_status_string",
             "pkm_backward_values_noalloc", "pkm_slot_usage", "pkm_backward",
-            "pkm_forward_train", "pkm_backward_train")
+            "pkm_forward_train", "pkm_backward_train", "pkm_set_option", "pkm_get_option")
 
 
 class PKMError(RuntimeError):
@@ -79,6 +82,10 @@ def lib() -> ctypes.CDLL:
         L.pkm_trace_enable.restype = ctypes.c_int
         L.pkm_trace_read.argtypes = [ctypes.c_int, P, ctypes.c_int, P, P]
         L.pkm_trace_read.restype = ctypes.c_int
+        L.pkm_set_option.argtypes = [ctypes.c_int, ctypes.c_int]
+        L.pkm_set_option.restype = ctypes.c_int
+        L.pkm_get_option.argtypes = [ctypes.c_int]
+        L.pkm_get_option.restype = ctypes.c_int
         L.pkm_status_string.argtypes = [ctypes.c_int]
         L.pkm_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -90,6 +97,42 @@ lib()  # fail loudly at import when the library is missing
 
 def pkm_status_string(code: int) -> str:
     return lib().pkm_status_string(int(code)).decode()
+
+
+def pkm_set_option(option: int, value: int) -> None:
+    rc = lib().pkm_set_option(int(option), int(value))
+    if rc != PKM_OK:
+        raise PKMError("pkm_set_option", rc)
+
+
+def pkm_get_option(option: int) -> int:
+    rc = int(lib().pkm_get_option(int(option)))
+    if rc < 0:
+        raise PKMError("pkm_get_option", rc)
+    return rc
+
+
+class options:
+    """Context manager that sets the library's implementation switches and restores
+    them on exit: ``with options(path="simt"): ...`` (path: "auto", "tc" or "simt";
+    subbatches: 1..4)."""
+
+    def __init__(self, path: Optional[str] = None, subbatches: Optional[int] = None):
+        self.want = {}
+        if path is not None:
+            self.want[PKM_OPT_PATH] = _PATHS[path]
+        if subbatches is not None:
+            self.want[PKM_OPT_SUBBATCHES] = int(subbatches)
+
+    def __enter__(self):
+        self.old = {o: pkm_get_option(o) for o in self.want}
+        for o, v in self.want.items():
+            pkm_set_option(o, v)
+        return self
+
+    def __exit__(self, *exc):
+        for o, v in self.old.items():
+            pkm_set_option(o, v)
 
 
 def make_shape(B, d_model, H, dq, n, k, v, dtype, bn_eps=1e-5) -> pkm_shape:

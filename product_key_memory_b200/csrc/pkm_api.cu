@@ -5,6 +5,7 @@
 
 #include <nvtx3/nvToolsExt.h>
 
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -22,15 +23,35 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 // Which implementation of the forward runs: the small-batch kernels for a few
 // tokens, else the tensor-core kernels where the shape fits their tiles, else the
-// CUDA-core kernels. PKM_PATH=simt or =tc pins one of the large-batch paths (tests
-// compare the paths on the same inputs).
+// CUDA-core kernels. The option PKM_OPT_PATH pins one of the large-batch paths
+// (tests compare the paths on the same inputs).
 enum class Path { kTensor, kSimt, kSmall };
 
+// Process-wide implementation switches (pkm_set_option). The environment variables
+// PKM_PATH (auto | tc | simt) and PKM_SUBBATCHES (1..4) give their initial values and
+// are read once, at the first call that needs them.
+std::atomic<int> g_opt_path{PKM_PATH_AUTO};
+std::atomic<int> g_opt_subbatches{1};
+
+void init_options() {
+  static std::once_flag once;
+  std::call_once(once, [] {
+    const char* p = getenv("PKM_PATH");
+    if (p && strcmp(p, "simt") == 0) g_opt_path = PKM_PATH_SIMT;
+    if (p && strcmp(p, "tc") == 0) g_opt_path = PKM_PATH_TC;
+    const char* sb = getenv("PKM_SUBBATCHES");
+    if (sb) {
+      const int v = atoi(sb);
+      g_opt_subbatches = v < 1 ? 1 : (v > 4 ? 4 : v);
+    }
+  });
+}
+
 Path choose_path(const pkm_shape* s) {
-  const char* env = getenv("PKM_PATH");
-  if (env && strcmp(env, "simt") == 0) return Path::kSimt;
-  const bool pin_tc = env && strcmp(env, "tc") == 0;
-  if (!pin_tc &&
+  init_options();
+  const int pin = g_opt_path.load(std::memory_order_relaxed);
+  if (pin == PKM_PATH_SIMT) return Path::kSimt;
+  if (pin != PKM_PATH_TC &&
       pkm::small_supported(s->B, s->d_model, s->H, s->dq, s->n, s->k, s->v, s->dtype))
     return Path::kSmall;
   return pkm::tc_supported(s->dtype, s->d_model, s->H, s->dq, s->n, s->k) ? Path::kTensor
@@ -80,13 +101,11 @@ struct ForwardWs {
   int* list_i;      // [B][H][2][32]
 };
 
-// Tokens per pipelined sub-batch of the tensor-core path: PKM_SUBBATCHES (1..4,
+// Tokens per pipelined sub-batch of the tensor-core path: PKM_OPT_SUBBATCHES (1..4,
 // default 1) sub-batches of at least 2048 tokens, a multiple of the 128-token tile.
 int64_t sub_batch_tokens(int64_t B) {
-  const char* env = getenv("PKM_SUBBATCHES");
-  int64_t want = env ? atoi(env) : 1;
-  if (want < 1) want = 1;
-  if (want > 4) want = 4;
+  init_options();
+  const int64_t want = g_opt_subbatches.load(std::memory_order_relaxed);
   int64_t S = B / 2048;
   if (S > want) S = want;
   if (S < 1) S = 1;
@@ -279,6 +298,29 @@ int aux_resources(int n, cudaStream_t* aux, cudaEvent_t* evs) {
 }  // namespace
 
 extern "C" {
+
+int pkm_set_option(int option, int value) {
+  init_options();
+  if (option == PKM_OPT_PATH) {
+    if (value != PKM_PATH_AUTO && value != PKM_PATH_TC && value != PKM_PATH_SIMT)
+      return PKM_ERR_INVALID_ARG;
+    g_opt_path = value;
+    return PKM_OK;
+  }
+  if (option == PKM_OPT_SUBBATCHES) {
+    if (value < 1 || value > 4) return PKM_ERR_INVALID_ARG;
+    g_opt_subbatches = value;
+    return PKM_OK;
+  }
+  return PKM_ERR_INVALID_ARG;
+}
+
+int pkm_get_option(int option) {
+  init_options();
+  if (option == PKM_OPT_PATH) return g_opt_path.load();
+  if (option == PKM_OPT_SUBBATCHES) return g_opt_subbatches.load();
+  return PKM_ERR_INVALID_ARG;
+}
 
 int pkm_trace_enable(int on) {
   std::lock_guard<std::mutex> lk(g_trace_mu);
@@ -503,12 +545,26 @@ cudaError_t run_forward(const pkm_shape* s, const LayerArgs& a, const ForwardWs&
       e = pkm::launch_select_gather(a, w.list_s, w.list_i, out, indices, weights, scores, st);
     tr.end(st);
     launches = 3;
+  } else if (sub_batch_tokens(s->B) >= s->B) {
+    // One batch: the three launches in order on the caller's stream.
+    tr.begin(0, st);
+    e = pkm::launch_query_tc(a, w.planes, st);
+    tr.end(st);
+    tr.begin(1, st);
+    if (e == cudaSuccess) e = pkm::launch_score_topk_tc(a, w.planes, w.list_s, w.list_i, st);
+    tr.end(st);
+    tr.begin(2, st);
+    if (e == cudaSuccess)
+      e = pkm::launch_select_gather(a, w.list_s, w.list_i, out, indices, weights, scores, st);
+    tr.end(st);
+    launches = 3;
   } else {
-    // Pipelined over sub-batches: the query network and per-half search of sub-batch
-    // i+1 run on the caller's stream while the gather of sub-batch i runs on a second
-    // stream (it is bound by HBM, the others by the tensor cores and ALUs). The second
-    // stream waits for each sub-batch's lists and the caller's stream waits for the
-    // last gather, so the call stays ordered on `stream`.
+    // Pipelined over sub-batches (PKM_OPT_SUBBATCHES > 1): the query network and
+    // per-half search of sub-batch i+1 run on the caller's stream while the gather of
+    // sub-batch i runs on the library's second stream (it is bound by HBM, the others
+    // by the tensor cores and ALUs). The second stream waits for each sub-batch's
+    // lists and the caller's stream waits for the last gather, so the call stays
+    // ordered on `stream`.
     const int64_t sub = sub_batch_tokens(s->B);
     const int nsub = static_cast<int>((s->B + sub - 1) / sub);
     cudaStream_t aux;

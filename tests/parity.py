@@ -34,6 +34,19 @@ def allclose_report(name, got, ref, rtol=RTOL, atol=ATOL):
     return float(err.max()) if err.size else 0.0
 
 
+def grad_report(name, got, ref, rtol=RTOL, atol=ATOL):
+    """Gradient tensor against the oracle with the stated bar |got - ref| <=
+    atol + rtol |ref| elementwise (no scaling with the tensor's size). Prints and
+    returns the worst error as a fraction of its element's bar (<= 1 passes)."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64).reshape(got.shape)
+    allclose_report(name, got, ref, rtol, atol)
+    frac = float((np.abs(got - ref) / (atol + rtol * np.abs(ref))).max()) if got.size else 0.0
+    print("%s: worst error %.3g of the bar, max |ref| %.3g" % (
+        name, frac, float(np.abs(ref).max()) if ref.size else 0.0))
+    return frac
+
+
 def compare_forward(gpu: dict, ref: dict, values_cpu: torch.Tensor, n: int, *,
                     rtol=RTOL, atol=ATOL, rel_tie=REL_TIE, max_exempt_frac=0.01):
     """gpu: numpy out/indices/weights/scores for the same tokens as ref (oracle with

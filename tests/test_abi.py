@@ -4,6 +4,8 @@ CUDA call (so these run without a GPU)."""
 import ctypes
 import os
 import re
+import subprocess
+import sys
 
 import pytest
 
@@ -39,22 +41,49 @@ def _shape(**kw):
     return P.make_shape(**base)
 
 
-def test_workspace_sizes(monkeypatch):
+def test_workspace_sizes():
     s = _shape()
     lists = 16384 * 4 * 2 * 32 * 8            # best 32 per half: fp32 score + int32 id
     fw = P.pkm_workspace_size(s)
     # tensor-core path: status + three bf16 q planes per token of a sub-batch + lists
     assert fw >= 256 + 16384 * 2048 * 6 + lists
-    monkeypatch.setenv("PKM_SUBBATCHES", "4")
-    assert 256 + 4096 * 2048 * 6 + lists <= P.pkm_workspace_size(s) < fw
-    monkeypatch.delenv("PKM_SUBBATCHES")
-    monkeypatch.setenv("PKM_PATH", "simt")
-    # CUDA-core path: fp32 q for every token
-    assert P.pkm_workspace_size(s) >= 256 + 16384 * 2048 * 4 + lists
-    monkeypatch.delenv("PKM_PATH")
+    with P.options(subbatches=4):
+        assert 256 + 4096 * 2048 * 6 + lists <= P.pkm_workspace_size(s) < fw
+    with P.options(path="simt"):
+        # CUDA-core path: fp32 q for every token
+        assert P.pkm_workspace_size(s) >= 256 + 16384 * 2048 * 4 + lists
+    assert P.pkm_workspace_size(s) == fw
     bw = P.pkm_workspace_size(s, True)
     assert bw >= 256 + 4 * (2 * 1024 * 1024 + 16384 * 4 * 32)
     assert P.pkm_workspace_size(_shape(B=0)) > 0
+
+
+def test_options_set_get_and_reject():
+    assert P.pkm_get_option(P.PKM_OPT_PATH) == P.PKM_PATH_AUTO
+    assert P.pkm_get_option(P.PKM_OPT_SUBBATCHES) == 1
+    with P.options(path="tc", subbatches=3):
+        assert P.pkm_get_option(P.PKM_OPT_PATH) == P.PKM_PATH_TC
+        assert P.pkm_get_option(P.PKM_OPT_SUBBATCHES) == 3
+    assert P.pkm_get_option(P.PKM_OPT_PATH) == P.PKM_PATH_AUTO
+    assert P.pkm_get_option(P.PKM_OPT_SUBBATCHES) == 1
+    L = P.lib()
+    assert L.pkm_set_option(P.PKM_OPT_PATH, 7) == -1
+    assert L.pkm_set_option(P.PKM_OPT_SUBBATCHES, 0) == -1
+    assert L.pkm_set_option(P.PKM_OPT_SUBBATCHES, 5) == -1
+    assert L.pkm_set_option(9, 1) == -1
+    assert L.pkm_get_option(9) == -1
+    assert P.pkm_get_option(P.PKM_OPT_SUBBATCHES) == 1
+
+
+def test_environment_gives_initial_options():
+    """PKM_PATH / PKM_SUBBATCHES are read once, as the initial option values."""
+    code = ("import product_key_memory_b200 as P; "
+            "print(P.pkm_get_option(P.PKM_OPT_PATH), P.pkm_get_option(P.PKM_OPT_SUBBATCHES))")
+    env = dict(os.environ, PKM_PATH="simt", PKM_SUBBATCHES="3", PYTHONPATH=ROOT)
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True,
+                       timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.split() == ["2", "3"]
 
 
 @pytest.mark.parametrize("kw,code", [

@@ -3,10 +3,9 @@ the C ABI.
 
 Both sides hold the same picks fixed: the device forward's indices and weights
 (fp32) go to the oracle as they are, so near-ties in the forward play no part.
-Tolerance for every gradient tensor G: |got - ref| <= 2e-3 |ref| + 1e-4 max(1, max|ref|).
-The second term scales the absolute bar with the tensor's size: grad_W_q,
-grad_bn_* and grad_subkeys are fp32 sums over thousands of tokens whose terms
-cancel, so an element near zero carries the rounding of its large terms.
+Tolerance for every element of every gradient tensor: |got - ref| <= 1e-4 + 2e-3 |ref|
+(the stated bar, with no scaling by the tensor's size). Each check prints its worst
+error as a fraction of that bar.
 """
 import concurrent.futures as cf
 import os
@@ -17,7 +16,7 @@ import torch
 
 import oracle
 import synth
-from parity import allclose_report
+from parity import grad_report
 
 pytestmark = pytest.mark.gpu
 
@@ -32,23 +31,11 @@ def _P():
 
 
 def _grad_check(name, got, ref):
-    ref = np.asarray(ref, np.float64)
-    scale = max(1.0, float(np.abs(ref).max()) if ref.size else 1.0)
-    return allclose_report(name, got, ref, rtol=2e-3, atol=1e-4 * scale)
+    return grad_report(name, got, ref)
 
 
 def _with_path(path):
-    class _Ctx:
-        def __enter__(self):
-            self.old = os.environ.get("PKM_PATH")
-            os.environ["PKM_PATH"] = path
-
-        def __exit__(self, *a):
-            if self.old is None:
-                os.environ.pop("PKM_PATH", None)
-            else:
-                os.environ["PKM_PATH"] = self.old
-    return _Ctx()
+    return _P().options(path=path)
 
 
 def _device_forward_backward(L, w, gout, path="auto", want=NAMES, init_values=None):
@@ -171,8 +158,9 @@ def test_partial_requests_leave_the_rest_alone():
     _compare_all(L, w, idx, wt, gout, g, _oracle_full(L, idx, wt, gout, w), init_values=init)
 
 
-def test_matches_value_backward_bit_for_bit():
-    """grad_scores and grad_values come from the same kernels as pkm_backward_values."""
+def test_matches_value_backward():
+    """grad_scores and grad_values come from the same kernels as pkm_backward_values:
+    grad_scores equal bit for bit, grad_values within fp32 summation-order rounding."""
     w = synth.WORKLOADS["c512"].with_(B=300, n=256)
     L = synth.make_layer(w)
     gout = synth.make_grad_out(w)

@@ -14,7 +14,7 @@ import torch
 
 import oracle
 import synth
-from parity import allclose_report, compare_forward, to_numpy
+from parity import allclose_report, compare_forward, grad_report, to_numpy
 
 pytestmark = pytest.mark.gpu
 
@@ -24,19 +24,8 @@ def _P():
     return mod
 
 
-class _Path:
-    def __init__(self, path):
-        self.path = path
-
-    def __enter__(self):
-        self.old = os.environ.get("PKM_PATH")
-        os.environ["PKM_PATH"] = self.path
-
-    def __exit__(self, *a):
-        if self.old is None:
-            os.environ.pop("PKM_PATH", None)
-        else:
-            os.environ["PKM_PATH"] = self.old
+def _Path(path):
+    return _P().options(path=path)
 
 
 def _layer(name, **kw):
@@ -93,9 +82,7 @@ def test_running_statistics_momentum_limits():
 
 
 def _grad_check(name, got, ref):
-    ref = np.asarray(ref, np.float64)
-    scale = max(1.0, float(np.abs(ref).max()) if ref.size else 1.0)
-    return allclose_report(name, got, ref, rtol=2e-3, atol=1e-4 * scale)
+    return grad_report(name, got, ref)
 
 
 def _check_backward(L, w, path="auto"):

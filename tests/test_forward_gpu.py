@@ -39,20 +39,13 @@ def _to_dev(L):
 
 
 def _gpu_forward(L, w, path="auto"):
-    old = os.environ.get("PKM_PATH")
-    os.environ["PKM_PATH"] = path
-    try:
+    with _lib().options(path=path):
         d = _to_dev(L)
         out, idx, wt, sc = _lib().pkm_forward(d["x"], d["W_q"], d["bn_mean"], d["bn_var"],
                                               d["bn_gamma"], d["bn_beta"], d["subkeys"],
                                               d["values"], k=w.k)
         torch.cuda.synchronize()
         return to_numpy(out, idx, wt, sc)
-    finally:
-        if old is None:
-            os.environ.pop("PKM_PATH", None)
-        else:
-            os.environ["PKM_PATH"] = old
 
 
 def _check(L, w, rows=None, path="auto", **kw):

@@ -24,23 +24,13 @@ def _P():
 
 
 def _forward(L, w, path=None):
-    old = os.environ.get("PKM_PATH")
-    if path is None:
-        os.environ.pop("PKM_PATH", None)
-    else:
-        os.environ["PKM_PATH"] = path
-    try:
+    with _P().options(path=path or "auto"):
         d = {k: v.cuda() for k, v in L.items()}
         out, idx, wt, sc = _P().pkm_forward(d["x"], d["W_q"], d["bn_mean"], d["bn_var"],
                                             d["bn_gamma"], d["bn_beta"], d["subkeys"],
                                             d["values"], k=w.k)
         torch.cuda.synchronize()
         return to_numpy(out, idx, wt, sc)
-    finally:
-        if old is None:
-            os.environ.pop("PKM_PATH", None)
-        else:
-            os.environ["PKM_PATH"] = old
 
 
 def _check(L, w):
