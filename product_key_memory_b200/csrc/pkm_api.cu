@@ -96,7 +96,7 @@ int validate_shape(const pkm_shape* s) {
 struct ForwardWs {
   int* status;
   float* q;         // SIMT path: fp32 q [B][H*dq]
-  void* planes;     // tensor path: bf16 q planes [3][sub][H*dq] of one sub-batch
+  void* planes;     // tensor path: bf16 q planes [kScorePlanes][sub][H*dq] of a sub-batch
   float* list_s;    // [B][H][2][32] best 32 per half (any order)
   int* list_i;      // [B][H][2][32]
 };
@@ -118,7 +118,8 @@ size_t forward_ws(const pkm_shape* s, ForwardWs* w, char* base) {
   const int64_t F = static_cast<int64_t>(s->H) * s->dq;
   const Path path = choose_path(s);
   const size_t qbytes = path == Path::kTensor
-                            ? static_cast<size_t>(sub_batch_tokens(s->B)) * F * 6
+                            ? static_cast<size_t>(sub_batch_tokens(s->B)) * F * 2 *
+                                  pkm::kScorePlanes
                             : static_cast<size_t>(s->B) * F * 4;
   // The small-batch path keeps each chunk's best 32 before merging them.
   const int64_t L = path == Path::kSmall

@@ -1,6 +1,7 @@
 // pkm_tc.cu -- tensor-core (tcgen05 / TMEM / TMA) kernels for sm_100a:
 //
-//   query_tc_kernel        q = BN(x W_q^T), written as three bf16 planes hi/mid/lo
+//   query_tc_kernel        q = BN(x W_q^T), written as bf16 planes hi/lo (the forward)
+//                          or acc = x W_q^T as hi/mid/lo (batch statistics, backward)
 //   score_topk_tc_kernel   s = q_half C^T per (128-token tile, head, half), scored in
 //                          256-sub-key chunks into TMEM; one epilogue thread per row
 //                          keeps the row's best 32 sub-keys: the scores never reach HBM
@@ -24,9 +25,12 @@
 //
 // Precision: q is an fp32 result. Rounding it to bf16 before scoring would move
 // scores by ~1e-3 relative, far more than the gaps that decide which keys are
-// kept, so the query kernel writes q = hi + mid + lo (three bf16 values, exact to
-// ~2^-24 relative) and the scoring kernel issues three MMAs per K step into one fp32
-// accumulator. Sub-keys are bf16 and exact.
+// kept, so the query kernel writes q = hi + lo (hi = RN(q), lo = RN(q - hi): the
+// residual is at most 2^-16 |q|, about 2^-18 |q| on average) and the scoring kernel
+// issues two MMAs per K step into one fp32 accumulator. That residual is at the
+// level of the tensor cores' own fp32 accumulation error on these sums (about
+// 1e-5 absolute on per-half scores near 3), and far below the 1e-5 relative window
+// in which two keys count as tied. Sub-keys are bf16 and exact.
 #include <mutex>
 
 #include "pkm_common.cuh"
@@ -56,8 +60,8 @@ constexpr uint32_t kQABytes = kRowsPerTile * kKBlock * 2;  // 16 KiB
 constexpr uint32_t kQBBytes = kColsPerMma * kKBlock * 2;   // 32 KiB
 constexpr uint32_t kQStageBytes = kQABytes + kQBBytes;
 constexpr int kQMaxF = 4096;  // BN scale/shift of every feature live in shared memory
-// Output staging: per epilogue warp, its 32 rows x 32 columns of each of the 3 planes
-// (64-byte rows, 64-byte swizzle), written to HBM by TMA tensor stores.
+// Output staging: per epilogue warp, its 32 rows x 32 columns of each plane (up to 3;
+// 64-byte rows, 64-byte swizzle), written to HBM by TMA tensor stores.
 constexpr uint32_t kQStagePlane = 32 * 32 * 2;             // 2 KiB
 constexpr uint32_t kQStageWarp = 3 * kQStagePlane;         // 6 KiB
 
@@ -70,7 +74,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) query_tc_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
     const __grid_constant__ CUtensorMap tm_out, const float* __restrict__ mean,
     const float* __restrict__ var, const float* __restrict__ gamma,
-    const float* __restrict__ beta, float eps, int B, int d, int F, int raw_acc, int* status) {
+    const float* __restrict__ beta, float eps, int B, int d, int F, int raw_acc, int nplanes,
+    int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* stages = align1024(smem_raw);
   float* scale_s = reinterpret_cast<float*>(stages + kQStages * kQStageBytes);
@@ -221,6 +226,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) query_tc_kernel(
         for (int i = 0; i < 32; i += 2) {
           const float q0 = fmaf(v[i], scale_s[f0 + i], shift_s[f0 + i]);
           const float q1 = fmaf(v[i + 1], scale_s[f0 + i + 1], shift_s[f0 + i + 1]);
+          // hi = RN(q), mid = RN(q - hi), lo = RN(q - hi - mid); the forward's two
+          // planes are hi and mid.
           split3_pair(q0, q1, ph_[i / 2], pm[i / 2], pl[i / 2]);
         }
         // The previous group's stores must have read the staging tile before it is
@@ -234,8 +241,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) query_tc_kernel(
               make_uint4(ph_[4 * c], ph_[4 * c + 1], ph_[4 * c + 2], ph_[4 * c + 3]);
           *reinterpret_cast<uint4*>(my_row + kQStagePlane + pos) =
               make_uint4(pm[4 * c], pm[4 * c + 1], pm[4 * c + 2], pm[4 * c + 3]);
-          *reinterpret_cast<uint4*>(my_row + 2 * kQStagePlane + pos) =
-              make_uint4(pl[4 * c], pl[4 * c + 1], pl[4 * c + 2], pl[4 * c + 3]);
+          if (nplanes == 3)
+            *reinterpret_cast<uint4*>(my_row + 2 * kQStagePlane + pos) =
+                make_uint4(pl[4 * c], pl[4 * c + 1], pl[4 * c + 2], pl[4 * c + 3]);
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -244,7 +252,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) query_tc_kernel(
           // Rows past B in a partly filled box lie outside the tensor map and are not
           // written; a box that starts past B is not issued at all.
 #pragma unroll
-          for (int p = 0; p < 3; ++p) tma_store_3d(&tm_out, stg + p * kQStagePlane, f0, row0, p);
+          for (int p = 0; p < 3; ++p)
+            if (p < nplanes) tma_store_3d(&tm_out, stg + p * kQStagePlane, f0, row0, p);
           bulk_commit();
         }
       }
@@ -276,9 +285,9 @@ constexpr int kSStages = kSSets == 2 ? 3 : 2;
 constexpr CUtensorMapSwizzle kSSwizzle =
     kSK == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
 constexpr uint32_t kSPlaneBytes = kRowsPerTile * kSK * 2;           // 8 KiB
-constexpr uint32_t kSABytes = 3 * kSPlaneBytes;                     // 24 KiB
+constexpr uint32_t kSABytes = kScorePlanes * kSPlaneBytes;          // 16 KiB
 constexpr uint32_t kSBBytes = kColsPerMma * kSK * 2;                // 16 KiB
-constexpr uint32_t kSStageBytes = kSABytes + kSBBytes;              // 40 KiB
+constexpr uint32_t kSStageBytes = kSABytes + kSBBytes;              // 32 KiB
 constexpr int kList = kMaxK;          // entries per per-half list (the best 32, any order)
 constexpr int kSStep = 8;             // columns read from TMEM per step
 constexpr int kSNewCap = 32;          // survivors logged between two merges
@@ -347,7 +356,10 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
   const int nunits = mt * HS;
   const int nchunks = n / kColsPerMma;
   const int kiters = half / kSK;
-  // This CTA's units are blockIdx.x + j * gridDim.x; set s takes the j with j % 2 == s.
+  // This CTA's units are nunits - 1 - (blockIdx.x + j * gridDim.x); set s takes the j
+  // with j % 2 == s. Units run from the last token tile down: the query kernel writes
+  // the q planes in tile order, so the most recently written tiles, the ones most
+  // likely still in L2, are scored first.
   const int myunits = nunits > static_cast<int>(blockIdx.x)
                           ? (nunits - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1
                           : 0;
@@ -380,7 +392,7 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- TMA producer: per K step three q planes + one sub-key tile, in
+      // ---------------- TMA producer: per K step the q planes + one sub-key tile, in
       // the order the MMA issuer consumes them (chunks of the two sets interleaved)
       uint32_t s = 0, ph = 0;
       uint32_t issued_phase[kSStages];
@@ -392,7 +404,7 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
           for (int set = 0; set < kSSets && ok; ++set) {
             const int j = j0 + set;
             if (j >= myunits) break;
-            const int u = blockIdx.x + j * gridDim.x;
+            const int u = nunits - 1 - static_cast<int>(blockIdx.x + j * gridDim.x);
             const int m = u / HS, hs = u - m * HS;
             const int xq = (hs >> 1) * dq + (hs & 1) * half;
             for (int kb = 0; kb < kiters; ++kb) {
@@ -400,7 +412,7 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
               uint8_t* a = stages + s * kSStageBytes;
               mbar_arrive_expect_tx(&full[s], kSStageBytes);
 #pragma unroll
-              for (int p = 0; p < 3; ++p)
+              for (int p = 0; p < kScorePlanes; ++p)
                 tma_load_3d(a + p * kSPlaneBytes, &tm_planes, &full[s], xq + kb * kSK,
                             m * kRowsPerTile, p);
               tma_load_2d(a + kSABytes, &tm_keys, &full[s], kb * kSK, hs * n + c * kColsPerMma);
@@ -421,7 +433,7 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      // ---------------- MMA issuer: chunk of 256 sub-keys = kiters x 3 planes x 2 MMAs
+      // ---------------- MMA issuer: chunk of 256 sub-keys = kiters x planes x 2 MMAs
       const uint32_t idesc = idesc_bf16_f32(kRowsPerTile, kColsPerMma);
       uint32_t s = 0, ph = 0;
       int uses[kSSets] = {};  // chunks written into each set's accumulators so far
@@ -442,7 +454,7 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
               const uint32_t a = smem_addr(stages + s * kSStageBytes);
               const uint32_t bb = a + kSABytes;
 #pragma unroll
-              for (int p = 0; p < 3; ++p)
+              for (int p = 0; p < kScorePlanes; ++p)
 #pragma unroll
                 for (int jj = 0; jj < kSK / 16; ++jj) {
                   const uint64_t ad = kSK == 32 ? sw64_desc(a + p * kSPlaneBytes, jj * 32)
@@ -479,7 +491,7 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
     constexpr int kStepsPerChunk = kColsPerMma / kSStep;
     int uses = 0;
     for (int j = set; j < myunits; j += kSSets) {
-      const int u = blockIdx.x + j * gridDim.x;
+      const int u = nunits - 1 - static_cast<int>(blockIdx.x + j * gridDim.x);
       const int m = u / HS, hs = u - m * HS;
       float Ls[32];
 #pragma unroll
@@ -703,6 +715,7 @@ bool tc_supported(int dtype, int d_model, int H, int dq, int n, int k) {
 
 cudaError_t launch_query_tc(const LayerArgs& a, void* planes, cudaStream_t st) {
   const int F = a.H * a.dq;
+  const int nplanes = a.raw_acc ? 3 : kScorePlanes;
   CUtensorMap tm_x, tm_w;
   const cuuint64_t xd[2] = {static_cast<cuuint64_t>(a.d_model), static_cast<cuuint64_t>(a.B)};
   const cuuint64_t xs[1] = {static_cast<cuuint64_t>(a.d_model) * 2};
@@ -710,7 +723,8 @@ cudaError_t launch_query_tc(const LayerArgs& a, void* planes, cudaStream_t st) {
   const cuuint64_t wd[2] = {static_cast<cuuint64_t>(a.d_model), static_cast<cuuint64_t>(F)};
   const cuuint32_t wb[2] = {kKBlock, kColsPerMma};
   CUtensorMap tm_out;
-  const cuuint64_t od[3] = {static_cast<cuuint64_t>(F), static_cast<cuuint64_t>(a.B), 3};
+  const cuuint64_t od[3] = {static_cast<cuuint64_t>(F), static_cast<cuuint64_t>(a.B),
+                            static_cast<cuuint64_t>(nplanes)};
   const cuuint64_t os[2] = {static_cast<cuuint64_t>(F) * 2, static_cast<cuuint64_t>(F) * 2 * a.B};
   const cuuint32_t ob[3] = {32, 32, 1};
   if (!make_map(&tm_x, a.x, 2, xd, xs, xb) || !make_map(&tm_w, a.W_q, 2, wd, xs, wb) ||
@@ -724,7 +738,7 @@ cudaError_t launch_query_tc(const LayerArgs& a, void* planes, cudaStream_t st) {
   query_tc_kernel<<<grid, kTcThreads, smem, st>>>(tm_x, tm_w, tm_out, a.bn_mean, a.bn_var,
                                                   a.bn_gamma, a.bn_beta, a.bn_eps,
                                                   static_cast<int>(a.B), a.d_model, F, a.raw_acc,
-                                                  a.status);
+                                                  nplanes, a.status);
   return cudaGetLastError();
 }
 
@@ -733,7 +747,8 @@ cudaError_t launch_score_topk_tc(const LayerArgs& a, const void* planes, float* 
   const int F = a.H * a.dq;
   const int half = a.dq / 2;
   CUtensorMap tm_p, tm_k;
-  const cuuint64_t pd[3] = {static_cast<cuuint64_t>(F), static_cast<cuuint64_t>(a.B), 3};
+  const cuuint64_t pd[3] = {static_cast<cuuint64_t>(F), static_cast<cuuint64_t>(a.B),
+                            static_cast<cuuint64_t>(kScorePlanes)};
   const cuuint64_t ps[2] = {static_cast<cuuint64_t>(F) * 2, static_cast<cuuint64_t>(F) * 2 * a.B};
   const cuuint32_t pb[3] = {kSK, kRowsPerTile, 1};
   const cuuint64_t kd[2] = {static_cast<cuuint64_t>(half),

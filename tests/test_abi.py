@@ -45,10 +45,10 @@ def test_workspace_sizes():
     s = _shape()
     lists = 16384 * 4 * 2 * 32 * 8            # best 32 per half: fp32 score + int32 id
     fw = P.pkm_workspace_size(s)
-    # tensor-core path: status + three bf16 q planes per token of a sub-batch + lists
-    assert fw >= 256 + 16384 * 2048 * 6 + lists
+    # tensor-core path: status + two bf16 q planes per token of a sub-batch + lists
+    assert fw >= 256 + 16384 * 2048 * 4 + lists
     with P.options(subbatches=4):
-        assert 256 + 4096 * 2048 * 6 + lists <= P.pkm_workspace_size(s) < fw
+        assert 256 + 4096 * 2048 * 4 + lists <= P.pkm_workspace_size(s) < fw
     with P.options(path="simt"):
         # CUDA-core path: fp32 q for every token
         assert P.pkm_workspace_size(s) >= 256 + 16384 * 2048 * 4 + lists
