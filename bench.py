@@ -479,6 +479,21 @@ def run_c512_and_backward(args, dev, P, hbm, bf16, stream, world, barrier,
             "algorithmic_bytes": bytes_alg, "achieved_gbs": bytes_alg / (bwd_ms * 1e-3) / 1e9,
             "frac_of_hbm": bytes_alg / (bwd_ms * 1e-3) / 1e9 / hbm,
             "stage_ms": [m / max(1, bcalls) for m in bstage[:2]]}
+        # The same call on skewed picks: every pick from 40 of the 262,144 slots (about
+        # 13,000 picks per touched row), the case a per-pick atomic scatter serialises on.
+        hidx, hw = synth.random_selection(B, w.H, w.k, w.n * w.n, seed=77, hot_rows=40)
+        hidx, hw = hidx.to(dev), hw.to(dev)
+
+        def bwd_hot():
+            P.pkm_backward_values(d["values"], hidx, hw, gout, gv, gs, w.n, workspace=bws)
+
+        for _ in range(max(3, args.warmup)):
+            bwd_hot()
+        hot_ms = timed(bwd_hot, args.steps)
+        res["backward"]["skewed"] = {
+            "picks_from_slots": 40, "ms_per_step": hot_ms,
+            "value": world * B / (hot_ms / 1e3), "unit": UNIT,
+            "vs_uniform": hot_ms / bwd_ms}
     P.pkm_trace_enable(False)
 
     # Full backward on the same picks: every gradient of the layer (x, W_q, BatchNorm

@@ -105,9 +105,12 @@ size_t pkm_workspace_size(const pkm_shape* s, int for_backward);
  *   scores   [B][H][k]  fp32   kept key scores s1[i] + s2[j]; may be NULL
  * workspace: device scratch of at least pkm_workspace_size(s, 0) bytes, 256-byte
  *   aligned; its contents on entry do not matter.
- * Batches of at most 128 tokens (H <= 8) take the small-batch kernels, which spread
- * W_q, the sub-keys and the heads over all SMs for latency; their three launches
- * overlap through programmatic dependent launch on `stream`. Larger batches run
+ * Batches of at most 128 tokens (H <= 8) take the small-batch path, which spreads
+ * W_q, the sub-keys and the heads over all SMs for latency: three kernels that
+ * overlap through programmatic dependent launch on `stream`, or, with
+ * PKM_PATH_SMALL_FUSED, one cooperative kernel (one block per SM, its query, scoring
+ * and gather phases separated by grid-wide barriers whose waits are bounded like the
+ * pipelines'). Larger batches run
  * three kernels on `stream` (query network, per-half scores and top-k, candidate
  * top-k + softmax + gather). With PKM_OPT_SUBBATCHES > 1, large batches of
  * tensor-core shapes are processed in up to that many sub-batches; the value gather
@@ -135,9 +138,12 @@ int pkm_forward(const pkm_shape* s, const void* x, const void* W_q, const float*
  *   grad_out    [B][v]     dtype
  *   grad_values [n*n][v]   fp32   ACCUMULATED into (the caller zeroes it once)
  *   grad_scores [B][H][k]  fp32   overwritten; may be NULL
- * Picks are grouped by slot with a counting sort, so each touched row is read and
- * written once per group rather than once per pick. Slot ids outside [0, n*n) are
- * skipped and counted in the status word (PKM_ERR_DEVICE).
+ * Picks are grouped by slot with a stable radix sort, so each slot's picks are summed
+ * in pick order and each touched row is read and written once, whatever the number of
+ * picks that hit it (large groups are split over several blocks whose partial sums are
+ * added in a fixed order). The result is bit-for-bit the same on every run, and no
+ * row is updated with atomics. Slot ids outside [0, n*n) are skipped and counted in
+ * the status word (PKM_ERR_DEVICE).
  * Only B, H, n, k, v and dtype of the shape are read; d_model, dq and bn_eps are
  * ignored.
  * workspace: at least pkm_workspace_size(s, 1) bytes, 256-byte aligned.
@@ -232,10 +238,10 @@ int pkm_backward_train(const pkm_shape* s, const void* x, const void* W_q,
  * host that passes device pointers but no allocator). Arguments and results are
  * those of pkm_backward_values; the caller still passes inputs and outputs.
  *
- * Scratch: one fixed 16 MiB device array inside libpkm.so, held on every GPU that
- * loads the library until the process exits. Limits: n*n <= 1,048,576 slots and
- * B*H*k <= 2,097,152 picks; larger shapes return PKM_ERR_UNSUPPORTED before any
- * launch. The call allocates nothing (no cudaMalloc, no library allocator).
+ * Scratch: one fixed device array of about 40.3 MiB inside libpkm.so, held on every
+ * GPU that loads the library until the process exits. Limits: n*n <= 1,048,576 slots,
+ * B*H*k <= 2,097,152 picks and v <= 2048; larger shapes return PKM_ERR_UNSUPPORTED
+ * before any launch. The call allocates nothing (no cudaMalloc, no library allocator).
  * The first call on a device looks up the array's device address with that device
  * current; make that first call before any stream capture. All calls share the
  * one array (each call clears what must start at zero), so calls that overlap on
@@ -289,14 +295,17 @@ int pkm_trace_read(int pass, double* stage_ms, int max_stages, int64_t* calls,
 /*
  * Implementation switches (a convenience of this library; the pages have no
  * counterpart). Process-wide, for every device; a change applies to calls made after
- * it. The environment variables PKM_PATH (auto | tc | simt) and PKM_SUBBATCHES (1..4)
+ * it. The environment variables PKM_PATH (auto | tc | simt | small_fused) and
+ * PKM_SUBBATCHES (1..4)
  * give the initial values and are read once, at the first call that needs them.
  *   PKM_OPT_PATH        PKM_PATH_AUTO (default): small-batch kernels for up to 128
  *                       tokens, else the tensor-core kernels where the layer fits
  *                       their tiles (bf16, d_model and dq/2 multiples of 64, n a
  *                       multiple of 256, H*dq <= 4096), else the CUDA-core kernels;
  *                       PKM_PATH_TC: never the small-batch kernels;
- *                       PKM_PATH_SIMT: always the CUDA-core kernels.
+ *                       PKM_PATH_SIMT: always the CUDA-core kernels;
+ *                       PKM_PATH_SMALL_FUSED: as AUTO, but small batches run as one
+ *                       cooperative kernel instead of three kernels.
  *   PKM_OPT_SUBBATCHES  1 (default) to 4: sub-batches of the pipelined tensor-core
  *                       forward (see pkm_forward). The forward's workspace size
  *                       depends on it: query it after setting the option.
@@ -304,7 +313,7 @@ int pkm_trace_read(int pass, double* stage_ms, int max_stages, int64_t* calls,
  * pkm_get_option returns the current value or PKM_ERR_INVALID_ARG.
  */
 enum { PKM_OPT_PATH = 0, PKM_OPT_SUBBATCHES = 1 };
-enum { PKM_PATH_AUTO = 0, PKM_PATH_TC = 1, PKM_PATH_SIMT = 2 };
+enum { PKM_PATH_AUTO = 0, PKM_PATH_TC = 1, PKM_PATH_SIMT = 2, PKM_PATH_SMALL_FUSED = 3 };
 int pkm_set_option(int option, int value);
 int pkm_get_option(int option);
 

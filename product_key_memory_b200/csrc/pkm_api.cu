@@ -28,7 +28,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 enum class Path { kTensor, kSimt, kSmall };
 
 // Process-wide implementation switches (pkm_set_option). The environment variables
-// PKM_PATH (auto | tc | simt) and PKM_SUBBATCHES (1..4) give their initial values and
+// PKM_PATH (auto | tc | simt | small_fused) and PKM_SUBBATCHES (1..4) give their initial values and
 // are read once, at the first call that needs them.
 std::atomic<int> g_opt_path{PKM_PATH_AUTO};
 std::atomic<int> g_opt_subbatches{1};
@@ -39,6 +39,7 @@ void init_options() {
     const char* p = getenv("PKM_PATH");
     if (p && strcmp(p, "simt") == 0) g_opt_path = PKM_PATH_SIMT;
     if (p && strcmp(p, "tc") == 0) g_opt_path = PKM_PATH_TC;
+    if (p && strcmp(p, "small_fused") == 0) g_opt_path = PKM_PATH_SMALL_FUSED;
     const char* sb = getenv("PKM_SUBBATCHES");
     if (sb) {
       const int v = atoi(sb);
@@ -161,7 +162,8 @@ size_t forward_train_ws(const pkm_shape* s, ForwardWs* fw, TrainWs* tw, char* ba
 }
 
 size_t backward_ws(const pkm_shape* s, pkm::BackwardWs* w, char* base) {
-  return pkm::backward_ws_bytes(s->B, s->H, s->k, static_cast<int64_t>(s->n) * s->n, w, base);
+  return pkm::backward_ws_bytes(s->B, s->H, s->k, static_cast<int64_t>(s->n) * s->n, s->v, w,
+                               base);
 }
 
 // ---------------------------------------------------------------------------
@@ -303,7 +305,8 @@ extern "C" {
 int pkm_set_option(int option, int value) {
   init_options();
   if (option == PKM_OPT_PATH) {
-    if (value != PKM_PATH_AUTO && value != PKM_PATH_TC && value != PKM_PATH_SIMT)
+    if (value != PKM_PATH_AUTO && value != PKM_PATH_TC && value != PKM_PATH_SIMT &&
+        value != PKM_PATH_SMALL_FUSED)
       return PKM_ERR_INVALID_ARG;
     g_opt_path = value;
     return PKM_OK;
@@ -531,9 +534,17 @@ cudaError_t run_forward(const pkm_shape* s, const LayerArgs& a, const ForwardWs&
   const Path path = choose_path(s);
   if (path == Path::kSmall) {
     tr.begin(2, st);
-    e = pkm::launch_forward_small(a, w.q, w.list_s, w.list_i, out, indices, weights, scores, st);
+    if (g_opt_path.load(std::memory_order_relaxed) == PKM_PATH_SMALL_FUSED &&
+        pkm::small_fused_supported(s->d_model, s->H, s->dq, s->n, s->v, s->dtype)) {
+      e = pkm::launch_forward_small_fused(a, w.q, w.list_s, w.list_i, out, indices, weights,
+                                          scores, st);
+      launches = 1;
+    } else {
+      e = pkm::launch_forward_small(a, w.q, w.list_s, w.list_i, out, indices, weights, scores,
+                                    st);
+      launches = 3;
+    }
     tr.end(st);
-    launches = 3;
   } else if (path == Path::kSimt) {
     tr.begin(0, st);
     e = pkm::launch_query_bn_simt(a, w.q, st);
@@ -630,7 +641,8 @@ int pkm_forward(const pkm_shape* s, const void* x, const void* W_q, const float*
   forward_ws(s, &w, static_cast<char*>(workspace));
   LayerArgs a{s->B, s->d_model, s->H, s->dq, s->n, s->k, s->v, s->dtype, s->bn_eps,
               x, W_q, bn_mean, bn_var, bn_gamma, bn_beta, subkeys, values, w.status, 0};
-  if (cudaMemsetAsync(w.status, 0, sizeof(int), st) != cudaSuccess) return PKM_ERR_CUDA;
+  // The status word and the small-batch kernel's grid-barrier counter after it.
+  if (cudaMemsetAsync(w.status, 0, 2 * sizeof(int), st) != cudaSuccess) return PKM_ERR_CUDA;
   Tracer tr(0);
   int launches = 0;
   tr.begin(3, st);
@@ -672,7 +684,7 @@ int pkm_forward_train(const pkm_shape* s, const void* x, const void* W_q,
   a.bn_mean = batch_mean;
   a.bn_var = batch_var;
   a.raw_acc = 0;
-  if (cudaMemsetAsync(w.status, 0, sizeof(int), st) != cudaSuccess) return PKM_ERR_CUDA;
+  if (cudaMemsetAsync(w.status, 0, 2 * sizeof(int), st) != cudaSuccess) return PKM_ERR_CUDA;
   Tracer tr(0);
   int launches = 0;
   tr.begin(3, st);
@@ -727,7 +739,8 @@ int pkm_backward_values(const pkm_shape* s, const void* values, const int32_t* i
       });
   tr.end(st);
   tr.end(st);
-  tr.finish(e == cudaSuccess, grad_scores ? 7 : 6);
+  tr.finish(e == cudaSuccess, pkm::backward_values_launches(static_cast<int64_t>(s->n) * s->n,
+                                                           grad_scores != nullptr, true));
   return e == cudaSuccess ? PKM_OK : PKM_ERR_CUDA;
 }
 

@@ -7,12 +7,18 @@
 //   grad wrt kept score j:  w_j (g_j - sum_l w_l g_l),  g_j = <grad_out[t], V[slot_j]>
 //   grad wrt V[slot]:       sum over the picks of that slot of w * grad_out[t]
 //
-// The value gradient groups the B*H*k picks by slot with a counting sort
-// (histogram, exclusive scan, scatter), then one warp walks each window of 32
-// sorted picks, sums w * grad_out[t] per slot in registers and writes each slot's
-// row once: a plain read-modify-write when the slot's group lies inside the
-// window, a vector atomic add only for groups that cross a window edge. Hot slots
-// therefore cost one row update per window instead of one per pick.
+// The value gradient is deterministic and uses no atomics on rows:
+//   1. a stable LSD radix sort (8 bits per pass) groups the B*H*k picks by slot
+//      and keeps each slot's picks in pick order;
+//   2. one warp per window of 32 sorted picks takes every group that starts in its
+//      window: a group of at most kSmallGroup picks is summed in pick order in
+//      registers and its row is read and written once;
+//   3. a larger group becomes work items of at most kChunk picks: one block per item,
+//      eight warps on eight consecutive slices, their sums added in warp order;
+//   4. a group of more than kChunk picks writes one partial row per item, and one
+//      block per such group adds them in item order before its read-modify-write.
+// So every row's sum has the same order on every run, and hot slots are spread over
+// many blocks instead of serialising on one row.
 #include "pkm_common.cuh"
 #include "pkm_kernels.h"
 
@@ -26,19 +32,74 @@ static int64_t scan_blocks(int64_t slots) { return (slots + kScanBlock - 1) / kS
 
 static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-size_t backward_ws_bytes(int64_t B, int H, int k, int64_t slots, BackwardWs* carve, char* base) {
+// Radix sort geometry: each block of a pass owns kSortTile consecutive positions,
+// ranked in sub-tiles of kSortSub (eight warps x 16 steps of 32 keys).
+constexpr int kSortThreads = 256;
+constexpr int kSortWarps = kSortThreads / 32;
+constexpr int kSortSteps = 16;
+constexpr int kSortPerWarp = kSortSteps * 32;
+constexpr int kSortSub = kSortWarps * kSortPerWarp;     // 4096
+constexpr int kSortSubTiles = 4;
+constexpr int kSortTile = kSortSub * kSortSubTiles;     // 16384
+constexpr int kDigitBits = 8;
+constexpr int kDigits = 1 << kDigitBits;
+static_assert(kDigits == kSortThreads, "one thread per digit in the rank merge");
+
+// Group sizes: up to kSmallGroup picks a warp sums inline; larger groups are cut into
+// work items of at most kChunk picks, one block each.
+constexpr int kSmallGroup = kValueSmallGroup;
+constexpr int kChunk = kValueChunk;
+constexpr int kItemWarps = 8;
+static_assert(kSortTile == kSortTileKeys, "tile size shared with the workspace bound");
+
+static int64_t sort_blocks(int64_t E) { return (E + kSortTile - 1) / kSortTile; }
+
+// Radix passes for keys in [0, slots] (slots itself marks an id outside the table).
+static int sort_passes(int64_t slots) {
+  int bits = 0;
+  while (bits < 62 && (static_cast<int64_t>(1) << bits) <= slots) ++bits;
+  return (bits + kDigitBits - 1) / kDigitBits;
+}
+
+int backward_values_launches(int64_t slots, bool grad_scores, bool grad_values) {
+  return (grad_scores ? 1 : 0) + (grad_values ? 3 * sort_passes(slots) + 3 : 0);
+}
+
+size_t backward_ws_bytes(int64_t B, int H, int k, int64_t slots, int v, BackwardWs* carve,
+                         char* base) {
   const int64_t E = B * H * k;
+  const int64_t E1 = E > 0 ? E : 1;
+  const int64_t nblk = sort_blocks(E1);
+  // Hard bounds of the work lists: a group of more than kSmallGroup picks makes one
+  // item per kChunk picks, at most two per kChunk picks when it has more than kChunk.
+  const int64_t max_items = value_bwd_max_items(E);
+  const int64_t max_huge = value_bwd_max_huge(E);
+  const int64_t max_chunks = value_bwd_max_chunks(E);
   size_t off = kStatusBytes;
-  const size_t o_counts = off;   off += align256(sizeof(int) * slots);
-  const size_t o_offsets = off;  off += align256(sizeof(int) * (slots + 1));
-  const size_t o_partials = off; off += align256(sizeof(int) * (scan_blocks(slots) + 1));
-  const size_t o_order = off;    off += align256(sizeof(int) * (E > 0 ? E : 1));
+  const size_t o_ctr = off;      off += 256;
+  const size_t o_k0 = off;       off += align256(sizeof(int) * E1);
+  const size_t o_p0 = off;       off += align256(sizeof(int) * E1);
+  const size_t o_k1 = off;       off += align256(sizeof(int) * E1);
+  const size_t o_p1 = off;       off += align256(sizeof(int) * E1);
+  const size_t o_hist = off;     off += align256(sizeof(int) * kDigits * nblk);
+  const size_t o_items = off;    off += align256(sizeof(int4) * max_items);
+  const size_t o_huge = off;     off += align256(sizeof(int4) * max_huge);
+  const size_t o_scr = off;      off += align256(sizeof(float) * max_chunks * (v > 0 ? v : 1));
   if (carve && base) {
-    carve->counts = reinterpret_cast<int*>(base + o_counts);
-    carve->offsets = reinterpret_cast<int*>(base + o_offsets);
-    carve->partials = reinterpret_cast<int*>(base + o_partials);
-    carve->order = reinterpret_cast<int*>(base + o_order);
+    carve->ctr = reinterpret_cast<int*>(base + o_ctr);
+    carve->keys[0] = reinterpret_cast<int*>(base + o_k0);
+    carve->picks[0] = reinterpret_cast<int*>(base + o_p0);
+    carve->keys[1] = reinterpret_cast<int*>(base + o_k1);
+    carve->picks[1] = reinterpret_cast<int*>(base + o_p1);
+    carve->hist = reinterpret_cast<int*>(base + o_hist);
+    carve->items = reinterpret_cast<int4*>(base + o_items);
+    carve->huge = reinterpret_cast<int4*>(base + o_huge);
+    carve->scratch = reinterpret_cast<float*>(base + o_scr);
+    carve->max_items = max_items;
+    carve->max_huge = max_huge;
+    carve->max_chunks = max_chunks;
   }
+  (void)slots;
   return off;
 }
 
@@ -227,117 +288,446 @@ __global__ void slot_scatter_kernel(const int* __restrict__ indices, int64_t E, 
   }
 }
 
+// ------------------------------------------------------- stable LSD radix sort
+// Pass `first` reads the slot ids themselves (position p holds pick p); an id outside
+// [0, slots) sorts last under the key `slots` (recorded in the status word once per id
+// by the histogram pass). Later passes read the previous pass's (key, pick) pairs.
+__device__ __forceinline__ int sort_key(const int* keys, int64_t p, int64_t slots, int first) {
+  const int k = keys[p];
+  return (first && (k < 0 || k >= slots)) ? static_cast<int>(slots) : k;
+}
+
+// Digit counts of one tile, written digit-major: hist[d * nblk + block].
+__global__ void __launch_bounds__(kSortThreads) radix_hist_kernel(
+    const int* __restrict__ keys, int64_t E, int64_t slots, int shift, int first,
+    int* __restrict__ hist, int64_t nblk, int* status) {
+  __shared__ int h[kDigits];
+  h[threadIdx.x] = 0;
+  __syncthreads();
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * kSortTile;
+  for (int i = threadIdx.x; i < kSortTile; i += kSortThreads) {
+    const int64_t p = base + i;
+    if (p >= E) break;
+    const int raw = keys[p];
+    if (first && (raw < 0 || raw >= slots)) record_status(status, kDevBadSlot);
+    const int key = sort_key(keys, p, slots, first);
+    atomicAdd(&h[(key >> shift) & (kDigits - 1)], 1);  // a count: any order gives the same
+  }
+  __syncthreads();
+  hist[threadIdx.x * nblk + blockIdx.x] = h[threadIdx.x];
+}
+
+// Exclusive scan of the M digit-major counts, in place, by one block: each thread
+// scans a contiguous run, then the runs' totals are scanned across the block.
+__global__ void __launch_bounds__(1024) radix_scan_kernel(int* __restrict__ hist, int64_t M) {
+  __shared__ int warp_tot[32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t per = (M + 1023) / 1024;
+  const int64_t b = threadIdx.x * per;
+  const int64_t e = b + per < M ? b + per : M;
+  int sum = 0;
+  for (int64_t i = b; i < e; ++i) sum += hist[i];
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int wt = warp_tot[lane];
+    int wi = wt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += y;
+    }
+    warp_tot[lane] = wi - wt;
+  }
+  __syncthreads();
+  int run = warp_tot[warp] + incl - sum;
+  for (int64_t i = b; i < e; ++i) {
+    const int c = hist[i];
+    hist[i] = run;
+    run += c;
+  }
+}
+
+// Stable scatter of one tile: a key's new position is its digit's offset for this
+// block (the scan) + the keys of that digit before it in the tile. Ranks inside a
+// warp step come from __match_any_sync (lanes in order), steps and warps follow in
+// position order, so equal digits keep their order.
+__global__ void __launch_bounds__(kSortThreads) radix_scatter_kernel(
+    const int* __restrict__ keys_in, const int* __restrict__ picks_in, int64_t E,
+    int64_t slots, int shift, int first, const int* __restrict__ hist, int64_t nblk,
+    int* __restrict__ keys_out, int* __restrict__ picks_out) {
+  __shared__ int cnt[kSortWarps][kDigits];
+  __shared__ int base[kDigits];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const unsigned lower = (1u << lane) - 1u;
+  base[threadIdx.x] = hist[threadIdx.x * nblk + blockIdx.x];
+  for (int sub = 0; sub < kSortSubTiles; ++sub) {
+    for (int d = lane; d < kDigits; d += 32) cnt[warp][d] = 0;
+    __syncwarp();
+    const int64_t p0 = static_cast<int64_t>(blockIdx.x) * kSortTile +
+                       static_cast<int64_t>(sub) * kSortSub + warp * kSortPerWarp;
+    int key[kSortSteps], pick[kSortSteps], rank[kSortSteps];
+#pragma unroll
+    for (int r = 0; r < kSortSteps; ++r) {
+      const int64_t p = p0 + r * 32 + lane;
+      const bool valid = p < E;
+      key[r] = valid ? sort_key(keys_in, p, slots, first) : 0;
+      pick[r] = valid ? (picks_in ? picks_in[p] : static_cast<int>(p)) : 0;
+      const int d = valid ? (key[r] >> shift) & (kDigits - 1) : kDigits;
+      const unsigned peers = __match_any_sync(0xffffffffu, d);
+      const int before = __popc(peers & lower);
+      rank[r] = valid ? cnt[warp][d] + before : 0;
+      __syncwarp();
+      if (valid && before == 0) cnt[warp][d] += __popc(peers);
+      __syncwarp();
+    }
+    __syncthreads();
+    {
+      // Digit d's positions for this sub-tile: the block's earlier keys, then the
+      // warps in order.
+      const int d = threadIdx.x;
+      int run = base[d];
+#pragma unroll
+      for (int w = 0; w < kSortWarps; ++w) {
+        const int c = cnt[w][d];
+        cnt[w][d] = run;
+        run += c;
+      }
+      base[d] = run;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < kSortSteps; ++r) {
+      const int64_t p = p0 + r * 32 + lane;
+      if (p < E) {
+        const int pos = cnt[warp][(key[r] >> shift) & (kDigits - 1)] + rank[r];
+        keys_out[pos] = key[r];
+        picks_out[pos] = pick[r];
+      }
+    }
+    __syncthreads();
+  }
+}
+
 // ----------------------------------------------------------- segmented row sums
-// One warp per window of 32 sorted picks; total_ptr points at the number of valid
-// picks (the last entry of the sort's offsets). Group bounds inside the window come from the
-// sorted keys themselves (a ballot on key changes); the keys just before and after
-// the window tell whether the first and last groups continue into a neighbour.
+// Position just past the group of key r that contains position s (keys sorted
+// ascending): the first position q > s with key != r, or E. The warp probes 32
+// positions at once, first at distances 1, 2, 4, ... from s, then evenly inside the
+// bracket that holds the end (about 32x narrower per round).
+__device__ int64_t group_end(const int* __restrict__ skey, int64_t E, int64_t s, int r) {
+  const int lane = threadIdx.x & 31;
+  int64_t q = s + (static_cast<int64_t>(1) << lane);
+  if (q > E) q = E;
+  bool past = q >= E || skey[q] != r;
+  unsigned b = __ballot_sync(0xffffffffu, past);   // lane 31 reaches E: never empty
+  int j = __ffs(b) - 1;
+  int64_t hi = __shfl_sync(0xffffffffu, q, j);
+  const int64_t qp = __shfl_sync(0xffffffffu, q, j > 0 ? j - 1 : 0);
+  int64_t lo = j == 0 ? s + 1 : qp + 1;
+  // Invariant: the key at lo - 1 is r, and hi is E or holds another key.
+  while (lo < hi) {
+    const int64_t span = hi - lo;
+    q = lo + span * lane / 32;
+    past = skey[q] != r;
+    b = __ballot_sync(0xffffffffu, past);
+    if (b == 0) {
+      lo = lo + span * 31 / 32 + 1;
+    } else {
+      j = __ffs(b) - 1;
+      const int64_t qj = __shfl_sync(0xffffffffu, q, j);
+      const int64_t qb = __shfl_sync(0xffffffffu, q, j > 0 ? j - 1 : 0);
+      hi = qj;
+      if (j > 0) lo = qb + 1;
+    }
+  }
+  return hi;
+}
+
+// acc += sum over the sorted positions [a, b) in order of w[pick] * grad_out[token];
+// each lane holds the vectors lane, lane + 32, ... of the row.
 template <typename T, int MAXV>
-__global__ void __launch_bounds__(128) segment_rows_kernel(
-    const int* __restrict__ order, const int* __restrict__ total_ptr,
-    const int* __restrict__ indices, const float* __restrict__ weights,
-    const T* __restrict__ grad_out, int HK, int v, float* __restrict__ grad_values) {
+__device__ __forceinline__ void sum_picks(const int* __restrict__ spick, int64_t a, int64_t b,
+                                          const float* __restrict__ weights,
+                                          const T* __restrict__ grad_out, int HK, int v,
+                                          float (&acc)[MAXV][Vec<T>::kPer]) {
   constexpr int VPER = Vec<T>::kPer;
   const int lane = threadIdx.x & 31;
-  const int total = *total_ptr;
   const int nvec = v / VPER;
-  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  for (int64_t win = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-       win * 32 < total; win += nwarps) {
-    const int w0 = static_cast<int>(win * 32);
-    const int w1 = min(w0 + 32, total);
-    int e_l = 0, r_l = -1;
-    float wt_l = 0.f;
-    if (w0 + lane < w1) {
-      e_l = order[w0 + lane];
-      r_l = indices[e_l];
-      wt_l = weights[e_l];
+  for (int64_t c0 = a; c0 < b; c0 += 32) {
+    int e_l = 0;
+    float w_l = 0.f;
+    if (c0 + lane < b) {
+      e_l = spick[c0 + lane];
+      w_l = weights[e_l];
     }
-    // Keys of the picks just outside the window (-1: none).
-    int edge = -1;
-    if (lane == 0 && w0 > 0) edge = indices[order[w0 - 1]];
-    if (lane == 1 && w1 < total) edge = indices[order[w1]];
-    const int prev_r = __shfl_sync(0xffffffffu, edge, 0);
-    const int next_r = __shfl_sync(0xffffffffu, edge, 1);
-    int i = w0;
-    while (i < w1) {
-      const int r = __shfl_sync(0xffffffffu, r_l, i - w0);
-      const unsigned change = __ballot_sync(0xffffffffu, lane > i - w0 && r_l != r);
-      const int end = change ? w0 + __ffs(change) - 1 : w1;
-      const bool whole = (i > w0 || prev_r != r) && (end < w1 || next_r != r);
-      float* grow = grad_values + static_cast<int64_t>(r) * v;
-      // A slot group that lies inside this window is owned by this warp: load its row
-      // now so the HBM read overlaps the sums below. A group that crosses a window edge
-      // is added with vector atomics instead.
-      float4 old[MAXV][VPER / 4];
-      float acc[MAXV][VPER];
+    const int nb = static_cast<int>(b - c0 < 32 ? b - c0 : 32);
+    int j = 0;
+    for (; j + 1 < nb; j += 2) {  // two picks in flight
+      const int ea = __shfl_sync(0xffffffffu, e_l, j);
+      const int eb = __shfl_sync(0xffffffffu, e_l, j + 1);
+      const float wa = __shfl_sync(0xffffffffu, w_l, j);
+      const float wb = __shfl_sync(0xffffffffu, w_l, j + 1);
+      const T* ga = grad_out + static_cast<int64_t>(ea / HK) * v;
+      const T* gb = grad_out + static_cast<int64_t>(eb / HK) * v;
+      uint4 ra[MAXV], rb[MAXV];
 #pragma unroll
       for (int m = 0; m < MAXV; ++m) {
         const int vec = lane + 32 * m;
-#pragma unroll
-        for (int q = 0; q < VPER; q += 4) {
-          old[m][q / 4] = (whole && vec < nvec)
-                              ? *reinterpret_cast<const float4*>(grow + vec * VPER + q)
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
-          acc[m][q] = acc[m][q + 1] = acc[m][q + 2] = acc[m][q + 3] = 0.f;
-        }
+        ra[m] = vec < nvec ? __ldg(reinterpret_cast<const uint4*>(ga + vec * VPER)) : make_uint4(0, 0, 0, 0);
+        rb[m] = vec < nvec ? __ldg(reinterpret_cast<const uint4*>(gb + vec * VPER)) : make_uint4(0, 0, 0, 0);
       }
-      int j = i;
-      for (; j + 1 < end; j += 2) {  // two picks in flight
-        const int ea = __shfl_sync(0xffffffffu, e_l, j - w0);
-        const int eb = __shfl_sync(0xffffffffu, e_l, j + 1 - w0);
-        const float wa = __shfl_sync(0xffffffffu, wt_l, j - w0);
-        const float wb = __shfl_sync(0xffffffffu, wt_l, j + 1 - w0);
-        const T* ga = grad_out + static_cast<int64_t>(ea / HK) * v;
-        const T* gb = grad_out + static_cast<int64_t>(eb / HK) * v;
-        uint4 ra[MAXV], rb[MAXV];
 #pragma unroll
-        for (int m = 0; m < MAXV; ++m) {
-          const int vec = lane + 32 * m;
-          ra[m] = vec < nvec ? __ldg(reinterpret_cast<const uint4*>(ga + vec * VPER)) : make_uint4(0, 0, 0, 0);
-          rb[m] = vec < nvec ? __ldg(reinterpret_cast<const uint4*>(gb + vec * VPER)) : make_uint4(0, 0, 0, 0);
-        }
+      for (int m = 0; m < MAXV; ++m) {
+        float fa[VPER], fb[VPER];
+        Vec<T>::widen(ra[m], fa);
+        Vec<T>::widen(rb[m], fb);
 #pragma unroll
-        for (int m = 0; m < MAXV; ++m) {
-          float fa[VPER], fb[VPER];
-          Vec<T>::widen(ra[m], fa);
-          Vec<T>::widen(rb[m], fb);
-#pragma unroll
-          for (int q = 0; q < VPER; ++q) acc[m][q] = fmaf(wb, fb[q], fmaf(wa, fa[q], acc[m][q]));
-        }
+        for (int q = 0; q < VPER; ++q) acc[m][q] = fmaf(wb, fb[q], fmaf(wa, fa[q], acc[m][q]));
       }
-      if (j < end) {
-        const int ea = __shfl_sync(0xffffffffu, e_l, j - w0);
-        const float wa = __shfl_sync(0xffffffffu, wt_l, j - w0);
-        const T* ga = grad_out + static_cast<int64_t>(ea / HK) * v;
-#pragma unroll
-        for (int m = 0; m < MAXV; ++m) {
-          const int vec = lane + 32 * m;
-          if (vec < nvec) {
-            float fa[VPER];
-            Vec<T>::widen(__ldg(reinterpret_cast<const uint4*>(ga + vec * VPER)), fa);
-#pragma unroll
-            for (int q = 0; q < VPER; ++q) acc[m][q] = fmaf(wa, fa[q], acc[m][q]);
-          }
-        }
-      }
+    }
+    if (j < nb) {
+      const int ea = __shfl_sync(0xffffffffu, e_l, j);
+      const float wa = __shfl_sync(0xffffffffu, w_l, j);
+      const T* ga = grad_out + static_cast<int64_t>(ea / HK) * v;
 #pragma unroll
       for (int m = 0; m < MAXV; ++m) {
         const int vec = lane + 32 * m;
         if (vec < nvec) {
+          float fa[VPER];
+          Vec<T>::widen(__ldg(reinterpret_cast<const uint4*>(ga + vec * VPER)), fa);
 #pragma unroll
-          for (int q = 0; q < VPER; q += 4) {
-            float4* p = reinterpret_cast<float4*>(grow + vec * VPER + q);
-            const float4 o = old[m][q / 4];
-            if (whole)
-              *p = make_float4(o.x + acc[m][q], o.y + acc[m][q + 1], o.z + acc[m][q + 2],
-                               o.w + acc[m][q + 3]);
-            else
-              atomicAdd(p, make_float4(acc[m][q], acc[m][q + 1], acc[m][q + 2], acc[m][q + 3]));
-          }
+          for (int q = 0; q < VPER; ++q) acc[m][q] = fmaf(wa, fa[q], acc[m][q]);
         }
       }
-      i = end;
+    }
+  }
+}
+
+// acc += the picks at window lanes [j0, j1) in order, each lane l holding pick e_l with
+// weight w_l (the window's own loads, handed out by shuffles).
+template <typename T, int MAXV>
+__device__ __forceinline__ void sum_window_picks(int e_l, float w_l, int j0, int j1,
+                                                 const T* __restrict__ grad_out, int HK, int v,
+                                                 float (&acc)[MAXV][Vec<T>::kPer]) {
+  constexpr int VPER = Vec<T>::kPer;
+  const int lane = threadIdx.x & 31;
+  const int nvec = v / VPER;
+  int j = j0;
+  for (; j + 1 < j1; j += 2) {  // two picks in flight
+    const int ea = __shfl_sync(0xffffffffu, e_l, j);
+    const int eb = __shfl_sync(0xffffffffu, e_l, j + 1);
+    const float wa = __shfl_sync(0xffffffffu, w_l, j);
+    const float wb = __shfl_sync(0xffffffffu, w_l, j + 1);
+    const T* ga = grad_out + static_cast<int64_t>(ea / HK) * v;
+    const T* gb = grad_out + static_cast<int64_t>(eb / HK) * v;
+    uint4 ra[MAXV], rb[MAXV];
+#pragma unroll
+    for (int m = 0; m < MAXV; ++m) {
+      const int vec = lane + 32 * m;
+      ra[m] = vec < nvec ? __ldg(reinterpret_cast<const uint4*>(ga + vec * VPER)) : make_uint4(0, 0, 0, 0);
+      rb[m] = vec < nvec ? __ldg(reinterpret_cast<const uint4*>(gb + vec * VPER)) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int m = 0; m < MAXV; ++m) {
+      float fa[VPER], fb[VPER];
+      Vec<T>::widen(ra[m], fa);
+      Vec<T>::widen(rb[m], fb);
+#pragma unroll
+      for (int q = 0; q < VPER; ++q) acc[m][q] = fmaf(wb, fb[q], fmaf(wa, fa[q], acc[m][q]));
+    }
+  }
+  if (j < j1) {
+    const int ea = __shfl_sync(0xffffffffu, e_l, j);
+    const float wa = __shfl_sync(0xffffffffu, w_l, j);
+    const T* ga = grad_out + static_cast<int64_t>(ea / HK) * v;
+#pragma unroll
+    for (int m = 0; m < MAXV; ++m) {
+      const int vec = lane + 32 * m;
+      if (vec < nvec) {
+        float fa[VPER];
+        Vec<T>::widen(__ldg(reinterpret_cast<const uint4*>(ga + vec * VPER)), fa);
+#pragma unroll
+        for (int q = 0; q < VPER; ++q) acc[m][q] = fmaf(wa, fa[q], acc[m][q]);
+      }
+    }
+  }
+}
+
+// One warp per window of 32 sorted picks; the warp takes every group that starts in
+// its window. Groups of at most kSmallGroup picks: summed here and the row written
+// once (the only writer of that row). Larger groups: appended to the work lists.
+template <typename T, int MAXV>
+__global__ void __launch_bounds__(128) segment_small_kernel(
+    const int* __restrict__ skey, const int* __restrict__ spick, int64_t E, int64_t slots,
+    const float* __restrict__ weights, const T* __restrict__ grad_out, int HK, int v,
+    float* __restrict__ grad_values, int* __restrict__ ctr, int4* __restrict__ items,
+    int4* __restrict__ huge) {
+  constexpr int VPER = Vec<T>::kPer;
+  const int lane = threadIdx.x & 31;
+  const int nvec = v / VPER;
+  const int end_key = static_cast<int>(slots);  // past the table: never a group
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t win = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       win * 32 < E; win += nwarps) {
+    const int64_t w0 = win * 32;
+    const int key = w0 + lane < E ? skey[w0 + lane] : end_key;
+    // The window's picks and weights, loaded once: groups inside the window take them
+    // by shuffles, so a group's row reads wait for one round trip, not three.
+    int e_l = 0;
+    float w_l = 0.f;
+    if (w0 + lane < E && key < end_key) {
+      e_l = spick[w0 + lane];
+      w_l = weights[e_l];
+    }
+    int prev = __shfl_up_sync(0xffffffffu, key, 1);
+    if (lane == 0) prev = w0 > 0 ? skey[w0 - 1] : -1;
+    unsigned starts = __ballot_sync(0xffffffffu, key < end_key && key != prev);
+    while (starts) {
+      const int s = __ffs(starts) - 1;
+      starts &= starts - 1;
+      const int r = __shfl_sync(0xffffffffu, key, s);
+      const unsigned change = __ballot_sync(0xffffffffu, lane > s && key != r);
+      const int64_t g0 = w0 + s;
+      const int64_t g1 = change ? w0 + __ffs(change) - 1 : group_end(skey, E, w0 + 31, r);
+      const int64_t size = g1 - g0;
+      if (size <= kSmallGroup) {
+        float* grow = grad_values + static_cast<int64_t>(r) * v;
+        float4 old[MAXV][VPER / 4];
+        float acc[MAXV][VPER];
+#pragma unroll
+        for (int m = 0; m < MAXV; ++m) {
+          const int vec = lane + 32 * m;
+#pragma unroll
+          for (int q = 0; q < VPER; q += 4) {
+            old[m][q / 4] = vec < nvec ? *reinterpret_cast<const float4*>(grow + vec * VPER + q)
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+            acc[m][q] = acc[m][q + 1] = acc[m][q + 2] = acc[m][q + 3] = 0.f;
+          }
+        }
+        const int in_end = static_cast<int>((g1 < w0 + 32 ? g1 : w0 + 32) - w0);
+        sum_window_picks<T, MAXV>(e_l, w_l, s, in_end, grad_out, HK, v, acc);
+        if (g1 > w0 + 32) sum_picks<T, MAXV>(spick, w0 + 32, g1, weights, grad_out, HK, v, acc);
+#pragma unroll
+        for (int m = 0; m < MAXV; ++m) {
+          const int vec = lane + 32 * m;
+          if (vec < nvec) {
+#pragma unroll
+            for (int q = 0; q < VPER; q += 4) {
+              const float4 o = old[m][q / 4];
+              *reinterpret_cast<float4*>(grow + vec * VPER + q) =
+                  make_float4(o.x + acc[m][q], o.y + acc[m][q + 1], o.z + acc[m][q + 2],
+                              o.w + acc[m][q + 3]);
+            }
+          }
+        }
+      } else if (size <= kChunk) {
+        if (lane == 0) items[atomicAdd(&ctr[0], 1)] = make_int4(static_cast<int>(g0),
+                                                                static_cast<int>(size), r, -1);
+      } else {
+        // One item per kChunk picks, each writing a partial row; the group's own entry
+        // in `huge` lists the partial rows in item order.
+        const int nch = static_cast<int>((size + kChunk - 1) / kChunk);
+        int i0 = 0, c0 = 0;
+        if (lane == 0) {
+          i0 = atomicAdd(&ctr[0], nch);
+          c0 = atomicAdd(&ctr[2], nch);
+          huge[atomicAdd(&ctr[1], 1)] = make_int4(r, c0, nch, 0);
+        }
+        i0 = __shfl_sync(0xffffffffu, i0, 0);
+        c0 = __shfl_sync(0xffffffffu, c0, 0);
+        for (int c = lane; c < nch; c += 32) {
+          const int64_t a = g0 + static_cast<int64_t>(c) * kChunk;
+          const int64_t n = size - static_cast<int64_t>(c) * kChunk;
+          items[i0 + c] = make_int4(static_cast<int>(a), static_cast<int>(n < kChunk ? n : kChunk),
+                                    r, c0 + c);
+        }
+      }
+    }
+  }
+}
+
+// One block per work item {start, picks, slot, dest}: eight warps sum eight
+// consecutive slices in pick order, then the slices are added in warp order. dest < 0:
+// the row is read and written once; else the sum is partial row `dest` of a huge group.
+template <typename T, int MAXV>
+__global__ void __launch_bounds__(kItemWarps * 32) segment_items_kernel(
+    const int* __restrict__ spick, const float* __restrict__ weights,
+    const T* __restrict__ grad_out, int HK, int v, const int* __restrict__ ctr,
+    const int4* __restrict__ items, float* __restrict__ grad_values,
+    float* __restrict__ scratch) {
+  constexpr int VPER = Vec<T>::kPer;
+  extern __shared__ float4 red4[];  // [kItemWarps][v / 4]
+  float* red = reinterpret_cast<float*>(red4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nvec = v / VPER;
+  const int nitems = ctr[0];
+  for (int it = blockIdx.x; it < nitems; it += gridDim.x) {
+    const int4 item = items[it];
+    const int per = (item.y + kItemWarps - 1) / kItemWarps;
+    const int64_t end = static_cast<int64_t>(item.x) + item.y;
+    int64_t a = static_cast<int64_t>(item.x) + static_cast<int64_t>(warp) * per;
+    int64_t b = a + per;
+    if (a > end) a = end;
+    if (b > end) b = end;
+    float acc[MAXV][VPER];
+#pragma unroll
+    for (int m = 0; m < MAXV; ++m)
+#pragma unroll
+      for (int q = 0; q < VPER; ++q) acc[m][q] = 0.f;
+    sum_picks<T, MAXV>(spick, a, b, weights, grad_out, HK, v, acc);
+#pragma unroll
+    for (int m = 0; m < MAXV; ++m) {
+      const int vec = lane + 32 * m;
+      if (vec < nvec) {
+#pragma unroll
+        for (int q = 0; q < VPER; ++q) red[warp * v + vec * VPER + q] = acc[m][q];
+      }
+    }
+    __syncthreads();
+    for (int c = threadIdx.x * 4; c < v; c += kItemWarps * 32 * 4) {
+      float4 sum = *reinterpret_cast<const float4*>(red + c);
+#pragma unroll
+      for (int w = 1; w < kItemWarps; ++w) {
+        const float4 x = *reinterpret_cast<const float4*>(red + w * v + c);
+        sum = make_float4(sum.x + x.x, sum.y + x.y, sum.z + x.z, sum.w + x.w);
+      }
+      if (item.w < 0) {
+        float4* g = reinterpret_cast<float4*>(grad_values + static_cast<int64_t>(item.z) * v + c);
+        const float4 o = *g;
+        *g = make_float4(o.x + sum.x, o.y + sum.y, o.z + sum.z, o.w + sum.w);
+      } else {
+        *reinterpret_cast<float4*>(scratch + static_cast<int64_t>(item.w) * v + c) = sum;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// One block per group of more than kChunk picks: its partial rows added in item order,
+// then one read-modify-write of the row.
+__global__ void __launch_bounds__(256) segment_huge_kernel(const int* __restrict__ ctr,
+                                                           const int4* __restrict__ huge,
+                                                           const float* __restrict__ scratch,
+                                                           int v, float* __restrict__ grad_values) {
+  const int nh = ctr[1];
+  for (int g = blockIdx.x; g < nh; g += gridDim.x) {
+    const int4 h = huge[g];
+    for (int c = threadIdx.x * 4; c < v; c += 256 * 4) {
+      float4 sum = *reinterpret_cast<const float4*>(scratch + static_cast<int64_t>(h.y) * v + c);
+      for (int i = 1; i < h.z; ++i) {
+        const float4 x =
+            *reinterpret_cast<const float4*>(scratch + static_cast<int64_t>(h.y + i) * v + c);
+        sum = make_float4(sum.x + x.x, sum.y + x.y, sum.z + x.z, sum.w + x.w);
+      }
+      float4* gr = reinterpret_cast<float4*>(grad_values + static_cast<int64_t>(h.x) * v + c);
+      const float4 o = *gr;
+      *gr = make_float4(o.x + sum.x, o.y + sum.y, o.z + sum.z, o.w + sum.w);
     }
   }
 }
@@ -363,6 +753,31 @@ cudaError_t launch_counting_sort(const int* keys, int64_t E, int64_t slots, cons
   return cudaGetLastError();
 }
 
+// Stable sort of the picks by slot; returns which ping-pong buffer holds the result.
+static cudaError_t sort_picks_by_slot(const int* indices, int64_t E, int64_t slots,
+                                      const BackwardWs& ws, int* status, cudaStream_t st,
+                                      int* which) {
+  const int64_t nblk = sort_blocks(E);
+  const int passes = sort_passes(slots);
+  const int* kin = indices;
+  const int* pin = nullptr;
+  int cur = 0;
+  for (int ps = 0; ps < passes; ++ps) {
+    const int shift = kDigitBits * ps;
+    const int first = ps == 0;
+    radix_hist_kernel<<<static_cast<unsigned>(nblk), kSortThreads, 0, st>>>(
+        kin, E, slots, shift, first, ws.hist, nblk, status);
+    radix_scan_kernel<<<1, 1024, 0, st>>>(ws.hist, kDigits * nblk);
+    radix_scatter_kernel<<<static_cast<unsigned>(nblk), kSortThreads, 0, st>>>(
+        kin, pin, E, slots, shift, first, ws.hist, nblk, ws.keys[cur], ws.picks[cur]);
+    kin = ws.keys[cur];
+    pin = ws.picks[cur];
+    cur ^= 1;
+  }
+  *which = cur ^ 1;
+  return cudaGetLastError();
+}
+
 template <typename T, int MAXV>
 static cudaError_t launch_bwd_t(int64_t B, int H, int k, int v, int64_t slots, const void* values,
                                 const int* indices, const float* weights, const void* grad_out,
@@ -379,13 +794,24 @@ static cudaError_t launch_bwd_t(int64_t B, int H, int k, int v, int64_t slots, c
   }
   between_stages();
   if (!grad_values) return cudaGetLastError();
-  cudaError_t e = launch_counting_sort(indices, E, slots, ws, status, st);
+  cudaError_t e = cudaMemsetAsync(ws.ctr, 0, 4 * sizeof(int), st);
   if (e != cudaSuccess) return e;
+  int which = 0;
+  e = sort_picks_by_slot(indices, E, slots, ws, status, st, &which);
+  if (e != cudaSuccess) return e;
+  const int* skey = ws.keys[which];
+  const int* spick = ws.picks[which];
   const int64_t windows = (E + 31) / 32;
   const int64_t sblocks = (windows + 3) / 4;
   const unsigned sgrid = static_cast<unsigned>(sblocks < 148 * 64 ? sblocks : 148 * 64);
-  segment_rows_kernel<T, MAXV><<<sgrid > 0 ? sgrid : 1, 128, 0, st>>>(
-      ws.order, ws.offsets + slots, indices, weights, G, H * k, v, grad_values);
+  segment_small_kernel<T, MAXV><<<sgrid > 0 ? sgrid : 1, 128, 0, st>>>(
+      skey, spick, E, slots, weights, G, H * k, v, grad_values, ws.ctr, ws.items, ws.huge);
+  const size_t smem = sizeof(float) * kItemWarps * v;
+  e = set_max_smem(reinterpret_cast<const void*>(segment_items_kernel<T, MAXV>), smem);
+  if (e != cudaSuccess) return e;
+  segment_items_kernel<T, MAXV><<<2 * 148, kItemWarps * 32, smem, st>>>(
+      spick, weights, G, H * k, v, ws.ctr, ws.items, grad_values, ws.scratch);
+  segment_huge_kernel<<<148, 256, 0, st>>>(ws.ctr, ws.huge, ws.scratch, v, grad_values);
   return cudaGetLastError();
 }
 

@@ -456,7 +456,8 @@ size_t backward_full_ws_bytes(const LayerArgs& a, bool tensor_path, FullBackward
   const int64_t E2 = 2 * E > 0 ? 2 * E : 1;
   const int64_t tslots = 2LL * a.H * a.n;
   BackwardWs vws;
-  size_t off = backward_ws_bytes(a.B, a.H, a.k, static_cast<int64_t>(a.n) * a.n, &vws, base);
+  size_t off = backward_ws_bytes(a.B, a.H, a.k, static_cast<int64_t>(a.n) * a.n, a.v, &vws,
+                                base);
   const size_t o_gs = off;      off += al256(sizeof(float) * (E > 0 ? E : 1));
   const size_t o_acc = off;     off += al256(sizeof(float) * a.B * F);
   const size_t o_q = off;       off += al256(sizeof(float) * a.B * F);
@@ -530,7 +531,7 @@ static cudaError_t launch_full_t(const LayerArgs& a, bool tensor_path, bool bn_t
   e = launch_backward_values(a.B, a.H, a.k, a.v, a.dtype, slots, a.values, indices, weights,
                              grad_out, grad_values, w.g_s, w.values, a.status, st, [] {});
   if (e != cudaSuccess) return e;
-  *launches += grad_values ? 7 : 1;
+  *launches += backward_values_launches(slots, true, grad_values != nullptr);
   if (grad_scores) {
     e = cudaMemcpyAsync(grad_scores, w.g_s, sizeof(float) * E, cudaMemcpyDeviceToDevice, st);
     if (e != cudaSuccess) return e;

@@ -40,12 +40,49 @@ cudaError_t launch_select_gather(const LayerArgs& a, const float* list_s, const 
 
 // Value backward (pkm_backward.cu).
 struct BackwardWs {
+  // Counting sort (launch_counting_sort: the full backward's sub-key grouping).
   int* counts;    // [slots]
   int* offsets;   // [slots + 1]
   int* partials;  // [scan blocks + 1]
-  int* order;     // [B*H*k] pick ids grouped by slot
+  int* order;     // [E] ids grouped by key
+  // Value gradient: stable radix sort of the picks by slot, then work lists.
+  int* keys[2];   // [E] slot ids, ping-pong between sort passes
+  int* picks[2];  // [E] pick ids (t*H*k + h*k + j), ping-pong
+  int* hist;      // [256][sort blocks] digit counts, then their exclusive scan
+  int* ctr;       // [4] work-list lengths: items, huge groups, scratch rows
+  int4* items;    // [max_items] {start, picks, slot, scratch row or -1}
+  int4* huge;     // [max_huge] {slot, first scratch row, rows, 0}
+  float* scratch; // [max_chunks][v] partial row sums of huge groups
+  int64_t max_items, max_huge, max_chunks;
 };
-size_t backward_ws_bytes(int64_t B, int H, int k, int64_t slots, BackwardWs* carve, char* base);
+size_t backward_ws_bytes(int64_t B, int H, int k, int64_t slots, int v, BackwardWs* carve,
+                         char* base);
+
+// Value-gradient geometry: radix-sort tile, the largest group a warp sums inline, the
+// picks per work item; and the workspace bytes for E picks and rows of v floats, laid
+// out as backward_ws_bytes carves them (status word, list lengths, two key and two
+// pick buffers, digit counts, work lists, partial rows). A compile-time function so
+// that the fixed scratch of pkm_backward_values_noalloc is sized by the same sum.
+constexpr int kSortTileKeys = 16384;
+constexpr int kValueSmallGroup = 256;
+constexpr int kValueChunk = 4096;
+constexpr size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+constexpr int64_t value_bwd_max_items(int64_t E) {
+  return E / (kValueSmallGroup + 1) + E / (kValueChunk / 2) + 2;
+}
+constexpr int64_t value_bwd_max_huge(int64_t E) { return E / (kValueChunk + 1) + 1; }
+constexpr int64_t value_bwd_max_chunks(int64_t E) { return E / (kValueChunk / 2) + 1; }
+constexpr size_t value_bwd_ws_bytes(int64_t E, int v) {
+  return 256 + 256 + 4 * round256(4 * static_cast<size_t>(E > 0 ? E : 1)) +
+         round256(4 * 256 * static_cast<size_t>(((E > 0 ? E : 1) + kSortTileKeys - 1) /
+                                                kSortTileKeys)) +
+         round256(16 * static_cast<size_t>(value_bwd_max_items(E))) +
+         round256(16 * static_cast<size_t>(value_bwd_max_huge(E))) +
+         round256(4 * static_cast<size_t>(value_bwd_max_chunks(E)) *
+                  static_cast<size_t>(v > 0 ? v : 1));
+}
+// Kernels one pkm_backward_values call launches.
+int backward_values_launches(int64_t slots, bool grad_scores, bool grad_values);
 cudaError_t launch_backward_values(int64_t B, int H, int k, int v, int dtype, int64_t slots,
                                    const void* values, const int* indices, const float* weights,
                                    const void* grad_out, float* grad_values, float* grad_scores,
@@ -99,6 +136,12 @@ bool small_supported(int64_t B, int d_model, int H, int dq, int n, int k, int v,
 size_t small_chunk_entries(int64_t B, int H, int n);
 cudaError_t launch_forward_small(const LayerArgs& a, float* q, float* chunk_s, int* chunk_i,
                                  float* out, int* idx, float* w, float* sc, cudaStream_t st);
+// The same forward as one cooperative launch with grid-wide barriers (one CTA per SM);
+// the barrier counter is the int after a.status, zeroed by the caller.
+bool small_fused_supported(int d_model, int H, int dq, int n, int v, int dtype);
+cudaError_t launch_forward_small_fused(const LayerArgs& a, float* q, float* chunk_s,
+                                       int* chunk_i, float* out, int* idx, float* w, float* sc,
+                                       cudaStream_t st);
 
 // 16-byte vectors of a v-wide row each lane of a warp holds, rounded up to the kernel
 // instantiations (1, 2, 4 or 8); 0 when a row is wider than 8 vectors per lane.

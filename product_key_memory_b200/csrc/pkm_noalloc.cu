@@ -10,22 +10,25 @@
 // the inputs and outputs.
 //
 // The scratch is the file-scope array below. Every GPU that loads this library
-// holds it (16 MiB) until the process exits. Host code only sees a host-side
+// holds it (about 40 MiB) until the process exits. Host code only sees a host-side
 // stand-in under that name, so the array's device address is looked up with
 // cudaGetSymbolAddress, once per device, the first time the entry point runs on
 // that device (with that device current).
 #include <mutex>
 
 #include "../../include/pkm.h"
+#include "pkm_kernels.h"
 
 namespace {
 
-// Limits of the fixed scratch: n*n slots and B*H*k picks.
+// Limits of the fixed scratch: n*n slots, B*H*k picks and the value width (a bf16 row
+// of at most 2048 elements is the widest the kernels take).
 constexpr long long kNoAllocMaxSlots = 1LL << 20;  // 1,048,576 slots (n <= 1024)
 constexpr long long kNoAllocMaxPicks = 1LL << 21;  // 2,097,152 picks
-// Same layout as the workspace of pkm_backward_values at those limits: status word,
-// slot counts, slot offsets (+1), scan partials, pick order (each 256-byte aligned).
-constexpr size_t kNoAllocBytes = 256 + (4u << 20) + ((4u << 20) + 256) + 1280 + (8u << 20);
+constexpr int kNoAllocMaxV = 2048;
+// The workspace of pkm_backward_values at those limits (its sort buffers, work lists
+// and partial rows): about 40.3 MiB.
+constexpr size_t kNoAllocBytes = pkm::value_bwd_ws_bytes(kNoAllocMaxPicks, kNoAllocMaxV);
 
 __device__ __align__(256) unsigned char g_pkm_noalloc_scratch[kNoAllocBytes];
 
@@ -65,13 +68,15 @@ extern "C" int pkm_backward_values_noalloc(const pkm_shape* s, const void* value
   }
   const long long slots = static_cast<long long>(s->n) * s->n;
   const long long picks = s->B * s->H * static_cast<long long>(s->k);
-  if (slots > kNoAllocMaxSlots || picks > kNoAllocMaxPicks || need > kNoAllocBytes)
+  if (slots > kNoAllocMaxSlots || picks > kNoAllocMaxPicks || s->v > kNoAllocMaxV ||
+      need > kNoAllocBytes)
     return PKM_ERR_UNSUPPORTED;
   void* scratch = nullptr;
   const int rc = scratch_on_current_device(&scratch);
   if (rc != PKM_OK) return rc;
-  // The regular entry point zeroes the status word and the slot counts on the
-  // stream before its kernels use them, so the previous call's contents do not leak.
+  // The regular entry point zeroes the status word and the work-list lengths on the
+  // stream before its kernels use them, and every other part of the scratch is written
+  // before it is read, so the previous call's contents do not leak.
   return pkm_backward_values(s, values, indices, weights, grad_out, grad_values, grad_scores,
                              scratch, kNoAllocBytes, stream);
 }

@@ -23,6 +23,8 @@
 #include "pkm_common.cuh"
 #include "pkm_kernels.h"
 #include "pkm_select.cuh"
+#include "pkm_tc.h"
+#include "pkm_tcgen05.cuh"
 
 namespace pkm {
 
@@ -483,6 +485,421 @@ __global__ void __launch_bounds__(kSmallWarps * 32) gather_small_kernel(
 }
 
 // ---------------------------------------------------------------------------
+// The same forward as ONE cooperative launch (one CTA per SM), its three phases
+// separated by grid-wide barriers instead of kernel boundaries:
+//   Q  query network: CTA = a group of 16 features for all tokens (W_q rows staged
+//      once); meanwhile the sub-keys of the CTA's first scoring unit stream into
+//      shared memory with asynchronous copies, since they do not depend on q
+//   S  scores: CTA = (head-half, 64 sub-keys): scores for every token and each
+//      token's best 32 of the chunk
+//   G  gather: CTA = token: the chunk lists of all heads merged per half (one warp
+//      per half), exact top-k of the pruned candidates and softmax (one warp per
+//      head), then the H*k weighted value rows over 8 warps, added in warp order.
+// A barrier is a counter in the workspace (zeroed by the host before the launch):
+// each CTA adds one and waits, bounded by the pipelines' wait limit, until every CTA
+// has; on a timeout the kernel records it in the status word and returns. The
+// arithmetic is that of the three-kernel path above (fp32 q and dot products, the
+// same selection order and candidate pruning).
+// ---------------------------------------------------------------------------
+struct FusedArgs {
+  const void* x;
+  const void* W;
+  const float* mean;
+  const float* var;
+  const float* gamma;
+  const float* beta;
+  const void* subkeys;
+  const void* values;
+  float eps;
+  int B, d, H, dq, n, k, v;
+  float* q;        // [B][H*dq] fp32
+  float* cs;       // [B][H][2][nchunks][32] chunk lists
+  int* ci;
+  float* out;
+  int* idx;
+  float* w;
+  float* sc;
+  int* status;
+  unsigned* barrier;
+};
+
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(tc::smem_addr(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+// Returns false (every thread of the CTA) once the wait limit has passed.
+__device__ bool fused_grid_sync(unsigned* counter, unsigned target, int* status, int* ok_s) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    __threadfence();
+    atomicAdd(counter, 1u);
+    unsigned seen;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(seen) : "l"(counter) : "memory");
+    if (seen < target) {
+      const uint64_t t0 = tc::global_timer_ns();
+      for (;;) {
+        __nanosleep(32);
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(seen) : "l"(counter) : "memory");
+        if (seen >= target) break;
+        if (tc::global_timer_ns() - t0 > tc::kWaitLimitNs) {
+          record_status(status, kDevTimeout);
+          ok = 0;
+          break;
+        }
+      }
+    }
+    *ok_s = ok;
+  }
+  __syncthreads();
+  return *ok_s != 0;
+}
+
+// Shared-memory layout (bytes) of the fused kernel: region A holds phase Q's W_q
+// group and x rows, later phase G's lists and per-warp row sums; region B holds the
+// scoring unit's sub-key rows and the warps' query halves.
+struct FusedSmem {
+  size_t a, b, total;
+};
+__host__ __device__ inline FusedSmem fused_smem(int d, int H, int dq, int n, int v, int esz) {
+  const int half = dq / 2;
+  const int nchunks = (n + kSChunk - 1) / kSChunk;
+  const size_t q_bytes = static_cast<size_t>(kQFeat + kQTok) * d * esz;
+  const size_t lists = static_cast<size_t>(2 * H) * nchunks * kMaxK * 8;
+  const size_t merged = static_cast<size_t>(2 * H) * kMaxK * 8;
+  const size_t picks = static_cast<size_t>(H) * kMaxK * 8;
+  const size_t red = static_cast<size_t>(kSmallWarps) * v * 4;
+  const size_t g_bytes = lists + merged + picks + red;
+  FusedSmem m;
+  m.a = ((q_bytes > g_bytes ? q_bytes : g_bytes) + 15) & ~static_cast<size_t>(15);
+  const size_t rows = (static_cast<size_t>(esz) * kSChunk * (half + (esz == 2 ? 2 : 1)) + 15) &
+                      ~static_cast<size_t>(15);
+  m.b = rows + sizeof(float) * kSmallWarps * 2 * half;
+  m.total = m.a + m.b + sizeof(int) * kMaxPairs;
+  return m;
+}
+
+template <typename T, int MAXV>
+__global__ void __launch_bounds__(kSmallWarps * 32, 1) forward_small_fused_kernel(FusedArgs a) {
+  constexpr int VPER = Vec<T>::kPer;
+  extern __shared__ __align__(16) unsigned char fs_raw[];
+  __shared__ int ok_s;
+  __shared__ int npairs_s;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int B = a.B, d = a.d, H = a.H, dq = a.dq, n = a.n, k = a.k, v = a.v;
+  const int F = H * dq, half = dq >> 1;
+  const int esz = static_cast<int>(sizeof(T));
+  const FusedSmem L = fused_smem(d, H, dq, n, v, esz);
+  unsigned char* regA = fs_raw;
+  unsigned char* regB = fs_raw + L.a;
+  int* pairs = reinterpret_cast<int*>(fs_raw + L.a + L.b);
+  const int nchunks = (n + kSChunk - 1) / kSChunk;
+  const int NQ = (F + kQFeat - 1) / kQFeat;
+  const int NS = 2 * H * nchunks;
+  const unsigned G = gridDim.x;
+  const T* X = static_cast<const T*>(a.x);
+  const T* W = static_cast<const T*>(a.W);
+  const T* C = static_cast<const T*>(a.subkeys);
+  const int ld = half + (sizeof(T) == 2 ? 2 : 1);  // padded sub-key row (elements)
+  T* rows_s = reinterpret_cast<T*>(regB);
+  float* qs = reinterpret_cast<float*>(
+      regB + ((sizeof(T) * kSChunk * ld + 15) & ~static_cast<size_t>(15)));
+  const int row_words_c = half * esz / 4;         // words of one sub-key row
+  const int ld_words = ld * esz / 4;
+
+  if (threadIdx.x == 0) npairs_s = build_pairs(k, pairs);
+
+  // Sub-keys of this CTA's first scoring unit: asynchronous copies into region B,
+  // waited for at the start of phase S.
+  if (static_cast<int>(blockIdx.x) < NS) {
+    const int u = blockIdx.x;
+    const int hs = u / nchunks, chunk = u - hs * nchunks;
+    const int c0 = chunk * kSChunk;
+    const int nr = min(kSChunk, n - c0);
+    const uint32_t* src =
+        reinterpret_cast<const uint32_t*>(C + (static_cast<int64_t>(hs) * n + c0) * half);
+    uint32_t* dst = reinterpret_cast<uint32_t*>(rows_s);
+    for (int i = threadIdx.x; i < kSChunk * row_words_c; i += blockDim.x) {
+      const int r = i / row_words_c, c = i - r * row_words_c;
+      if (r < nr) cp_async4(dst + r * ld_words + c, src + i);
+      else dst[r * ld_words + c] = 0u;
+    }
+  }
+
+  // ---------------- phase Q
+  {
+    T* ws = reinterpret_cast<T*>(regA);  // [kQFeat][d]
+    T* xs = ws + kQFeat * d;             // [kQTok][d]
+    const int row_words = d * esz / 4;
+    for (int g = blockIdx.x; g < NQ; g += G) {
+      const int f0 = g * kQFeat;
+      const int nf = min(kQFeat, F - f0);
+      __syncthreads();
+      stage_rows(reinterpret_cast<const uint32_t*>(W + static_cast<int64_t>(f0) * d),
+                 reinterpret_cast<uint32_t*>(ws), kQFeat, nf, row_words, row_words);
+      for (int t0 = 0; t0 < B; t0 += kQTok) {
+        __syncthreads();
+        stage_rows(reinterpret_cast<const uint32_t*>(X + static_cast<int64_t>(t0) * d),
+                   reinterpret_cast<uint32_t*>(xs), kQTok, min(kQTok, B - t0), row_words,
+                   row_words);
+        __syncthreads();
+        const int t = t0 + warp;
+        if (t >= B) continue;  // warp-uniform
+        float acc[kQFeat];
+#pragma unroll
+        for (int j = 0; j < kQFeat; ++j) acc[j] = 0.f;
+        const T* xr = xs + warp * d;
+        if constexpr (sizeof(T) == 2) {
+          const uint32_t* xw = reinterpret_cast<const uint32_t*>(xr);
+          const uint32_t* ww = reinterpret_cast<const uint32_t*>(ws);
+          const int dw = d >> 1;
+          for (int c0 = 0; c0 < dw; c0 += 32 * 4) {
+            uint32_t xv[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int c = c0 + lane + 32 * u;
+              xv[u] = c < dw ? xw[c] : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int c = c0 + lane + 32 * u;
+              if (c < dw) {
+                const float xa = bf16_lo(xv[u]), xb = bf16_hi(xv[u]);
+#pragma unroll
+                for (int j = 0; j < kQFeat; ++j) {
+                  const uint32_t wv = ww[j * dw + c];
+                  acc[j] = fmaf(xb, bf16_hi(wv), fmaf(xa, bf16_lo(wv), acc[j]));
+                }
+              }
+            }
+          }
+        } else {
+          for (int c0 = 0; c0 < d; c0 += 32 * 8) {
+            float xv[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int c = c0 + lane + 32 * u;
+              xv[u] = c < d ? load_elem(xr, c) : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int c = c0 + lane + 32 * u;
+              if (c < d) {
+#pragma unroll
+                for (int j = 0; j < kQFeat; ++j)
+                  acc[j] = fmaf(xv[u], load_elem(ws, j * d + c), acc[j]);
+              }
+            }
+          }
+        }
+#pragma unroll
+        for (int m = 16, c = kQFeat / 2; c >= 1; m >>= 1, c >>= 1) {
+          const bool up = (lane & m) != 0;
+#pragma unroll
+          for (int i = 0; i < c; ++i) {
+            const float send = up ? acc[i] : acc[i + c];
+            const float keep = up ? acc[i + c] : acc[i];
+            acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+          }
+        }
+        const float sum = acc[0] + __shfl_xor_sync(0xffffffffu, acc[0], 1);
+        const int j = lane >> 1;
+        if ((lane & 1) == 0 && j < nf) {
+          const int f = f0 + j;
+          const float sc = a.gamma[f] / sqrtf(a.var[f] + a.eps);
+          a.q[static_cast<int64_t>(t) * F + f] = fmaf(sum, sc, a.beta[f] - a.mean[f] * sc);
+        }
+      }
+    }
+  }
+  if (!fused_grid_sync(a.barrier, G, a.status, &ok_s)) return;
+
+  // ---------------- phase S
+  for (int u = blockIdx.x; u < NS; u += G) {
+    const int hs = u / nchunks, chunk = u - hs * nchunks;
+    const int h = hs >> 1, side = hs & 1;
+    const int c0 = chunk * kSChunk;
+    if (u == static_cast<int>(blockIdx.x)) {
+      cp_async_wait_all();
+    } else {
+      __syncthreads();
+      stage_rows(reinterpret_cast<const uint32_t*>(C + (static_cast<int64_t>(hs) * n + c0) * half),
+                 reinterpret_cast<uint32_t*>(rows_s), kSChunk, min(kSChunk, n - c0),
+                 row_words_c, ld_words);
+    }
+    __syncthreads();
+    float* qw = qs + warp * 2 * half;
+    const bool v0 = c0 + lane < n, v1 = c0 + 32 + lane < n;
+    const T* r0 = rows_s + lane * ld;
+    const T* r1 = rows_s + (lane + 32) * ld;
+    for (int tb = warp * 2; tb < B; tb += kSmallWarps * 2) {
+      // This warp's two tokens' query halves (written by other CTAs: read from L2).
+      for (int i = lane; i < 2 * half; i += 32) {
+        const int uu = i / half, e = i - uu * half;
+        const int t = tb + uu;
+        qw[i] = t < B ? __ldcg(a.q + static_cast<int64_t>(t) * F + h * dq + side * half + e)
+                      : 0.f;
+      }
+      __syncwarp();
+      for (int uu = 0; uu < 2; ++uu) {
+        const int t = tb + uu;
+        if (t >= B) break;
+        const float* qq = qw + uu * half;
+        float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+        for (int e = 0; e < half; e += 2) {
+          const float2 qv = *reinterpret_cast<const float2*>(qq + e);
+          float x0a, x0b, x1a, x1b;
+          if constexpr (sizeof(T) == 2) {
+            const uint32_t w0 = *reinterpret_cast<const uint32_t*>(r0 + e);
+            const uint32_t w1 = *reinterpret_cast<const uint32_t*>(r1 + e);
+            x0a = bf16_lo(w0); x0b = bf16_hi(w0);
+            x1a = bf16_lo(w1); x1b = bf16_hi(w1);
+          } else {
+            x0a = load_elem(r0, e); x0b = load_elem(r0, e + 1);
+            x1a = load_elem(r1, e); x1b = load_elem(r1, e + 1);
+          }
+          a0 = fmaf(qv.x, x0a, a0);
+          a1 = fmaf(qv.x, x1a, a1);
+          b0 = fmaf(qv.y, x0b, b0);
+          b1 = fmaf(qv.y, x1b, b1);
+        }
+        a0 += b0;
+        a1 += b1;
+        float s0 = v0 ? a0 : -INFINITY, s1 = v1 ? a1 : -INFINITY;
+        int i0 = v0 ? c0 + lane : kIdPad, i1 = v1 ? c0 + 32 + lane : kIdPad;
+        warp_sort32(s0, i0);
+        warp_sort32(s1, i1);
+        warp_merge32(s0, i0, s1, i1);
+        const int64_t o =
+            ((((static_cast<int64_t>(t) * H + h) * 2 + side) * nchunks + chunk) << 5) + lane;
+        a.cs[o] = s0;
+        a.ci[o] = i0;
+      }
+      __syncwarp();
+    }
+  }
+  if (!fused_grid_sync(a.barrier, 2 * G, a.status, &ok_s)) return;
+
+  // ---------------- phase G
+  const int list_len = 2 * H * nchunks * kMaxK;
+  float* ls = reinterpret_cast<float*>(regA);            // [2H][nchunks][32]
+  int* li = reinterpret_cast<int*>(ls + list_len);
+  float* ms = reinterpret_cast<float*>(li + list_len);   // [2H][32] merged halves
+  int* mi = reinterpret_cast<int*>(ms + 2 * H * kMaxK);
+  int* prow = mi + 2 * H * kMaxK;                        // [H][k] picked slots
+  float* pw = reinterpret_cast<float*>(prow + H * kMaxK);
+  float* red = pw + H * kMaxK;                           // [8][v]
+  const int nvec = v / VPER;
+  for (int t = blockIdx.x; t < B; t += G) {
+    __syncthreads();
+    const int64_t src = static_cast<int64_t>(t) * list_len;
+    for (int i = threadIdx.x; i < list_len; i += blockDim.x) {
+      ls[i] = __ldcg(a.cs + src + i);
+      li[i] = __ldcg(a.ci + src + i);
+    }
+    __syncthreads();
+    for (int hs = warp; hs < 2 * H; hs += kSmallWarps) {
+      const int base = hs * nchunks * kMaxK;
+      float bs = ls[base + lane];
+      int bi = li[base + lane];
+      for (int c = 1; c < nchunks; ++c) {
+        const float cs = ls[base + c * kMaxK + lane];
+        const int ci = li[base + c * kMaxK + lane];
+        const float ks = __shfl_sync(0xffffffffu, bs, 31);
+        const int ki = __shfl_sync(0xffffffffu, bi, 31);
+        const float c0s = __shfl_sync(0xffffffffu, cs, 0);
+        const int c0i = __shfl_sync(0xffffffffu, ci, 0);
+        if (better(c0s, c0i, ks, ki)) warp_merge32(bs, bi, cs, ci);
+      }
+      ms[hs * kMaxK + lane] = bs;
+      mi[hs * kMaxK + lane] = bi;
+    }
+    __syncthreads();
+    if (warp < H) {
+      const int h = warp;
+      float bs;
+      int bi;
+      select_candidates(ms[2 * h * kMaxK + lane], mi[2 * h * kMaxK + lane],
+                        ms[(2 * h + 1) * kMaxK + lane], mi[(2 * h + 1) * kMaxK + lane], pairs,
+                        npairs_s, n, bs, bi);
+      const float mx = __shfl_sync(0xffffffffu, bs, 0);
+      const float e = lane < k ? expf(bs - mx) : 0.f;
+      const float den = warp_sum(e);
+      const float wt = e / den;
+      if (lane < k) {
+        const int64_t o = (static_cast<int64_t>(t) * H + h) * k + lane;
+        a.idx[o] = bi;
+        a.w[o] = wt;
+        if (a.sc) a.sc[o] = bs;
+        prow[h * k + lane] = bi;
+        pw[h * k + lane] = wt;
+      }
+    }
+    __syncthreads();
+    // The H*k weighted rows, rows warp, warp + 8, ... of each warp 4 at a time.
+    const int HK = H * k;
+    const T* Vt = static_cast<const T*>(a.values);
+    float acc[MAXV][VPER];
+#pragma unroll
+    for (int m = 0; m < MAXV; ++m)
+#pragma unroll
+      for (int e = 0; e < VPER; ++e) acc[m][e] = 0.f;
+    for (int r0 = warp; r0 < HK; r0 += 4 * kSmallWarps) {
+      uint4 raw[4][MAXV];
+      float wr[4];
+#pragma unroll
+      for (int uu = 0; uu < 4; ++uu) {
+        const int r = r0 + uu * kSmallWarps;
+        bool live = r < HK;
+        int row = live ? prow[r] : 0;
+        if (live && (row < 0 || row >= n * n)) {  // only reachable with NaN scores
+          if (lane == 0) record_status(a.status, kDevBadSlot);
+          live = false;
+          row = 0;
+        }
+        wr[uu] = live ? pw[r] : 0.f;
+        const T* rp = Vt + static_cast<int64_t>(row) * v;
+#pragma unroll
+        for (int m = 0; m < MAXV; ++m) {
+          const int vec = lane + 32 * m;
+          raw[uu][m] = (live && vec < nvec) ? ld_stream_v4(rp + vec * VPER)
+                                            : make_uint4(0, 0, 0, 0);
+        }
+      }
+#pragma unroll
+      for (int uu = 0; uu < 4; ++uu)
+#pragma unroll
+        for (int m = 0; m < MAXV; ++m) {
+          float f[VPER];
+          Vec<T>::widen(raw[uu][m], f);
+#pragma unroll
+          for (int e = 0; e < VPER; ++e) acc[m][e] = fmaf(wr[uu], f[e], acc[m][e]);
+        }
+    }
+    float* my = red + warp * v;
+#pragma unroll
+    for (int m = 0; m < MAXV; ++m) {
+      const int vec = lane + 32 * m;
+      if (vec < nvec) {
+#pragma unroll
+        for (int e = 0; e < VPER; ++e) my[vec * VPER + e] = acc[m][e];
+      }
+    }
+    __syncthreads();
+    for (int c = threadIdx.x; c < v; c += blockDim.x) {
+      float sum = red[c];
+#pragma unroll
+      for (int ww = 1; ww < kSmallWarps; ++ww) sum += red[ww * v + c];
+      a.out[static_cast<int64_t>(t) * v + c] = sum;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
 static size_t query_small_smem(int d, int dtype) {
@@ -540,6 +957,57 @@ static cudaError_t launch_gather_small(const LayerArgs& a, const float* cs, cons
   return cudaLaunchKernelEx(&cfg, gather_small_kernel<T, MAXV>, cs, ci,
                             static_cast<const T*>(a.values), a.H, a.n, a.k, a.v, out, idx, w,
                             sc, a.status);
+}
+
+template <typename T, int MAXV>
+static cudaError_t launch_fused_t(const LayerArgs& a, float* q, float* cs, int* ci, float* out,
+                                  int* idx, float* w, float* sc, cudaStream_t st) {
+  const FusedSmem m = fused_smem(a.d_model, a.H, a.dq, a.n, a.v, a.dtype == 0 ? 4 : 2);
+  const void* kern = reinterpret_cast<const void*>(forward_small_fused_kernel<T, MAXV>);
+  cudaError_t e = set_max_smem(kern, m.total);
+  if (e != cudaSuccess) return e;
+  FusedArgs fa;
+  fa.x = a.x; fa.W = a.W_q; fa.mean = a.bn_mean; fa.var = a.bn_var; fa.gamma = a.bn_gamma;
+  fa.beta = a.bn_beta; fa.subkeys = a.subkeys; fa.values = a.values; fa.eps = a.bn_eps;
+  fa.B = static_cast<int>(a.B); fa.d = a.d_model; fa.H = a.H; fa.dq = a.dq; fa.n = a.n;
+  fa.k = a.k; fa.v = a.v; fa.q = q; fa.cs = cs; fa.ci = ci; fa.out = out; fa.idx = idx;
+  fa.w = w; fa.sc = sc; fa.status = a.status;
+  // The grid barriers' counter: the word after the status word (the caller zeroes both).
+  fa.barrier = reinterpret_cast<unsigned*>(a.status + 1);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(sm_count()), 1, 1);  // one CTA per SM
+  cfg.blockDim = dim3(kSmallWarps * 32, 1, 1);
+  cfg.dynamicSmemBytes = m.total;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident: the barriers can end
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, forward_small_fused_kernel<T, MAXV>, fa);
+}
+
+bool small_fused_supported(int d_model, int H, int dq, int n, int v, int dtype) {
+  const FusedSmem m = fused_smem(d_model, H, dq, n, v, dtype == 0 ? 4 : 2);
+  return m.total <= 200 * 1024 && H <= kSmallWarps;
+}
+
+cudaError_t launch_forward_small_fused(const LayerArgs& a, float* q, float* chunk_s,
+                                       int* chunk_i, float* out, int* idx, float* w, float* sc,
+                                       cudaStream_t st) {
+#define PKM_FUSED(T)                                                                     \
+  switch (row_vecs_per_lane(a.v, a.dtype)) {                                             \
+    case 1: return launch_fused_t<T, 1>(a, q, chunk_s, chunk_i, out, idx, w, sc, st);    \
+    case 2: return launch_fused_t<T, 2>(a, q, chunk_s, chunk_i, out, idx, w, sc, st);    \
+    case 4: return launch_fused_t<T, 4>(a, q, chunk_s, chunk_i, out, idx, w, sc, st);    \
+    case 8: return launch_fused_t<T, 8>(a, q, chunk_s, chunk_i, out, idx, w, sc, st);    \
+  }                                                                                      \
+  return cudaErrorInvalidValue;
+  if (a.dtype == 0) {
+    PKM_FUSED(float)
+  }
+  PKM_FUSED(uint16_t)
+#undef PKM_FUSED
 }
 
 template <typename T>

@@ -3,7 +3,8 @@
 Both sides get the same indices and weights: the oracle's forward picks, rounded
 to fp32 for the device. Tolerance: 1e-4 absolute + 2e-3 relative on grad_scores
 and on every touched row of grad_values; untouched rows must stay exactly as the
-caller left them.
+caller left them. The value gradient sums each slot's picks in a fixed order, so two
+runs on the same inputs must agree bit for bit, whatever the group sizes.
 """
 import numpy as np
 import pytest
@@ -119,3 +120,38 @@ def test_backward_bad_slot_is_reported_not_written():
     contrib = (w32.double() * keep).reshape(-1, 1) * gout.double().repeat_interleave(H * k, 0)
     ref.index_add_(0, good.clamp(0, n * n - 1).reshape(-1).long(), contrib)
     torch.testing.assert_close(gv.cpu().double(), ref, rtol=2e-3, atol=1e-4)
+
+
+def _skewed(B, H, k, n, v, hot, seed):
+    idx, w32 = synth.random_selection(B, H, k, n * n, seed=seed, hot_rows=hot)
+    g = synth.generator(seed + 1)
+    values = (torch.randn(n * n, v, generator=g) / 16).to(torch.bfloat16)
+    gout = torch.randn(B, v, generator=g).to(torch.bfloat16)
+    return values, idx.numpy(), w32.numpy(), gout
+
+
+@pytest.mark.parametrize("B,hot", [(4096, 40), (600, 64), (300, 2000)])
+def test_backward_group_sizes_against_oracle(B, hot):
+    """Every pick from `hot` slots: groups of ~13,000 picks (split into work items with
+    partial rows), ~1,200 picks (one work item each) and ~19 picks (summed inline)."""
+    values, idx, w32, gout = _skewed(B, 4, 32, 256, 256, hot, seed=21 + hot)
+    gv, gs = _run(values, idx, w32, gout, 256)
+    _compare(values, idx, w32, gout, gv, gs)
+
+
+@pytest.mark.parametrize("hot", [0, 40])
+def test_backward_is_bit_for_bit_repeatable(hot):
+    """Two runs on the same inputs (uniform picks, and picks from 40 hot slots on the
+    c512 table size) give identical grad_values and grad_scores."""
+    if hot:
+        values, idx, w32, gout = _skewed(4096, 4, 32, 512, 1024, hot, seed=31)
+    else:
+        idx_t, w_t = synth.random_selection(4096, 4, 32, 512 * 512, seed=33)
+        g = synth.generator(34)
+        values = (torch.randn(512 * 512, 1024, generator=g) / 32).to(torch.bfloat16)
+        gout = torch.randn(4096, 1024, generator=g).to(torch.bfloat16)
+        idx, w32 = idx_t.numpy(), w_t.numpy()
+    gv1, gs1 = _run(values, idx, w32, gout, 512)
+    gv2, gs2 = _run(values, idx, w32, gout, 512)
+    assert torch.equal(gv1, gv2)
+    assert torch.equal(gs1, gs2)

@@ -33,37 +33,66 @@ def _forward(L, w, path=None):
         return to_numpy(out, idx, wt, sc)
 
 
-def _check(L, w):
-    g = _forward(L, w)
+def _check(L, w, path=None):
+    g = _forward(L, w, path)
     r = oracle.forward(L, w.H, w.dq, w.n, w.k, want_half=True)
     stats = compare_forward(g, r, L["values"], w.n)
     print(w.name, w.B, stats)
     return g, r
 
 
+# "auto": the three-kernel form; "small_fused": the single cooperative kernel.
+FORMS = ["auto", "small_fused"]
+
+
+@pytest.mark.parametrize("path", FORMS)
 @pytest.mark.parametrize("B", [1, 7, 64, 96, 128])
-def test_c1024_small_batches(B):
+def test_c1024_small_batches(B, path):
     w = synth.WORKLOADS["c1024"].with_(B=B)
-    _check(synth.make_layer(w), w)
+    _check(synth.make_layer(w), w, path)
 
 
-@pytest.mark.parametrize("name,B", [("c512", 33), ("wide", 16), ("tiny", 5)])
-def test_other_shapes(name, B):
+@pytest.mark.parametrize("path", FORMS)
+@pytest.mark.parametrize("name,B", [("c512", 33), ("wide", 16), ("wide", 128), ("tiny", 5)])
+def test_other_shapes(name, B, path):
     w = synth.WORKLOADS[name].with_(B=B)
-    _check(synth.make_layer(w), w)
+    _check(synth.make_layer(w), w, path)
 
 
+@pytest.mark.parametrize("path", FORMS)
 @pytest.mark.parametrize("k,n", [(1, 256), (3, 256), (8, 8), (32, 32)])
-def test_k_and_small_codebooks(k, n):
+def test_k_and_small_codebooks(k, n, path):
     w = synth.WORKLOADS["c512"].with_(B=9, n=n, k=k)
+    _check(synth.make_layer(w), w, path)
+
+
+def test_odd_half_query_goes_to_large_batch_kernels():
+    """fp32 with dq = 6 (halves of 3 elements): the small-batch scoring loop takes
+    element pairs, so such a layer runs on the large-batch CUDA-core kernels and must
+    still match the oracle."""
+    w = synth.WORKLOADS["tiny"].with_(B=4, dq=6)
     _check(synth.make_layer(w), w)
 
 
-def test_exact_ties_go_to_lower_slot():
+def test_fused_and_three_kernel_forms_agree():
+    """Same arithmetic in both forms: picks, weights and scores bit for bit; out up to
+    the order in which the H*k rows are added."""
+    w = synth.WORKLOADS["c1024"].with_(B=40)
+    L = synth.make_layer(w)
+    a = _forward(L, w, "small_fused")
+    b = _forward(L, w, "auto")
+    np.testing.assert_array_equal(a["indices"], b["indices"])
+    np.testing.assert_array_equal(a["weights"], b["weights"])
+    np.testing.assert_array_equal(a["scores"], b["scores"])
+    np.testing.assert_allclose(a["out"], b["out"], rtol=1e-5, atol=1e-6)
+
+
+@pytest.mark.parametrize("path", FORMS)
+def test_exact_ties_go_to_lower_slot(path):
     w = synth.WORKLOADS["c512"].with_(B=12, n=256)
     L = synth.make_layer(w)
     L["subkeys"][:, 0] = L["subkeys"][:, 0, :1]
-    g = _forward(L, w)
+    g = _forward(L, w, path)
     r = oracle.forward(L, w.H, w.dq, w.n, w.k, want_half=True)
     jstar = r["half"][:, :, 1].argmax(-1)
     expect = np.arange(w.k)[None, None, :] * w.n + jstar[..., None]
