@@ -238,7 +238,7 @@ int pkm_backward_train(const pkm_shape* s, const void* x, const void* W_q,
  * host that passes device pointers but no allocator). Arguments and results are
  * those of pkm_backward_values; the caller still passes inputs and outputs.
  *
- * Scratch: one fixed device array of about 40.3 MiB inside libpkm.so, held on every
+ * Scratch: one fixed device array of about 40.7 MiB inside libpkm.so, held on every
  * GPU that loads the library until the process exits. Limits: n*n <= 1,048,576 slots,
  * B*H*k <= 2,097,152 picks and v <= 2048; larger shapes return PKM_ERR_UNSUPPORTED
  * before any launch. The call allocates nothing (no cudaMalloc, no library allocator).

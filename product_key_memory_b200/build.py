@@ -21,11 +21,12 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libpkm.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
-# Test build: every pipeline wait of the tensor-core kernels gives up after 2 us (the
-# drains keep their full second), so tests can run the timeout path; see
-# tests/test_timeout_gpu.py. Loaded only through PKM_LIBRARY.
+# Test build: every pipeline wait of the tensor-core kernels gives up as soon as it is
+# not satisfied within one try (a 1 ns limit; the drains keep their full second), so
+# the first wait on a copy from HBM always runs out and tests exercise the timeout
+# path; see tests/test_timeout_gpu.py. Loaded only through PKM_LIBRARY.
 WAITTEST_LIB = os.path.join(HERE, "libpkm_waittest.so")
-WAITTEST_DEFINES = ("-DPKM_WAIT_LIMIT_NS=2000ull", "-DPKM_TRY_WAIT_HINT_NS=100")
+WAITTEST_DEFINES = ("-DPKM_WAIT_LIMIT_NS=1ull", "-DPKM_TRY_WAIT_HINT_NS=100")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",

@@ -39,8 +39,8 @@ constexpr int kSortWarps = kSortThreads / 32;
 constexpr int kSortSteps = 16;
 constexpr int kSortPerWarp = kSortSteps * 32;
 constexpr int kSortSub = kSortWarps * kSortPerWarp;     // 4096
-constexpr int kSortSubTiles = 4;
-constexpr int kSortTile = kSortSub * kSortSubTiles;     // 16384
+constexpr int kSortSubTiles = 1;
+constexpr int kSortTile = kSortSub * kSortSubTiles;     // 4096
 constexpr int kDigitBits = 8;
 constexpr int kDigits = 1 << kDigitBits;
 static_assert(kDigits == kSortThreads, "one thread per digit in the rank merge");
@@ -297,28 +297,44 @@ __device__ __forceinline__ int sort_key(const int* keys, int64_t p, int64_t slot
   return (first && (k < 0 || k >= slots)) ? static_cast<int>(slots) : k;
 }
 
-// Digit counts of one tile, written digit-major: hist[d * nblk + block].
+// Digit counts of one tile, written digit-major: hist[d * nblk + block]. Each thread
+// loads its kSortSteps keys before counting; a warp adds each distinct digit of a step
+// once (the lanes sharing it found by __match_any_sync).
 __global__ void __launch_bounds__(kSortThreads) radix_hist_kernel(
     const int* __restrict__ keys, int64_t E, int64_t slots, int shift, int first,
     int* __restrict__ hist, int64_t nblk, int* status) {
   __shared__ int h[kDigits];
   h[threadIdx.x] = 0;
-  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const unsigned lower = (1u << lane) - 1u;
   const int64_t base = static_cast<int64_t>(blockIdx.x) * kSortTile;
-  for (int i = threadIdx.x; i < kSortTile; i += kSortThreads) {
-    const int64_t p = base + i;
-    if (p >= E) break;
-    const int raw = keys[p];
-    if (first && (raw < 0 || raw >= slots)) record_status(status, kDevBadSlot);
-    const int key = sort_key(keys, p, slots, first);
-    atomicAdd(&h[(key >> shift) & (kDigits - 1)], 1);  // a count: any order gives the same
+  int raw[kSortSteps];
+#pragma unroll
+  for (int r = 0; r < kSortSteps; ++r) {
+    const int64_t p = base + r * kSortThreads + threadIdx.x;
+    raw[r] = p < E ? keys[p] : 0;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < kSortSteps; ++r) {
+    const int64_t p = base + r * kSortThreads + threadIdx.x;
+    const bool valid = p < E;
+    int key = raw[r];
+    if (first && valid && (key < 0 || key >= slots)) {
+      record_status(status, kDevBadSlot);
+      key = static_cast<int>(slots);
+    }
+    const int d = valid ? (key >> shift) & (kDigits - 1) : kDigits;
+    const unsigned peers = __match_any_sync(0xffffffffu, d);
+    if (valid && (peers & lower) == 0) atomicAdd(&h[d], __popc(peers));  // a count: any order
   }
   __syncthreads();
   hist[threadIdx.x * nblk + blockIdx.x] = h[threadIdx.x];
 }
 
 // Exclusive scan of the M digit-major counts, in place, by one block: each thread
-// scans a contiguous run, then the runs' totals are scanned across the block.
+// scans a contiguous run (loaded 8 at a time), then the runs' totals are scanned
+// across the block.
 __global__ void __launch_bounds__(1024) radix_scan_kernel(int* __restrict__ hist, int64_t M) {
   __shared__ int warp_tot[32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -326,7 +342,13 @@ __global__ void __launch_bounds__(1024) radix_scan_kernel(int* __restrict__ hist
   const int64_t b = threadIdx.x * per;
   const int64_t e = b + per < M ? b + per : M;
   int sum = 0;
-  for (int64_t i = b; i < e; ++i) sum += hist[i];
+  for (int64_t i0 = b; i0 < e; i0 += 8) {
+    int c[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) c[u] = i0 + u < e ? hist[i0 + u] : 0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) sum += c[u];
+  }
   int incl = sum;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -347,10 +369,15 @@ __global__ void __launch_bounds__(1024) radix_scan_kernel(int* __restrict__ hist
   }
   __syncthreads();
   int run = warp_tot[warp] + incl - sum;
-  for (int64_t i = b; i < e; ++i) {
-    const int c = hist[i];
-    hist[i] = run;
-    run += c;
+  for (int64_t i0 = b; i0 < e; i0 += 8) {
+    int c[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) c[u] = i0 + u < e ? hist[i0 + u] : 0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (i0 + u < e) hist[i0 + u] = run;
+      run += c[u];
+    }
   }
 }
 

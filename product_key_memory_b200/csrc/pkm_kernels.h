@@ -63,7 +63,7 @@ size_t backward_ws_bytes(int64_t B, int H, int k, int64_t slots, int v, Backward
 // out as backward_ws_bytes carves them (status word, list lengths, two key and two
 // pick buffers, digit counts, work lists, partial rows). A compile-time function so
 // that the fixed scratch of pkm_backward_values_noalloc is sized by the same sum.
-constexpr int kSortTileKeys = 16384;
+constexpr int kSortTileKeys = 4096;
 constexpr int kValueSmallGroup = 256;
 constexpr int kValueChunk = 4096;
 constexpr size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }

@@ -273,27 +273,27 @@ __global__ void __launch_bounds__(kTcThreads, 1) query_tc_kernel(
 // Two epilogue warp sets work on alternate units of the CTA, each with its own TMEM
 // accumulator (256 columns) and its own survivor log, so two warps share each SM
 // sub-partition. The MMA issuer interleaves the two sets' chunks.
-#ifndef PKM_SCORE_SETS
-#define PKM_SCORE_SETS 2
-#endif
-constexpr int kSSets = PKM_SCORE_SETS;
-constexpr int kSBufPerSet = 2 / kSSets;  // TMEM accumulators (256 columns) per set
+constexpr int kSSets = 2;
 constexpr int kSEpiWarps = 4 * kSSets;
 constexpr int kSThreads = 64 + 32 * kSEpiWarps;
-constexpr int kSK = kSSets == 2 ? 32 : 64;                          // K per stage
-constexpr int kSStages = kSSets == 2 ? 3 : 2;
-constexpr CUtensorMapSwizzle kSSwizzle =
-    kSK == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+constexpr int kSK = 32;                                             // K per stage
+constexpr int kSStages = 3;
+constexpr CUtensorMapSwizzle kSSwizzle = CU_TENSOR_MAP_SWIZZLE_64B;
 constexpr uint32_t kSPlaneBytes = kRowsPerTile * kSK * 2;           // 8 KiB
 constexpr uint32_t kSABytes = kScorePlanes * kSPlaneBytes;          // 16 KiB
 constexpr uint32_t kSBBytes = kColsPerMma * kSK * 2;                // 16 KiB
 constexpr uint32_t kSStageBytes = kSABytes + kSBBytes;              // 32 KiB
 constexpr int kList = kMaxK;          // entries per per-half list (the best 32, any order)
 constexpr int kSStep = 8;             // columns read from TMEM per step
-constexpr int kSNewCap = 32;          // survivors logged between two merges
+constexpr int kSSteps = kColsPerMma / kSStep;  // steps per chunk
+constexpr int kSNewCap = 48;          // survivors logged between two merges
+constexpr int kSMidMerge = kSNewCap - 2 * kSStep;  // fresh entries that force a merge
+                                                   // inside a chunk (two steps' room left)
+constexpr int kSEndMerge = 8;         // fresh entries worth a merge at a chunk's end
 constexpr int kSLogCap = kList + kSNewCap;
 constexpr int kSTrash = kSLogCap;     // slot written (and dropped) past a full log
 constexpr int kSLogRows = kSLogCap + 1;
+static_assert(kSSteps % 2 == 0, "the step loop alternates two load buffers");
 
 size_t score_tc_smem_bytes() {
   // stages + per-set log: fp32 scores and 16-bit ids for 128 rows + barriers
@@ -442,9 +442,9 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
         for (int c = 0; c < nchunks && ok; ++c)
           for (int set = 0; set < kSSets && ok; ++set) {
             if (j0 + set >= myunits) break;
-            // Accumulator b of this set; its uses alternate between the set's buffers.
-            const int b = set * kSBufPerSet + uses[set] % kSBufPerSet;
-            const uint32_t tph = (uses[set] / kSBufPerSet) & 1;
+            // Set `set` owns accumulator `set`; its uses alternate the barrier phase.
+            const int b = set;
+            const uint32_t tph = uses[set] & 1;
             if (!mbar_wait(&tempty[b], tph ^ 1, status, abort)) { ok = false; break; }
             tc_fence_after();
             const uint32_t d_tmem = tmem_base + b * kColsPerMma;
@@ -456,12 +456,9 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
 #pragma unroll
               for (int p = 0; p < kScorePlanes; ++p)
 #pragma unroll
-                for (int jj = 0; jj < kSK / 16; ++jj) {
-                  const uint64_t ad = kSK == 32 ? sw64_desc(a + p * kSPlaneBytes, jj * 32)
-                                                : sw128_desc(a + p * kSPlaneBytes, jj * 32);
-                  const uint64_t bd = kSK == 32 ? sw64_desc(bb, jj * 32) : sw128_desc(bb, jj * 32);
-                  mma_bf16(d_tmem, ad, bd, idesc, (kb | p | jj) != 0);
-                }
+                for (int jj = 0; jj < kSK / 16; ++jj)
+                  mma_bf16(d_tmem, sw64_desc(a + p * kSPlaneBytes, jj * 32), sw64_desc(bb, jj * 32),
+                           idesc, (kb | p | jj) != 0);
               mma_commit(&empty[s]);
               if (++s == kSStages) { s = 0; ph ^= 1; }
             }
@@ -478,6 +475,10 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
     // Ls holds the 32 largest scores seen so far (values only, sorted); the log in
     // shared memory holds (score, id) of every element that can still be among the
     // best 32. Columns arrive in increasing sub-key id, so the log is in id order.
+    // A chunk is read 8 columns per step with the next step's TMEM load in flight, and
+    // the accumulator goes back to the MMA issuer as soon as its last columns are read:
+    // the merge that normally follows a chunk runs after that, while the MMAs of the
+    // set's next chunk proceed.
     const int set = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
@@ -488,7 +489,7 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
     // s_row + e * kSStrideS (score) and i_row + e * kSStrideI (id).
     constexpr uint32_t kSStrideS = kRowsPerTile * 4, kSStrideI = kRowsPerTile * 2;
     const uint32_t s_row = smem_addr(lg_s + r), i_row = smem_addr(lg_i + r);
-    constexpr int kStepsPerChunk = kColsPerMma / kSStep;
+    const uint32_t acc0 = tmem_base + lane_addr + set * kColsPerMma;  // this set's accumulator
     int uses = 0;
     for (int j = set; j < myunits; j += kSSets) {
       const int u = nunits - 1 - static_cast<int>(blockIdx.x + j * gridDim.x);
@@ -503,53 +504,32 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
       float thr = -INFINITY;   // v > thr  <=>  v >= tau0 && v > tau_run
       int cnt = 0, kept = 0;   // log entries; entries kept by the last merge
       bool ok = true;
-      const int nsteps = nchunks * kStepsPerChunk;
-      int bsel = set * kSBufPerSet;
-      uint32_t col0 = tmem_base + lane_addr + bsel * kColsPerMma;
-#pragma unroll 1
-      for (int st = 0; st <= nsteps; ++st) {
-        const bool flush = st == nsteps;
-        const int c = st / kStepsPerChunk, sc = st - c * kStepsPerChunk;
-        float v[kSStep];
-        if (!flush) {
-          if (sc == 0) {
-            const int uc = uses + c;
-            bsel = set * kSBufPerSet + uc % kSBufPerSet;
-            col0 = tmem_base + lane_addr + bsel * kColsPerMma;
-            if (!warp_wait(&tfull[bsel], (uc / kSBufPerSet) & 1, status, abort)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            if (c == 0) {
-              // The maxima of the 64 groups of 4 columns are 64 different scores of the
-              // chunk, so its 32nd best (and the row's) is at least the 32nd largest.
-              float mx[64];
+
+      // Branch-free filter of 8 columns: every score is written to the next free log
+      // slot, which only advances when the score is kept (a rejected one is overwritten).
+      auto filter = [&](const uint32_t (&rv)[8], int id0) {
+        uint32_t as = s_row + cnt * kSStrideS, ai = i_row + cnt * kSStrideI;
 #pragma unroll
-              for (int g = 0; g < 8; ++g) {
-                float w[32];
-                tmem_ld32(col0 + g * 32, w);
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                  mx[g * 8 + i] = fmaxf(fmaxf(w[4 * i], w[4 * i + 1]),
-                                        fmaxf(w[4 * i + 2], w[4 * i + 3]));
-              }
-              tau0 = kth32_of_64(mx);
-              thr = fmaxf(nextafterf(tau0, -INFINITY), tau_run);
-            }
-          }
-          tmem_ld8(col0 + sc * kSStep, v);
-          if (sc == kStepsPerChunk - 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[bsel]);
+        for (int i = 0; i < kSStep; ++i) {
+          const float v = __uint_as_float(rv[i]);
+          sts_f32(as, v);
+          sts_u16(ai, static_cast<uint16_t>(id0 + i));
+          if (v > thr) {
+            as += kSStrideS;
+            ai += kSStrideI;
           }
         }
-        // Merge when the next step could overflow the log, and once at the end.
-        const int fresh = cnt - kept;
-        if (__any_sync(0xffffffffu, flush ? fresh > 0 : fresh > kSNewCap - kSStep)) {
+        cnt = static_cast<int>((as - s_row) / kSStrideS);
+      };
+
+      // Merge every fresh log entry into Ls (32 at a time), raise tau_run and compact
+      // the log to the entries that can still be among the best 32.
+      auto merge = [&]() {
+#pragma unroll 1
+        for (int base = kept; __any_sync(0xffffffffu, base < cnt); base += 32) {
+          const int fresh = cnt - base;
           float b[32];
-          const uint32_t fresh_at = s_row + kept * kSStrideS;
+          const uint32_t fresh_at = s_row + base * kSStrideS;
 #pragma unroll
           for (int q = 0; q < 32; ++q)
             b[q] = q < fresh ? lds_f32(fresh_at + q * kSStrideS) : -INFINITY;
@@ -562,73 +542,105 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
             for (int i = 0; i < 32; ++i) {
               const int jj = i ^ stride;
               if (jj > i) {
-                const float a = Ls[i], bb = Ls[jj];
-                Ls[i] = fmaxf(a, bb);
-                Ls[jj] = fminf(a, bb);
+                const float x0 = Ls[i], x1 = Ls[jj];
+                Ls[i] = fmaxf(x0, x1);
+                Ls[jj] = fminf(x0, x1);
               }
             }
-          tau_run = Ls[31];
-          // Branch-free in-place compaction to the entries >= tau_run: each entry is
-          // rewritten either to slot w (w <= e, so nothing unread is overwritten) or to
-          // the trash slot. That keeps the current best 32 plus any later entry tied
-          // with the 32nd score.
-          // Every entry is written to the current write slot, which only advances for a
-          // kept entry (w <= e, so nothing unread is overwritten).
-          const int cmax = __reduce_max_sync(0xffffffffu, cnt);
-          uint32_t ws = s_row, wi = i_row;
+        }
+        tau_run = Ls[31];
+        // Branch-free in-place compaction to the entries >= tau_run: every entry is
+        // written to the current write slot, which only advances for a kept entry (w <= e,
+        // so nothing unread is overwritten). That keeps the current best 32 plus any
+        // later entry tied with the 32nd score.
+        const int cmax = __reduce_max_sync(0xffffffffu, cnt);
+        uint32_t ws = s_row, wi = i_row;
 #pragma unroll 4
-          for (int e = 0; e < cmax; ++e) {
-            const float sv = lds_f32(s_row + e * kSStrideS);
-            const uint16_t iv = lds_u16(i_row + e * kSStrideI);
-            sts_f32(ws, sv);
-            sts_u16(wi, iv);
-            if (e < cnt && sv >= tau_run) {
-              ws += kSStrideS;
-              wi += kSStrideI;
-            }
+        for (int e = 0; e < cmax; ++e) {
+          const float sv = lds_f32(s_row + e * kSStrideS);
+          const uint16_t iv = lds_u16(i_row + e * kSStrideI);
+          sts_f32(ws, sv);
+          sts_u16(wi, iv);
+          if (e < cnt && sv >= tau_run) {
+            ws += kSStrideS;
+            wi += kSStrideI;
           }
-          int w = static_cast<int>((ws - s_row) / kSStrideS);
-          if (__any_sync(0xffffffffu, w > kList)) {
-            // Rare: ties at the 32nd score. Of the entries equal to tau_run keep the first
-            // `eq` in id order (eq = how many of the best 32 scores equal it), so the log
-            // is exactly the best 32 by (score desc, id asc).
-            int eq = 0;
+        }
+        int w = static_cast<int>((ws - s_row) / kSStrideS);
+        if (__any_sync(0xffffffffu, w > kList)) {
+          // Rare: ties at the 32nd score. Of the entries equal to tau_run keep the first
+          // `eq` in id order (eq = how many of the best 32 scores equal it), so the log
+          // is exactly the best 32 by (score desc, id asc).
+          int eq = 0;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) eq += Ls[i] == tau_run ? 1 : 0;
-            const int wmax = __reduce_max_sync(0xffffffffu, w);
-            int w2 = 0;
-            for (int e = 0; e < wmax; ++e) {
-              const float sv = lg_s[e * kRowsPerTile + r];
-              const uint16_t iv = lg_i[e * kRowsPerTile + r];
-              const bool tie = e < w && sv == tau_run && eq > 0;
-              const bool keep = e < w && (sv > tau_run || tie);
-              eq -= tie ? 1 : 0;
-              const int dst = keep ? w2 : kSTrash;
-              lg_s[dst * kRowsPerTile + r] = sv;
-              lg_i[dst * kRowsPerTile + r] = iv;
-              w2 += keep ? 1 : 0;
-            }
-            w = w2;
+          for (int i = 0; i < 32; ++i) eq += Ls[i] == tau_run ? 1 : 0;
+          const int wmax = __reduce_max_sync(0xffffffffu, w);
+          int w2 = 0;
+          for (int e = 0; e < wmax; ++e) {
+            const float sv = lg_s[e * kRowsPerTile + r];
+            const uint16_t iv = lg_i[e * kRowsPerTile + r];
+            const bool tie = e < w && sv == tau_run && eq > 0;
+            const bool keep = e < w && (sv > tau_run || tie);
+            eq -= tie ? 1 : 0;
+            const int dst = keep ? w2 : kSTrash;
+            lg_s[dst * kRowsPerTile + r] = sv;
+            lg_i[dst * kRowsPerTile + r] = iv;
+            w2 += keep ? 1 : 0;
           }
-          cnt = w;
-          kept = w;
+          w = w2;
+        }
+        cnt = w;
+        kept = w;
+        thr = fmaxf(nextafterf(tau0, -INFINITY), tau_run);
+      };
+
+#pragma unroll 1
+      for (int c = 0; c < nchunks; ++c) {
+        if (!warp_wait(&tfull[set], (uses + c) & 1, status, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (c == 0) {
+          // The maxima of the 64 groups of 4 columns are 64 different scores of the
+          // chunk, so its 32nd best (and the row's) is at least the 32nd largest.
+          float mx[64];
+#pragma unroll
+          for (int g = 0; g < 8; ++g) {
+            float w[32];
+            tmem_ld32(acc0 + g * 32, w);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              mx[g * 8 + i] = fmaxf(fmaxf(w[4 * i], w[4 * i + 1]), fmaxf(w[4 * i + 2], w[4 * i + 3]));
+          }
+          tau0 = kth32_of_64(mx);
           thr = fmaxf(nextafterf(tau0, -INFINITY), tau_run);
         }
-        if (!flush) {
-          // Branch-free filter: every score is written to the next free log slot, which
-          // only advances when the score is kept (a rejected one is overwritten).
-          const int id0 = c * kColsPerMma + sc * kSStep;
-          uint32_t as = s_row + cnt * kSStrideS, ai = i_row + cnt * kSStrideI;
-#pragma unroll
-          for (int i = 0; i < kSStep; ++i) {
-            sts_f32(as, v[i]);
-            sts_u16(ai, static_cast<uint16_t>(id0 + i));
-            if (v[i] > thr) {
-              as += kSStrideS;
-              ai += kSStrideI;
-            }
+        const int id_base = c * kColsPerMma;
+        const bool last_chunk = c == nchunks - 1;
+        uint32_t ra[8], rb[8];
+        tmem_ld8_issue(acc0, ra);
+#pragma unroll 1
+        for (int st = 0; st < kSSteps; st += 2) {
+          tmem_wait_ld8(ra);
+          tmem_ld8_issue(acc0 + (st + 1) * kSStep, rb);
+          filter(ra, id_base + st * kSStep);
+          tmem_wait_ld8(rb);
+          const bool chunk_end = st + 2 >= kSSteps;
+          if (!chunk_end) {
+            tmem_ld8_issue(acc0 + (st + 2) * kSStep, ra);
+          } else {
+            // Every column of the accumulator has been read: hand it back.
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[set]);
           }
-          cnt = static_cast<int>((as - s_row) / kSStrideS);
+          filter(rb, id_base + (st + 1) * kSStep);
+          // Merge when the next two steps could overflow the log, after a chunk when
+          // enough is fresh, and after the unit's last chunk whenever anything is.
+          const int fresh = cnt - kept;
+          const int limit = !chunk_end ? kSMidMerge : (last_chunk ? 0 : kSEndMerge);
+          if (__any_sync(0xffffffffu, fresh > limit)) merge();
         }
       }
       uses += nchunks;

@@ -1,7 +1,8 @@
 """The timeout path of the tensor-core kernels, run on the GPU without a hang.
 
-The test build of the library (libpkm_waittest.so: every pipeline wait gives up
-after 2 us, the drains keep their full second) is loaded in a child process through
+The test build of the library (libpkm_waittest.so: every pipeline wait gives up as
+soon as one try does not satisfy it, so the first wait on a copy from HBM always runs
+out; the drains keep their full second) is loaded in a child process through
 PKM_LIBRARY. Its forward and full backward must return, record the timeout in the
 workspace status word (pkm_device_status -> PKM_ERR_DEVICE), leave the CUDA context
 usable, and exit cleanly. Nothing is done to the GPU that a normal call does not do:
