@@ -523,7 +523,7 @@ def run_c512_and_backward(args, dev, P, hbm, bf16, stream, world, barrier,
             "algorithmic_bytes": full_bytes, "gemm_flops": full_flops,
             "step_roofline_frac": max(t_mem, t_gemm) * 1e3 / full_ms}
     if "latency" in parts:
-        res["small_batch"] = run_latency(args, dev, P)
+        res["small_batch"] = run_latency(args, dev, P, with_wide="wide" not in parts)
     if "train" in parts:
         # One training step of the layer with BatchNorm in training mode: the forward
         # on batch statistics (running statistics updated), then the full backward
@@ -594,6 +594,8 @@ def run_c512_and_backward(args, dev, P, hbm, bf16, stream, world, barrier,
                    "step_roofline_frac": max(t_mem, t_gemm) * 1e3 / fwd_ms,
                    "stage_ms": [m / max(1, calls) for m in stage_ms[:3]],
                    "gather_gbs": per_token_bytes(w) * B / (stage_ms[2] / max(1, calls) * 1e-3) / 1e9}
+    if "small_batch" in res:
+        res["small_batch"].update(latency_table(args, dev, P, "wide", d, (64, 96, 112, 128)))
     return res
 
 
@@ -602,39 +604,64 @@ def pruned_pairs(k: int) -> int:
     return sum(k // (a + 1) for a in range(k))
 
 
-def run_latency(args, dev, P):
-    """Forward latency for a few tokens on the 1024^2-slot layer (the serving case):
-    calls issued back to back on one stream, device time per call from CUDA events
-    around 200 calls; caches warm (one token touches 128 value rows)."""
+def latency_table(args, dev, P, wname, d, Bs):
+    """Forward latency of a few tokens on the layer d (device tensors of workload
+    wname): calls issued back to back on one stream, device time per call from CUDA
+    events around 200 calls; caches warm (one token touches H*k value rows). Each
+    batch size through the default choice, each small-batch form forced (the single
+    cooperative kernel "small_fused", the three kernels "small_split") and the
+    large-batch tensor-core kernels ("tc"): the data behind the cut-offs."""
+    w0 = synth.WORKLOADS[wname]
+    res = {}
+    for path in ("auto", "small_fused", "small_split", "tc"):
+        for B in Bs:
+            x = d["x"][:B].contiguous()
+            out = torch.empty(B, w0.v, device=dev)
+            idx = torch.empty(B, w0.H, w0.k, dtype=torch.int32, device=dev)
+            wts = torch.empty(B, w0.H, w0.k, device=dev)
+            with P.options(path=path):
+                shape = P.make_shape(B, w0.d_model, w0.H, w0.dq, w0.n, w0.k, w0.v,
+                                     w0.torch_dtype)
+                ws = P.alloc_workspace(shape, False, dev)
+
+                def call():
+                    P.pkm_forward(x, d["W_q"], d["bn_mean"], d["bn_var"], d["bn_gamma"],
+                                  d["bn_beta"], d["subkeys"], d["values"], k=w0.k, out=out,
+                                  indices=idx, weights=wts, want_scores=False, workspace=ws)
+
+                for _ in range(max(3, args.warmup) * 4):
+                    call()
+                torch.cuda.synchronize(dev)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                n = 200
+                a.record()
+                for _ in range(n):
+                    call()
+                b.record()
+                torch.cuda.synchronize(dev)
+            key = ("" if wname == "c1024" else wname + " ") + "B=%d" % B
+            key += "" if path == "auto" else " " + path
+            res[key] = a.elapsed_time(b) / n * 1e3
+    return res
+
+
+def run_latency(args, dev, P, with_wide=False):
+    """Small-batch latency on the 1024^2-slot layer (1 to 128 tokens). The wide layer's
+    entries are added where that layer is built (run_c512_and_backward), or here when
+    with_wide is set (the latency part run alone)."""
     w0 = synth.WORKLOADS["c1024"]
-    L = synth.make_layer(w0.with_(B=64))
+    L = synth.make_layer(w0.with_(B=128))
     d = {k: v.to(dev) for k, v in L.items()}
-    res = {"workload": "c1024 layer (1024^2 slots, H=4, k=32, v=1024, bf16), B tokens per call",
+    res = {"workload": "c1024 layer (1024^2 slots, H=4, k=32, v=1024, bf16) and the wide "
+                       "layer (d_model 1600, H=8, v=1600), B tokens per call",
            "unit": "us per call"}
-    for B in (1, 16, 64):
-        x = d["x"][:B].contiguous()
-        out = torch.empty(B, w0.v, device=dev)
-        idx = torch.empty(B, w0.H, w0.k, dtype=torch.int32, device=dev)
-        wts = torch.empty(B, w0.H, w0.k, device=dev)
-        shape = P.make_shape(B, w0.d_model, w0.H, w0.dq, w0.n, w0.k, w0.v, w0.torch_dtype)
-        ws = P.alloc_workspace(shape, False, dev)
-
-        def call():
-            P.pkm_forward(x, d["W_q"], d["bn_mean"], d["bn_var"], d["bn_gamma"], d["bn_beta"],
-                          d["subkeys"], d["values"], k=w0.k, out=out, indices=idx,
-                          weights=wts, want_scores=False, workspace=ws)
-
-        for _ in range(max(3, args.warmup) * 4):
-            call()
-        torch.cuda.synchronize(dev)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        n = 200
-        a.record()
-        for _ in range(n):
-            call()
-        b.record()
-        torch.cuda.synchronize(dev)
-        res["B=%d" % B] = a.elapsed_time(b) / n * 1e3
+    res.update(latency_table(args, dev, P, "c1024", d, (1, 4, 8, 16, 32, 64, 96, 112, 128)))
+    del d, L
+    if with_wide:
+        L = synth.make_layer(synth.WORKLOADS["wide"].with_(B=128))
+        d = {k: v.to(dev) for k, v in L.items()}
+        del L
+        res.update(latency_table(args, dev, P, "wide", d, (64, 96, 112, 128)))
     return res
 
 

@@ -105,12 +105,12 @@ size_t pkm_workspace_size(const pkm_shape* s, int for_backward);
  *   scores   [B][H][k]  fp32   kept key scores s1[i] + s2[j]; may be NULL
  * workspace: device scratch of at least pkm_workspace_size(s, 0) bytes, 256-byte
  *   aligned; its contents on entry do not matter.
- * Batches of at most 128 tokens (H <= 8) take the small-batch path, which spreads
- * W_q, the sub-keys and the heads over all SMs for latency: three kernels that
- * overlap through programmatic dependent launch on `stream`, or, with
- * PKM_PATH_SMALL_FUSED, one cooperative kernel (one block per SM, its query, scoring
- * and gather phases separated by grid-wide barriers whose waits are bounded like the
- * pipelines'). Larger batches run
+ * Batches of at most 112 tokens (H <= 8) take the small-batch path, which spreads
+ * W_q, the sub-keys and the heads over all SMs for latency: from 8 to 32 tokens one
+ * cooperative kernel (one block per SM, its query, scoring and gather phases
+ * separated by grid-wide barriers whose waits are bounded like the pipelines'),
+ * otherwise three kernels that overlap through programmatic dependent launch on
+ * `stream` (PKM_OPT_PATH can force either form). Larger batches run
  * three kernels on `stream` (query network, per-half scores and top-k, candidate
  * top-k + softmax + gather). With PKM_OPT_SUBBATCHES > 1, large batches of
  * tensor-core shapes are processed in up to that many sub-batches; the value gather
@@ -238,7 +238,7 @@ int pkm_backward_train(const pkm_shape* s, const void* x, const void* W_q,
  * host that passes device pointers but no allocator). Arguments and results are
  * those of pkm_backward_values; the caller still passes inputs and outputs.
  *
- * Scratch: one fixed device array of about 40.7 MiB inside libpkm.so, held on every
+ * Scratch: one fixed device array of about 44.2 MiB inside libpkm.so, held on every
  * GPU that loads the library until the process exits. Limits: n*n <= 1,048,576 slots,
  * B*H*k <= 2,097,152 picks and v <= 2048; larger shapes return PKM_ERR_UNSUPPORTED
  * before any launch. The call allocates nothing (no cudaMalloc, no library allocator).
@@ -295,7 +295,7 @@ int pkm_trace_read(int pass, double* stage_ms, int max_stages, int64_t* calls,
 /*
  * Implementation switches (a convenience of this library; the pages have no
  * counterpart). Process-wide, for every device; a change applies to calls made after
- * it. The environment variables PKM_PATH (auto | tc | simt | small_fused) and
+ * it. The environment variables PKM_PATH (auto | tc | simt | small_fused | small_split) and
  * PKM_SUBBATCHES (1..4)
  * give the initial values and are read once, at the first call that needs them.
  *   PKM_OPT_PATH        PKM_PATH_AUTO (default): small-batch kernels for up to 128
@@ -304,8 +304,10 @@ int pkm_trace_read(int pass, double* stage_ms, int max_stages, int64_t* calls,
  *                       multiple of 256, H*dq <= 4096), else the CUDA-core kernels;
  *                       PKM_PATH_TC: never the small-batch kernels;
  *                       PKM_PATH_SIMT: always the CUDA-core kernels;
- *                       PKM_PATH_SMALL_FUSED: as AUTO, but small batches run as one
- *                       cooperative kernel instead of three kernels.
+ *                       PKM_PATH_SMALL_FUSED: as AUTO, but every small batch runs as
+ *                       the one cooperative kernel;
+ *                       PKM_PATH_SMALL_SPLIT: as AUTO, but every small batch runs as
+ *                       the three kernels.
  *   PKM_OPT_SUBBATCHES  1 (default) to 4: sub-batches of the pipelined tensor-core
  *                       forward (see pkm_forward). The forward's workspace size
  *                       depends on it: query it after setting the option.
@@ -313,7 +315,13 @@ int pkm_trace_read(int pass, double* stage_ms, int max_stages, int64_t* calls,
  * pkm_get_option returns the current value or PKM_ERR_INVALID_ARG.
  */
 enum { PKM_OPT_PATH = 0, PKM_OPT_SUBBATCHES = 1 };
-enum { PKM_PATH_AUTO = 0, PKM_PATH_TC = 1, PKM_PATH_SIMT = 2, PKM_PATH_SMALL_FUSED = 3 };
+enum {
+  PKM_PATH_AUTO = 0,
+  PKM_PATH_TC = 1,
+  PKM_PATH_SIMT = 2,
+  PKM_PATH_SMALL_FUSED = 3,
+  PKM_PATH_SMALL_SPLIT = 4
+};
 int pkm_set_option(int option, int value);
 int pkm_get_option(int option);
 

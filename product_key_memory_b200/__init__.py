@@ -22,9 +22,9 @@ LIB_PATH = os.environ.get("PKM_LIBRARY") or os.path.join(_HERE, "libpkm.so")
 PKM_F32, PKM_BF16 = 0, 1
 PKM_OK = 0
 PKM_OPT_PATH, PKM_OPT_SUBBATCHES = 0, 1
-PKM_PATH_AUTO, PKM_PATH_TC, PKM_PATH_SIMT, PKM_PATH_SMALL_FUSED = 0, 1, 2, 3
+PKM_PATH_AUTO, PKM_PATH_TC, PKM_PATH_SIMT, PKM_PATH_SMALL_FUSED, PKM_PATH_SMALL_SPLIT = range(5)
 _PATHS = {"auto": PKM_PATH_AUTO, "tc": PKM_PATH_TC, "simt": PKM_PATH_SIMT,
-          "small_fused": PKM_PATH_SMALL_FUSED}
+          "small_fused": PKM_PATH_SMALL_FUSED, "small_split": PKM_PATH_SMALL_SPLIT}
 _STATUS = {0: "PKM_OK", -1: "PKM_ERR_INVALID_ARG", -2: "PKM_ERR_UNSUPPORTED",
            -3: "PKM_ERR_WORKSPACE", -4: "PKM_ERR_CUDA", -5: "PKM_ERR_DEVICE"}
 
@@ -115,8 +115,8 @@ def pkm_get_option(option: int) -> int:
 
 class options:
     """Context manager that sets the library's implementation switches and restores
-    them on exit: ``with options(path="simt"): ...`` (path: "auto", "tc", "simt" or
-    "small_fused"; subbatches: 1..4)."""
+    them on exit: ``with options(path="simt"): ...`` (path: "auto", "tc", "simt",
+    "small_fused" or "small_split"; subbatches: 1..4)."""
 
     def __init__(self, path: Optional[str] = None, subbatches: Optional[int] = None):
         self.want = {}

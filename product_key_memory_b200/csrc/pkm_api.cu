@@ -28,7 +28,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 enum class Path { kTensor, kSimt, kSmall };
 
 // Process-wide implementation switches (pkm_set_option). The environment variables
-// PKM_PATH (auto | tc | simt | small_fused) and PKM_SUBBATCHES (1..4) give their initial values and
+// PKM_PATH (auto | tc | simt | small_fused | small_split) and PKM_SUBBATCHES (1..4) give their initial values and
 // are read once, at the first call that needs them.
 std::atomic<int> g_opt_path{PKM_PATH_AUTO};
 std::atomic<int> g_opt_subbatches{1};
@@ -40,6 +40,7 @@ void init_options() {
     if (p && strcmp(p, "simt") == 0) g_opt_path = PKM_PATH_SIMT;
     if (p && strcmp(p, "tc") == 0) g_opt_path = PKM_PATH_TC;
     if (p && strcmp(p, "small_fused") == 0) g_opt_path = PKM_PATH_SMALL_FUSED;
+    if (p && strcmp(p, "small_split") == 0) g_opt_path = PKM_PATH_SMALL_SPLIT;
     const char* sb = getenv("PKM_SUBBATCHES");
     if (sb) {
       const int v = atoi(sb);
@@ -100,6 +101,7 @@ struct ForwardWs {
   void* planes;     // tensor path: bf16 q planes [kScorePlanes][sub][H*dq] of a sub-batch
   float* list_s;    // [B][H][2][32] best 32 per half (any order)
   int* list_i;      // [B][H][2][32]
+  float* part;      // small-batch path: [B][H][v] each head's output row
 };
 
 // Tokens per pipelined sub-batch of the tensor-core path: PKM_OPT_SUBBATCHES (1..4,
@@ -130,12 +132,15 @@ size_t forward_ws(const pkm_shape* s, ForwardWs* w, char* base) {
   const size_t o_q = off;  off += align256(qbytes);
   const size_t o_ls = off; off += align256(sizeof(float) * L);
   const size_t o_li = off; off += align256(sizeof(int) * L);
+  const size_t o_pt = off;
+  off += align256(path == Path::kSmall ? sizeof(float) * s->B * s->H * s->v : 0);
   if (w && base) {
     w->status = reinterpret_cast<int*>(base);
     w->q = reinterpret_cast<float*>(base + o_q);
     w->planes = base + o_q;
     w->list_s = reinterpret_cast<float*>(base + o_ls);
     w->list_i = reinterpret_cast<int*>(base + o_li);
+    w->part = reinterpret_cast<float*>(base + o_pt);
   }
   return off;
 }
@@ -306,7 +311,7 @@ int pkm_set_option(int option, int value) {
   init_options();
   if (option == PKM_OPT_PATH) {
     if (value != PKM_PATH_AUTO && value != PKM_PATH_TC && value != PKM_PATH_SIMT &&
-        value != PKM_PATH_SMALL_FUSED)
+        value != PKM_PATH_SMALL_FUSED && value != PKM_PATH_SMALL_SPLIT)
       return PKM_ERR_INVALID_ARG;
     g_opt_path = value;
     return PKM_OK;
@@ -534,10 +539,13 @@ cudaError_t run_forward(const pkm_shape* s, const LayerArgs& a, const ForwardWs&
   const Path path = choose_path(s);
   if (path == Path::kSmall) {
     tr.begin(2, st);
-    if (g_opt_path.load(std::memory_order_relaxed) == PKM_PATH_SMALL_FUSED &&
+    const int pin = g_opt_path.load(std::memory_order_relaxed);
+    if (pin != PKM_PATH_SMALL_SPLIT &&
+        (pin == PKM_PATH_SMALL_FUSED ||
+         (s->B >= pkm::kSmallFusedMinB && s->B <= pkm::kSmallFusedMaxB)) &&
         pkm::small_fused_supported(s->d_model, s->H, s->dq, s->n, s->v, s->dtype)) {
-      e = pkm::launch_forward_small_fused(a, w.q, w.list_s, w.list_i, out, indices, weights,
-                                          scores, st);
+      e = pkm::launch_forward_small_fused(a, w.q, w.list_s, w.list_i, w.part, out, indices,
+                                          weights, scores, st);
       launches = 1;
     } else {
       e = pkm::launch_forward_small(a, w.q, w.list_s, w.list_i, out, indices, weights, scores,

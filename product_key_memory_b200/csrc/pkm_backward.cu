@@ -41,9 +41,10 @@ constexpr int kSortPerWarp = kSortSteps * 32;
 constexpr int kSortSub = kSortWarps * kSortPerWarp;     // 4096
 constexpr int kSortSubTiles = 1;
 constexpr int kSortTile = kSortSub * kSortSubTiles;     // 4096
-constexpr int kDigitBits = 8;
-constexpr int kDigits = 1 << kDigitBits;
-static_assert(kDigits == kSortThreads, "one thread per digit in the rank merge");
+constexpr int kDigitBits = 11;
+constexpr int kDigits = 1 << kDigitBits;                // 2048
+constexpr int kDigitsPerThread = kDigits / kSortThreads;  // 8
+static_assert(kDigits % kSortThreads == 0, "digits split evenly over the threads");
 
 // Group sizes: up to kSmallGroup picks a warp sums inline; larger groups are cut into
 // work items of at most kChunk picks, one block each.
@@ -76,7 +77,7 @@ size_t backward_ws_bytes(int64_t B, int H, int k, int64_t slots, int v, Backward
   const int64_t max_huge = value_bwd_max_huge(E);
   const int64_t max_chunks = value_bwd_max_chunks(E);
   size_t off = kStatusBytes;
-  const size_t o_ctr = off;      off += 256;
+  const size_t o_ctr = off;      off += 8448;  // list lengths [4], digit totals [64, 2112)
   const size_t o_k0 = off;       off += align256(sizeof(int) * E1);
   const size_t o_p0 = off;       off += align256(sizeof(int) * E1);
   const size_t o_k1 = off;       off += align256(sizeof(int) * E1);
@@ -304,7 +305,8 @@ __global__ void __launch_bounds__(kSortThreads) radix_hist_kernel(
     const int* __restrict__ keys, int64_t E, int64_t slots, int shift, int first,
     int* __restrict__ hist, int64_t nblk, int* status) {
   __shared__ int h[kDigits];
-  h[threadIdx.x] = 0;
+#pragma unroll
+  for (int i = 0; i < kDigitsPerThread; ++i) h[threadIdx.x + i * kSortThreads] = 0;
   const int lane = threadIdx.x & 31;
   const unsigned lower = (1u << lane) - 1u;
   const int64_t base = static_cast<int64_t>(blockIdx.x) * kSortTile;
@@ -329,56 +331,35 @@ __global__ void __launch_bounds__(kSortThreads) radix_hist_kernel(
     if (valid && (peers & lower) == 0) atomicAdd(&h[d], __popc(peers));  // a count: any order
   }
   __syncthreads();
-  hist[threadIdx.x * nblk + blockIdx.x] = h[threadIdx.x];
+#pragma unroll
+  for (int i = 0; i < kDigitsPerThread; ++i) {
+    const int d = threadIdx.x + i * kSortThreads;
+    hist[d * nblk + blockIdx.x] = h[d];
+  }
 }
 
-// Exclusive scan of the M digit-major counts, in place, by one block: each thread
-// scans a contiguous run (loaded 8 at a time), then the runs' totals are scanned
-// across the block.
-__global__ void __launch_bounds__(1024) radix_scan_kernel(int* __restrict__ hist, int64_t M) {
-  __shared__ int warp_tot[32];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t per = (M + 1023) / 1024;
-  const int64_t b = threadIdx.x * per;
-  const int64_t e = b + per < M ? b + per : M;
-  int sum = 0;
-  for (int64_t i0 = b; i0 < e; i0 += 8) {
-    int c[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) c[u] = i0 + u < e ? hist[i0 + u] : 0;
-#pragma unroll
-    for (int u = 0; u < 8; ++u) sum += c[u];
-  }
-  int incl = sum;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  if (lane == 31) warp_tot[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    const int wt = warp_tot[lane];
-    int wi = wt;
+// Per digit, the exclusive scan of its counts over the blocks, in place (one warp per
+// digit, the row read 32 counts at a time), and the digit's total.
+__global__ void __launch_bounds__(256) radix_scan_kernel(int* __restrict__ hist, int64_t nblk,
+                                                        int* __restrict__ totals) {
+  const int lane = threadIdx.x & 31;
+  const int d = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (d >= kDigits) return;
+  int* row = hist + static_cast<int64_t>(d) * nblk;
+  int run = 0;
+  for (int64_t b0 = 0; b0 < nblk; b0 += 32) {
+    const int64_t b = b0 + lane;
+    const int c = b < nblk ? row[b] : 0;
+    int incl = c;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, wi, o);
-      if (lane >= o) wi += y;
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
     }
-    warp_tot[lane] = wi - wt;
+    if (b < nblk) row[b] = run + incl - c;
+    run += __shfl_sync(0xffffffffu, incl, 31);
   }
-  __syncthreads();
-  int run = warp_tot[warp] + incl - sum;
-  for (int64_t i0 = b; i0 < e; i0 += 8) {
-    int c[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) c[u] = i0 + u < e ? hist[i0 + u] : 0;
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      if (i0 + u < e) hist[i0 + u] = run;
-      run += c[u];
-    }
-  }
+  if (lane == 0) totals[d] = run;
 }
 
 // Stable scatter of one tile: a key's new position is its digit's offset for this
@@ -388,15 +369,44 @@ __global__ void __launch_bounds__(1024) radix_scan_kernel(int* __restrict__ hist
 __global__ void __launch_bounds__(kSortThreads) radix_scatter_kernel(
     const int* __restrict__ keys_in, const int* __restrict__ picks_in, int64_t E,
     int64_t slots, int shift, int first, const int* __restrict__ hist, int64_t nblk,
-    int* __restrict__ keys_out, int* __restrict__ picks_out) {
-  __shared__ int cnt[kSortWarps][kDigits];
-  __shared__ int base[kDigits];
+    const int* __restrict__ totals, int* __restrict__ keys_out, int* __restrict__ picks_out) {
+  extern __shared__ int sc_smem[];
+  int (*cnt)[kDigits] = reinterpret_cast<int (*)[kDigits]>(sc_smem);  // [kSortWarps][kDigits]
+  int* base = sc_smem + kSortWarps * kDigits;                         // [kDigits]
+  __shared__ int warp_tot[kSortWarps];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned lower = (1u << lane) - 1u;
-  base[threadIdx.x] = hist[threadIdx.x * nblk + blockIdx.x];
+  {
+    // Digit d starts after every smaller digit's keys (the exclusive scan of the
+    // totals; thread t holds digits [8t, 8t + 8)) and this digit's keys in earlier
+    // blocks.
+    const int d0 = threadIdx.x * kDigitsPerThread;
+    int t[kDigitsPerThread];
+    int sum = 0;
+#pragma unroll
+    for (int i = 0; i < kDigitsPerThread; ++i) {
+      t[i] = totals[d0 + i];
+      sum += t[i];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    int run = incl - sum;
+    for (int w = 0; w < warp; ++w) run += warp_tot[w];
+#pragma unroll
+    for (int i = 0; i < kDigitsPerThread; ++i) {
+      base[d0 + i] = run + hist[static_cast<int64_t>(d0 + i) * nblk + blockIdx.x];
+      run += t[i];
+    }
+  }
   for (int sub = 0; sub < kSortSubTiles; ++sub) {
     for (int d = lane; d < kDigits; d += 32) cnt[warp][d] = 0;
-    __syncwarp();
+    __syncthreads();  // base complete, counters zeroed
     const int64_t p0 = static_cast<int64_t>(blockIdx.x) * kSortTile +
                        static_cast<int64_t>(sub) * kSortSub + warp * kSortPerWarp;
     int key[kSortSteps], pick[kSortSteps], rank[kSortSteps];
@@ -415,10 +425,11 @@ __global__ void __launch_bounds__(kSortThreads) radix_scatter_kernel(
       __syncwarp();
     }
     __syncthreads();
-    {
+#pragma unroll
+    for (int i = 0; i < kDigitsPerThread; ++i) {
       // Digit d's positions for this sub-tile: the block's earlier keys, then the
       // warps in order.
-      const int d = threadIdx.x;
+      const int d = threadIdx.x + i * kSortThreads;
       int run = base[d];
 #pragma unroll
       for (int w = 0; w < kSortWarps; ++w) {
@@ -603,14 +614,19 @@ __global__ void __launch_bounds__(128) segment_small_kernel(
   for (int64_t win = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
        win * 32 < E; win += nwarps) {
     const int64_t w0 = win * 32;
+    // Keys, picks and weights of this window and of the next one, loaded together:
+    // groups that start here and end within the next window need no further loads.
     const int key = w0 + lane < E ? skey[w0 + lane] : end_key;
-    // The window's picks and weights, loaded once: groups inside the window take them
-    // by shuffles, so a group's row reads wait for one round trip, not three.
-    int e_l = 0;
-    float w_l = 0.f;
-    if (w0 + lane < E && key < end_key) {
+    const int key_b = w0 + 32 + lane < E ? skey[w0 + 32 + lane] : end_key;
+    int e_l = 0, e_b = 0;
+    float w_l = 0.f, w_b = 0.f;
+    if (key < end_key) {
       e_l = spick[w0 + lane];
       w_l = weights[e_l];
+    }
+    if (key_b < end_key) {
+      e_b = spick[w0 + 32 + lane];
+      w_b = weights[e_b];
     }
     int prev = __shfl_up_sync(0xffffffffu, key, 1);
     if (lane == 0) prev = w0 > 0 ? skey[w0 - 1] : -1;
@@ -620,8 +636,11 @@ __global__ void __launch_bounds__(128) segment_small_kernel(
       starts &= starts - 1;
       const int r = __shfl_sync(0xffffffffu, key, s);
       const unsigned change = __ballot_sync(0xffffffffu, lane > s && key != r);
+      const unsigned change_b = __ballot_sync(0xffffffffu, key_b != r);
       const int64_t g0 = w0 + s;
-      const int64_t g1 = change ? w0 + __ffs(change) - 1 : group_end(skey, E, w0 + 31, r);
+      const int64_t g1 = change     ? w0 + __ffs(change) - 1
+                         : change_b ? w0 + 32 + __ffs(change_b) - 1
+                                    : group_end(skey, E, w0 + 63, r);
       const int64_t size = g1 - g0;
       if (size <= kSmallGroup) {
         float* grow = grad_values + static_cast<int64_t>(r) * v;
@@ -637,9 +656,14 @@ __global__ void __launch_bounds__(128) segment_small_kernel(
             acc[m][q] = acc[m][q + 1] = acc[m][q + 2] = acc[m][q + 3] = 0.f;
           }
         }
-        const int in_end = static_cast<int>((g1 < w0 + 32 ? g1 : w0 + 32) - w0);
-        sum_window_picks<T, MAXV>(e_l, w_l, s, in_end, grad_out, HK, v, acc);
-        if (g1 > w0 + 32) sum_picks<T, MAXV>(spick, w0 + 32, g1, weights, grad_out, HK, v, acc);
+        // In pick order: this window's lanes, the next window's lanes, then the rest.
+        const int in_a = static_cast<int>((g1 < w0 + 32 ? g1 : w0 + 32) - w0);
+        sum_window_picks<T, MAXV>(e_l, w_l, s, in_a, grad_out, HK, v, acc);
+        if (g1 > w0 + 32) {
+          const int in_b = static_cast<int>((g1 < w0 + 64 ? g1 : w0 + 64) - (w0 + 32));
+          sum_window_picks<T, MAXV>(e_b, w_b, 0, in_b, grad_out, HK, v, acc);
+        }
+        if (g1 > w0 + 64) sum_picks<T, MAXV>(spick, w0 + 64, g1, weights, grad_out, HK, v, acc);
 #pragma unroll
         for (int m = 0; m < MAXV; ++m) {
           const int vec = lane + 32 * m;
@@ -781,10 +805,14 @@ cudaError_t launch_counting_sort(const int* keys, int64_t E, int64_t slots, cons
 }
 
 // Stable sort of the picks by slot; returns which ping-pong buffer holds the result.
+constexpr size_t kScatterSmem = sizeof(int) * (kSortWarps + 1) * kDigits;  // 72 KiB
+
 static cudaError_t sort_picks_by_slot(const int* indices, int64_t E, int64_t slots,
                                       const BackwardWs& ws, int* status, cudaStream_t st,
                                       int* which) {
   const int64_t nblk = sort_blocks(E);
+  cudaError_t e = set_max_smem(reinterpret_cast<const void*>(radix_scatter_kernel), kScatterSmem);
+  if (e != cudaSuccess) return e;
   const int passes = sort_passes(slots);
   const int* kin = indices;
   const int* pin = nullptr;
@@ -794,9 +822,10 @@ static cudaError_t sort_picks_by_slot(const int* indices, int64_t E, int64_t slo
     const int first = ps == 0;
     radix_hist_kernel<<<static_cast<unsigned>(nblk), kSortThreads, 0, st>>>(
         kin, E, slots, shift, first, ws.hist, nblk, status);
-    radix_scan_kernel<<<1, 1024, 0, st>>>(ws.hist, kDigits * nblk);
-    radix_scatter_kernel<<<static_cast<unsigned>(nblk), kSortThreads, 0, st>>>(
-        kin, pin, E, slots, shift, first, ws.hist, nblk, ws.keys[cur], ws.picks[cur]);
+    radix_scan_kernel<<<kDigits / 8, 256, 0, st>>>(ws.hist, nblk, ws.ctr + 64);
+    radix_scatter_kernel<<<static_cast<unsigned>(nblk), kSortThreads, kScatterSmem, st>>>(
+        kin, pin, E, slots, shift, first, ws.hist, nblk, ws.ctr + 64, ws.keys[cur],
+        ws.picks[cur]);
     kin = ws.keys[cur];
     pin = ws.picks[cur];
     cur ^= 1;

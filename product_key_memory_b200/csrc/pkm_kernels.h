@@ -48,8 +48,9 @@ struct BackwardWs {
   // Value gradient: stable radix sort of the picks by slot, then work lists.
   int* keys[2];   // [E] slot ids, ping-pong between sort passes
   int* picks[2];  // [E] pick ids (t*H*k + h*k + j), ping-pong
-  int* hist;      // [256][sort blocks] digit counts, then their exclusive scan
-  int* ctr;       // [4] work-list lengths: items, huge groups, scratch rows
+  int* hist;      // [2048][sort blocks] digit counts, then their scan over the blocks
+  int* ctr;       // [4] work-list lengths: items, huge groups, scratch rows; [64, 2112)
+                  // the radix pass's digit totals
   int4* items;    // [max_items] {start, picks, slot, scratch row or -1}
   int4* huge;     // [max_huge] {slot, first scratch row, rows, 0}
   float* scratch; // [max_chunks][v] partial row sums of huge groups
@@ -73,9 +74,9 @@ constexpr int64_t value_bwd_max_items(int64_t E) {
 constexpr int64_t value_bwd_max_huge(int64_t E) { return E / (kValueChunk + 1) + 1; }
 constexpr int64_t value_bwd_max_chunks(int64_t E) { return E / (kValueChunk / 2) + 1; }
 constexpr size_t value_bwd_ws_bytes(int64_t E, int v) {
-  return 256 + 256 + 4 * round256(4 * static_cast<size_t>(E > 0 ? E : 1)) +
-         round256(4 * 256 * static_cast<size_t>(((E > 0 ? E : 1) + kSortTileKeys - 1) /
-                                                kSortTileKeys)) +
+  return 256 + 8448 + 4 * round256(4 * static_cast<size_t>(E > 0 ? E : 1)) +
+         round256(4 * 2048 * static_cast<size_t>(((E > 0 ? E : 1) + kSortTileKeys - 1) /
+                                                 kSortTileKeys)) +
          round256(16 * static_cast<size_t>(value_bwd_max_items(E))) +
          round256(16 * static_cast<size_t>(value_bwd_max_huge(E))) +
          round256(4 * static_cast<size_t>(value_bwd_max_chunks(E)) *
@@ -131,17 +132,26 @@ cudaError_t launch_bn_train_dacc(const float* g_q, const float* acc, const float
 // Small-batch forward (pkm_small.cu): B <= kSmallMaxB tokens, three launches that
 // spread the parameters over every SM. Workspace: q fp32 [B][H*dq] and chunk lists of
 // small_chunk_entries() (score, id) entries.
-constexpr int kSmallMaxB = 128;  // measured crossover with the tensor-core path
+// Measured crossover with the tensor-core path (bench.py small_batch): at 128 tokens the
+// tensor-core kernels are faster on the 1024^2 layer (115 vs 121 us) and on the wide
+// layer (265 vs 292 us), at 96 the small-batch kernels (90 vs 110, 224 vs 264 us).
+constexpr int kSmallMaxB = 112;
 bool small_supported(int64_t B, int d_model, int H, int dq, int n, int k, int v, int dtype);
 size_t small_chunk_entries(int64_t B, int H, int n);
 cudaError_t launch_forward_small(const LayerArgs& a, float* q, float* chunk_s, int* chunk_i,
                                  float* out, int* idx, float* w, float* sc, cudaStream_t st);
 // The same forward as one cooperative launch with grid-wide barriers (one CTA per SM);
-// the barrier counter is the int after a.status, zeroed by the caller.
+// the barrier counter is the int after a.status, zeroed by the caller. `part` holds
+// [B][H][v] floats. Default for batches of kSmallFusedMinB to kSmallFusedMaxB tokens,
+// where it measured faster (37 vs 45 us at 16 tokens on the 1024^2 layer); for one
+// token the three kernels' programmatic overlap wins (27 vs 29 us), and above 32 tokens
+// they spread the token loops over more blocks (67 vs 87 us at 64).
+constexpr int kSmallFusedMinB = 8;
+constexpr int kSmallFusedMaxB = 32;
 bool small_fused_supported(int d_model, int H, int dq, int n, int v, int dtype);
 cudaError_t launch_forward_small_fused(const LayerArgs& a, float* q, float* chunk_s,
-                                       int* chunk_i, float* out, int* idx, float* w, float* sc,
-                                       cudaStream_t st);
+                                       int* chunk_i, float* part, float* out, int* idx, float* w,
+                                       float* sc, cudaStream_t st);
 
 // 16-byte vectors of a v-wide row each lane of a warp holds, rounded up to the kernel
 // instantiations (1, 2, 4 or 8); 0 when a row is wider than 8 vectors per lane.

@@ -10,7 +10,7 @@
 // the inputs and outputs.
 //
 // The scratch is the file-scope array below. Every GPU that loads this library
-// holds it (about 40.7 MiB) until the process exits. Host code only sees a host-side
+// holds it (about 44.2 MiB) until the process exits. Host code only sees a host-side
 // stand-in under that name, so the array's device address is looked up with
 // cudaGetSymbolAddress, once per device, the first time the entry point runs on
 // that device (with that device current).
@@ -27,7 +27,7 @@ constexpr long long kNoAllocMaxSlots = 1LL << 20;  // 1,048,576 slots (n <= 1024
 constexpr long long kNoAllocMaxPicks = 1LL << 21;  // 2,097,152 picks
 constexpr int kNoAllocMaxV = 2048;
 // The workspace of pkm_backward_values at those limits (its sort buffers, work lists
-// and partial rows): about 40.7 MiB.
+// and partial rows): about 44.2 MiB.
 constexpr size_t kNoAllocBytes = pkm::value_bwd_ws_bytes(kNoAllocMaxPicks, kNoAllocMaxV);
 
 __device__ __align__(256) unsigned char g_pkm_noalloc_scratch[kNoAllocBytes];

@@ -485,21 +485,23 @@ __global__ void __launch_bounds__(kSmallWarps * 32) gather_small_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// The same forward as ONE cooperative launch (one CTA per SM), its three phases
-// separated by grid-wide barriers instead of kernel boundaries:
+// The same forward as ONE cooperative launch (one CTA per SM), its phases separated by
+// grid-wide barriers instead of kernel boundaries:
 //   Q  query network: CTA = a group of 16 features for all tokens (W_q rows staged
-//      once); meanwhile the sub-keys of the CTA's first scoring unit stream into
-//      shared memory with asynchronous copies, since they do not depend on q
+//      once); meanwhile the sub-keys of the CTA's first scoring unit are prefetched
+//      into L2, since they do not depend on q
 //   S  scores: CTA = (head-half, 64 sub-keys): scores for every token and each
 //      token's best 32 of the chunk
-//   G  gather: CTA = token: the chunk lists of all heads merged per half (one warp
-//      per half), exact top-k of the pruned candidates and softmax (one warp per
-//      head), then the H*k weighted value rows over 8 warps, added in warp order.
-// A barrier is a counter in the workspace (zeroed by the host before the launch):
-// each CTA adds one and waits, bounded by the pipelines' wait limit, until every CTA
-// has; on a timeout the kernel records it in the status word and returns. The
-// arithmetic is that of the three-kernel path above (fp32 q and dot products, the
-// same selection order and candidate pruning).
+//   G1 gather: CTA = (token, head): the chunk lists merged per half (one warp per
+//      half), exact top-k of the pruned candidates and softmax, the head's k weighted
+//      value rows over 8 warps (all in flight), added in warp order into the head's
+//      row of a workspace array
+//   G2 CTA = token: the heads' rows added in head order into out
+// A barrier is a counter in the workspace (zeroed by the host before the launch): each
+// CTA adds one and waits, bounded by the pipelines' wait limit, until every CTA has; on
+// a timeout the kernel records it in the status word and returns. The arithmetic is
+// that of the three-kernel path above (fp32 q and dot products, the same selection
+// order and candidate pruning; each head's rows in the same order, heads in head order).
 // ---------------------------------------------------------------------------
 struct FusedArgs {
   const void* x;
@@ -515,6 +517,7 @@ struct FusedArgs {
   float* q;        // [B][H*dq] fp32
   float* cs;       // [B][H][2][nchunks][32] chunk lists
   int* ci;
+  float* part;     // [B][H][v] each head's output row
   float* out;
   int* idx;
   float* w;
@@ -522,14 +525,6 @@ struct FusedArgs {
   int* status;
   unsigned* barrier;
 };
-
-__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(tc::smem_addr(dst)), "l"(src)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.wait_all;" ::: "memory");
-}
 
 // Returns false (every thread of the CTA) once the wait limit has passed.
 __device__ bool fused_grid_sync(unsigned* counter, unsigned target, int* status, int* ok_s) {
@@ -569,9 +564,9 @@ __host__ __device__ inline FusedSmem fused_smem(int d, int H, int dq, int n, int
   const int half = dq / 2;
   const int nchunks = (n + kSChunk - 1) / kSChunk;
   const size_t q_bytes = static_cast<size_t>(kQFeat + kQTok) * d * esz;
-  const size_t lists = static_cast<size_t>(2 * H) * nchunks * kMaxK * 8;
-  const size_t merged = static_cast<size_t>(2 * H) * kMaxK * 8;
-  const size_t picks = static_cast<size_t>(H) * kMaxK * 8;
+  const size_t lists = static_cast<size_t>(2) * nchunks * kMaxK * 8;
+  const size_t merged = static_cast<size_t>(2) * kMaxK * 8;
+  const size_t picks = static_cast<size_t>(kMaxK) * 8;
   const size_t red = static_cast<size_t>(kSmallWarps) * v * 4;
   const size_t g_bytes = lists + merged + picks + red;
   FusedSmem m;
@@ -613,21 +608,17 @@ __global__ void __launch_bounds__(kSmallWarps * 32, 1) forward_small_fused_kerne
 
   if (threadIdx.x == 0) npairs_s = build_pairs(k, pairs);
 
-  // Sub-keys of this CTA's first scoring unit: asynchronous copies into region B,
-  // waited for at the start of phase S.
+  // Sub-keys of this CTA's first scoring unit: prefetched into L2 now (one request per
+  // 128-byte line), since they do not depend on q; phase S stages them from there.
   if (static_cast<int>(blockIdx.x) < NS) {
     const int u = blockIdx.x;
     const int hs = u / nchunks, chunk = u - hs * nchunks;
     const int c0 = chunk * kSChunk;
     const int nr = min(kSChunk, n - c0);
-    const uint32_t* src =
-        reinterpret_cast<const uint32_t*>(C + (static_cast<int64_t>(hs) * n + c0) * half);
-    uint32_t* dst = reinterpret_cast<uint32_t*>(rows_s);
-    for (int i = threadIdx.x; i < kSChunk * row_words_c; i += blockDim.x) {
-      const int r = i / row_words_c, c = i - r * row_words_c;
-      if (r < nr) cp_async4(dst + r * ld_words + c, src + i);
-      else dst[r * ld_words + c] = 0u;
-    }
+    const char* src = reinterpret_cast<const char*>(C + (static_cast<int64_t>(hs) * n + c0) * half);
+    const int lines = (nr * half * esz + 127) / 128;
+    for (int i = threadIdx.x; i < lines; i += blockDim.x)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(src + 128 * i));
   }
 
   // ---------------- phase Q
@@ -723,26 +714,34 @@ __global__ void __launch_bounds__(kSmallWarps * 32, 1) forward_small_fused_kerne
     const int hs = u / nchunks, chunk = u - hs * nchunks;
     const int h = hs >> 1, side = hs & 1;
     const int c0 = chunk * kSChunk;
-    if (u == static_cast<int>(blockIdx.x)) {
-      cp_async_wait_all();
-    } else {
-      __syncthreads();
-      stage_rows(reinterpret_cast<const uint32_t*>(C + (static_cast<int64_t>(hs) * n + c0) * half),
-                 reinterpret_cast<uint32_t*>(rows_s), kSChunk, min(kSChunk, n - c0),
-                 row_words_c, ld_words);
-    }
+    __syncthreads();
+    stage_rows(reinterpret_cast<const uint32_t*>(C + (static_cast<int64_t>(hs) * n + c0) * half),
+               reinterpret_cast<uint32_t*>(rows_s), kSChunk, min(kSChunk, n - c0),
+               row_words_c, ld_words);
     __syncthreads();
     float* qw = qs + warp * 2 * half;
     const bool v0 = c0 + lane < n, v1 = c0 + 32 + lane < n;
     const T* r0 = rows_s + lane * ld;
     const T* r1 = rows_s + (lane + 32) * ld;
     for (int tb = warp * 2; tb < B; tb += kSmallWarps * 2) {
-      // This warp's two tokens' query halves (written by other CTAs: read from L2).
-      for (int i = lane; i < 2 * half; i += 32) {
-        const int uu = i / half, e = i - uu * half;
-        const int t = tb + uu;
-        qw[i] = t < B ? __ldcg(a.q + static_cast<int64_t>(t) * F + h * dq + side * half + e)
+      // This warp's two tokens' query halves (written by other CTAs: read from L2), 16
+      // loads in flight per lane before any is stored.
+      for (int i0 = 0; i0 < 2 * half; i0 += 32 * 16) {
+        float qv[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int i = i0 + lane + 32 * u;
+          const int uu = i / half, e = i - uu * half;
+          const int t = tb + uu;
+          qv[u] = (i < 2 * half && t < B)
+                      ? __ldcg(a.q + static_cast<int64_t>(t) * F + h * dq + side * half + e)
                       : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int i = i0 + lane + 32 * u;
+          if (i < 2 * half) qw[i] = qv[u];
+        }
       }
       __syncwarp();
       for (int uu = 0; uu < 2; ++uu) {
@@ -784,26 +783,41 @@ __global__ void __launch_bounds__(kSmallWarps * 32, 1) forward_small_fused_kerne
   }
   if (!fused_grid_sync(a.barrier, 2 * G, a.status, &ok_s)) return;
 
-  // ---------------- phase G
-  const int list_len = 2 * H * nchunks * kMaxK;
-  float* ls = reinterpret_cast<float*>(regA);            // [2H][nchunks][32]
+  // ---------------- phase G1: block = (token, head)
+  const int list_len = 2 * nchunks * kMaxK;              // this head's two halves
+  float* ls = reinterpret_cast<float*>(regA);            // [2][nchunks][32]
   int* li = reinterpret_cast<int*>(ls + list_len);
-  float* ms = reinterpret_cast<float*>(li + list_len);   // [2H][32] merged halves
-  int* mi = reinterpret_cast<int*>(ms + 2 * H * kMaxK);
-  int* prow = mi + 2 * H * kMaxK;                        // [H][k] picked slots
-  float* pw = reinterpret_cast<float*>(prow + H * kMaxK);
-  float* red = pw + H * kMaxK;                           // [8][v]
+  float* ms = reinterpret_cast<float*>(li + list_len);   // [2][32] merged halves
+  int* mi = reinterpret_cast<int*>(ms + 2 * kMaxK);
+  int* prow = mi + 2 * kMaxK;                            // [k] picked slots
+  float* pw = reinterpret_cast<float*>(prow + kMaxK);
+  float* red = pw + kMaxK;                               // [8][v]
   const int nvec = v / VPER;
-  for (int t = blockIdx.x; t < B; t += G) {
+  const T* Vt = static_cast<const T*>(a.values);
+  for (int u = blockIdx.x; u < B * H; u += G) {  // u = token * H + head
     __syncthreads();
-    const int64_t src = static_cast<int64_t>(t) * list_len;
-    for (int i = threadIdx.x; i < list_len; i += blockDim.x) {
-      ls[i] = __ldcg(a.cs + src + i);
-      li[i] = __ldcg(a.ci + src + i);
+    const int64_t src = static_cast<int64_t>(u) * list_len;
+    for (int i0 = 0; i0 < list_len; i0 += blockDim.x * 4) {
+      float sv[4];
+      int iv[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int i = i0 + threadIdx.x + q * blockDim.x;
+        sv[q] = i < list_len ? __ldcg(a.cs + src + i) : 0.f;
+        iv[q] = i < list_len ? __ldcg(a.ci + src + i) : 0;
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int i = i0 + threadIdx.x + q * blockDim.x;
+        if (i < list_len) {
+          ls[i] = sv[q];
+          li[i] = iv[q];
+        }
+      }
     }
     __syncthreads();
-    for (int hs = warp; hs < 2 * H; hs += kSmallWarps) {
-      const int base = hs * nchunks * kMaxK;
+    if (warp < 2) {  // warp `side` merges that half's chunk lists in chunk order
+      const int base = warp * nchunks * kMaxK;
       float bs = ls[base + lane];
       int bi = li[base + lane];
       for (int c = 1; c < nchunks; ++c) {
@@ -815,46 +829,43 @@ __global__ void __launch_bounds__(kSmallWarps * 32, 1) forward_small_fused_kerne
         const int c0i = __shfl_sync(0xffffffffu, ci, 0);
         if (better(c0s, c0i, ks, ki)) warp_merge32(bs, bi, cs, ci);
       }
-      ms[hs * kMaxK + lane] = bs;
-      mi[hs * kMaxK + lane] = bi;
+      ms[warp * kMaxK + lane] = bs;
+      mi[warp * kMaxK + lane] = bi;
     }
     __syncthreads();
-    if (warp < H) {
-      const int h = warp;
+    if (warp == 0) {
       float bs;
       int bi;
-      select_candidates(ms[2 * h * kMaxK + lane], mi[2 * h * kMaxK + lane],
-                        ms[(2 * h + 1) * kMaxK + lane], mi[(2 * h + 1) * kMaxK + lane], pairs,
-                        npairs_s, n, bs, bi);
+      select_candidates(ms[lane], mi[lane], ms[kMaxK + lane], mi[kMaxK + lane], pairs, npairs_s,
+                        n, bs, bi);
       const float mx = __shfl_sync(0xffffffffu, bs, 0);
       const float e = lane < k ? expf(bs - mx) : 0.f;
       const float den = warp_sum(e);
       const float wt = e / den;
       if (lane < k) {
-        const int64_t o = (static_cast<int64_t>(t) * H + h) * k + lane;
+        const int64_t o = static_cast<int64_t>(u) * k + lane;
         a.idx[o] = bi;
         a.w[o] = wt;
         if (a.sc) a.sc[o] = bs;
-        prow[h * k + lane] = bi;
-        pw[h * k + lane] = wt;
+        prow[lane] = bi;
+        pw[lane] = wt;
       }
     }
     __syncthreads();
-    // The H*k weighted rows, rows warp, warp + 8, ... of each warp 4 at a time.
-    const int HK = H * k;
-    const T* Vt = static_cast<const T*>(a.values);
+    // The head's k weighted rows, rows warp, warp + 8, ... all in flight at once.
     float acc[MAXV][VPER];
 #pragma unroll
     for (int m = 0; m < MAXV; ++m)
 #pragma unroll
       for (int e = 0; e < VPER; ++e) acc[m][e] = 0.f;
-    for (int r0 = warp; r0 < HK; r0 += 4 * kSmallWarps) {
-      uint4 raw[4][MAXV];
-      float wr[4];
+    {
+      constexpr int kRows = kMaxK / kSmallWarps;  // 4
+      uint4 raw[kRows][MAXV];
+      float wr[kRows];
 #pragma unroll
-      for (int uu = 0; uu < 4; ++uu) {
-        const int r = r0 + uu * kSmallWarps;
-        bool live = r < HK;
+      for (int uu = 0; uu < kRows; ++uu) {
+        const int r = warp + uu * kSmallWarps;
+        bool live = r < k;
         int row = live ? prow[r] : 0;
         if (live && (row < 0 || row >= n * n)) {  // only reachable with NaN scores
           if (lane == 0) record_status(a.status, kDevBadSlot);
@@ -871,7 +882,7 @@ __global__ void __launch_bounds__(kSmallWarps * 32, 1) forward_small_fused_kerne
         }
       }
 #pragma unroll
-      for (int uu = 0; uu < 4; ++uu)
+      for (int uu = 0; uu < kRows; ++uu)
 #pragma unroll
         for (int m = 0; m < MAXV; ++m) {
           float f[VPER];
@@ -890,11 +901,26 @@ __global__ void __launch_bounds__(kSmallWarps * 32, 1) forward_small_fused_kerne
       }
     }
     __syncthreads();
+    float* prt = a.part + static_cast<int64_t>(u) * v;  // this head's row of the output
     for (int c = threadIdx.x; c < v; c += blockDim.x) {
       float sum = red[c];
 #pragma unroll
       for (int ww = 1; ww < kSmallWarps; ++ww) sum += red[ww * v + c];
-      a.out[static_cast<int64_t>(t) * v + c] = sum;
+      prt[c] = sum;
+    }
+  }
+  if (!fused_grid_sync(a.barrier, 3 * G, a.status, &ok_s)) return;
+
+  // ---------------- phase G2: block = token, the heads' rows added in head order
+  for (int t = blockIdx.x; t < B; t += G) {
+    const float* prt = a.part + static_cast<int64_t>(t) * H * v;
+    for (int c = threadIdx.x * 4; c < v; c += blockDim.x * 4) {
+      float4 sum = __ldcg(reinterpret_cast<const float4*>(prt + c));
+      for (int hh = 1; hh < H; ++hh) {
+        const float4 x = __ldcg(reinterpret_cast<const float4*>(prt + hh * v + c));
+        sum = make_float4(sum.x + x.x, sum.y + x.y, sum.z + x.z, sum.w + x.w);
+      }
+      *reinterpret_cast<float4*>(a.out + static_cast<int64_t>(t) * v + c) = sum;
     }
   }
 }
@@ -960,8 +986,8 @@ static cudaError_t launch_gather_small(const LayerArgs& a, const float* cs, cons
 }
 
 template <typename T, int MAXV>
-static cudaError_t launch_fused_t(const LayerArgs& a, float* q, float* cs, int* ci, float* out,
-                                  int* idx, float* w, float* sc, cudaStream_t st) {
+static cudaError_t launch_fused_t(const LayerArgs& a, float* q, float* cs, int* ci, float* part,
+                                  float* out, int* idx, float* w, float* sc, cudaStream_t st) {
   const FusedSmem m = fused_smem(a.d_model, a.H, a.dq, a.n, a.v, a.dtype == 0 ? 4 : 2);
   const void* kern = reinterpret_cast<const void*>(forward_small_fused_kernel<T, MAXV>);
   cudaError_t e = set_max_smem(kern, m.total);
@@ -970,7 +996,8 @@ static cudaError_t launch_fused_t(const LayerArgs& a, float* q, float* cs, int* 
   fa.x = a.x; fa.W = a.W_q; fa.mean = a.bn_mean; fa.var = a.bn_var; fa.gamma = a.bn_gamma;
   fa.beta = a.bn_beta; fa.subkeys = a.subkeys; fa.values = a.values; fa.eps = a.bn_eps;
   fa.B = static_cast<int>(a.B); fa.d = a.d_model; fa.H = a.H; fa.dq = a.dq; fa.n = a.n;
-  fa.k = a.k; fa.v = a.v; fa.q = q; fa.cs = cs; fa.ci = ci; fa.out = out; fa.idx = idx;
+  fa.k = a.k; fa.v = a.v; fa.q = q; fa.cs = cs; fa.ci = ci; fa.part = part; fa.out = out;
+  fa.idx = idx;
   fa.w = w; fa.sc = sc; fa.status = a.status;
   // The grid barriers' counter: the word after the status word (the caller zeroes both).
   fa.barrier = reinterpret_cast<unsigned*>(a.status + 1);
@@ -993,14 +1020,14 @@ bool small_fused_supported(int d_model, int H, int dq, int n, int v, int dtype) 
 }
 
 cudaError_t launch_forward_small_fused(const LayerArgs& a, float* q, float* chunk_s,
-                                       int* chunk_i, float* out, int* idx, float* w, float* sc,
-                                       cudaStream_t st) {
+                                       int* chunk_i, float* part, float* out, int* idx, float* w,
+                                       float* sc, cudaStream_t st) {
 #define PKM_FUSED(T)                                                                     \
   switch (row_vecs_per_lane(a.v, a.dtype)) {                                             \
-    case 1: return launch_fused_t<T, 1>(a, q, chunk_s, chunk_i, out, idx, w, sc, st);    \
-    case 2: return launch_fused_t<T, 2>(a, q, chunk_s, chunk_i, out, idx, w, sc, st);    \
-    case 4: return launch_fused_t<T, 4>(a, q, chunk_s, chunk_i, out, idx, w, sc, st);    \
-    case 8: return launch_fused_t<T, 8>(a, q, chunk_s, chunk_i, out, idx, w, sc, st);    \
+    case 1: return launch_fused_t<T, 1>(a, q, chunk_s, chunk_i, part, out, idx, w, sc, st);    \
+    case 2: return launch_fused_t<T, 2>(a, q, chunk_s, chunk_i, part, out, idx, w, sc, st);    \
+    case 4: return launch_fused_t<T, 4>(a, q, chunk_s, chunk_i, part, out, idx, w, sc, st);    \
+    case 8: return launch_fused_t<T, 8>(a, q, chunk_s, chunk_i, part, out, idx, w, sc, st);    \
   }                                                                                      \
   return cudaErrorInvalidValue;
   if (a.dtype == 0) {

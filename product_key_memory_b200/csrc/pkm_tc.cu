@@ -53,34 +53,39 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 }
 
 // ===========================================================================
-// Query network: q = BN(x W_q^T) -> bf16 planes [3][B][F]
+// Query network: q = BN(x W_q^T) -> NP bf16 planes [NP][B][F]
 // ===========================================================================
-constexpr int kQStages = 3;
 constexpr uint32_t kQABytes = kRowsPerTile * kKBlock * 2;  // 16 KiB
 constexpr uint32_t kQBBytes = kColsPerMma * kKBlock * 2;   // 32 KiB
 constexpr uint32_t kQStageBytes = kQABytes + kQBBytes;
-constexpr int kQMaxF = 4096;  // BN scale/shift of every feature live in shared memory
-// Output staging: per epilogue warp, its 32 rows x 32 columns of each plane (up to 3;
-// 64-byte rows, 64-byte swizzle), written to HBM by TMA tensor stores.
+constexpr int kQMaxF = 4096;  // features (the planes' row length fits one tensor map box run)
+// Output staging: per epilogue warp, its 32 rows x 32 columns of each plane (64-byte
+// rows, 64-byte swizzle), written to HBM by TMA tensor stores.
 constexpr uint32_t kQStagePlane = 32 * 32 * 2;             // 2 KiB
-constexpr uint32_t kQStageWarp = 3 * kQStagePlane;         // 6 KiB
+// Operand stages: four with two output planes (the forward), three with three.
+__host__ __device__ constexpr int query_stages(int np) { return np == 2 ? 4 : 3; }
 
+template <int NP>
 size_t query_tc_smem_bytes() {
-  return 1024 + kQStages * kQStageBytes + 2 * kQMaxF * sizeof(float) + kEpiWarps * kQStageWarp +
-         256;
+  return 1024 + query_stages(NP) * kQStageBytes + kEpiWarps * NP * kQStagePlane + 256;
 }
 
+// NP = 2: q = BN(acc) as hi, mid (the forward's scoring planes); NP = 3: acc itself
+// (raw_acc) as hi, mid, lo. The BatchNorm scale and shift of a column are formed in the
+// epilogue from the parameters in global memory (L1-resident after the first tiles),
+// so shared memory holds only operand stages and output staging.
+template <int NP>
 __global__ void __launch_bounds__(kTcThreads, 1) query_tc_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
     const __grid_constant__ CUtensorMap tm_out, const float* __restrict__ mean,
     const float* __restrict__ var, const float* __restrict__ gamma,
-    const float* __restrict__ beta, float eps, int B, int d, int F, int raw_acc, int nplanes,
+    const float* __restrict__ beta, float eps, int B, int d, int F, int raw_acc,
     int* status) {
+  constexpr int kQStages = query_stages(NP);
+  constexpr uint32_t kQStageWarp = NP * kQStagePlane;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* stages = align1024(smem_raw);
-  float* scale_s = reinterpret_cast<float*>(stages + kQStages * kQStageBytes);
-  float* shift_s = scale_s + kQMaxF;
-  uint8_t* staging = reinterpret_cast<uint8_t*>(shift_s + kQMaxF);  // [kEpiWarps][6 KiB]
+  uint8_t* staging = stages + kQStages * kQStageBytes;  // [kEpiWarps][NP planes]
   uint64_t* full = reinterpret_cast<uint64_t*>(staging + kEpiWarps * kQStageWarp);
   uint64_t* empty = full + kQStages;
   uint64_t* tfull = empty + kQStages;
@@ -95,11 +100,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) query_tc_kernel(
   const int ntiles = mt * nt;
   const int kiters = d / kKBlock;
 
-  for (int f = threadIdx.x; f < F; f += blockDim.x) {
-    const float sc = raw_acc ? 1.f : gamma[f] / sqrtf(var[f] + eps);
-    scale_s[f] = sc;
-    shift_s[f] = raw_acc ? 0.f : beta[f] - mean[f] * sc;
-  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < kQStages; ++s) {
       mbar_init(&full[s], 1);
@@ -223,12 +223,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) query_tc_kernel(
         const int f0 = nn * kColsPerMma + g * 32;
         uint32_t ph_[16], pm[16], pl[16];
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const float q0 = fmaf(v[i], scale_s[f0 + i], shift_s[f0 + i]);
-          const float q1 = fmaf(v[i + 1], scale_s[f0 + i + 1], shift_s[f0 + i + 1]);
+        for (int i = 0; i < 32; i += 4) {
+          float q[4] = {v[i], v[i + 1], v[i + 2], v[i + 3]};
+          if (!raw_acc) {
+            const float4 gm = __ldg(reinterpret_cast<const float4*>(gamma + f0 + i));
+            const float4 vr = __ldg(reinterpret_cast<const float4*>(var + f0 + i));
+            const float4 mu = __ldg(reinterpret_cast<const float4*>(mean + f0 + i));
+            const float4 bt = __ldg(reinterpret_cast<const float4*>(beta + f0 + i));
+            const float g4[4] = {gm.x, gm.y, gm.z, gm.w}, v4[4] = {vr.x, vr.y, vr.z, vr.w};
+            const float m4[4] = {mu.x, mu.y, mu.z, mu.w}, b4[4] = {bt.x, bt.y, bt.z, bt.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              // rsqrtf: a few ulp from 1/sqrt, far below the 2^-16 |q| of the planes' split.
+              const float sc = g4[u] * rsqrtf(v4[u] + eps);
+              q[u] = fmaf(q[u], sc, b4[u] - m4[u] * sc);
+            }
+          }
           // hi = RN(q), mid = RN(q - hi), lo = RN(q - hi - mid); the forward's two
           // planes are hi and mid.
-          split3_pair(q0, q1, ph_[i / 2], pm[i / 2], pl[i / 2]);
+          split3_pair(q[0], q[1], ph_[i / 2], pm[i / 2], pl[i / 2]);
+          split3_pair(q[2], q[3], ph_[i / 2 + 1], pm[i / 2 + 1], pl[i / 2 + 1]);
         }
         // The previous group's stores must have read the staging tile before it is
         // overwritten.
@@ -241,7 +255,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) query_tc_kernel(
               make_uint4(ph_[4 * c], ph_[4 * c + 1], ph_[4 * c + 2], ph_[4 * c + 3]);
           *reinterpret_cast<uint4*>(my_row + kQStagePlane + pos) =
               make_uint4(pm[4 * c], pm[4 * c + 1], pm[4 * c + 2], pm[4 * c + 3]);
-          if (nplanes == 3)
+          if (NP == 3)
             *reinterpret_cast<uint4*>(my_row + 2 * kQStagePlane + pos) =
                 make_uint4(pl[4 * c], pl[4 * c + 1], pl[4 * c + 2], pl[4 * c + 3]);
         }
@@ -252,8 +266,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) query_tc_kernel(
           // Rows past B in a partly filled box lie outside the tensor map and are not
           // written; a box that starts past B is not issued at all.
 #pragma unroll
-          for (int p = 0; p < 3; ++p)
-            if (p < nplanes) tma_store_3d(&tm_out, stg + p * kQStagePlane, f0, row0, p);
+          for (int p = 0; p < NP; ++p) tma_store_3d(&tm_out, stg + p * kQStagePlane, f0, row0, p);
           bulk_commit();
         }
       }
@@ -287,10 +300,13 @@ constexpr int kList = kMaxK;          // entries per per-half list (the best 32,
 constexpr int kSStep = 8;             // columns read from TMEM per step
 constexpr int kSSteps = kColsPerMma / kSStep;  // steps per chunk
 constexpr int kSNewCap = 48;          // survivors logged between two merges
-constexpr int kSMidMerge = kSNewCap - 2 * kSStep;  // fresh entries that force a merge
-                                                   // inside a chunk (two steps' room left)
 constexpr int kSEndMerge = 8;         // fresh entries worth a merge at a chunk's end
 constexpr int kSLogCap = kList + kSNewCap;
+constexpr int kSMidMerge = kSNewCap - 2 * kSStep;  // fresh entries that force a merge
+                                                   // inside a chunk
+constexpr int kSFull = kSLogCap - 2 * kSStep;      // entries that force one (room for two
+                                                   // more steps left)
+constexpr int kSCompactAt = kSLogCap - 4 * kSStep; // entries above which a merge compacts
 constexpr int kSTrash = kSLogCap;     // slot written (and dropped) past a full log
 constexpr int kSLogRows = kSLogCap + 1;
 static_assert(kSSteps % 2 == 0, "the step loop alternates two load buffers");
@@ -522,9 +538,10 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
         cnt = static_cast<int>((as - s_row) / kSStrideS);
       };
 
-      // Merge every fresh log entry into Ls (32 at a time), raise tau_run and compact
-      // the log to the entries that can still be among the best 32.
-      auto merge = [&]() {
+      // Merge every fresh log entry into Ls (32 at a time) and raise tau_run. Entries
+      // below tau_run can stay in the log: it is compacted to the entries that can
+      // still be among the best 32 only when it is filling up, and after the unit.
+      auto merge = [&](bool last) {
 #pragma unroll 1
         for (int base = kept; __any_sync(0xffffffffu, base < cnt); base += 32) {
           const int fresh = cnt - base;
@@ -549,6 +566,11 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
             }
         }
         tau_run = Ls[31];
+        thr = fmaxf(nextafterf(tau0, -INFINITY), tau_run);
+        if (!__any_sync(0xffffffffu, last || cnt > kSCompactAt)) {
+          kept = cnt;
+          return;
+        }
         // Branch-free in-place compaction to the entries >= tau_run: every entry is
         // written to the current write slot, which only advances for a kept entry (w <= e,
         // so nothing unread is overwritten). That keeps the current best 32 plus any
@@ -591,7 +613,6 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
         }
         cnt = w;
         kept = w;
-        thr = fmaxf(nextafterf(tau0, -INFINITY), tau_run);
       };
 
 #pragma unroll 1
@@ -636,11 +657,12 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
             if (lane == 0) mbar_arrive(&tempty[set]);
           }
           filter(rb, id_base + (st + 1) * kSStep);
-          // Merge when the next two steps could overflow the log, after a chunk when
-          // enough is fresh, and after the unit's last chunk whenever anything is.
+          // Merge when enough is fresh or the next two steps could overflow the log, after
+          // a chunk when enough is fresh, and after the unit's last chunk always.
           const int fresh = cnt - kept;
-          const int limit = !chunk_end ? kSMidMerge : (last_chunk ? 0 : kSEndMerge);
-          if (__any_sync(0xffffffffu, fresh > limit)) merge();
+          const int limit = !chunk_end ? kSMidMerge : kSEndMerge;
+          const bool unit_end = chunk_end && last_chunk;
+          if (__any_sync(0xffffffffu, unit_end || fresh > limit || cnt > kSFull)) merge(unit_end);
         }
       }
       uses += nchunks;
@@ -742,15 +764,26 @@ cudaError_t launch_query_tc(const LayerArgs& a, void* planes, cudaStream_t st) {
   if (!make_map(&tm_x, a.x, 2, xd, xs, xb) || !make_map(&tm_w, a.W_q, 2, wd, xs, wb) ||
       !make_map(&tm_out, planes, 3, od, os, ob, CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
-  const size_t smem = query_tc_smem_bytes();
-  cudaError_t e = set_max_smem(reinterpret_cast<const void*>(query_tc_kernel), smem);
-  if (e != cudaSuccess) return e;
   const int64_t tiles = ((a.B + kRowsPerTile - 1) / kRowsPerTile) * (F / kColsPerMma);
   const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
-  query_tc_kernel<<<grid, kTcThreads, smem, st>>>(tm_x, tm_w, tm_out, a.bn_mean, a.bn_var,
-                                                  a.bn_gamma, a.bn_beta, a.bn_eps,
-                                                  static_cast<int>(a.B), a.d_model, F, a.raw_acc,
-                                                  nplanes, a.status);
+  static_assert(kScorePlanes == 2, "the forward's query kernel writes two planes");
+  if (nplanes == 2) {
+    const size_t smem = query_tc_smem_bytes<2>();
+    cudaError_t e = set_max_smem(reinterpret_cast<const void*>(query_tc_kernel<2>), smem);
+    if (e != cudaSuccess) return e;
+    query_tc_kernel<2><<<grid, kTcThreads, smem, st>>>(tm_x, tm_w, tm_out, a.bn_mean, a.bn_var,
+                                                       a.bn_gamma, a.bn_beta, a.bn_eps,
+                                                       static_cast<int>(a.B), a.d_model, F,
+                                                       a.raw_acc, a.status);
+  } else {
+    const size_t smem = query_tc_smem_bytes<3>();
+    cudaError_t e = set_max_smem(reinterpret_cast<const void*>(query_tc_kernel<3>), smem);
+    if (e != cudaSuccess) return e;
+    query_tc_kernel<3><<<grid, kTcThreads, smem, st>>>(tm_x, tm_w, tm_out, a.bn_mean, a.bn_var,
+                                                       a.bn_gamma, a.bn_beta, a.bn_eps,
+                                                       static_cast<int>(a.B), a.d_model, F,
+                                                       a.raw_acc, a.status);
+  }
   return cudaGetLastError();
 }
 

@@ -1,5 +1,6 @@
-"""GPU parity of the small-batch forward (B <= 128 tokens: pkm_forward picks the
-small-batch kernels by itself) against the fp64 oracle, through the C ABI.
+"""GPU parity of the small-batch forward (B <= 112 tokens: pkm_forward picks the
+small-batch kernels by itself) against the fp64 oracle, through the C ABI, in both
+forms: the single cooperative kernel and the three kernels.
 
 Same bar as tests/test_forward_gpu.py: indices bit-exact except fp64 near-ties
 within 1e-5 relative of the k-th score; weights, kept scores and out within
@@ -41,19 +42,20 @@ def _check(L, w, path=None):
     return g, r
 
 
-# "auto": the three-kernel form; "small_fused": the single cooperative kernel.
-FORMS = ["auto", "small_fused"]
+# The two small-batch forms, each forced: the single cooperative kernel and the three
+# kernels ("auto" picks the first up to 32 tokens and the second above).
+FORMS = ["small_fused", "small_split"]
 
 
 @pytest.mark.parametrize("path", FORMS)
-@pytest.mark.parametrize("B", [1, 7, 64, 96, 128])
+@pytest.mark.parametrize("B", [1, 7, 8, 32, 64, 96, 112])
 def test_c1024_small_batches(B, path):
     w = synth.WORKLOADS["c1024"].with_(B=B)
     _check(synth.make_layer(w), w, path)
 
 
 @pytest.mark.parametrize("path", FORMS)
-@pytest.mark.parametrize("name,B", [("c512", 33), ("wide", 16), ("wide", 128), ("tiny", 5)])
+@pytest.mark.parametrize("name,B", [("c512", 33), ("wide", 16), ("wide", 112), ("tiny", 5)])
 def test_other_shapes(name, B, path):
     w = synth.WORKLOADS[name].with_(B=B)
     _check(synth.make_layer(w), w, path)
@@ -80,7 +82,7 @@ def test_fused_and_three_kernel_forms_agree():
     w = synth.WORKLOADS["c1024"].with_(B=40)
     L = synth.make_layer(w)
     a = _forward(L, w, "small_fused")
-    b = _forward(L, w, "auto")
+    b = _forward(L, w, "small_split")
     np.testing.assert_array_equal(a["indices"], b["indices"])
     np.testing.assert_array_equal(a["weights"], b["weights"])
     np.testing.assert_array_equal(a["scores"], b["scores"])
