@@ -106,7 +106,7 @@ size_t pkm_workspace_size(const pkm_shape* s, int for_backward);
  * workspace: device scratch of at least pkm_workspace_size(s, 0) bytes, 256-byte
  *   aligned; its contents on entry do not matter.
  * Batches of at most 112 tokens (H <= 8) take the small-batch path, which spreads
- * W_q, the sub-keys and the heads over all SMs for latency: from 8 to 32 tokens one
+ * W_q, the sub-keys and the heads over all SMs for latency: from 4 to 32 tokens one
  * cooperative kernel (one block per SM, its query, scoring and gather phases
  * separated by grid-wide barriers whose waits are bounded like the pipelines'),
  * otherwise three kernels that overlap through programmatic dependent launch on
@@ -114,8 +114,8 @@ size_t pkm_workspace_size(const pkm_shape* s, int for_backward);
  * three kernels on `stream` (query network, per-half scores and top-k, candidate
  * top-k + softmax + gather). With PKM_OPT_SUBBATCHES > 1, large batches of
  * tensor-core shapes are processed in up to that many sub-batches; the value gather
- * of one sub-batch then runs on a second stream owned by the library (one per
- * device) while the next sub-batch is scored on `stream`. Event waits order both
+ * of one sub-batch then runs on the library's helper stream (one per device) while
+ * the next sub-batch is scored on `stream`. Event waits order both
  * ways, so all of the call's work is complete when `stream` reaches the point after
  * the call.
  * Returns PKM_OK or a status code above.
@@ -146,6 +146,11 @@ int pkm_forward(const pkm_shape* s, const void* x, const void* W_q, const float*
  * the status word (PKM_ERR_DEVICE).
  * Only B, H, n, k, v and dtype of the shape are read; d_model, dq and bn_eps are
  * ignored.
+ * With grad_scores requested the two results are computed concurrently: the slot
+ * grouping and row sums run on the library's helper stream (one per device, highest
+ * priority) while grad_scores is computed on `stream`; event waits order both ways,
+ * so all of the call's work is complete when `stream` reaches the point after the
+ * call (CUDA-graph capture of `stream` takes the helper stream's work in with it).
  * workspace: at least pkm_workspace_size(s, 1) bytes, 256-byte aligned.
  */
 int pkm_backward_values(const pkm_shape* s, const void* values, const int32_t* indices,
@@ -178,6 +183,9 @@ int pkm_backward_values(const pkm_shape* s, const void* values, const int32_t* i
  * are added atomically. Slot ids outside [0, n*n) are skipped and counted in the
  * status word. 2*B*H*k must stay below 2^31 (PKM_ERR_UNSUPPORTED otherwise: the
  * sub-key grouping sorts two contributions per pick with 32-bit positions).
+ * grad_values, when requested, is computed on the library's helper stream alongside
+ * the rest (as in pkm_backward_values), joined back into `stream` before the call's
+ * end.
  * workspace: at least pkm_workspace_size(s, 3) bytes, 256-byte aligned.
  */
 int pkm_backward(const pkm_shape* s, const void* x, const void* W_q, const float* bn_mean,

@@ -274,7 +274,10 @@ class Tracer {
 };
 
 // ---------------------------------------------------------------------------
-// Second stream per device for the pipelined forward, plus ordering events.
+// Second stream per device (highest priority, so its blocks are scheduled ahead of the
+// caller's when both have work queued) for the parts of a call that are independent
+// of the rest: the value-gradient rows of the backward passes and the gathers of the
+// pipelined forward. Plus ordering events.
 // ---------------------------------------------------------------------------
 constexpr int kMaxDevices = 64;
 std::mutex g_aux_mu;
@@ -289,7 +292,10 @@ int aux_resources(int n, cudaStream_t* aux, cudaEvent_t* evs) {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PKM_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_aux_mu);
   if (!g_aux_stream[dev]) {
-    if (cudaStreamCreateWithFlags(&g_aux_stream[dev], cudaStreamNonBlocking) != cudaSuccess)
+    int least = 0, greatest = 0;
+    if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess ||
+        cudaStreamCreateWithPriority(&g_aux_stream[dev], cudaStreamNonBlocking, greatest) !=
+            cudaSuccess)
       return PKM_ERR_CUDA;
     for (int i = 0; i < 64; ++i) {
       cudaEvent_t e;
@@ -300,6 +306,16 @@ int aux_resources(int n, cudaStream_t* aux, cudaEvent_t* evs) {
   *aux = g_aux_stream[dev];
   std::vector<cudaEvent_t>& pool = g_sync_events[dev];
   for (int i = 0; i < n; ++i) evs[i] = pool[(g_sync_next[dev]++) % pool.size()];
+  return PKM_OK;
+}
+
+// The helper stream with a fork and a join event, for a call that splits in two.
+int side_stream(pkm::SideStream* side) {
+  cudaEvent_t ev[2];
+  const int rc = aux_resources(2, &side->st, ev);
+  if (rc != PKM_OK) return rc;
+  side->fork = ev[0];
+  side->join = ev[1];
   return PKM_OK;
 }
 
@@ -437,13 +453,15 @@ int backward_full_impl(const pkm_shape* s, bool bn_training, const void* x, cons
   pkm::FullBackwardWs w;
   pkm::backward_full_ws_bytes(a, tensor, &w, static_cast<char*>(workspace));
   if (cudaMemsetAsync(workspace, 0, sizeof(int), st) != cudaSuccess) return PKM_ERR_CUDA;
+  pkm::SideStream side;
+  if (grad_values && side_stream(&side) != PKM_OK) return PKM_ERR_CUDA;
   Tracer tr(1);
   tr.begin(3, st);
   int launches = 0;
   const cudaError_t e = pkm::launch_backward_full(a, tensor, bn_training, indices, weights,
                                                   grad_out, grad_x, grad_W_q, grad_bn_gamma,
                                                   grad_bn_beta, grad_subkeys, grad_values,
-                                                  grad_scores, w, st, &launches);
+                                                  grad_scores, w, side, st, &launches);
   tr.end(st);
   tr.finish(e == cudaSuccess, launches);
   return e == cudaSuccess ? PKM_OK : PKM_ERR_CUDA;
@@ -734,18 +752,34 @@ int pkm_backward_values(const pkm_shape* s, const void* values, const int32_t* i
   backward_ws(s, &w, static_cast<char*>(workspace));
   int* status = static_cast<int*>(workspace);
   if (cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess) return PKM_ERR_CUDA;
+  const int64_t slots = static_cast<int64_t>(s->n) * s->n;
+  // The two parts are independent: with both asked for, the value rows (sort + row
+  // sums) run on the helper stream while the kept-score gradients stream the value
+  // rows on the caller's stream.
+  const bool split = grad_scores != nullptr;
+  pkm::SideStream side;
+  if (split && side_stream(&side) != PKM_OK) return PKM_ERR_CUDA;
   // Stages: 0 grad wrt kept scores, 1 slot grouping + row sums into grad_values,
   // 3 the whole call.
   Tracer tr(1);
   tr.begin(3, st);
-  tr.begin(0, st);
-  cudaError_t e = pkm::launch_backward_values(
-      s->B, s->H, s->k, s->v, s->dtype, static_cast<int64_t>(s->n) * s->n, values, indices,
-      weights, grad_out, grad_values, grad_scores, w, status, st, [&] {
-        tr.end(st);
-        tr.begin(1, st);
-      });
-  tr.end(st);
+  cudaError_t e = split ? pkm::side_fork(side, st) : cudaSuccess;
+  const cudaStream_t vs = split ? side.st : st;
+  tr.begin(1, vs);
+  if (e == cudaSuccess)
+    e = pkm::launch_value_rows(s->B, s->H, s->k, s->v, s->dtype, slots, indices, weights,
+                               grad_out, grad_values, w, status, vs);
+  tr.end(vs);
+  if (split) {
+    tr.begin(0, st);
+    if (e == cudaSuccess)
+      e = pkm::launch_grad_scores(s->B, s->H, s->k, s->v, s->dtype, slots, values, indices,
+                                  weights, grad_out, grad_scores, status, st);
+    tr.end(st);
+    // Always join, even after an error.
+    const cudaError_t e2 = pkm::side_join(side, st);
+    if (e == cudaSuccess) e = e2;
+  }
   tr.end(st);
   tr.finish(e == cudaSuccess, pkm::backward_values_launches(static_cast<int64_t>(s->n) * s->n,
                                                            grad_scores != nullptr, true));

@@ -834,22 +834,29 @@ static cudaError_t sort_picks_by_slot(const int* indices, int64_t E, int64_t slo
   return cudaGetLastError();
 }
 
+// B1: gradients of the kept scores (reads the picked value rows and grad_out).
 template <typename T, int MAXV>
-static cudaError_t launch_bwd_t(int64_t B, int H, int k, int v, int64_t slots, const void* values,
-                                const int* indices, const float* weights, const void* grad_out,
-                                float* grad_values, float* grad_scores, const BackwardWs& ws,
-                                int* status, cudaStream_t st,
-                                const std::function<void()>& between_stages) {
+static cudaError_t launch_scores_t(int64_t B, int H, int k, int v, int64_t slots,
+                                   const void* values, const int* indices, const float* weights,
+                                   const void* grad_out, float* grad_scores, int* status,
+                                   cudaStream_t st) {
+  const unsigned grid = static_cast<unsigned>((B + 3) / 4);
+  grad_scores_kernel<T, MAXV><<<grid, 128, 0, st>>>(static_cast<const T*>(values),
+                                                    static_cast<const T*>(grad_out), indices,
+                                                    weights, B, H, k, v, slots, grad_scores,
+                                                    status);
+  return cudaGetLastError();
+}
+
+// B2: stable sort of the picks by slot, then each slot's picks summed into its row of
+// grad_values (needs only the indices, weights and grad_out: independent of B1).
+template <typename T, int MAXV>
+static cudaError_t launch_rows_t(int64_t B, int H, int k, int v, int64_t slots,
+                                 const int* indices, const float* weights, const void* grad_out,
+                                 float* grad_values, const BackwardWs& ws, int* status,
+                                 cudaStream_t st) {
   const int64_t E = B * H * k;
-  const T* V = static_cast<const T*>(values);
   const T* G = static_cast<const T*>(grad_out);
-  if (grad_scores) {
-    const unsigned grid = static_cast<unsigned>((B + 3) / 4);
-    grad_scores_kernel<T, MAXV><<<grid, 128, 0, st>>>(V, G, indices, weights, B, H, k, v, slots,
-                                                      grad_scores, status);
-  }
-  between_stages();
-  if (!grad_values) return cudaGetLastError();
   cudaError_t e = cudaMemsetAsync(ws.ctr, 0, 4 * sizeof(int), st);
   if (e != cudaSuccess) return e;
   int which = 0;
@@ -871,32 +878,42 @@ static cudaError_t launch_bwd_t(int64_t B, int H, int k, int v, int64_t slots, c
   return cudaGetLastError();
 }
 
-cudaError_t launch_backward_values(int64_t B, int H, int k, int v, int dtype, int64_t slots,
-                                   const void* values, const int* indices, const float* weights,
-                                   const void* grad_out, float* grad_values, float* grad_scores,
-                                   const BackwardWs& ws, int* status, cudaStream_t st,
-                                   const std::function<void()>& between_stages) {
-  const int m = row_vecs_per_lane(v, dtype);
-#define PKM_BWD(T, M)                                                                        \
-  return launch_bwd_t<T, M>(B, H, k, v, slots, values, indices, weights, grad_out, grad_values, \
-                            grad_scores, ws, status, st, between_stages)
-  if (dtype == 0) {
-    switch (m) {
-      case 1: PKM_BWD(float, 1);
-      case 2: PKM_BWD(float, 2);
-      case 4: PKM_BWD(float, 4);
-      case 8: PKM_BWD(float, 8);
-    }
-  } else {
-    switch (m) {
-      case 1: PKM_BWD(uint16_t, 1);
-      case 2: PKM_BWD(uint16_t, 2);
-      case 4: PKM_BWD(uint16_t, 4);
-      case 8: PKM_BWD(uint16_t, 8);
-    }
-  }
-#undef PKM_BWD
-  return cudaErrorInvalidValue;
+#define PKM_BWD_DISPATCH(FN, ...)                          \
+  do {                                                     \
+    const int m_ = row_vecs_per_lane(v, dtype);            \
+    if (dtype == 0) {                                      \
+      switch (m_) {                                        \
+        case 1: return FN<float, 1>(__VA_ARGS__);          \
+        case 2: return FN<float, 2>(__VA_ARGS__);          \
+        case 4: return FN<float, 4>(__VA_ARGS__);          \
+        case 8: return FN<float, 8>(__VA_ARGS__);          \
+      }                                                    \
+    } else {                                               \
+      switch (m_) {                                        \
+        case 1: return FN<uint16_t, 1>(__VA_ARGS__);       \
+        case 2: return FN<uint16_t, 2>(__VA_ARGS__);       \
+        case 4: return FN<uint16_t, 4>(__VA_ARGS__);       \
+        case 8: return FN<uint16_t, 8>(__VA_ARGS__);       \
+      }                                                    \
+    }                                                      \
+    return cudaErrorInvalidValue;                          \
+  } while (0)
+
+cudaError_t launch_grad_scores(int64_t B, int H, int k, int v, int dtype, int64_t slots,
+                               const void* values, const int* indices, const float* weights,
+                               const void* grad_out, float* grad_scores, int* status,
+                               cudaStream_t st) {
+  PKM_BWD_DISPATCH(launch_scores_t, B, H, k, v, slots, values, indices, weights, grad_out,
+                   grad_scores, status, st);
 }
+
+cudaError_t launch_value_rows(int64_t B, int H, int k, int v, int dtype, int64_t slots,
+                              const int* indices, const float* weights, const void* grad_out,
+                              float* grad_values, const BackwardWs& ws, int* status,
+                              cudaStream_t st) {
+  PKM_BWD_DISPATCH(launch_rows_t, B, H, k, v, slots, indices, weights, grad_out, grad_values, ws,
+                   status, st);
+}
+#undef PKM_BWD_DISPATCH
 
 }  // namespace pkm

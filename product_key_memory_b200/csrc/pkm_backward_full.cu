@@ -519,7 +519,7 @@ static cudaError_t launch_full_t(const LayerArgs& a, bool tensor_path, bool bn_t
                                  const int* indices,
                                  const float* weights, const void* grad_out, float* grad_x,
                                  float* grad_W, float* grad_gamma, float* grad_beta,
-                                 float* grad_subkeys, float* grad_values, float* grad_scores,
+                                 float* grad_subkeys, float* grad_scores,
                                  const FullBackwardWs& w, cudaStream_t st, int* launches) {
   const int64_t F = static_cast<int64_t>(a.H) * a.dq;
   const int64_t E = a.B * a.H * static_cast<int64_t>(a.k);
@@ -527,11 +527,12 @@ static cudaError_t launch_full_t(const LayerArgs& a, bool tensor_path, bool bn_t
   const int half = a.dq / 2;
   const bool vec = (half % 8) == 0;
   cudaError_t e;
-  // 1. kept-score gradients (into the workspace) and, if asked, the value gradients.
-  e = launch_backward_values(a.B, a.H, a.k, a.v, a.dtype, slots, a.values, indices, weights,
-                             grad_out, grad_values, w.g_s, w.values, a.status, st, [] {});
+  // 1. kept-score gradients (into the workspace); the value gradients are launched by
+  //    the caller.
+  e = launch_grad_scores(a.B, a.H, a.k, a.v, a.dtype, slots, a.values, indices, weights,
+                         grad_out, w.g_s, a.status, st);
   if (e != cudaSuccess) return e;
-  *launches += backward_values_launches(slots, true, grad_values != nullptr);
+  *launches += 1;
   if (grad_scores) {
     e = cudaMemcpyAsync(grad_scores, w.g_s, sizeof(float) * E, cudaMemcpyDeviceToDevice, st);
     if (e != cudaSuccess) return e;
@@ -629,14 +630,37 @@ cudaError_t launch_backward_full(const LayerArgs& a, bool tensor_path, bool bn_t
                                  const float* weights, const void* grad_out, float* grad_x,
                                  float* grad_W, float* grad_gamma, float* grad_beta,
                                  float* grad_subkeys, float* grad_values, float* grad_scores,
-                                 const FullBackwardWs& w, cudaStream_t st, int* launches) {
-  if (a.dtype == 0)
-    return launch_full_t<float>(a, tensor_path, bn_training, indices, weights, grad_out, grad_x, grad_W,
-                                grad_gamma, grad_beta, grad_subkeys, grad_values, grad_scores, w,
-                                st, launches);
-  return launch_full_t<uint16_t>(a, tensor_path, bn_training, indices, weights, grad_out, grad_x, grad_W,
-                                 grad_gamma, grad_beta, grad_subkeys, grad_values, grad_scores, w,
-                                 st, launches);
+                                 const FullBackwardWs& w, const SideStream& side,
+                                 cudaStream_t st, int* launches) {
+  const int64_t slots = static_cast<int64_t>(a.n) * a.n;
+  cudaError_t e = cudaSuccess;
+  const bool split = grad_values && side.st;
+  if (grad_values) {
+    // The value gradients need only the picks and grad_out: on the side stream their
+    // row read-modify-writes (HBM) overlap the GEMMs and the sub-key work below.
+    if (split) e = side_fork(side, st);
+    if (e == cudaSuccess)
+      e = launch_value_rows(a.B, a.H, a.k, a.v, a.dtype, slots, indices, weights, grad_out,
+                            grad_values, w.values, a.status, split ? side.st : st);
+    *launches += backward_values_launches(slots, false, true);
+  }
+  if (e == cudaSuccess) {
+    if (a.dtype == 0)
+      e = launch_full_t<float>(a, tensor_path, bn_training, indices, weights, grad_out, grad_x,
+                               grad_W, grad_gamma, grad_beta, grad_subkeys, grad_scores, w, st,
+                               launches);
+    else
+      e = launch_full_t<uint16_t>(a, tensor_path, bn_training, indices, weights, grad_out,
+                                  grad_x, grad_W, grad_gamma, grad_beta, grad_subkeys,
+                                  grad_scores, w, st, launches);
+  }
+  // Always join, even after an error, so the caller's stream never runs ahead of work
+  // already queued on the side stream.
+  if (split) {
+    const cudaError_t e2 = side_join(side, st);
+    if (e == cudaSuccess) e = e2;
+  }
+  return e;
 }
 
 }  // namespace pkm

@@ -6,7 +6,6 @@
 #include <stddef.h>
 #include <stdint.h>
 
-#include <functional>
 
 namespace pkm {
 
@@ -84,11 +83,34 @@ constexpr size_t value_bwd_ws_bytes(int64_t E, int v) {
 }
 // Kernels one pkm_backward_values call launches.
 int backward_values_launches(int64_t slots, bool grad_scores, bool grad_values);
-cudaError_t launch_backward_values(int64_t B, int H, int k, int v, int dtype, int64_t slots,
-                                   const void* values, const int* indices, const float* weights,
-                                   const void* grad_out, float* grad_values, float* grad_scores,
-                                   const BackwardWs& ws, int* status, cudaStream_t st,
-                                   const std::function<void()>& between_stages);
+// B1: gradients of the kept scores into grad_scores.
+cudaError_t launch_grad_scores(int64_t B, int H, int k, int v, int dtype, int64_t slots,
+                               const void* values, const int* indices, const float* weights,
+                               const void* grad_out, float* grad_scores, int* status,
+                               cudaStream_t st);
+// B2: picks sorted by slot, each slot's weighted grad_out rows added to grad_values.
+// Independent of B1 (reads indices, weights and grad_out only).
+cudaError_t launch_value_rows(int64_t B, int H, int k, int v, int dtype, int64_t slots,
+                              const int* indices, const float* weights, const void* grad_out,
+                              float* grad_values, const BackwardWs& ws, int* status,
+                              cudaStream_t st);
+
+// A second stream for work of a call that is independent of the rest of it: `fork` is
+// recorded on the caller's stream and waited on by the side stream before the side
+// work; `join` is recorded on the side stream after it and waited on by the caller's
+// stream, so the call stays ordered on the caller's stream.
+struct SideStream {
+  cudaStream_t st = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+inline cudaError_t side_fork(const SideStream& s, cudaStream_t st) {
+  cudaError_t e = cudaEventRecord(s.fork, st);
+  return e == cudaSuccess ? cudaStreamWaitEvent(s.st, s.fork, 0) : e;
+}
+inline cudaError_t side_join(const SideStream& s, cudaStream_t st) {
+  cudaError_t e = cudaEventRecord(s.join, s.st);
+  return e == cudaSuccess ? cudaStreamWaitEvent(st, s.join, 0) : e;
+}
 
 cudaError_t launch_counting_sort(const int* keys, int64_t E, int64_t slots, const BackwardWs& ws,
                                  int* status, cudaStream_t st);
@@ -114,7 +136,8 @@ cudaError_t launch_backward_full(const LayerArgs& a, bool tensor_path, bool bn_t
                                  const float* weights, const void* grad_out, float* grad_x,
                                  float* grad_W, float* grad_gamma, float* grad_beta,
                                  float* grad_subkeys, float* grad_values, float* grad_scores,
-                                 const FullBackwardWs& w, cudaStream_t st, int* launches);
+                                 const FullBackwardWs& w, const SideStream& side,
+                                 cudaStream_t st, int* launches);
 
 // BatchNorm in training mode (pkm_bn_train.cu). Batch statistics of acc (three bf16
 // planes, or fp32 when planes is null) in chunks of kStatChunk tokens; part holds
@@ -143,10 +166,10 @@ cudaError_t launch_forward_small(const LayerArgs& a, float* q, float* chunk_s, i
 // The same forward as one cooperative launch with grid-wide barriers (one CTA per SM);
 // the barrier counter is the int after a.status, zeroed by the caller. `part` holds
 // [B][H][v] floats. Default for batches of kSmallFusedMinB to kSmallFusedMaxB tokens,
-// where it measured faster (37 vs 45 us at 16 tokens on the 1024^2 layer); for one
-// token the three kernels' programmatic overlap wins (27 vs 29 us), and above 32 tokens
-// they spread the token loops over more blocks (67 vs 87 us at 64).
-constexpr int kSmallFusedMinB = 8;
+// where it measured faster (31 vs 32 us at 4 tokens, 37 vs 46 at 16, on the 1024^2
+// layer); for one token the three kernels' programmatic overlap wins (27 vs 29 us),
+// and above 32 tokens they spread the token loops over more blocks (67 vs 88 us at 64).
+constexpr int kSmallFusedMinB = 4;
 constexpr int kSmallFusedMaxB = 32;
 bool small_fused_supported(int d_model, int H, int dq, int n, int v, int dtype);
 cudaError_t launch_forward_small_fused(const LayerArgs& a, float* q, float* chunk_s,

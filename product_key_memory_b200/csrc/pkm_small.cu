@@ -816,21 +816,34 @@ __global__ void __launch_bounds__(kSmallWarps * 32, 1) forward_small_fused_kerne
       }
     }
     __syncthreads();
-    if (warp < 2) {  // warp `side` merges that half's chunk lists in chunk order
-      const int base = warp * nchunks * kMaxK;
-      float bs = ls[base + lane];
-      int bi = li[base + lane];
-      for (int c = 1; c < nchunks; ++c) {
-        const float cs = ls[base + c * kMaxK + lane];
-        const int ci = li[base + c * kMaxK + lane];
+    // Each half's chunk lists merged as a tree over the 8 warps (as in
+    // gather_small_kernel): at stride st the list at 2 st i + st is merged into the
+    // list at 2 st i.
+    for (int st = 1; st < nchunks; st <<= 1) {
+      const int per_side = (nchunks + 2 * st - 1) / (2 * st);
+      for (int item = warp; item < 2 * per_side; item += kSmallWarps) {
+        const int side = item / per_side, i = item - side * per_side;
+        const int a0 = 2 * st * i, b0 = a0 + st;
+        if (b0 >= nchunks) continue;  // warp-uniform
+        const int pa = ((side * nchunks + a0) << 5) + lane;
+        const int pb = ((side * nchunks + b0) << 5) + lane;
+        float bs = ls[pa];
+        int bi = li[pa];
+        const float cs = ls[pb];
+        const int ci = li[pb];
         const float ks = __shfl_sync(0xffffffffu, bs, 31);
         const int ki = __shfl_sync(0xffffffffu, bi, 31);
         const float c0s = __shfl_sync(0xffffffffu, cs, 0);
         const int c0i = __shfl_sync(0xffffffffu, ci, 0);
         if (better(c0s, c0i, ks, ki)) warp_merge32(bs, bi, cs, ci);
+        ls[pa] = bs;
+        li[pa] = bi;
       }
-      ms[warp * kMaxK + lane] = bs;
-      mi[warp * kMaxK + lane] = bi;
+      __syncthreads();
+    }
+    if (warp < 2) {
+      ms[warp * kMaxK + lane] = ls[((warp * nchunks) << 5) + lane];
+      mi[warp * kMaxK + lane] = li[((warp * nchunks) << 5) + lane];
     }
     __syncthreads();
     if (warp == 0) {
