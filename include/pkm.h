@@ -106,11 +106,13 @@ size_t pkm_workspace_size(const pkm_shape* s, int for_backward);
  * workspace: device scratch of at least pkm_workspace_size(s, 0) bytes, 256-byte
  *   aligned; its contents on entry do not matter.
  * Batches of at most 112 tokens (H <= 8) take the small-batch path, which spreads
- * W_q, the sub-keys and the heads over all SMs for latency: from 4 to 32 tokens one
+ * W_q, the sub-keys and the heads over all SMs for latency: from 9 to 32 tokens one
  * cooperative kernel (one block per SM, its query, scoring and gather phases
  * separated by grid-wide barriers whose waits are bounded like the pipelines'),
  * otherwise three kernels that overlap through programmatic dependent launch on
- * `stream` (PKM_OPT_PATH can force either form). Larger batches run
+ * `stream` (PKM_OPT_PATH can force either form). Up to 8 tokens the query and
+ * scoring stages give a warp one W_q row or 8 sub-keys for all tokens, its lanes
+ * splitting the dot products (rows of 16-byte multiples). Larger batches run
  * three kernels on `stream` (query network, per-half scores and top-k, candidate
  * top-k + softmax + gather). With PKM_OPT_SUBBATCHES > 1, large batches of
  * tensor-core shapes are processed in up to that many sub-batches; the value gather

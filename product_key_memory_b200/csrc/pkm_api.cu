@@ -101,7 +101,8 @@ struct ForwardWs {
   void* planes;     // tensor path: bf16 q planes [kScorePlanes][sub][H*dq] of a sub-batch
   float* list_s;    // [B][H][2][32] best 32 per half (any order)
   int* list_i;      // [B][H][2][32]
-  float* part;      // small-batch path: [B][H][v] each head's output row
+  float* part;      // small-batch path: [B][H][v] each head's output row, then [B]
+                    // per-token counts (single-kernel form)
 };
 
 // Tokens per pipelined sub-batch of the tensor-core path: PKM_OPT_SUBBATCHES (1..4,
@@ -133,7 +134,9 @@ size_t forward_ws(const pkm_shape* s, ForwardWs* w, char* base) {
   const size_t o_ls = off; off += align256(sizeof(float) * L);
   const size_t o_li = off; off += align256(sizeof(int) * L);
   const size_t o_pt = off;
-  off += align256(path == Path::kSmall ? sizeof(float) * s->B * s->H * s->v : 0);
+  off += align256(path == Path::kSmall
+                      ? sizeof(float) * s->B * s->H * s->v + sizeof(unsigned) * s->B
+                      : 0);
   if (w && base) {
     w->status = reinterpret_cast<int*>(base);
     w->q = reinterpret_cast<float*>(base + o_q);

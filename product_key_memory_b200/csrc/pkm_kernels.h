@@ -165,11 +165,14 @@ cudaError_t launch_forward_small(const LayerArgs& a, float* q, float* chunk_s, i
                                  float* out, int* idx, float* w, float* sc, cudaStream_t st);
 // The same forward as one cooperative launch with grid-wide barriers (one CTA per SM);
 // the barrier counter is the int after a.status, zeroed by the caller. `part` holds
-// [B][H][v] floats. Default for batches of kSmallFusedMinB to kSmallFusedMaxB tokens,
-// where it measured faster (31 vs 32 us at 4 tokens, 37 vs 46 at 16, on the 1024^2
-// layer); for one token the three kernels' programmatic overlap wins (27 vs 29 us),
-// and above 32 tokens they spread the token loops over more blocks (67 vs 88 us at 64).
-constexpr int kSmallFusedMinB = 4;
+// [B][H][v] floats followed by B unsigned per-token counts (zeroed by the kernel).
+// Default for batches of kSmallFusedMinB to kSmallFusedMaxB tokens, where it measured
+// faster (35 vs 45 us at 16 tokens, 49 vs 53 at 32, on the 1024^2 layer). Up to 8
+// tokens both forms run in decode mode (a warp per W_q row / per 8 sub-keys) and the
+// three kernels win (19 vs 23 us for one token, 27 vs 31 for 8: their query grid has
+// more blocks, and programmatic launch overlaps the stages); above 32 tokens the three
+// kernels spread the token loops over more blocks (67 vs 86 us at 64).
+constexpr int kSmallFusedMinB = 9;
 constexpr int kSmallFusedMaxB = 32;
 bool small_fused_supported(int d_model, int H, int dq, int n, int v, int dtype);
 cudaError_t launch_forward_small_fused(const LayerArgs& a, float* q, float* chunk_s,

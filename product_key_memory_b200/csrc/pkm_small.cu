@@ -99,6 +99,180 @@ __device__ __forceinline__ void stage_rows(const uint32_t* __restrict__ src, uin
 }
 
 // ---------------------------------------------------------------------------
+// Decode mode: batches of at most kDecodeB tokens. The kernels below give each warp a
+// token, so with one token a single warp of every block does that block's work. In
+// decode mode a warp instead takes one W_q row (query) or kDecodeKeys sub-keys
+// (scoring) for every token, its lanes splitting the contraction: lane L reads the
+// 16-byte chunks L, L + 32, ... of each row straight from global memory, all in flight
+// together, and accumulates their elements in order with fmaf; the lanes' partial sums
+// are then added by an xor tree over lane masks 16, 8, 4, 2, 1 (every lane ends with
+// the same total). Both small-batch forms use these functions and the same decode_mode
+// test, so their results stay identical.
+// ---------------------------------------------------------------------------
+constexpr int kDecodeB = 8;
+constexpr int kDecodeRowVecs = 8;  // 16-byte chunks per lane of a W_q row: d*esz <= 4 KiB
+constexpr int kDecodeKeyVecs = 2;  // of a sub-key row: (dq/2)*esz <= 1 KiB
+constexpr int kDecodeKeys = kSChunk / kSmallWarps;  // sub-keys per warp (8)
+
+__host__ __device__ inline bool decode_mode(int64_t B, int d, int dq, int esz) {
+  const int rb = d * esz, kb = (dq / 2) * esz;
+  return B >= 1 && B <= kDecodeB && rb % 16 == 0 && kb % 16 == 0 &&
+         rb <= 16 * 32 * kDecodeRowVecs && kb <= 16 * 32 * kDecodeKeyVecs;
+}
+
+__device__ __forceinline__ float xor_tree_sum(float p) {
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) p += __shfl_xor_sync(0xffffffffu, p, m);
+  return p;
+}
+
+// q[t][f] for every token t < B (one warp): W_q row f against each token's x row, then
+// the BatchNorm affine map as in the kernels below.
+template <typename T, int RV>
+__device__ __forceinline__ void decode_query_row(const T* __restrict__ x, const T* __restrict__ W,
+                                                 const float* __restrict__ mean,
+                                                 const float* __restrict__ var,
+                                                 const float* __restrict__ gamma,
+                                                 const float* __restrict__ beta, float eps,
+                                                 int B, int d, int F, int f,
+                                                 float* __restrict__ q) {
+  constexpr int VPER = Vec<T>::kPer;
+  const int lane = threadIdx.x & 31;
+  const int nch = d / VPER;  // 16-byte chunks per row
+  const uint4* wr = reinterpret_cast<const uint4*>(W + static_cast<int64_t>(f) * d);
+  uint4 wv[RV];
+#pragma unroll
+  for (int i = 0; i < RV; ++i) {
+    const int c = lane + 32 * i;
+    wv[i] = c < nch ? __ldg(wr + c) : make_uint4(0, 0, 0, 0);
+  }
+  float sc = 0.f, sh = 0.f;
+  if (lane == 0) {
+    sc = gamma[f] / sqrtf(var[f] + eps);
+    sh = beta[f] - mean[f] * sc;
+  }
+  // Two tokens at a time, so that both x rows' loads are in flight together.
+  for (int t = 0; t < B; t += 2) {
+    const bool two = t + 1 < B;  // warp-uniform
+    const uint4* xr0 = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t) * d);
+    const uint4* xr1 = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(t + 1) * d);
+    uint4 xv0[RV], xv1[RV];
+#pragma unroll
+    for (int i = 0; i < RV; ++i) {
+      const int c = lane + 32 * i;
+      xv0[i] = c < nch ? __ldg(xr0 + c) : make_uint4(0, 0, 0, 0);
+      xv1[i] = (two && c < nch) ? __ldg(xr1 + c) : make_uint4(0, 0, 0, 0);
+    }
+    float p0 = 0.f, p1 = 0.f;
+#pragma unroll
+    for (int i = 0; i < RV; ++i) {
+      if (lane + 32 * i < nch) {
+        float x0[VPER], x1[VPER], wf[VPER];
+        Vec<T>::widen(xv0[i], x0);
+        Vec<T>::widen(xv1[i], x1);
+        Vec<T>::widen(wv[i], wf);
+#pragma unroll
+        for (int e = 0; e < VPER; ++e) {
+          p0 = fmaf(x0[e], wf[e], p0);
+          p1 = fmaf(x1[e], wf[e], p1);
+        }
+      }
+    }
+    p0 = xor_tree_sum(p0);
+    p1 = xor_tree_sum(p1);
+    if (lane == 0) {
+      q[static_cast<int64_t>(t) * F + f] = fmaf(p0, sc, sh);
+      if (two) q[static_cast<int64_t>(t + 1) * F + f] = fmaf(p1, sc, sh);
+    }
+  }
+}
+
+// This warp's kDecodeKeys sub-key rows c0 + kDecodeKeys * warp + r of head-half hs
+// (rows past n read as zeros).
+template <typename T, int KV>
+__device__ __forceinline__ void decode_load_keys(const T* __restrict__ C, int n, int half, int hs,
+                                                 int c0, uint4 (&kv)[kDecodeKeys][KV]) {
+  constexpr int VPER = Vec<T>::kPer;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nch = half / VPER;
+#pragma unroll
+  for (int r = 0; r < kDecodeKeys; ++r) {
+    const int c = c0 + kDecodeKeys * warp + r;
+    const uint4* kr = reinterpret_cast<const uint4*>(C + (static_cast<int64_t>(hs) * n + c) * half);
+#pragma unroll
+    for (int i = 0; i < KV; ++i) {
+      const int ch = lane + 32 * i;
+      kv[r][i] = (c < n && ch < nch) ? __ldg(kr + ch) : make_uint4(0, 0, 0, 0);
+    }
+  }
+}
+
+// Scores of those rows against each token's query half (fp32, from global memory),
+// written to sc[t][kDecodeKeys * warp + r] (kSChunk floats per token).
+template <typename T, int KV>
+__device__ __forceinline__ void decode_score_keys(const float* __restrict__ q, int B, int F,
+                                                  int dq, int hs, const uint4 (&kv)[kDecodeKeys][KV],
+                                                  float* sc) {
+  constexpr int VPER = Vec<T>::kPer;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int half = dq >> 1;
+  const int nch = half / VPER;
+  const int off = (hs >> 1) * dq + (hs & 1) * half;
+  for (int t = 0; t < B; ++t) {
+    const float* qt = q + static_cast<int64_t>(t) * F + off;
+    float qf[KV][VPER];
+#pragma unroll
+    for (int i = 0; i < KV; ++i) {
+      const int ch = lane + 32 * i;
+#pragma unroll
+      for (int e = 0; e < VPER; e += 4) {
+        const float4 v4 = ch < nch ? __ldcg(reinterpret_cast<const float4*>(qt + ch * VPER + e))
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+        qf[i][e] = v4.x;
+        qf[i][e + 1] = v4.y;
+        qf[i][e + 2] = v4.z;
+        qf[i][e + 3] = v4.w;
+      }
+    }
+    float p[kDecodeKeys];
+#pragma unroll
+    for (int r = 0; r < kDecodeKeys; ++r) {
+      p[r] = 0.f;
+#pragma unroll
+      for (int i = 0; i < KV; ++i) {
+        if (lane + 32 * i < nch) {
+          float kf[VPER];
+          Vec<T>::widen(kv[r][i], kf);
+#pragma unroll
+          for (int e = 0; e < VPER; ++e) p[r] = fmaf(qf[i][e], kf[e], p[r]);
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kDecodeKeys; ++r) p[r] = xor_tree_sum(p[r]);
+    if (lane == 0) {
+#pragma unroll
+      for (int r = 0; r < kDecodeKeys; ++r) sc[t * kSChunk + kDecodeKeys * warp + r] = p[r];
+    }
+  }
+}
+
+// Token t's best 32 of the chunk's kSChunk scores (one warp; rows past n excluded), in
+// the order the kernels below write chunk lists.
+__device__ __forceinline__ void decode_chunk_list(const float* sc, int t, int c0, int n,
+                                                  float& s0, int& i0) {
+  const int lane = threadIdx.x & 31;
+  const bool v0 = c0 + lane < n, v1 = c0 + 32 + lane < n;
+  s0 = v0 ? sc[t * kSChunk + lane] : -INFINITY;
+  float s1 = v1 ? sc[t * kSChunk + 32 + lane] : -INFINITY;
+  i0 = v0 ? c0 + lane : kIdPad;
+  int i1 = v1 ? c0 + 32 + lane : kIdPad;
+  warp_sort32(s0, i0);
+  warp_sort32(s1, i1);
+  warp_merge32(s0, i0, s1, i1);
+}
+
+// ---------------------------------------------------------------------------
 // q[t][f] = (sum_c x[t][c] W[f][c]) * scale[f] + shift[f], scale = gamma / sqrt(var + eps),
 // shift = beta - mean * scale (the tensor-core epilogue's form). CTA = 16 features x 8
 // tokens: the 16 rows of W_q and the 8 rows of x staged in shared memory, one warp
@@ -281,6 +455,50 @@ __global__ void __launch_bounds__(kSmallWarps * 32) score_small_kernel(
     warp_sort32(s1, i1);
     warp_merge32(s0, i0, s1, i1);
     const int64_t o = ((((static_cast<int64_t>(t) * H + h) * 2 + side) * nchunks + chunk) << 5) + lane;
+    chunk_s[o] = s0;
+    chunk_i[o] = i0;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Decode mode of the three-kernel form (at most kDecodeB tokens): the two kernels
+// above with a warp per W_q row / per kDecodeKeys sub-keys instead of per token. Kept
+// apart from them so that their register budgets stay small.
+// ---------------------------------------------------------------------------
+template <typename T, int RV>
+__global__ void __launch_bounds__(kSmallWarps * 32) query_decode_kernel(
+    const T* __restrict__ x, const T* __restrict__ W, const float* __restrict__ mean,
+    const float* __restrict__ var, const float* __restrict__ gamma,
+    const float* __restrict__ beta, float eps, int B, int d, int F, float* __restrict__ q) {
+  allow_dependents();
+  const int f = blockIdx.x * kSmallWarps + (threadIdx.x >> 5);
+  if (f < F) decode_query_row<T, RV>(x, W, mean, var, gamma, beta, eps, B, d, F, f, q);
+}
+
+// Grid (chunks, 2H): block = 64 sub-keys of one head-half for every token; warp t then
+// writes token t's chunk list.
+template <typename T, int KV>
+__global__ void __launch_bounds__(kSmallWarps * 32) score_decode_kernel(
+    const float* __restrict__ q, const T* __restrict__ subkeys, int B, int H, int dq, int n,
+    float* __restrict__ chunk_s, int* __restrict__ chunk_i) {
+  __shared__ float scs[kDecodeB * kSChunk];
+  const int chunk = blockIdx.x, hs = blockIdx.y;
+  const int h = hs >> 1, side = hs & 1;
+  const int c0 = chunk * kSChunk;
+  const int nchunks = (n + kSChunk - 1) / kSChunk;
+  allow_dependents();
+  uint4 kv[kDecodeKeys][KV];
+  decode_load_keys<T, KV>(subkeys, n, dq >> 1, hs, c0, kv);
+  wait_prior_grid();  // q comes from the query kernel
+  decode_score_keys<T, KV>(q, B, H * dq, dq, hs, kv, scs);
+  __syncthreads();
+  const int t = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (t < B) {
+    float s0;
+    int i0;
+    decode_chunk_list(scs, t, c0, n, s0, i0);
+    const int64_t o =
+        ((((static_cast<int64_t>(t) * H + h) * 2 + side) * nchunks + chunk) << 5) + lane;
     chunk_s[o] = s0;
     chunk_i[o] = i0;
   }
@@ -492,14 +710,15 @@ __global__ void __launch_bounds__(kSmallWarps * 32) gather_small_kernel(
 //      into L2, since they do not depend on q
 //   S  scores: CTA = (head-half, 64 sub-keys): scores for every token and each
 //      token's best 32 of the chunk
-//   G1 gather: CTA = (token, head): the chunk lists merged per half (one warp per
-//      half), exact top-k of the pruned candidates and softmax, the head's k weighted
-//      value rows over 8 warps (all in flight), added in warp order into the head's
-//      row of a workspace array
-//   G2 CTA = token: the heads' rows added in head order into out
-// A barrier is a counter in the workspace (zeroed by the host before the launch): each
-// CTA adds one and waits, bounded by the pipelines' wait limit, until every CTA has; on
-// a timeout the kernel records it in the status word and returns. The arithmetic is
+//   G  gather: CTA = (token, head): the chunk lists merged per half (a tree over the
+//      8 warps), exact top-k of the pruned candidates and softmax, the head's k
+//      weighted value rows over 8 warps (all in flight), added in warp order into the
+//      head's row of a workspace array; the token's last head to finish (a per-token
+//      count) adds the H rows in head order into out
+// With at most kDecodeB tokens, Q and S run in decode mode (above). A barrier is a
+// counter in the workspace (zeroed by the host before the launch): each CTA adds one
+// and waits, bounded by the pipelines' wait limit, until every CTA has; on a timeout
+// the kernel records it in the status word and returns. The arithmetic is
 // that of the three-kernel path above (fp32 q and dot products, the same selection
 // order and candidate pruning; each head's rows in the same order, heads in head order).
 // ---------------------------------------------------------------------------
@@ -514,10 +733,12 @@ struct FusedArgs {
   const void* values;
   float eps;
   int B, d, H, dq, n, k, v;
+  int decode;      // decode_mode(B, d, dq, esz)
   float* q;        // [B][H*dq] fp32
   float* cs;       // [B][H][2][nchunks][32] chunk lists
   int* ci;
   float* part;     // [B][H][v] each head's output row
+  unsigned* tok_done;  // [B] heads of the token finished (phase G)
   float* out;
   int* idx;
   float* w;
@@ -574,6 +795,8 @@ __host__ __device__ inline FusedSmem fused_smem(int d, int H, int dq, int n, int
   const size_t rows = (static_cast<size_t>(esz) * kSChunk * (half + (esz == 2 ? 2 : 1)) + 15) &
                       ~static_cast<size_t>(15);
   m.b = rows + sizeof(float) * kSmallWarps * 2 * half;
+  const size_t dec = sizeof(float) * kDecodeB * kSChunk;  // decode mode's chunk scores
+  if (m.b < dec) m.b = dec;
   m.total = m.a + m.b + sizeof(int) * kMaxPairs;
   return m;
 }
@@ -584,6 +807,7 @@ __global__ void __launch_bounds__(kSmallWarps * 32, 1) forward_small_fused_kerne
   extern __shared__ __align__(16) unsigned char fs_raw[];
   __shared__ int ok_s;
   __shared__ int npairs_s;
+  __shared__ int last_s;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int B = a.B, d = a.d, H = a.H, dq = a.dq, n = a.n, k = a.k, v = a.v;
   const int F = H * dq, half = dq >> 1;
@@ -607,6 +831,9 @@ __global__ void __launch_bounds__(kSmallWarps * 32, 1) forward_small_fused_kerne
   const int ld_words = ld * esz / 4;
 
   if (threadIdx.x == 0) npairs_s = build_pairs(k, pairs);
+  // Per-token head counts of phase G, zeroed before the first barrier.
+  if (blockIdx.x == 0)
+    for (int t = threadIdx.x; t < B; t += blockDim.x) a.tok_done[t] = 0u;
 
   // Sub-keys of this CTA's first scoring unit: prefetched into L2 now (one request per
   // 128-byte line), since they do not depend on q; phase S stages them from there.
@@ -622,7 +849,12 @@ __global__ void __launch_bounds__(kSmallWarps * 32, 1) forward_small_fused_kerne
   }
 
   // ---------------- phase Q
-  {
+  if (a.decode) {  // warp = W_q row, all tokens
+    for (int f = static_cast<int>(blockIdx.x) * kSmallWarps + warp; f < F;
+         f += static_cast<int>(G) * kSmallWarps)
+      decode_query_row<T, kDecodeRowVecs>(X, W, a.mean, a.var, a.gamma, a.beta, a.eps, B, d,
+                                          F, f, a.q);
+  } else {
     T* ws = reinterpret_cast<T*>(regA);  // [kQFeat][d]
     T* xs = ws + kQFeat * d;             // [kQTok][d]
     const int row_words = d * esz / 4;
@@ -710,6 +942,28 @@ __global__ void __launch_bounds__(kSmallWarps * 32, 1) forward_small_fused_kerne
   if (!fused_grid_sync(a.barrier, G, a.status, &ok_s)) return;
 
   // ---------------- phase S
+  if (a.decode) {  // warp = kDecodeKeys sub-keys, all tokens; warp t selects token t's list
+    float* scs = reinterpret_cast<float*>(regB);  // [kDecodeB][kSChunk]
+    for (int u = blockIdx.x; u < NS; u += G) {
+      const int hs = u / nchunks, chunk = u - hs * nchunks;
+      const int h = hs >> 1, side = hs & 1;
+      const int c0 = chunk * kSChunk;
+      uint4 kv[kDecodeKeys][kDecodeKeyVecs];
+      decode_load_keys<T, kDecodeKeyVecs>(C, n, half, hs, c0, kv);
+      __syncthreads();  // the previous unit's lists have been read from scs
+      decode_score_keys<T, kDecodeKeyVecs>(a.q, B, F, dq, hs, kv, scs);
+      __syncthreads();
+      if (warp < B) {
+        float s0;
+        int i0;
+        decode_chunk_list(scs, warp, c0, n, s0, i0);
+        const int64_t o =
+            ((((static_cast<int64_t>(warp) * H + h) * 2 + side) * nchunks + chunk) << 5) + lane;
+        a.cs[o] = s0;
+        a.ci[o] = i0;
+      }
+    }
+  } else
   for (int u = blockIdx.x; u < NS; u += G) {
     const int hs = u / nchunks, chunk = u - hs * nchunks;
     const int h = hs >> 1, side = hs & 1;
@@ -783,7 +1037,7 @@ __global__ void __launch_bounds__(kSmallWarps * 32, 1) forward_small_fused_kerne
   }
   if (!fused_grid_sync(a.barrier, 2 * G, a.status, &ok_s)) return;
 
-  // ---------------- phase G1: block = (token, head)
+  // ---------------- phase G: block = (token, head)
   const int list_len = 2 * nchunks * kMaxK;              // this head's two halves
   float* ls = reinterpret_cast<float*>(regA);            // [2][nchunks][32]
   int* li = reinterpret_cast<int*>(ls + list_len);
@@ -921,19 +1175,24 @@ __global__ void __launch_bounds__(kSmallWarps * 32, 1) forward_small_fused_kerne
       for (int ww = 1; ww < kSmallWarps; ++ww) sum += red[ww * v + c];
       prt[c] = sum;
     }
-  }
-  if (!fused_grid_sync(a.barrier, 3 * G, a.status, &ok_s)) return;
-
-  // ---------------- phase G2: block = token, the heads' rows added in head order
-  for (int t = blockIdx.x; t < B; t += G) {
-    const float* prt = a.part + static_cast<int64_t>(t) * H * v;
-    for (int c = threadIdx.x * 4; c < v; c += blockDim.x * 4) {
-      float4 sum = __ldcg(reinterpret_cast<const float4*>(prt + c));
-      for (int hh = 1; hh < H; ++hh) {
-        const float4 x = __ldcg(reinterpret_cast<const float4*>(prt + hh * v + c));
-        sum = make_float4(sum.x + x.x, sum.y + x.y, sum.z + x.z, sum.w + x.w);
+    // The token's last head to finish adds its H rows in head order into out (each
+    // writer fences its row before the count, the last one fences before reading).
+    const int t = u / H;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) last_s = atomicAdd(a.tok_done + t, 1u) == static_cast<unsigned>(H - 1);
+    __syncthreads();
+    if (last_s) {
+      __threadfence();
+      const float* rows_t = a.part + static_cast<int64_t>(t) * H * v;
+      for (int c = threadIdx.x * 4; c < v; c += blockDim.x * 4) {
+        float4 sum = __ldcg(reinterpret_cast<const float4*>(rows_t + c));
+        for (int hh = 1; hh < H; ++hh) {
+          const float4 x = __ldcg(reinterpret_cast<const float4*>(rows_t + hh * v + c));
+          sum = make_float4(sum.x + x.x, sum.y + x.y, sum.z + x.z, sum.w + x.w);
+        }
+        *reinterpret_cast<float4*>(a.out + static_cast<int64_t>(t) * v + c) = sum;
       }
-      *reinterpret_cast<float4*>(a.out + static_cast<int64_t>(t) * v + c) = sum;
     }
   }
 }
@@ -1010,6 +1269,8 @@ static cudaError_t launch_fused_t(const LayerArgs& a, float* q, float* cs, int* 
   fa.beta = a.bn_beta; fa.subkeys = a.subkeys; fa.values = a.values; fa.eps = a.bn_eps;
   fa.B = static_cast<int>(a.B); fa.d = a.d_model; fa.H = a.H; fa.dq = a.dq; fa.n = a.n;
   fa.k = a.k; fa.v = a.v; fa.q = q; fa.cs = cs; fa.ci = ci; fa.part = part; fa.out = out;
+  fa.tok_done = reinterpret_cast<unsigned*>(part + a.B * a.H * a.v);
+  fa.decode = decode_mode(a.B, a.d_model, a.dq, a.dtype == 0 ? 4 : 2) ? 1 : 0;
   fa.idx = idx;
   fa.w = w; fa.sc = sc; fa.status = a.status;
   // The grid barriers' counter: the word after the status word (the caller zeroes both).
@@ -1058,25 +1319,52 @@ static cudaError_t launch_small_t(const LayerArgs& a, float* q, float* cs, int* 
   size_t smem = query_small_smem(a.d_model, a.dtype);
   cudaError_t e = set_max_smem(reinterpret_cast<const void*>(query_small_kernel<T>), smem);
   if (e != cudaSuccess) return e;
-  dim3 gq((F + kQFeat - 1) / kQFeat, (B + kQTok - 1) / kQTok);
-  query_small_kernel<T><<<gq, kSmallWarps * 32, smem, st>>>(
-      static_cast<const T*>(a.x), static_cast<const T*>(a.W_q), a.bn_mean, a.bn_var, a.bn_gamma,
-      a.bn_beta, a.bn_eps, B, a.d_model, F, q);
-  smem = score_small_smem(a.dq, a.dtype);
-  e = set_max_smem(reinterpret_cast<const void*>(score_small_kernel<T>), smem);
-  if (e != cudaSuccess) return e;
+  const bool decode = decode_mode(B, a.d_model, a.dq, a.dtype == 0 ? 4 : 2);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((a.n + kSChunk - 1) / kSChunk, a.H * 2, (B + kSTok - 1) / kSTok);
   cfg.blockDim = dim3(kSmallWarps * 32, 1, 1);
-  cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, score_small_kernel<T>, static_cast<const float*>(q),
-                         static_cast<const T*>(a.subkeys), B, a.H, a.dq, a.n, cs, ci);
+  if (decode) {
+    // 16-byte chunks per lane of a W_q row and of a sub-key row.
+    const int esz = a.dtype == 0 ? 4 : 2;
+    const int rv = (a.d_model * esz / 16 + 31) / 32, kv = ((a.dq / 2) * esz / 16 + 31) / 32;
+    const unsigned gq = static_cast<unsigned>((F + kSmallWarps - 1) / kSmallWarps);
+    const T* xp = static_cast<const T*>(a.x);
+    const T* wp = static_cast<const T*>(a.W_q);
+#define PKM_QDEC(RV)                                                                     \
+  query_decode_kernel<T, RV><<<gq, kSmallWarps * 32, 0, st>>>(xp, wp, a.bn_mean, a.bn_var, \
+                                                             a.bn_gamma, a.bn_beta, a.bn_eps, \
+                                                             B, a.d_model, F, q)
+    if (rv <= 1) PKM_QDEC(1);
+    else if (rv <= 2) PKM_QDEC(2);
+    else if (rv <= 4) PKM_QDEC(4);
+    else PKM_QDEC(8);
+#undef PKM_QDEC
+    cfg.gridDim = dim3((a.n + kSChunk - 1) / kSChunk, a.H * 2, 1);
+    cfg.dynamicSmemBytes = 0;
+    const float* qc = q;
+    const T* kp = static_cast<const T*>(a.subkeys);
+    e = kv <= 1 ? cudaLaunchKernelEx(&cfg, score_decode_kernel<T, 1>, qc, kp, B, a.H, a.dq, a.n,
+                                     cs, ci)
+                : cudaLaunchKernelEx(&cfg, score_decode_kernel<T, 2>, qc, kp, B, a.H, a.dq, a.n,
+                                     cs, ci);
+  } else {
+    dim3 gq((F + kQFeat - 1) / kQFeat, (B + kQTok - 1) / kQTok);
+    query_small_kernel<T><<<gq, kSmallWarps * 32, smem, st>>>(
+        static_cast<const T*>(a.x), static_cast<const T*>(a.W_q), a.bn_mean, a.bn_var,
+        a.bn_gamma, a.bn_beta, a.bn_eps, B, a.d_model, F, q);
+    smem = score_small_smem(a.dq, a.dtype);
+    e = set_max_smem(reinterpret_cast<const void*>(score_small_kernel<T>), smem);
+    if (e != cudaSuccess) return e;
+    cfg.gridDim = dim3((a.n + kSChunk - 1) / kSChunk, a.H * 2, (B + kSTok - 1) / kSTok);
+    cfg.dynamicSmemBytes = smem;
+    e = cudaLaunchKernelEx(&cfg, score_small_kernel<T>, static_cast<const float*>(q),
+                           static_cast<const T*>(a.subkeys), B, a.H, a.dq, a.n, cs, ci);
+  }
   if (e != cudaSuccess) return e;
   switch (row_vecs_per_lane(a.v, a.dtype)) {
     case 1: return launch_gather_small<T, 1>(a, cs, ci, out, idx, w, sc, st);

@@ -55,16 +55,21 @@ def test_c1024_small_batches(B, path):
 
 
 @pytest.mark.parametrize("path", FORMS)
-@pytest.mark.parametrize("name,B", [("c512", 33), ("wide", 16), ("wide", 112), ("tiny", 5)])
+@pytest.mark.parametrize("name,B", [("c512", 33), ("wide", 4), ("wide", 16), ("wide", 112),
+                                    ("tiny", 5)])
 def test_other_shapes(name, B, path):
     w = synth.WORKLOADS[name].with_(B=B)
     _check(synth.make_layer(w), w, path)
 
 
 @pytest.mark.parametrize("path", FORMS)
-@pytest.mark.parametrize("k,n", [(1, 256), (3, 256), (8, 8), (32, 32)])
-def test_k_and_small_codebooks(k, n, path):
-    w = synth.WORKLOADS["c512"].with_(B=9, n=n, k=k)
+@pytest.mark.parametrize("B", [3, 9])
+@pytest.mark.parametrize("k,n", [(1, 256), (3, 256), (8, 8), (32, 32), (32, 100)])
+def test_k_and_small_codebooks(k, n, B, path):
+    """3 tokens take the decode mode (a warp per W_q row or per 8 sub-keys, lanes over
+    the contraction), 9 tokens the token-per-warp kernels; n = 8, 32, 100 leave the
+    last 64-sub-key chunk ragged."""
+    w = synth.WORKLOADS["c512"].with_(B=B, n=n, k=k)
     _check(synth.make_layer(w), w, path)
 
 
@@ -76,10 +81,12 @@ def test_odd_half_query_goes_to_large_batch_kernels():
     _check(synth.make_layer(w), w)
 
 
-def test_fused_and_three_kernel_forms_agree():
-    """Same arithmetic in both forms: picks, weights and scores bit for bit; out up to
-    the order in which the H*k rows are added."""
-    w = synth.WORKLOADS["c1024"].with_(B=40)
+@pytest.mark.parametrize("B", [3, 40])
+def test_fused_and_three_kernel_forms_agree(B):
+    """Same arithmetic in both forms (3 tokens: decode mode; 40: token per warp): picks,
+    weights and scores bit for bit; out up to the order in which the H*k rows are
+    added."""
+    w = synth.WORKLOADS["c1024"].with_(B=B)
     L = synth.make_layer(w)
     a = _forward(L, w, "small_fused")
     b = _forward(L, w, "small_split")
@@ -90,8 +97,9 @@ def test_fused_and_three_kernel_forms_agree():
 
 
 @pytest.mark.parametrize("path", FORMS)
-def test_exact_ties_go_to_lower_slot(path):
-    w = synth.WORKLOADS["c512"].with_(B=12, n=256)
+@pytest.mark.parametrize("B", [2, 12])
+def test_exact_ties_go_to_lower_slot(path, B):
+    w = synth.WORKLOADS["c512"].with_(B=B, n=256)
     L = synth.make_layer(w)
     L["subkeys"][:, 0] = L["subkeys"][:, 0, :1]
     g = _forward(L, w, path)
