@@ -54,9 +54,9 @@ FLUSH_BYTES = 256 << 20
 # keyed by (kernel_sha(), workload, tokens); reported as null once the kernel's source
 # has changed since the capture.
 TRAFFIC = {
-    # c1024 at 4096 tokens: dram read 960.7 MB + write 4.7 MB, scaled x4 to the
+    # c1024 at 4096 tokens: dram read 956.5 MB + write 7.8 MB, scaled x4 to the
     # 16384-token launch (the gather's traffic grows with the tokens).
-    ("b442ea1a5c72b593", "c1024", 16384): 3.862e9,
+    ("ab6394527d8d2580", "c1024", 16384): 3.857e9,
 }
 
 
