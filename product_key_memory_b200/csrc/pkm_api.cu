@@ -183,10 +183,11 @@ constexpr int kPasses = 2;
 
 struct TraceSpan {
   int stage;
-  cudaEvent_t start, stop;
+  int start, stop;  // indices into TraceCall::events
 };
 struct TraceCall {
   int pass;
+  std::vector<cudaEvent_t> events;  // each recorded once; spans may share them
   std::vector<TraceSpan> spans;
 };
 
@@ -230,30 +231,19 @@ class Tracer {
   }
   // Spans nest: end() closes the most recently begun span that is still open. Every
   // span is also an NVTX range (host side; profilers attach the launches inside it).
-  void begin(int stage, cudaStream_t st) {
-    nvtxRangePushA(stage_name(call_.pass, stage));
-    ++nvtx_open_;
-    if (!on_) return;
-    std::lock_guard<std::mutex> lk(g_trace_mu);
-    TraceSpan sp{stage, take_timing_event(), take_timing_event()};
-    if (!sp.start || !sp.stop) {
-      if (sp.start) g_event_pool.push_back(sp.start);
-      if (sp.stop) g_event_pool.push_back(sp.stop);
-      on_ = false;
-      return;
-    }
-    cudaEventRecord(sp.start, st);
-    open_.push_back(call_.spans.size());
-    call_.spans.push_back(sp);
-  }
-  void end(cudaStream_t st) {
-    if (nvtx_open_ > 0) {
-      nvtxRangePop();
-      --nvtx_open_;
-    }
-    if (!on_ || open_.empty()) return;
-    cudaEventRecord(call_.spans[open_.back()].stop, st);
-    open_.pop_back();
+  void begin(int stage, cudaStream_t st) { open_span(stage, record(st)); }
+  void end(cudaStream_t st) { close_span(record(st)); }
+  // The same at the point of the stream where the previous begin / end / next recorded
+  // its event (one event for both): only where nothing has been issued to `st` since.
+  // Each timing event recorded between two kernels delays the second one, so a call
+  // records one event per stage boundary.
+  void begin_here(int stage, cudaStream_t st) { open_span(stage, reuse(st)); }
+  void end_here(cudaStream_t st) { close_span(reuse(st)); }
+  // End the innermost open span and begin `stage` at one event (nothing in between).
+  void next(int stage, cudaStream_t st) {
+    const int ev = record(st);
+    close_span(ev);
+    open_span(stage, ev);
   }
   void finish(bool ok, int launches) {
     std::lock_guard<std::mutex> lk(g_trace_mu);
@@ -262,18 +252,53 @@ class Tracer {
     if (ok && open_.empty()) {
       g_trace_pending.push_back(call_);
     } else {
-      for (const TraceSpan& sp : call_.spans) {
-        g_event_pool.push_back(sp.start);
-        g_event_pool.push_back(sp.stop);
-      }
+      for (cudaEvent_t e : call_.events) g_event_pool.push_back(e);
     }
   }
 
  private:
+  // Index of a newly recorded event (-1 when tracing is off or out of events).
+  int record(cudaStream_t st) {
+    if (!on_) return -1;
+    cudaEvent_t e;
+    {
+      std::lock_guard<std::mutex> lk(g_trace_mu);
+      e = take_timing_event();
+    }
+    if (!e) {
+      on_ = false;
+      return -1;
+    }
+    cudaEventRecord(e, st);
+    call_.events.push_back(e);
+    last_ = static_cast<int>(call_.events.size()) - 1;
+    last_st_ = st;
+    return last_;
+  }
+  int reuse(cudaStream_t st) { return (on_ && last_ >= 0 && last_st_ == st) ? last_ : record(st); }
+  void open_span(int stage, int ev) {
+    nvtxRangePushA(stage_name(call_.pass, stage));
+    ++nvtx_open_;
+    if (!on_ || ev < 0) return;
+    open_.push_back(call_.spans.size());
+    call_.spans.push_back(TraceSpan{stage, ev, -1});
+  }
+  void close_span(int ev) {
+    if (nvtx_open_ > 0) {
+      nvtxRangePop();
+      --nvtx_open_;
+    }
+    if (!on_ || open_.empty() || ev < 0) return;
+    call_.spans[open_.back()].stop = ev;
+    open_.pop_back();
+  }
+
   bool on_ = false;
   int nvtx_open_ = 0;
   TraceCall call_;
   std::vector<size_t> open_;
+  int last_ = -1;
+  cudaStream_t last_st_ = nullptr;
 };
 
 // ---------------------------------------------------------------------------
@@ -371,13 +396,13 @@ int pkm_trace_read(int pass, double* stage_ms, int max_stages, int64_t* calls,
       continue;
     }
     for (const TraceSpan& sp : c.spans) {
-      if (cudaEventSynchronize(sp.stop) != cudaSuccess) rc = PKM_ERR_CUDA;
+      const cudaEvent_t a = c.events[sp.start], b = c.events[sp.stop];
+      if (cudaEventSynchronize(b) != cudaSuccess) rc = PKM_ERR_CUDA;
       float ms = 0.f;
-      if (cudaEventElapsedTime(&ms, sp.start, sp.stop) != cudaSuccess) rc = PKM_ERR_CUDA;
+      if (cudaEventElapsedTime(&ms, a, b) != cudaSuccess) rc = PKM_ERR_CUDA;
       if (sp.stage < max_stages) stage_ms[sp.stage] += ms;
-      g_event_pool.push_back(sp.start);
-      g_event_pool.push_back(sp.stop);
     }
+    for (cudaEvent_t e : c.events) g_event_pool.push_back(e);
     ++n;
   }
   g_trace_pending.swap(keep);
@@ -559,7 +584,7 @@ cudaError_t run_forward(const pkm_shape* s, const LayerArgs& a, const ForwardWs&
   int launches = 0;
   const Path path = choose_path(s);
   if (path == Path::kSmall) {
-    tr.begin(2, st);
+    tr.begin_here(2, st);
     const int pin = g_opt_path.load(std::memory_order_relaxed);
     if (pin != PKM_PATH_SMALL_SPLIT &&
         (pin == PKM_PATH_SMALL_FUSED ||
@@ -575,26 +600,22 @@ cudaError_t run_forward(const pkm_shape* s, const LayerArgs& a, const ForwardWs&
     }
     tr.end(st);
   } else if (path == Path::kSimt) {
-    tr.begin(0, st);
+    tr.begin_here(0, st);
     e = pkm::launch_query_bn_simt(a, w.q, st);
-    tr.end(st);
-    tr.begin(1, st);
+    tr.next(1, st);
     if (e == cudaSuccess) e = pkm::launch_subkey_topk_simt(a, w.q, w.list_s, w.list_i, st);
-    tr.end(st);
-    tr.begin(2, st);
+    tr.next(2, st);
     if (e == cudaSuccess)
       e = pkm::launch_select_gather(a, w.list_s, w.list_i, out, indices, weights, scores, st);
     tr.end(st);
     launches = 3;
   } else if (sub_batch_tokens(s->B) >= s->B) {
     // One batch: the three launches in order on the caller's stream.
-    tr.begin(0, st);
+    tr.begin_here(0, st);
     e = pkm::launch_query_tc(a, w.planes, st);
-    tr.end(st);
-    tr.begin(1, st);
+    tr.next(1, st);
     if (e == cudaSuccess) e = pkm::launch_score_topk_tc(a, w.planes, w.list_s, w.list_i, st);
-    tr.end(st);
-    tr.begin(2, st);
+    tr.next(2, st);
     if (e == cudaSuccess)
       e = pkm::launch_select_gather(a, w.list_s, w.list_i, out, indices, weights, scores, st);
     tr.end(st);
@@ -621,10 +642,9 @@ cudaError_t run_forward(const pkm_shape* s, const LayerArgs& a, const ForwardWs&
       ai.x = static_cast<const char*>(x) + t0 * s->d_model * xsz;
       float* ls = w.list_s + t0 * per_tok;
       int* li = w.list_i + t0 * per_tok;
-      tr.begin(0, st);
+      tr.begin_here(0, st);
       e = pkm::launch_query_tc(ai, w.planes, st);
-      tr.end(st);
-      tr.begin(1, st);
+      tr.next(1, st);
       if (e == cudaSuccess) e = pkm::launch_score_topk_tc(ai, w.planes, ls, li, st);
       tr.end(st);
       if (e == cudaSuccess) e = cudaEventRecord(ev[i], st);
@@ -676,7 +696,7 @@ int pkm_forward(const pkm_shape* s, const void* x, const void* W_q, const float*
   int launches = 0;
   tr.begin(3, st);
   const cudaError_t e = run_forward(s, a, w, out, indices, weights, scores, st, tr, &launches);
-  tr.end(st);
+  tr.end_here(st);  // the last stage's end, or a new event after the pipelined join
   tr.finish(e == cudaSuccess, launches);
   return e == cudaSuccess ? PKM_OK : PKM_ERR_CUDA;
 }
@@ -717,7 +737,7 @@ int pkm_forward_train(const pkm_shape* s, const void* x, const void* W_q,
   Tracer tr(0);
   int launches = 0;
   tr.begin(3, st);
-  tr.begin(0, st);
+  tr.begin_here(0, st);
   const bool tensor = choose_path(s) == Path::kTensor;
   cudaError_t e = tensor ? pkm::launch_query_tc(raw, tw.acc, st)
                          : pkm::launch_query_bn_simt(raw, static_cast<float*>(tw.acc), st);
@@ -729,7 +749,7 @@ int pkm_forward_train(const pkm_shape* s, const void* x, const void* W_q,
   tr.end(st);
   launches += 3;
   if (e == cudaSuccess) e = run_forward(s, a, w, out, indices, weights, scores, st, tr, &launches);
-  tr.end(st);
+  tr.end_here(st);
   tr.finish(e == cudaSuccess, launches);
   return e == cudaSuccess ? PKM_OK : PKM_ERR_CUDA;
 }
@@ -768,7 +788,7 @@ int pkm_backward_values(const pkm_shape* s, const void* values, const int32_t* i
   tr.begin(3, st);
   cudaError_t e = split ? pkm::side_fork(side, st) : cudaSuccess;
   const cudaStream_t vs = split ? side.st : st;
-  tr.begin(1, vs);
+  tr.begin_here(1, vs);  // shares the call's first event unless on the helper stream
   if (e == cudaSuccess)
     e = pkm::launch_value_rows(s->B, s->H, s->k, s->v, s->dtype, slots, indices, weights,
                                grad_out, grad_values, w, status, vs);
