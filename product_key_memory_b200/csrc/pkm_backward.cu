@@ -8,7 +8,8 @@
 //   grad wrt V[slot]:       sum over the picks of that slot of w * grad_out[t]
 //
 // The value gradient is deterministic and uses no atomics on rows:
-//   1. a stable LSD radix sort (8 bits per pass) groups the B*H*k picks by slot
+//   1. a stable LSD radix sort (11-bit digits, two passes up to 2^22 slots) groups
+//      the B*H*k picks by slot
 //      and keeps each slot's picks in pick order;
 //   2. one warp per window of 32 sorted picks takes every group that starts in its
 //      window: a group of at most kSmallGroup picks is summed in pick order in
@@ -170,7 +171,7 @@ __global__ void __launch_bounds__(128) grad_scores_kernel(
   }
 }
 
-// --------------------------------------------------------------- counting sort
+// ------------------------------------------- counting sort (full backward's sub-keys)
 __global__ void slot_histogram_kernel(const int* __restrict__ indices, int64_t E, int64_t slots,
                                       int* __restrict__ counts, int* status) {
   for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < E;
