@@ -542,10 +542,34 @@ __global__ void __launch_bounds__(kSmallWarps * 32) gather_small_kernel(
   if (threadIdx.x == 0) npairs_s = build_pairs(k, pairs);
   wait_prior_grid();  // the chunk lists come from the scoring kernel
   const int64_t src = (t * H + h) * list_words;
-  stage_rows(reinterpret_cast<const uint32_t*>(chunk_s + src), reinterpret_cast<uint32_t*>(cls),
-             1, 1, list_words, list_words);
-  stage_rows(reinterpret_cast<const uint32_t*>(chunk_i + src), reinterpret_cast<uint32_t*>(cli),
-             1, 1, list_words, list_words);
+  {
+    // Scores and ids in one pass (all of a thread's loads in flight before its stores).
+    // list_words is a multiple of 32 and the lists start 128-byte aligned.
+    const uint4* gs4 = reinterpret_cast<const uint4*>(chunk_s + src);
+    const uint4* gi4 = reinterpret_cast<const uint4*>(chunk_i + src);
+    uint4* ss4 = reinterpret_cast<uint4*>(cls);
+    uint4* si4 = reinterpret_cast<uint4*>(cli);
+    const int nv = list_words >> 2;
+    for (int b = threadIdx.x; b < nv; b += blockDim.x * 4) {
+      uint4 vs[4], vi[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = b + u * blockDim.x;
+        if (i < nv) {
+          vs[u] = __ldg(gs4 + i);
+          vi[u] = __ldg(gi4 + i);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = b + u * blockDim.x;
+        if (i < nv) {
+          ss4[i] = vs[u];
+          si4[i] = vi[u];
+        }
+      }
+    }
+  }
   __syncthreads();
 
   // (a) merge the chunk lists of each half, as a tree over the 8 warps: at stride st
