@@ -233,6 +233,24 @@ __device__ __forceinline__ void tmem_wait_ld8(uint32_t (&r)[8]) {
                : "memory");
 }
 
+// Shared-memory stores and loads at 32-bit shared-window addresses.
+__device__ __forceinline__ void sts_f32(uint32_t addr, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+__device__ __forceinline__ void sts_u16(uint32_t addr, uint16_t v) {
+  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
+}
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint16_t lds_u16(uint32_t addr) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr) : "memory");
+  return v;
+}
+
 // ------------------------------------------------------------- descriptors
 // Shared-memory matrix descriptor of a K-major operand tile stored as rows of 64 bf16
 // (128 bytes) with the 128-byte swizzle, 8-row groups 1024 bytes apart. The tile
