@@ -1,5 +1,6 @@
 // pkm_select_gather.cu -- exact top-k over the k x k product candidates, softmax,
-// and the weighted value read summed over heads. One warp per token.
+// and the weighted value read summed over heads. Persistent warps, each taking its
+// tokens' (token, head) units in order.
 //
 // "Large Memory Layers with Product Keys" (gptget.net summary, Methodology and the
 // Deep Analysis / Methodology list): the per-half sub-key sets are combined into

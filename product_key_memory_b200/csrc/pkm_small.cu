@@ -7,7 +7,9 @@
 // almost every SM idle and each stage is bound by one SM's bandwidth. Here every
 // stage spreads the layer's parameters over the whole GPU instead:
 //   query_small_kernel   q = BN(x W_q^T): CTA = 16 features x all tokens, its W_q rows
-//                        staged in shared memory, one warp per token (fp32 FMA)
+//                        staged in shared memory, one warp per token (fp32 FMA); up to
+//                        kDecodeB tokens query_decode_kernel / score_decode_kernel
+//                        instead give a warp one W_q row / 8 sub-keys for all tokens
 //   score_small_kernel   CTA = (64 sub-keys, head-half, 16 tokens): the chunk's scores
 //                        and its best 32 per token
 //   gather_small_kernel  CTA = (token, head), the H heads of a token one cluster:
