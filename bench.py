@@ -608,11 +608,14 @@ def pruned_pairs(k: int) -> int:
 
 def latency_table(args, dev, P, wname, d, Bs):
     """Forward latency of a few tokens on the layer d (device tensors of workload
-    wname): calls issued back to back on one stream, device time per call from CUDA
-    events around 200 calls; caches warm (one token touches H*k value rows). Each
-    batch size through the default choice, each small-batch form forced (the single
-    cooperative kernel "small_fused", the three kernels "small_split") and the
-    large-batch tensor-core kernels ("tc"): the data behind the cut-offs."""
+    wname), caches warm (one token touches H*k value rows). Each batch size through the
+    default choice, each small-batch form forced (the single cooperative kernel
+    "small_fused", the three kernels "small_split") and the large-batch tensor-core
+    kernels ("tc"): the data behind the cut-offs. Two timings per entry, CUDA events
+    around many calls issued back to back: "B=..": 10 calls captured in a CUDA graph,
+    replayed 20 times (the device's time per call, as a serving loop that replays
+    graphs sees it); "B=.. stream": 200 calls launched one by one from Python, which
+    on a slow host measures the host's launch time instead."""
     w0 = synth.WORKLOADS[wname]
     res = {}
     # The GPU's clocks ramp up under load: ~0.2 s of large-batch forwards first, so the
@@ -623,6 +626,7 @@ def latency_table(args, dev, P, wname, d, Bs):
         P.pkm_forward(x, d["W_q"], d["bn_mean"], d["bn_var"], d["bn_gamma"], d["bn_beta"],
                       d["subkeys"], d["values"], k=w0.k, want_scores=False)
         torch.cuda.synchronize(dev)
+    side = torch.cuda.Stream(dev)
     for path in ("auto", "small_fused", "small_split", "tc"):
         for B in Bs:
             x = d["x"][:B].contiguous()
@@ -649,9 +653,29 @@ def latency_table(args, dev, P, wname, d, Bs):
                     call()
                 b.record()
                 torch.cuda.synchronize(dev)
+                stream_us = a.elapsed_time(b) / n * 1e3
+                side.wait_stream(torch.cuda.current_stream(dev))
+                with torch.cuda.stream(side):
+                    call()
+                torch.cuda.current_stream(dev).wait_stream(side)
+                torch.cuda.synchronize(dev)
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    for _ in range(10):
+                        call()
+                g.replay()
+                torch.cuda.synchronize(dev)
+                a.record()
+                for _ in range(20):
+                    g.replay()
+                b.record()
+                torch.cuda.synchronize(dev)
+                graph_us = a.elapsed_time(b) / 200 * 1e3
+                del g
             key = ("" if wname == "c1024" else wname + " ") + "B=%d" % B
             key += "" if path == "auto" else " " + path
-            res[key] = a.elapsed_time(b) / n * 1e3
+            res[key] = graph_us
+            res[key + " stream"] = stream_us
     return res
 
 
@@ -664,7 +688,9 @@ def run_latency(args, dev, P, with_wide=False):
     d = {k: v.to(dev) for k, v in L.items()}
     res = {"workload": "c1024 layer (1024^2 slots, H=4, k=32, v=1024, bf16) and the wide "
                        "layer (d_model 1600, H=8, v=1600), B tokens per call",
-           "unit": "us per call"}
+           "unit": "us per call",
+           "timing": "plain keys: 10 calls in a CUDA graph replayed 20 times (device time "
+                     "per call); '... stream' keys: 200 calls launched one by one"}
     res.update(latency_table(args, dev, P, "c1024", d, (1, 4, 8, 16, 32, 64, 96, 112, 128)))
     del d, L
     if with_wide:

@@ -105,7 +105,8 @@ size_t pkm_workspace_size(const pkm_shape* s, int for_backward);
  *   scores   [B][H][k]  fp32   kept key scores s1[i] + s2[j]; may be NULL
  * workspace: device scratch of at least pkm_workspace_size(s, 0) bytes, 256-byte
  *   aligned; its contents on entry do not matter.
- * Batches of at most 112 tokens (H <= 8) take the small-batch path, which spreads
+ * Batches of at most 112 tokens (H <= 4; 96 with H <= 8) take the small-batch path
+ * (PKM_OPT_PATH small_fused / small_split: at most 112 for any H <= 8), which spreads
  * W_q, the sub-keys and the heads over all SMs for latency: from 9 to 32 tokens one
  * cooperative kernel (one block per SM, its query, scoring and gather phases
  * separated by grid-wide barriers whose waits are bounded like the pipelines'),

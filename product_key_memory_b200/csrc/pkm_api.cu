@@ -53,8 +53,12 @@ Path choose_path(const pkm_shape* s) {
   init_options();
   const int pin = g_opt_path.load(std::memory_order_relaxed);
   if (pin == PKM_PATH_SIMT) return Path::kSimt;
+  // A pinned small-batch form takes every batch the small-batch kernels support; the
+  // automatic choice only those up to the measured crossover for the head count.
+  const bool pinned_small = pin == PKM_PATH_SMALL_FUSED || pin == PKM_PATH_SMALL_SPLIT;
   if (pin != PKM_PATH_TC &&
-      pkm::small_supported(s->B, s->d_model, s->H, s->dq, s->n, s->k, s->v, s->dtype))
+      pkm::small_supported(s->B, s->d_model, s->H, s->dq, s->n, s->k, s->v, s->dtype) &&
+      (pinned_small || s->B <= pkm::small_auto_max_b(s->H)))
     return Path::kSmall;
   return pkm::tc_supported(s->dtype, s->d_model, s->H, s->dq, s->n, s->k) ? Path::kTensor
                                                                           : Path::kSimt;

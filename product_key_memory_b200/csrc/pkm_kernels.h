@@ -159,6 +159,11 @@ cudaError_t launch_bn_train_dacc(const float* g_q, const float* acc, const float
 // tensor-core kernels are faster on the 1024^2 layer (115 vs 121 us) and on the wide
 // layer (265 vs 292 us), at 96 the small-batch kernels (90 vs 110, 224 vs 264 us).
 constexpr int kSmallMaxB = 112;
+// Largest batch the automatic choice sends to the small-batch kernels: the measured
+// crossover with the tensor-core path (device time per call, graph replay) is about 112
+// tokens with H = 4 on the 1024^2 layer (111 vs 117 us at 112, 118 vs 117 at 128) and 96
+// with H = 8 on the wide layer (221 vs 221 us at 96, 264 vs 227 at 112).
+constexpr int small_auto_max_b(int H) { return H > 4 ? 96 : kSmallMaxB; }
 bool small_supported(int64_t B, int d_model, int H, int dq, int n, int k, int v, int dtype);
 size_t small_chunk_entries(int64_t B, int H, int n);
 cudaError_t launch_forward_small(const LayerArgs& a, float* q, float* chunk_s, int* chunk_i,

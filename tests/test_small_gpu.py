@@ -1,6 +1,7 @@
-"""GPU parity of the small-batch forward (B <= 112 tokens: pkm_forward picks the
-small-batch kernels by itself) against the fp64 oracle, through the C ABI, in both
-forms: the single cooperative kernel and the three kernels.
+"""GPU parity of the small-batch forward (up to 112 tokens with H <= 4, 96 with more
+heads: pkm_forward picks the small-batch kernels by itself; a pinned form takes up to
+112 tokens for any H <= 8) against the fp64 oracle, through the C ABI, in both forms:
+the single cooperative kernel and the three kernels.
 
 Same bar as tests/test_forward_gpu.py: indices bit-exact except fp64 near-ties
 within 1e-5 relative of the k-th score; weights, kept scores and out within

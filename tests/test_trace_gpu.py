@@ -34,6 +34,12 @@ def _forward(P, w, d, ws=None):
     ("c512", 4, "auto", (2,), 3),              # small batch, three kernels (decode mode)
     ("c512", 16, "auto", (2,), 1),             # small batch, one cooperative kernel
     ("tiny", 64, "simt", (0, 1, 2), 3),        # CUDA-core kernels (fp32)
+    # The automatic cut-off depends on the heads: H = 8 takes the small-batch kernels
+    # up to 96 tokens, the tensor-core kernels above; a pinned form keeps them to 112.
+    ("wide", 96, "auto", (2,), 3),
+    ("wide", 112, "auto", (0, 1, 2), 3),
+    ("wide", 112, "small_split", (2,), 3),
+    ("c1024", 112, "auto", (2,), 3),
 ])
 def test_forward_stages(name, B, path, stages, launches):
     P = _P()
