@@ -149,11 +149,11 @@ int pkm_forward(const pkm_shape* s, const void* x, const void* W_q, const float*
  * the status word (PKM_ERR_DEVICE).
  * Only B, H, n, k, v and dtype of the shape are read; d_model, dq and bn_eps are
  * ignored.
- * With grad_scores requested the two results are computed concurrently: the slot
- * grouping and row sums run on the library's helper stream (one per device, highest
- * priority) while grad_scores is computed on `stream`; event waits order both ways,
- * so all of the call's work is complete when `stream` reaches the point after the
- * call (CUDA-graph capture of `stream` takes the helper stream's work in with it).
+ * With grad_scores requested, the sort of the picks by slot runs on the library's
+ * helper stream (one per device, highest priority) while grad_scores is computed on
+ * `stream`, and the row sums follow on `stream`; event waits order both ways, so all
+ * of the call's work is complete when `stream` reaches the point after the call
+ * (CUDA-graph capture of `stream` takes the helper stream's work in with it).
  * workspace: at least pkm_workspace_size(s, 1) bytes, 256-byte aligned.
  */
 int pkm_backward_values(const pkm_shape* s, const void* values, const int32_t* indices,
@@ -186,9 +186,9 @@ int pkm_backward_values(const pkm_shape* s, const void* values, const int32_t* i
  * are added atomically. Slot ids outside [0, n*n) are skipped and counted in the
  * status word. 2*B*H*k must stay below 2^31 (PKM_ERR_UNSUPPORTED otherwise: the
  * sub-key grouping sorts two contributions per pick with 32-bit positions).
- * grad_values, when requested, is computed on the library's helper stream alongside
- * the rest (as in pkm_backward_values), joined back into `stream` before the call's
- * end.
+ * The other gradients' chain of kernels runs on the library's helper stream (highest
+ * priority) and grad_values, when requested, on `stream` beside it, joined back into
+ * `stream` before the call's end.
  * workspace: at least pkm_workspace_size(s, 3) bytes, 256-byte aligned.
  */
 int pkm_backward(const pkm_shape* s, const void* x, const void* W_q, const float* bn_mean,

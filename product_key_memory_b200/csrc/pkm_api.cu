@@ -780,9 +780,11 @@ int pkm_backward_values(const pkm_shape* s, const void* values, const int32_t* i
   int* status = static_cast<int*>(workspace);
   if (cudaMemsetAsync(status, 0, sizeof(int), st) != cudaSuccess) return PKM_ERR_CUDA;
   const int64_t slots = static_cast<int64_t>(s->n) * s->n;
-  // The two parts are independent: with both asked for, the value rows (sort + row
-  // sums) run on the helper stream while the kept-score gradients stream the value
-  // rows on the caller's stream.
+  // With both results asked for, the slot sort (ALU and L2 only) runs on the helper
+  // stream while the kept-score gradients stream the picked value rows from HBM on the
+  // caller's stream; the row sums (HBM read-modify-writes) follow on the caller's
+  // stream once both are done. Two HBM-bound kernels side by side only share the
+  // bandwidth, so they do not overlap each other.
   const bool split = grad_scores != nullptr;
   pkm::SideStream side;
   if (split && side_stream(&side) != PKM_OK) return PKM_ERR_CUDA;
@@ -791,12 +793,11 @@ int pkm_backward_values(const pkm_shape* s, const void* values, const int32_t* i
   Tracer tr(1);
   tr.begin(3, st);
   cudaError_t e = split ? pkm::side_fork(side, st) : cudaSuccess;
-  const cudaStream_t vs = split ? side.st : st;
-  tr.begin_here(1, vs);  // shares the call's first event unless on the helper stream
+  const cudaStream_t ss = split ? side.st : st;
+  tr.begin_here(1, ss);  // shares the call's first event unless on the helper stream
   if (e == cudaSuccess)
-    e = pkm::launch_value_rows(s->B, s->H, s->k, s->v, s->dtype, slots, indices, weights,
-                               grad_out, grad_values, w, status, vs);
-  tr.end(vs);
+    e = pkm::launch_value_sort(s->B, s->H, s->k, slots, indices, w, status, ss);
+  tr.end(ss);
   if (split) {
     tr.begin(0, st);
     if (e == cudaSuccess)
@@ -807,7 +808,12 @@ int pkm_backward_values(const pkm_shape* s, const void* values, const int32_t* i
     const cudaError_t e2 = pkm::side_join(side, st);
     if (e == cudaSuccess) e = e2;
   }
+  tr.begin(1, st);
+  if (e == cudaSuccess)
+    e = pkm::launch_value_segments(s->B, s->H, s->k, s->v, s->dtype, slots, weights, grad_out,
+                                   grad_values, w, st);
   tr.end(st);
+  tr.end_here(st);
   tr.finish(e == cudaSuccess, pkm::backward_values_launches(static_cast<int64_t>(s->n) * s->n,
                                                            grad_scores != nullptr, true));
   return e == cudaSuccess ? PKM_OK : PKM_ERR_CUDA;

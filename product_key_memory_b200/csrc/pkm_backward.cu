@@ -849,20 +849,28 @@ static cudaError_t launch_scores_t(int64_t B, int H, int k, int v, int64_t slots
   return cudaGetLastError();
 }
 
-// B2: stable sort of the picks by slot, then each slot's picks summed into its row of
-// grad_values (needs only the indices, weights and grad_out: independent of B1).
-template <typename T, int MAXV>
-static cudaError_t launch_rows_t(int64_t B, int H, int k, int v, int64_t slots,
-                                 const int* indices, const float* weights, const void* grad_out,
-                                 float* grad_values, const BackwardWs& ws, int* status,
-                                 cudaStream_t st) {
+// B2 in two parts. The sort of the picks by slot (reads only the indices; its keys and
+// pick ids stay in L2) ...
+static cudaError_t launch_sort_part(int64_t B, int H, int k, int64_t slots, const int* indices,
+                                    const BackwardWs& ws, int* status, cudaStream_t st) {
   const int64_t E = B * H * k;
-  const T* G = static_cast<const T*>(grad_out);
   cudaError_t e = cudaMemsetAsync(ws.ctr, 0, 4 * sizeof(int), st);
   if (e != cudaSuccess) return e;
   int which = 0;
-  e = sort_picks_by_slot(indices, E, slots, ws, status, st, &which);
-  if (e != cudaSuccess) return e;
+  return sort_picks_by_slot(indices, E, slots, ws, status, st, &which);
+}
+
+// ... and each slot's picks summed into its row of grad_values (reads the sorted picks,
+// weights and grad_out). Neither part needs B1's result.
+template <typename T, int MAXV>
+static cudaError_t launch_segments_t(int64_t B, int H, int k, int v, int64_t slots,
+                                     const float* weights, const void* grad_out,
+                                     float* grad_values, const BackwardWs& ws,
+                                     cudaStream_t st) {
+  const int64_t E = B * H * k;
+  const T* G = static_cast<const T*>(grad_out);
+  // sort_picks_by_slot alternates the two buffers, starting with 0.
+  const int which = (sort_passes(slots) - 1) & 1;
   const int* skey = ws.keys[which];
   const int* spick = ws.picks[which];
   const int64_t windows = (E + 31) / 32;
@@ -871,7 +879,7 @@ static cudaError_t launch_rows_t(int64_t B, int H, int k, int v, int64_t slots,
   segment_small_kernel<T, MAXV><<<sgrid > 0 ? sgrid : 1, 128, 0, st>>>(
       skey, spick, E, slots, weights, G, H * k, v, grad_values, ws.ctr, ws.items, ws.huge);
   const size_t smem = sizeof(float) * kItemWarps * v;
-  e = set_max_smem(reinterpret_cast<const void*>(segment_items_kernel<T, MAXV>), smem);
+  cudaError_t e = set_max_smem(reinterpret_cast<const void*>(segment_items_kernel<T, MAXV>), smem);
   if (e != cudaSuccess) return e;
   segment_items_kernel<T, MAXV><<<2 * 148, kItemWarps * 32, smem, st>>>(
       spick, weights, G, H * k, v, ws.ctr, ws.items, grad_values, ws.scratch);
@@ -908,12 +916,24 @@ cudaError_t launch_grad_scores(int64_t B, int H, int k, int v, int dtype, int64_
                    grad_scores, status, st);
 }
 
+cudaError_t launch_value_sort(int64_t B, int H, int k, int64_t slots, const int* indices,
+                              const BackwardWs& ws, int* status, cudaStream_t st) {
+  return launch_sort_part(B, H, k, slots, indices, ws, status, st);
+}
+
+cudaError_t launch_value_segments(int64_t B, int H, int k, int v, int dtype, int64_t slots,
+                                  const float* weights, const void* grad_out, float* grad_values,
+                                  const BackwardWs& ws, cudaStream_t st) {
+  PKM_BWD_DISPATCH(launch_segments_t, B, H, k, v, slots, weights, grad_out, grad_values, ws, st);
+}
+
 cudaError_t launch_value_rows(int64_t B, int H, int k, int v, int dtype, int64_t slots,
                               const int* indices, const float* weights, const void* grad_out,
                               float* grad_values, const BackwardWs& ws, int* status,
                               cudaStream_t st) {
-  PKM_BWD_DISPATCH(launch_rows_t, B, H, k, v, slots, indices, weights, grad_out, grad_values, ws,
-                   status, st);
+  const cudaError_t e = launch_value_sort(B, H, k, slots, indices, ws, status, st);
+  if (e != cudaSuccess) return e;
+  return launch_value_segments(B, H, k, v, dtype, slots, weights, grad_out, grad_values, ws, st);
 }
 #undef PKM_BWD_DISPATCH
 

@@ -635,24 +635,27 @@ cudaError_t launch_backward_full(const LayerArgs& a, bool tensor_path, bool bn_t
   const int64_t slots = static_cast<int64_t>(a.n) * a.n;
   cudaError_t e = cudaSuccess;
   const bool split = grad_values && side.st;
-  if (grad_values) {
-    // The value gradients need only the picks and grad_out: on the side stream their
-    // row read-modify-writes (HBM) overlap the GEMMs and the sub-key work below.
-    if (split) e = side_fork(side, st);
-    if (e == cudaSuccess)
-      e = launch_value_rows(a.B, a.H, a.k, a.v, a.dtype, slots, indices, weights, grad_out,
-                            grad_values, w.values, a.status, split ? side.st : st);
-    *launches += backward_values_launches(slots, false, true);
-  }
+  // The value gradients need only the picks and grad_out. The dependent chain of the
+  // rest (kept-score gradients, query recompute, sub-key and BatchNorm sums, GEMMs) runs
+  // on the helper stream, scheduled ahead of the caller's stream, and the value rows'
+  // sort and row sums fill the SMs it leaves idle on the caller's stream.
+  const cudaStream_t xs = split ? side.st : st;
+  if (split) e = side_fork(side, st);
   if (e == cudaSuccess) {
     if (a.dtype == 0)
       e = launch_full_t<float>(a, tensor_path, bn_training, indices, weights, grad_out, grad_x,
-                               grad_W, grad_gamma, grad_beta, grad_subkeys, grad_scores, w, st,
+                               grad_W, grad_gamma, grad_beta, grad_subkeys, grad_scores, w, xs,
                                launches);
     else
       e = launch_full_t<uint16_t>(a, tensor_path, bn_training, indices, weights, grad_out,
                                   grad_x, grad_W, grad_gamma, grad_beta, grad_subkeys,
-                                  grad_scores, w, st, launches);
+                                  grad_scores, w, xs, launches);
+  }
+  if (grad_values) {
+    if (e == cudaSuccess)
+      e = launch_value_rows(a.B, a.H, a.k, a.v, a.dtype, slots, indices, weights, grad_out,
+                            grad_values, w.values, a.status, st);
+    *launches += backward_values_launches(slots, false, true);
   }
   // Always join, even after an error, so the caller's stream never runs ahead of work
   // already queued on the side stream.

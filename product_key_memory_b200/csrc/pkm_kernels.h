@@ -88,8 +88,14 @@ cudaError_t launch_grad_scores(int64_t B, int H, int k, int v, int dtype, int64_
                                const void* values, const int* indices, const float* weights,
                                const void* grad_out, float* grad_scores, int* status,
                                cudaStream_t st);
-// B2: picks sorted by slot, each slot's weighted grad_out rows added to grad_values.
-// Independent of B1 (reads indices, weights and grad_out only).
+// B2: picks sorted by slot (launch_value_sort: indices only), then each slot's weighted
+// grad_out rows added to grad_values (launch_value_segments, same stream order after the
+// sort); launch_value_rows issues both. Independent of B1.
+cudaError_t launch_value_sort(int64_t B, int H, int k, int64_t slots, const int* indices,
+                              const BackwardWs& ws, int* status, cudaStream_t st);
+cudaError_t launch_value_segments(int64_t B, int H, int k, int v, int dtype, int64_t slots,
+                                  const float* weights, const void* grad_out, float* grad_values,
+                                  const BackwardWs& ws, cudaStream_t st);
 cudaError_t launch_value_rows(int64_t B, int H, int k, int v, int dtype, int64_t slots,
                               const int* indices, const float* weights, const void* grad_out,
                               float* grad_values, const BackwardWs& ws, int* status,
