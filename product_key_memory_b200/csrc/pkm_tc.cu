@@ -521,16 +521,18 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
       int cnt = 0, kept = 0;   // log entries; entries kept by the last merge
       bool ok = true;
 
-      // Branch-free filter of 8 columns: every score is written to the next free log
-      // slot, which only advances when the score is kept (a rejected one is overwritten).
+      // Filter of 8 columns: a kept score and its id go to the next free log slot. The
+      // stores and the slot advance are predicated on the compare (no branch, so the
+      // warp's rows never diverge), and a rejected score costs no shared-memory store
+      // (storing every score and advancing only for kept ones measured 5 us slower).
       auto filter = [&](const uint32_t (&rv)[8], int id0) {
         uint32_t as = s_row + cnt * kSStrideS, ai = i_row + cnt * kSStrideI;
 #pragma unroll
         for (int i = 0; i < kSStep; ++i) {
           const float v = __uint_as_float(rv[i]);
-          sts_f32(as, v);
-          sts_u16(ai, static_cast<uint16_t>(id0 + i));
           if (v > thr) {
+            sts_f32(as, v);
+            sts_u16(ai, static_cast<uint16_t>(id0 + i));
             as += kSStrideS;
             ai += kSStrideI;
           }
