@@ -334,6 +334,24 @@ __device__ __forceinline__ void thread_sort32f(float (&x)[32]) {
       }
 }
 
+// Sort 16 floats held by one thread, largest first.
+__device__ __forceinline__ void thread_sort16f(float (&x)[16]) {
+#pragma unroll
+  for (int size = 2; size <= 16; size <<= 1)
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1)
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int j = i ^ stride;
+        if (j > i) {
+          const bool desc = (i & size) == 0 || size == 16;
+          const float a = x[i], b = x[j];
+          x[i] = desc ? fmaxf(a, b) : fminf(a, b);
+          x[j] = desc ? fminf(a, b) : fmaxf(a, b);
+        }
+      }
+}
+
 // 32nd largest of 64 floats: sort both halves, then the elementwise max of one half
 // and the other reversed is the best 32 (as a set); its minimum is the answer.
 __device__ __forceinline__ float kth32_of_64(float (&x)[64]) {
@@ -540,21 +558,32 @@ __global__ void __launch_bounds__(kSThreads, 1) score_topk_tc_kernel(
         cnt = static_cast<int>((as - s_row) / kSStrideS);
       };
 
-      // Merge every fresh log entry into Ls (32 at a time) and raise tau_run. Entries
+      // Merge every fresh log entry into Ls (32 at a time; a round in which no row of the
+      // warp has more than 16 fresh entries sorts 16) and raise tau_run. Entries
       // below tau_run can stay in the log: it is compacted to the entries that can
       // still be among the best 32 only when it is filling up, and after the unit.
       auto merge = [&](bool last) {
 #pragma unroll 1
         for (int base = kept; __any_sync(0xffffffffu, base < cnt); base += 32) {
           const int fresh = cnt - base;
-          float b[32];
           const uint32_t fresh_at = s_row + base * kSStrideS;
+          if (__reduce_max_sync(0xffffffffu, fresh) <= 16) {
+            float b[16];
 #pragma unroll
-          for (int q = 0; q < 32; ++q)
-            b[q] = q < fresh ? lds_f32(fresh_at + q * kSStrideS) : -INFINITY;
-          thread_sort32f(b);
+            for (int q = 0; q < 16; ++q)
+              b[q] = q < fresh ? lds_f32(fresh_at + q * kSStrideS) : -INFINITY;
+            thread_sort16f(b);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) Ls[i] = fmaxf(Ls[i], b[31 - i]);
+            for (int i = 16; i < 32; ++i) Ls[i] = fmaxf(Ls[i], b[31 - i]);
+          } else {
+            float b[32];
+#pragma unroll
+            for (int q = 0; q < 32; ++q)
+              b[q] = q < fresh ? lds_f32(fresh_at + q * kSStrideS) : -INFINITY;
+            thread_sort32f(b);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) Ls[i] = fmaxf(Ls[i], b[31 - i]);
+          }
 #pragma unroll
           for (int stride = 16; stride > 0; stride >>= 1)
 #pragma unroll
