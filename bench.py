@@ -597,13 +597,19 @@ def run_c512_and_backward(args, dev, P, hbm, bf16, stream, world, barrier,
                    "stage_ms": [m / max(1, calls) for m in stage_ms[:3]],
                    "gather_gbs": per_token_bytes(w) * B / (stage_ms[2] / max(1, calls) * 1e-3) / 1e9}
     if "small_batch" in res:
-        res["small_batch"].update(latency_table(args, dev, P, "wide", d, (64, 96, 112, 128)))
+        res["small_batch"].update(latency_table(args, dev, P, "wide", d, WIDE_LATENCY_B))
     return res
 
 
 def pruned_pairs(k: int) -> int:
     """Candidate pairs (a, b) of the two sorted per-half lists with (a+1)(b+1) <= k."""
     return sum(k // (a + 1) for a in range(k))
+
+
+# Batch sizes of the latency table: both sides of the automatic cut-off between the
+# small-batch kernels and the tensor-core path (384 tokens with H = 4, 240 with H = 8).
+C1024_LATENCY_B = (1, 4, 8, 16, 32, 64, 96, 128, 192, 256, 384, 448)
+WIDE_LATENCY_B = (64, 128, 192, 240, 256)
 
 
 def latency_table(args, dev, P, wname, d, Bs):
@@ -680,24 +686,24 @@ def latency_table(args, dev, P, wname, d, Bs):
 
 
 def run_latency(args, dev, P, with_wide=False):
-    """Small-batch latency on the 1024^2-slot layer (1 to 128 tokens). The wide layer's
+    """Small-batch latency on the 1024^2-slot layer (1 to 448 tokens). The wide layer's
     entries are added where that layer is built (run_c512_and_backward), or here when
     with_wide is set (the latency part run alone)."""
     w0 = synth.WORKLOADS["c1024"]
-    L = synth.make_layer(w0.with_(B=128))
+    L = synth.make_layer(w0.with_(B=max(C1024_LATENCY_B)))
     d = {k: v.to(dev) for k, v in L.items()}
     res = {"workload": "c1024 layer (1024^2 slots, H=4, k=32, v=1024, bf16) and the wide "
                        "layer (d_model 1600, H=8, v=1600), B tokens per call",
            "unit": "us per call",
            "timing": "plain keys: 10 calls in a CUDA graph replayed 20 times (device time "
                      "per call); '... stream' keys: 200 calls launched one by one"}
-    res.update(latency_table(args, dev, P, "c1024", d, (1, 4, 8, 16, 32, 64, 96, 112, 128)))
+    res.update(latency_table(args, dev, P, "c1024", d, C1024_LATENCY_B))
     del d, L
     if with_wide:
-        L = synth.make_layer(synth.WORKLOADS["wide"].with_(B=128))
+        L = synth.make_layer(synth.WORKLOADS["wide"].with_(B=max(WIDE_LATENCY_B)))
         d = {k: v.to(dev) for k, v in L.items()}
         del L
-        res.update(latency_table(args, dev, P, "wide", d, (64, 96, 112, 128)))
+        res.update(latency_table(args, dev, P, "wide", d, WIDE_LATENCY_B))
     return res
 
 

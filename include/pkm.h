@@ -105,13 +105,18 @@ size_t pkm_workspace_size(const pkm_shape* s, int for_backward);
  *   scores   [B][H][k]  fp32   kept key scores s1[i] + s2[j]; may be NULL
  * workspace: device scratch of at least pkm_workspace_size(s, 0) bytes, 256-byte
  *   aligned; its contents on entry do not matter.
- * Batches of at most 112 tokens (H <= 4; 96 with H <= 8) take the small-batch path
- * (PKM_OPT_PATH small_fused / small_split: at most 112 for any H <= 8), which spreads
- * W_q, the sub-keys and the heads over all SMs for latency: from 9 to 32 tokens one
- * cooperative kernel (one block per SM, its query, scoring and gather phases
- * separated by grid-wide barriers whose waits are bounded like the pipelines'),
- * otherwise three kernels that overlap through programmatic dependent launch on
- * `stream` (PKM_OPT_PATH can force either form). Up to 8 tokens the query and
+ * Small batches take the small-batch path, which spreads W_q, the sub-keys and the
+ * heads over all SMs for latency: up to 384 tokens with H <= 4 and 240 with H <= 8 on
+ * bf16 layers with d_model and dq/2 multiples of 32 and dq/2 <= 256 (whose query
+ * network and per-half scores there run as warp-level tensor-core tiles of 16 tokens),
+ * up to 112 / 96 tokens otherwise; a pinned form (PKM_OPT_PATH small_fused /
+ * small_split) takes up to 512 tokens for any H <= 8. By default it is three kernels
+ * that overlap through programmatic dependent launch on `stream`: the first waits on
+ * the device for the stream's earlier work and clears the status word itself, so
+ * back-to-back calls overlap too. PKM_PATH_SMALL_FUSED runs it as one cooperative
+ * kernel instead (one block per SM, its query, scoring and gather phases separated by
+ * grid-wide barriers whose waits are bounded like the pipelines'). Up to 4 tokens
+ * with H <= 4 (8 tokens on layers without the tensor-core tiles) the query and
  * scoring stages give a warp one W_q row or 8 sub-keys for all tokens, its lanes
  * splitting the dot products (rows of 16-byte multiples). Larger batches run
  * three kernels on `stream` (query network, per-half scores and top-k, candidate
@@ -309,16 +314,17 @@ int pkm_trace_read(int pass, double* stage_ms, int max_stages, int64_t* calls,
  * it. The environment variables PKM_PATH (auto | tc | simt | small_fused | small_split) and
  * PKM_SUBBATCHES (1..4)
  * give the initial values and are read once, at the first call that needs them.
- *   PKM_OPT_PATH        PKM_PATH_AUTO (default): small-batch kernels for up to 128
- *                       tokens, else the tensor-core kernels where the layer fits
+ *   PKM_OPT_PATH        PKM_PATH_AUTO (default): the small-batch kernels for small
+ *                       batches (see pkm_forward), else the tensor-core kernels where
+ *                       the layer fits
  *                       their tiles (bf16, d_model and dq/2 multiples of 64, n a
  *                       multiple of 256, H*dq <= 4096), else the CUDA-core kernels;
  *                       PKM_PATH_TC: never the small-batch kernels;
  *                       PKM_PATH_SIMT: always the CUDA-core kernels;
- *                       PKM_PATH_SMALL_FUSED: as AUTO, but every small batch runs as
- *                       the one cooperative kernel;
- *                       PKM_PATH_SMALL_SPLIT: as AUTO, but every small batch runs as
- *                       the three kernels.
+ *                       PKM_PATH_SMALL_FUSED: the small-batch path for every batch
+ *                       it supports (up to 512 tokens), as the one cooperative
+ *                       kernel;
+ *                       PKM_PATH_SMALL_SPLIT: the same, as the three kernels.
  *   PKM_OPT_SUBBATCHES  1 (default) to 4: sub-batches of the pipelined tensor-core
  *                       forward (see pkm_forward). The forward's workspace size
  *                       depends on it: query it after setting the option.

@@ -58,7 +58,7 @@ Path choose_path(const pkm_shape* s) {
   const bool pinned_small = pin == PKM_PATH_SMALL_FUSED || pin == PKM_PATH_SMALL_SPLIT;
   if (pin != PKM_PATH_TC &&
       pkm::small_supported(s->B, s->d_model, s->H, s->dq, s->n, s->k, s->v, s->dtype) &&
-      (pinned_small || s->B <= pkm::small_auto_max_b(s->H)))
+      (pinned_small || s->B <= pkm::small_auto_max_b(s->H, s->d_model, s->dq, s->dtype)))
     return Path::kSmall;
   return pkm::tc_supported(s->dtype, s->d_model, s->H, s->dq, s->n, s->k) ? Path::kTensor
                                                                           : Path::kSimt;
@@ -577,29 +577,33 @@ int validate_forward_args(const pkm_shape* s, const void* x, const void* W_q,
   return PKM_OK;
 }
 
-// The forward's launches for a validated call with B > 0 (status word already cleared).
+// Small-batch path: the single cooperative kernel (only when pinned) rather than the
+// three kernels.
+bool small_fused_chosen(const pkm_shape* s) {
+  return g_opt_path.load(std::memory_order_relaxed) == PKM_PATH_SMALL_FUSED &&
+         pkm::small_fused_supported(s->d_model, s->H, s->dq, s->n, s->v, s->dtype);
+}
+
+// The forward's launches for a validated call with B > 0. The status word is already
+// cleared, or (clear_status) the small-batch three-kernel form clears it itself.
 // Stages: 0 query network, 1 per-half scores + best 32, 2 candidate top-k + softmax +
 // gather; the caller brackets stage 3 (the whole call).
 cudaError_t run_forward(const pkm_shape* s, const LayerArgs& a, const ForwardWs& w, float* out,
                         int32_t* indices, float* weights, float* scores, cudaStream_t st,
-                        Tracer& tr, int* nlaunch) {
+                        Tracer& tr, int* nlaunch, bool clear_status) {
   const void* x = a.x;
   cudaError_t e = cudaSuccess;
   int launches = 0;
   const Path path = choose_path(s);
   if (path == Path::kSmall) {
     tr.begin_here(2, st);
-    const int pin = g_opt_path.load(std::memory_order_relaxed);
-    if (pin != PKM_PATH_SMALL_SPLIT &&
-        (pin == PKM_PATH_SMALL_FUSED ||
-         (s->B >= pkm::kSmallFusedMinB && s->B <= pkm::kSmallFusedMaxB)) &&
-        pkm::small_fused_supported(s->d_model, s->H, s->dq, s->n, s->v, s->dtype)) {
+    if (small_fused_chosen(s)) {
       e = pkm::launch_forward_small_fused(a, w.q, w.list_s, w.list_i, w.part, out, indices,
                                           weights, scores, st);
       launches = 1;
     } else {
       e = pkm::launch_forward_small(a, w.q, w.list_s, w.list_i, out, indices, weights, scores,
-                                    st);
+                                    clear_status ? w.status : nullptr, st);
       launches = 3;
     }
     tr.end(st);
@@ -694,12 +698,17 @@ int pkm_forward(const pkm_shape* s, const void* x, const void* W_q, const float*
   forward_ws(s, &w, static_cast<char*>(workspace));
   LayerArgs a{s->B, s->d_model, s->H, s->dq, s->n, s->k, s->v, s->dtype, s->bn_eps,
               x, W_q, bn_mean, bn_var, bn_gamma, bn_beta, subkeys, values, w.status, 0};
-  // The status word and the small-batch kernel's grid-barrier counter after it.
-  if (cudaMemsetAsync(w.status, 0, 2 * sizeof(int), st) != cudaSuccess) return PKM_ERR_CUDA;
+  // The status word and the small-batch kernel's grid-barrier counter after it. The
+  // small-batch three-kernel form clears the status word in its first kernel instead
+  // (it does not use the counter): one operation less between back-to-back calls.
+  const bool self_clear = choose_path(s) == Path::kSmall && !small_fused_chosen(s);
+  if (!self_clear && cudaMemsetAsync(w.status, 0, 2 * sizeof(int), st) != cudaSuccess)
+    return PKM_ERR_CUDA;
   Tracer tr(0);
   int launches = 0;
   tr.begin(3, st);
-  const cudaError_t e = run_forward(s, a, w, out, indices, weights, scores, st, tr, &launches);
+  const cudaError_t e =
+      run_forward(s, a, w, out, indices, weights, scores, st, tr, &launches, self_clear);
   tr.end_here(st);  // the last stage's end, or a new event after the pipelined join
   tr.finish(e == cudaSuccess, launches);
   return e == cudaSuccess ? PKM_OK : PKM_ERR_CUDA;
@@ -752,7 +761,8 @@ int pkm_forward_train(const pkm_shape* s, const void* x, const void* W_q,
                                    bn_running_var, st);
   tr.end(st);
   launches += 3;
-  if (e == cudaSuccess) e = run_forward(s, a, w, out, indices, weights, scores, st, tr, &launches);
+  if (e == cudaSuccess)
+    e = run_forward(s, a, w, out, indices, weights, scores, st, tr, &launches, false);
   tr.end_here(st);
   tr.finish(e == cudaSuccess, launches);
   return e == cudaSuccess ? PKM_OK : PKM_ERR_CUDA;

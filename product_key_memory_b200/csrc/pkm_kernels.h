@@ -161,30 +161,35 @@ cudaError_t launch_bn_train_dacc(const float* g_q, const float* acc, const float
 // Small-batch forward (pkm_small.cu): B <= kSmallMaxB tokens, three launches that
 // spread the parameters over every SM. Workspace: q fp32 [B][H*dq] and chunk lists of
 // small_chunk_entries() (score, id) entries.
-// Measured crossover with the tensor-core path (bench.py small_batch): at 128 tokens the
-// tensor-core kernels are faster on the 1024^2 layer (115 vs 121 us) and on the wide
-// layer (265 vs 292 us), at 96 the small-batch kernels (90 vs 110, 224 vs 264 us).
-constexpr int kSmallMaxB = 112;
+constexpr int kSmallMaxB = 512;
+// bf16 layers whose query network and per-half scores the small-batch kernels run as
+// tensor-core tiles above decode mode (d_model and dq/2 multiples of 32, dq/2 <= 256).
+bool small_mma_shape(int d_model, int dq, int dtype);
 // Largest batch the automatic choice sends to the small-batch kernels: the measured
-// crossover with the tensor-core path (device time per call, graph replay) is about 112
-// tokens with H = 4 on the 1024^2 layer (111 vs 117 us at 112, 118 vs 117 at 128) and 96
-// with H = 8 on the wide layer (221 vs 221 us at 96, 264 vs 227 at 112).
-constexpr int small_auto_max_b(int H) { return H > 4 ? 96 : kSmallMaxB; }
+// crossover with the tensor-core path (device time per call, CUDA-graph replay). With
+// the tensor-core tiles: about 390 tokens with H = 4 on the 1024^2 layer (118 vs 120 us
+// at 384, 127 vs 120 at 416) and 420 on the 512^2 layer (93 vs 104 us at 384, 110 vs
+// 103 at 448), about 250 with H = 8 on the wide layer (197 vs 224 us at 224, 228 vs 225
+// at 256). Without them (CUDA-core query and scores per token) 112 and 96 tokens.
+inline int small_auto_max_b(int H, int d_model, int dq, int dtype) {
+  if (small_mma_shape(d_model, dq, dtype)) return H > 4 ? 240 : 384;
+  return H > 4 ? 96 : 112;
+}
 bool small_supported(int64_t B, int d_model, int H, int dq, int n, int k, int v, int dtype);
 size_t small_chunk_entries(int64_t B, int H, int n);
+// clear: the call's status word, zeroed by the first kernel once the stream's earlier
+// work has finished (instead of a memset before the launch), or null.
 cudaError_t launch_forward_small(const LayerArgs& a, float* q, float* chunk_s, int* chunk_i,
-                                 float* out, int* idx, float* w, float* sc, cudaStream_t st);
+                                 float* out, int* idx, float* w, float* sc, int* clear,
+                                 cudaStream_t st);
 // The same forward as one cooperative launch with grid-wide barriers (one CTA per SM);
 // the barrier counter is the int after a.status, zeroed by the caller. `part` holds
-// [B][H][v] floats followed by B unsigned per-token counts (zeroed by the kernel).
-// Default for batches of kSmallFusedMinB to kSmallFusedMaxB tokens, where it measured
-// faster (35 vs 45 us at 16 tokens, 49 vs 53 at 32, on the 1024^2 layer). Up to 8
-// tokens both forms run in decode mode (a warp per W_q row / per 8 sub-keys) and the
-// three kernels win (19 vs 23 us for one token, 27 vs 31 for 8: their query grid has
-// more blocks, and programmatic launch overlaps the stages); above 32 tokens the three
-// kernels spread the token loops over more blocks (67 vs 86 us at 64).
-constexpr int kSmallFusedMinB = 9;
-constexpr int kSmallFusedMaxB = 32;
+// [B][H][v] floats followed by B unsigned per-token counts (zeroed by the kernel). Taken
+// only when pinned (PKM_OPT_PATH small_fused): the three kernels measured faster at
+// every batch size (12.1 vs 22.6 us for one token, 18.3 vs 24.6 for 16, 25.0 vs 30.7
+// for 32 on the 1024^2 layer), their first kernel overlapping the previous call's last
+// through programmatic launch and clearing the status word itself, where the single
+// kernel needs a memset of its barrier counter before each launch.
 bool small_fused_supported(int d_model, int H, int dq, int n, int v, int dtype);
 cudaError_t launch_forward_small_fused(const LayerArgs& a, float* q, float* chunk_s,
                                        int* chunk_i, float* part, float* out, int* idx, float* w,

@@ -21,6 +21,7 @@
 #include <cooperative_groups.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "pkm_common.cuh"
 #include "pkm_kernels.h"
@@ -44,6 +45,17 @@ __device__ __forceinline__ void allow_dependents() {
 }
 __device__ __forceinline__ void wait_prior_grid() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Prologue of the three-kernel form's first kernel, which is itself launched as a
+// programmatic dependent: its CTAs can be resident before the stream's previous kernel
+// ends, and wait here until that kernel's writes are visible (x and the parameters may
+// come from it). Then it clears the call's status word (clear, when the caller asks for
+// it instead of a memset before the launch) and lets the scoring kernel launch.
+__device__ __forceinline__ void first_kernel_prologue(int* clear) {
+  wait_prior_grid();
+  if (clear && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *clear = 0;
+  allow_dependents();
 }
 
 // Copy `words` 32-bit words from global to shared memory with every thread keeping
@@ -111,14 +123,32 @@ __device__ __forceinline__ void stage_rows(const uint32_t* __restrict__ src, uin
 // the same total). Both small-batch forms use these functions and the same decode_mode
 // test, so their results stay identical.
 // ---------------------------------------------------------------------------
-constexpr int kDecodeB = 8;
+constexpr int kDecodeB = 8;        // decode mode's largest batch
 constexpr int kDecodeRowVecs = 8;  // 16-byte chunks per lane of a W_q row: d*esz <= 4 KiB
 constexpr int kDecodeKeyVecs = 2;  // of a sub-key row: (dq/2)*esz <= 1 KiB
 constexpr int kDecodeKeys = kSChunk / kSmallWarps;  // sub-keys per warp (8)
+constexpr int kMmaMaxKB = 8;  // MMA tiles: 32-wide K-blocks of a sub-key row in registers
 
-__host__ __device__ inline bool decode_mode(int64_t B, int d, int dq, int esz) {
+// bf16 layers whose query network and per-half scores can run as the tensor-core tiles
+// below (d_model and dq/2 multiples of 32, dq/2 <= 256).
+__host__ __device__ inline bool mma_shape(int d, int dq, int esz) {
+  const int half = dq / 2;
+  return esz == 2 && d % 32 == 0 && half % 32 == 0 && half <= 32 * kMmaMaxKB;
+}
+
+// Largest batch decode mode takes. Where the tensor-core tiles can run instead they
+// measured faster from 6 tokens with H = 4 (1024^2 layer, us per call: 12.4 vs 16.3 for
+// one token, 15.8 vs 17.3 for 4, 18.9 vs 18.2 for 6, 21.8 vs 19.5 for 8) and from one
+// token with H = 8 (wide layer: 20.7 vs 19.9 for one, 29.6 vs 20.5 for 4): decode mode's
+// warps take the tokens one after another.
+__host__ __device__ inline int decode_max_b(int H, int d, int dq, int esz) {
+  if (!mma_shape(d, dq, esz)) return kDecodeB;
+  return H <= 4 ? 4 : 0;
+}
+
+__host__ __device__ inline bool decode_mode(int64_t B, int H, int d, int dq, int esz) {
   const int rb = d * esz, kb = (dq / 2) * esz;
-  return B >= 1 && B <= kDecodeB && rb % 16 == 0 && kb % 16 == 0 &&
+  return B >= 1 && B <= decode_max_b(H, d, dq, esz) && rb % 16 == 0 && kb % 16 == 0 &&
          rb <= 16 * 32 * kDecodeRowVecs && kb <= 16 * 32 * kDecodeKeyVecs;
 }
 
@@ -275,6 +305,229 @@ __device__ __forceinline__ void decode_chunk_list(const float* sc, int t, int c0
 }
 
 // ---------------------------------------------------------------------------
+// bf16 layers past decode mode: the query network and the per-half scores as
+// warp-level tensor-core products (mma.sync m16n8k16: bf16 operands, fp32
+// accumulation) on tiles of kMmaTok tokens, used by both small-batch forms.
+//
+// The operands go from global memory straight into the MMA fragments. A contraction
+// may run over its index in any order as long as both operands use the same one:
+// thread (g = lane / 4, t = lane % 4) of an MMA holds, for rows g and g + 8 of A and
+// column g of B, the k in {2t, 2t+1, 2t+8, 2t+9}; here those are the elements
+// 8t .. 8t+3 of a 32-wide K-block for the block's first MMA and 8t+4 .. 8t+7 for its
+// second, so a thread reads its 8 elements of a row as one 16-byte load.
+//
+// q stays an fp32 result ("Large Memory Layers with Product Keys", gptget.net summary,
+// Methodology: the query network is a linear map followed by batch normalisation):
+// the query tile accumulates x W_q^T in fp32, and the score tile splits q into
+// hi = RN_bf16(q) and lo = RN_bf16(q - hi) (residual at most 2^-16 |q|) with one fp32
+// accumulator per plane; sub-keys are bf16 and exact.
+// ---------------------------------------------------------------------------
+constexpr int kMmaTok = 16;     // tokens per tile (the MMA's M)
+constexpr int kMmaFeat = 16;    // features per query tile (two 8-wide MMA N tiles)
+constexpr int kMmaKSplit = kSmallWarps / 2;  // query tile: warps sharing an N tile's K
+constexpr int kMmaRedLd = kMmaFeat + 1;
+
+__host__ __device__ inline bool mma_mode(int64_t B, int H, int d, int dq, int esz) {
+  return mma_shape(d, dq, esz) && !decode_mode(B, H, d, dq, esz);
+}
+
+// Shared memory of the query tile: the K-split partial sums [kMmaKSplit][16][17].
+constexpr size_t kMmaQuerySmem = sizeof(float) * kMmaKSplit * kMmaTok * kMmaRedLd;
+
+// Shared memory of the score tile: q of its tokens as bf16 planes hi and lo,
+// [2][16][half + 32] (64 bytes of padding per row keep the fragment reads free of bank
+// conflicts), then the scores [16][kSChunk].
+__host__ __device__ inline size_t mma_score_smem(int half) {
+  return static_cast<size_t>(2) * kMmaTok * (half + 32) * 2 +
+         sizeof(float) * kMmaTok * kSChunk;
+}
+
+__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// The two MMAs of a 32-wide K-block: this thread's pieces of A rows g (ra) and g + 8
+// (rb) and of B column g (bv).
+__device__ __forceinline__ void mma_kblock(float (&c)[4], const uint4& ra, const uint4& rb,
+                                           const uint4& bv) {
+  mma16816(c, ra.x, rb.x, ra.y, rb.y, bv.x, bv.y);
+  mma16816(c, ra.z, rb.z, ra.w, rb.w, bv.z, bv.w);
+}
+
+// hi = RN_bf16(q), lo = RN_bf16(q - hi) of two consecutive elements, packed in pairs.
+__device__ __forceinline__ void split2_pair(float q0, float q1, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(q0, q1);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(q0 - __low2float(h), q1 - __high2float(h));
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+// q[t0 .. t0+15][f0 .. f0+15] = BN(x W_q^T) for the tokens below B (one CTA of 8 warps;
+// F is a multiple of 16). Warp w takes the 8 features f0 + 8 (w % 2) + [0, 8) over the
+// K-blocks kb = w / 2 (mod kMmaKSplit); the partial products of a feature are added in
+// K-split order through shared memory (red, kMmaQuerySmem bytes), then the BatchNorm
+// affine map as in the kernels above.
+__device__ void mma_query_tile(const uint16_t* __restrict__ X, const uint16_t* __restrict__ W,
+                               const float* __restrict__ mean, const float* __restrict__ var,
+                               const float* __restrict__ gamma, const float* __restrict__ beta,
+                               float eps, int B, int d, int F, int f0, int t0, float* red,
+                               float* __restrict__ q) {
+  constexpr int U = 4;  // K-blocks in flight per thread
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int nt = warp & 1, ks = warp >> 1;
+  const int nkb = d >> 5;
+  const int ra = t0 + g, rb = t0 + g + 8;
+  const bool oka = ra < B, okb = rb < B;
+  const uint4 z = make_uint4(0, 0, 0, 0);
+  const uint4* xa = reinterpret_cast<const uint4*>(X + static_cast<int64_t>(oka ? ra : 0) * d) + t;
+  const uint4* xb = reinterpret_cast<const uint4*>(X + static_cast<int64_t>(okb ? rb : 0) * d) + t;
+  const uint4* wr = reinterpret_cast<const uint4*>(W + static_cast<int64_t>(f0 + 8 * nt + g) * d) + t;
+  float c[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int kb0 = ks; kb0 < nkb; kb0 += U * kMmaKSplit) {
+    uint4 pa[U], pb[U], pw[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int kb = kb0 + u * kMmaKSplit;
+      const bool live = kb < nkb;
+      pa[u] = live && oka ? __ldg(xa + 4 * kb) : z;
+      pb[u] = live && okb ? __ldg(xb + 4 * kb) : z;
+      pw[u] = live ? __ldg(wr + 4 * kb) : z;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) mma_kblock(c, pa[u], pb[u], pw[u]);
+  }
+  float* rp = red + ks * kMmaTok * kMmaRedLd;
+  const int col = 8 * nt + 2 * t;
+  rp[g * kMmaRedLd + col] = c[0];
+  rp[g * kMmaRedLd + col + 1] = c[1];
+  rp[(g + 8) * kMmaRedLd + col] = c[2];
+  rp[(g + 8) * kMmaRedLd + col + 1] = c[3];
+  __syncthreads();
+  const int row = threadIdx.x / kMmaFeat, fc = threadIdx.x % kMmaFeat;  // 256 = 16 x 16
+  const int tok = t0 + row, f = f0 + fc;
+  if (tok < B) {
+    float s = red[row * kMmaRedLd + fc];
+#pragma unroll
+    for (int i = 1; i < kMmaKSplit; ++i) s += red[(i * kMmaTok + row) * kMmaRedLd + fc];
+    const float sc = gamma[f] / sqrtf(var[f] + eps);
+    q[static_cast<int64_t>(tok) * F + f] = fmaf(s, sc, beta[f] - mean[f] * sc);
+  }
+  __syncthreads();  // red is free again
+}
+
+// This warp's B fragments of a score tile: sub-keys c0 + 8 warp + g of head-half hs,
+// piece t of each 32-wide K-block (sub-keys past n read as zeros).
+__device__ __forceinline__ void mma_load_keys(const uint16_t* __restrict__ C, int n, int half,
+                                              int hs, int c0, uint4 (&kf)[kMmaMaxKB]) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int key = c0 + 8 * warp + (lane >> 2);
+  const bool ok = key < n;
+  const uint4* src = reinterpret_cast<const uint4*>(
+                         C + (static_cast<int64_t>(hs) * n + (ok ? key : 0)) * half) + (lane & 3);
+  const int nkb = half >> 5;
+#pragma unroll
+  for (int kb = 0; kb < kMmaMaxKB; ++kb)
+    kf[kb] = ok && kb < nkb ? __ldg(src + 4 * kb) : make_uint4(0, 0, 0, 0);
+}
+
+// Scores of the sub-keys c0 .. c0+63 of head-half hs (kf from mma_load_keys) against
+// the query halves of tokens t0 .. t0+15 below B, and each token's best 32 of them
+// into the chunk lists, as score_small_kernel writes them (one CTA of 8 warps; smem:
+// mma_score_smem(dq / 2) bytes, 16-byte aligned). q is read through L2 (__ldcg): in
+// the single-kernel form other CTAs wrote it during the same launch.
+__device__ void mma_score_tile(const float* q, const uint4 (&kf)[kMmaMaxKB], int B, int H,
+                               int dq, int n, int hs, int chunk, int t0, unsigned char* smem,
+                               float* __restrict__ cs, int* __restrict__ ci) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int half = dq >> 1, F = H * dq;
+  const int h = hs >> 1, side = hs & 1;
+  const int ld = half + 32;  // elements per plane row
+  uint16_t* qh = reinterpret_cast<uint16_t*>(smem);
+  uint16_t* ql = qh + kMmaTok * ld;
+  float* sc = reinterpret_cast<float*>(ql + kMmaTok * ld);  // [16][kSChunk]
+  const int c0 = chunk * kSChunk;
+  const int nchunks = (n + kSChunk - 1) / kSChunk;
+  __syncthreads();  // the previous tile has finished with the shared memory
+  const int per_row = half >> 2;  // float4 per query half
+  for (int i = threadIdx.x; i < kMmaTok * per_row; i += blockDim.x) {
+    const int r = i / per_row, e = (i - r * per_row) * 4;
+    const int tok = t0 + r;
+    const float4 v = tok < B ? __ldcg(reinterpret_cast<const float4*>(
+                                   q + static_cast<int64_t>(tok) * F + h * dq + side * half + e))
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+    uint32_t h0, l0, h1, l1;
+    split2_pair(v.x, v.y, h0, l0);
+    split2_pair(v.z, v.w, h1, l1);
+    *reinterpret_cast<uint2*>(qh + r * ld + e) = make_uint2(h0, h1);
+    *reinterpret_cast<uint2*>(ql + r * ld + e) = make_uint2(l0, l1);
+  }
+  __syncthreads();
+  float chi[4] = {0.f, 0.f, 0.f, 0.f}, clo[4] = {0.f, 0.f, 0.f, 0.f};
+  const int nkb = half >> 5;
+#pragma unroll
+  for (int kb = 0; kb < kMmaMaxKB; ++kb) {
+    if (kb < nkb) {
+      const int e = kb * 32 + 8 * t;
+      const uint4 ha = *reinterpret_cast<const uint4*>(qh + g * ld + e);
+      const uint4 hb = *reinterpret_cast<const uint4*>(qh + (g + 8) * ld + e);
+      const uint4 la = *reinterpret_cast<const uint4*>(ql + g * ld + e);
+      const uint4 lb = *reinterpret_cast<const uint4*>(ql + (g + 8) * ld + e);
+      mma_kblock(chi, ha, hb, kf[kb]);
+      mma_kblock(clo, la, lb, kf[kb]);
+    }
+  }
+  const int col = 8 * warp + 2 * t;
+  *reinterpret_cast<float2*>(sc + g * kSChunk + col) = make_float2(chi[0] + clo[0], chi[1] + clo[1]);
+  *reinterpret_cast<float2*>(sc + (g + 8) * kSChunk + col) =
+      make_float2(chi[2] + clo[2], chi[3] + clo[3]);
+  __syncthreads();
+  // Warp w selects for the tile's tokens w and w + 8.
+  for (int r = warp; r < kMmaTok; r += kSmallWarps) {
+    const int tok = t0 + r;
+    if (tok >= B) break;  // warp-uniform
+    float s0;
+    int i0;
+    decode_chunk_list(sc, r, c0, n, s0, i0);
+    const int64_t o =
+        ((((static_cast<int64_t>(tok) * H + h) * 2 + side) * nchunks + chunk) << 5) + lane;
+    cs[o] = s0;
+    ci[o] = i0;
+  }
+}
+
+// The three-kernel form's query and scoring kernels in that mode: CTA = (16 features,
+// 16 tokens) and CTA = (64 sub-keys, head-half, 16 tokens).
+__global__ void __launch_bounds__(kSmallWarps * 32) query_mma_kernel(
+    const uint16_t* __restrict__ x, const uint16_t* __restrict__ W,
+    const float* __restrict__ mean, const float* __restrict__ var,
+    const float* __restrict__ gamma, const float* __restrict__ beta, float eps, int B, int d,
+    int F, float* __restrict__ q, int* clear) {
+  __shared__ float red[kMmaKSplit * kMmaTok * kMmaRedLd];
+  first_kernel_prologue(clear);
+  mma_query_tile(x, W, mean, var, gamma, beta, eps, B, d, F, blockIdx.x * kMmaFeat,
+                 blockIdx.y * kMmaTok, red, q);
+}
+
+__global__ void __launch_bounds__(kSmallWarps * 32, 4) score_mma_kernel(
+    const float* __restrict__ q, const uint16_t* __restrict__ subkeys, int B, int H, int dq,
+    int n, float* __restrict__ chunk_s, int* __restrict__ chunk_i) {
+  extern __shared__ __align__(16) unsigned char sm_raw[];
+  allow_dependents();
+  uint4 kf[kMmaMaxKB];
+  mma_load_keys(subkeys, n, dq / 2, blockIdx.y, blockIdx.x * kSChunk, kf);
+  wait_prior_grid();  // q comes from the query kernel
+  mma_score_tile(q, kf, B, H, dq, n, blockIdx.y, blockIdx.x, blockIdx.z * kMmaTok, sm_raw,
+                 chunk_s, chunk_i);
+}
+
+// ---------------------------------------------------------------------------
 // q[t][f] = (sum_c x[t][c] W[f][c]) * scale[f] + shift[f], scale = gamma / sqrt(var + eps),
 // shift = beta - mean * scale (the tensor-core epilogue's form). CTA = 16 features x 8
 // tokens: the 16 rows of W_q and the 8 rows of x staged in shared memory, one warp
@@ -286,11 +539,12 @@ template <typename T>
 __global__ void __launch_bounds__(kSmallWarps * 32) query_small_kernel(
     const T* __restrict__ x, const T* __restrict__ W, const float* __restrict__ mean,
     const float* __restrict__ var, const float* __restrict__ gamma,
-    const float* __restrict__ beta, float eps, int B, int d, int F, float* __restrict__ q) {
+    const float* __restrict__ beta, float eps, int B, int d, int F, float* __restrict__ q,
+    int* clear) {
   extern __shared__ __align__(16) unsigned char qs_raw[];
   T* ws = reinterpret_cast<T*>(qs_raw);  // [kQFeat][d]
   T* xs = ws + kQFeat * d;               // [kQTok][d]
-  allow_dependents();
+  first_kernel_prologue(clear);
   const int f0 = blockIdx.x * kQFeat;
   const int nf = min(kQFeat, F - f0);
   const int t0 = blockIdx.y * kQTok;
@@ -471,8 +725,9 @@ template <typename T, int RV>
 __global__ void __launch_bounds__(kSmallWarps * 32) query_decode_kernel(
     const T* __restrict__ x, const T* __restrict__ W, const float* __restrict__ mean,
     const float* __restrict__ var, const float* __restrict__ gamma,
-    const float* __restrict__ beta, float eps, int B, int d, int F, float* __restrict__ q) {
-  allow_dependents();
+    const float* __restrict__ beta, float eps, int B, int d, int F, float* __restrict__ q,
+    int* clear) {
+  first_kernel_prologue(clear);
   const int f = blockIdx.x * kSmallWarps + (threadIdx.x >> 5);
   if (f < F) decode_query_row<T, RV>(x, W, mean, var, gamma, beta, eps, B, d, F, f, q);
 }
@@ -508,16 +763,19 @@ __global__ void __launch_bounds__(kSmallWarps * 32) score_decode_kernel(
 
 // ---------------------------------------------------------------------------
 // One CTA per (token, head); the H CTAs of a token form a thread-block cluster.
-// (a) Warps 0 and 1 merge the chunk lists of the head's two halves into each half's
-// best 32. (b) Warp 0: exact top-k of the pruned product candidates, softmax,
+// (a) The chunk lists of the head's two halves merged into each half's best 32, four
+// lists per warp in registers, then a tree over the warps. (b) Exact top-k of the
+// pruned product candidates (sorted 32 per warp, tree-merged), then warp 0: softmax,
 // indices / weights / scores. (c) The k weighted value rows, split over the 8 warps,
 // summed into the CTA's partial output in shared memory. (d) After a cluster
 // barrier, each CTA adds the H partial outputs of its slice of the columns in head
 // order through distributed shared memory and writes them to out[t]; a second
 // barrier keeps every CTA's shared memory alive until the others have read it.
 // ---------------------------------------------------------------------------
-template <typename T, int MAXV>
-__global__ void __launch_bounds__(kSmallWarps * 32) gather_small_kernel(
+// MINB: CTAs per SM the register budget is sized for (the launch picks 4 when a grid of
+// (token, head) CTAs would not fit on the GPU at once with the default budget).
+template <typename T, int MAXV, int MINB>
+__global__ void __launch_bounds__(kSmallWarps * 32, MINB) gather_small_kernel(
     const float* __restrict__ chunk_s, const int* __restrict__ chunk_i,
     const T* __restrict__ values, int H, int n, int k, int v, float* __restrict__ out,
     int* __restrict__ indices, float* __restrict__ weights, float* __restrict__ scores,
@@ -543,65 +801,52 @@ __global__ void __launch_bounds__(kSmallWarps * 32) gather_small_kernel(
   const int h = blockIdx.y;
   if (threadIdx.x == 0) npairs_s = build_pairs(k, pairs);
   wait_prior_grid();  // the chunk lists come from the scoring kernel
+  // The stream's next kernel may launch now: a later call's first kernel waits for this
+  // grid's end before it reads anything.
+  allow_dependents();
   const int64_t src = (t * H + h) * list_words;
-  {
-    // Scores and ids in one pass (all of a thread's loads in flight before its stores).
-    // list_words is a multiple of 32 and the lists start 128-byte aligned.
-    const uint4* gs4 = reinterpret_cast<const uint4*>(chunk_s + src);
-    const uint4* gi4 = reinterpret_cast<const uint4*>(chunk_i + src);
-    uint4* ss4 = reinterpret_cast<uint4*>(cls);
-    uint4* si4 = reinterpret_cast<uint4*>(cli);
-    const int nv = list_words >> 2;
-    for (int b = threadIdx.x; b < nv; b += blockDim.x * 4) {
-      uint4 vs[4], vi[4];
+
+  // (a) each half's best 32. Warp w takes up to 4 of a half's chunk lists straight into
+  // registers (lane j holding entry j of each) and merges them, two merges side by side
+  // and then one; the warps' lists (4 per half on the 1024^2 layer) are then merged as a
+  // tree in shared memory: at stride st the list at 2 st i + st into the list at 2 st i.
+  const int quads = (nchunks + 3) / 4;  // warp lists per half
+  for (int item = warp; item < 2 * quads; item += kSmallWarps) {
+    const int side = item / quads, qd = item - side * quads;
+    const int nl = min(4, nchunks - 4 * qd);
+    const int64_t g0 = src + ((side * nchunks + 4 * qd) << 5) + lane;
+    float ls4[4];
+    int li4[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = b + u * blockDim.x;
-        if (i < nv) {
-          vs[u] = __ldg(gs4 + i);
-          vi[u] = __ldg(gi4 + i);
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = b + u * blockDim.x;
-        if (i < nv) {
-          ss4[i] = vs[u];
-          si4[i] = vi[u];
-        }
-      }
+    for (int u = 0; u < 4; ++u) {
+      ls4[u] = u < nl ? __ldg(chunk_s + g0 + 32 * u) : -INFINITY;
+      li4[u] = u < nl ? __ldg(chunk_i + g0 + 32 * u) : kIdPad;
     }
+    warp_merge32(ls4[0], li4[0], ls4[1], li4[1]);
+    warp_merge32(ls4[2], li4[2], ls4[3], li4[3]);
+    warp_merge32(ls4[0], li4[0], ls4[2], li4[2]);
+    cls[((side * quads + qd) << 5) + lane] = ls4[0];
+    cli[((side * quads + qd) << 5) + lane] = li4[0];
   }
   __syncthreads();
-
-  // (a) merge the chunk lists of each half, as a tree over the 8 warps: at stride st
-  // the list at 2 st i + st is merged into the list at 2 st i (each list is read and
-  // written by one warp per round).
-  for (int st = 1; st < nchunks; st <<= 1) {
-    const int per_side = (nchunks + 2 * st - 1) / (2 * st);
+  for (int st = 1; st < quads; st <<= 1) {
+    const int per_side = (quads + 2 * st - 1) / (2 * st);
     for (int item = warp; item < 2 * per_side; item += kSmallWarps) {
       const int side = item / per_side, i = item - side * per_side;
       const int a0 = 2 * st * i, b0 = a0 + st;
-      if (b0 >= nchunks) continue;  // warp-uniform
-      const int pa = ((side * nchunks + a0) << 5) + lane, pb = ((side * nchunks + b0) << 5) + lane;
+      if (b0 >= quads) continue;  // warp-uniform
+      const int pa = ((side * quads + a0) << 5) + lane, pb = ((side * quads + b0) << 5) + lane;
       float bs = cls[pa];
       int bi = cli[pa];
-      const float cs = cls[pb];
-      const int ci = cli[pb];
-      // Merge only when the second list's best beats the first's 32nd.
-      const float ks = __shfl_sync(0xffffffffu, bs, 31);
-      const int ki = __shfl_sync(0xffffffffu, bi, 31);
-      const float c0s = __shfl_sync(0xffffffffu, cs, 0);
-      const int c0i = __shfl_sync(0xffffffffu, ci, 0);
-      if (better(c0s, c0i, ks, ki)) warp_merge32(bs, bi, cs, ci);
+      warp_merge32(bs, bi, cls[pb], cli[pb]);
       cls[pa] = bs;
       cli[pa] = bi;
     }
     __syncthreads();
   }
-  float* ls = cls;                          // half 0's best 32 at chunk 0, half 1's after
+  float* ls = cls;                          // half 0's best 32 at list 0, half 1's after
   int* li = cli;
-  const int l1 = nchunks << 5;
+  const int l1 = quads << 5;
 
   // (b) the pruned candidates in chunks of 32, one chunk per warp, each sorted; then
   // merged as a tree; warp 0 takes softmax and the head's picks.
@@ -759,7 +1004,8 @@ struct FusedArgs {
   const void* values;
   float eps;
   int B, d, H, dq, n, k, v;
-  int decode;      // decode_mode(B, d, dq, esz)
+  int decode;      // decode_mode(B, H, d, dq, esz)
+  int mma;         // mma_mode(B, H, d, dq, esz)
   float* q;        // [B][H*dq] fp32
   float* cs;       // [B][H][2][nchunks][32] chunk lists
   int* ci;
@@ -823,6 +1069,10 @@ __host__ __device__ inline FusedSmem fused_smem(int d, int H, int dq, int n, int
   m.b = rows + sizeof(float) * kSmallWarps * 2 * half;
   const size_t dec = sizeof(float) * kDecodeB * kSChunk;  // decode mode's chunk scores
   if (m.b < dec) m.b = dec;
+  if (esz == 2) {  // the tensor-core tiles
+    if (m.a < kMmaQuerySmem) m.a = kMmaQuerySmem;
+    if (m.b < mma_score_smem(half)) m.b = mma_score_smem(half);
+  }
   m.total = m.a + m.b + sizeof(int) * kMaxPairs;
   return m;
 }
@@ -880,6 +1130,16 @@ __global__ void __launch_bounds__(kSmallWarps * 32, 1) forward_small_fused_kerne
          f += static_cast<int>(G) * kSmallWarps)
       decode_query_row<T, kDecodeRowVecs>(X, W, a.mean, a.var, a.gamma, a.beta, a.eps, B, d,
                                           F, f, a.q);
+  } else if (a.mma) {  // CTA = (16 features, 16 tokens) tiles
+    float* red = reinterpret_cast<float*>(regA);
+    const int nfg = F / kMmaFeat;
+    const int ntiles = nfg * ((B + kMmaTok - 1) / kMmaTok);
+    for (int tile = blockIdx.x; tile < ntiles; tile += G) {
+      const int tg = tile / nfg, fg = tile - tg * nfg;
+      mma_query_tile(reinterpret_cast<const uint16_t*>(X), reinterpret_cast<const uint16_t*>(W),
+                     a.mean, a.var, a.gamma, a.beta, a.eps, B, d, F, fg * kMmaFeat,
+                     tg * kMmaTok, red, a.q);
+    }
   } else {
     T* ws = reinterpret_cast<T*>(regA);  // [kQFeat][d]
     T* xs = ws + kQFeat * d;             // [kQTok][d]
@@ -988,6 +1248,15 @@ __global__ void __launch_bounds__(kSmallWarps * 32, 1) forward_small_fused_kerne
         a.cs[o] = s0;
         a.ci[o] = i0;
       }
+    }
+  } else if (a.mma) {  // unit = (head-half, 64 sub-keys), its sub-keys in registers
+    const uint16_t* Cu = reinterpret_cast<const uint16_t*>(C);
+    for (int u = blockIdx.x; u < NS; u += G) {
+      const int hs = u / nchunks, chunk = u - hs * nchunks;
+      uint4 kf[kMmaMaxKB];
+      mma_load_keys(Cu, n, half, hs, chunk * kSChunk, kf);
+      for (int t0 = 0; t0 < B; t0 += kMmaTok)
+        mma_score_tile(a.q, kf, B, H, dq, n, hs, chunk, t0, regB, a.cs, a.ci);
     }
   } else
   for (int u = blockIdx.x; u < NS; u += G) {
@@ -1241,6 +1510,10 @@ static size_t gather_small_smem(int n, int v) {
   return sizeof(float) * (v + scratch) + kMaxPairs * 8 + kMaxK * 8 + sizeof(int) * kMaxPairs;
 }
 
+bool small_mma_shape(int d_model, int dq, int dtype) {
+  return mma_shape(d_model, dq, dtype == 0 ? 4 : 2);
+}
+
 bool small_supported(int64_t B, int d_model, int H, int dq, int n, int k, int v, int dtype) {
   constexpr size_t kLimit = 200 * 1024;
   const int esz = dtype == 0 ? 4 : 2;
@@ -1257,12 +1530,13 @@ size_t small_chunk_entries(int64_t B, int H, int n) {
   return static_cast<size_t>(B) * H * 2 * ((n + kSChunk - 1) / kSChunk) * kMaxK;
 }
 
-template <typename T, int MAXV>
-static cudaError_t launch_gather_small(const LayerArgs& a, const float* cs, const int* ci,
-                                       float* out, int* idx, float* w, float* sc,
-                                       cudaStream_t st) {
+template <typename T, int MAXV, int MINB>
+static cudaError_t launch_gather_small_t(const LayerArgs& a, const float* cs, const int* ci,
+                                         float* out, int* idx, float* w, float* sc,
+                                         cudaStream_t st) {
   const size_t smem = gather_small_smem(a.n, a.v);
-  cudaError_t e = set_max_smem(reinterpret_cast<const void*>(gather_small_kernel<T, MAXV>), smem);
+  const void* kern = reinterpret_cast<const void*>(gather_small_kernel<T, MAXV, MINB>);
+  cudaError_t e = set_max_smem(kern, smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(a.B), a.H, 1);
@@ -1278,9 +1552,45 @@ static cudaError_t launch_gather_small(const LayerArgs& a, const float* cs, cons
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, gather_small_kernel<T, MAXV>, cs, ci,
+  return cudaLaunchKernelEx(&cfg, gather_small_kernel<T, MAXV, MINB>, cs, ci,
                             static_cast<const T*>(a.values), a.H, a.n, a.k, a.v, out, idx, w,
                             sc, a.status);
+}
+
+// The default register budget keeps more loads in flight per CTA (c1024: 80 registers,
+// 3 CTAs per SM); when B * H CTAs would not all be resident at once with it, the launch
+// takes the 4-CTA-per-SM build (64 registers) instead: one wave rather than a second,
+// nearly empty one (47 vs 53 us per call at 112 tokens on the 1024^2 layer, while at 16
+// and 64 tokens the default build is 6 and 4 us faster).
+template <typename T, int MAXV>
+static cudaError_t launch_gather_small(const LayerArgs& a, const float* cs, const int* ci,
+                                       float* out, int* idx, float* w, float* sc,
+                                       cudaStream_t st) {
+  if constexpr (MAXV < 8) {
+    // Resident CTAs of the default build per SM, looked up once per shared-memory size.
+    static std::mutex mu;
+    static size_t seen_smem = 0;
+    static int seen_per_sm = 0;
+    const size_t smem = gather_small_smem(a.n, a.v);
+    int per_sm = 0;
+    {
+      std::lock_guard<std::mutex> lock(mu);
+      if (seen_smem != smem) {
+        const void* kern = reinterpret_cast<const void*>(gather_small_kernel<T, MAXV, 1>);
+        cudaError_t e = set_max_smem(kern, smem);
+        if (e == cudaSuccess)
+          e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&seen_per_sm, kern,
+                                                            kSmallWarps * 32, smem);
+        if (e != cudaSuccess) return e;
+        seen_smem = smem;
+      }
+      per_sm = seen_per_sm > 0 ? seen_per_sm : 1;
+    }
+    if (a.B * a.H > static_cast<int64_t>(per_sm) * sm_count())
+      return launch_gather_small_t<T, MAXV, 4>(a, cs, ci, out, idx, w, sc, st);
+    return launch_gather_small_t<T, MAXV, 1>(a, cs, ci, out, idx, w, sc, st);
+  }
+  return launch_gather_small_t<T, MAXV, 2>(a, cs, ci, out, idx, w, sc, st);
 }
 
 template <typename T, int MAXV>
@@ -1296,7 +1606,8 @@ static cudaError_t launch_fused_t(const LayerArgs& a, float* q, float* cs, int* 
   fa.B = static_cast<int>(a.B); fa.d = a.d_model; fa.H = a.H; fa.dq = a.dq; fa.n = a.n;
   fa.k = a.k; fa.v = a.v; fa.q = q; fa.cs = cs; fa.ci = ci; fa.part = part; fa.out = out;
   fa.tok_done = reinterpret_cast<unsigned*>(part + a.B * a.H * a.v);
-  fa.decode = decode_mode(a.B, a.d_model, a.dq, a.dtype == 0 ? 4 : 2) ? 1 : 0;
+  fa.decode = decode_mode(a.B, a.H, a.d_model, a.dq, a.dtype == 0 ? 4 : 2) ? 1 : 0;
+  fa.mma = mma_mode(a.B, a.H, a.d_model, a.dq, a.dtype == 0 ? 4 : 2) ? 1 : 0;
   fa.idx = idx;
   fa.w = w; fa.sc = sc; fa.status = a.status;
   // The grid barriers' counter: the word after the status word (the caller zeroes both).
@@ -1339,13 +1650,13 @@ cudaError_t launch_forward_small_fused(const LayerArgs& a, float* q, float* chun
 
 template <typename T>
 static cudaError_t launch_small_t(const LayerArgs& a, float* q, float* cs, int* ci, float* out,
-                                  int* idx, float* w, float* sc, cudaStream_t st) {
+                                  int* idx, float* w, float* sc, int* clear, cudaStream_t st) {
   const int F = a.H * a.dq;
   const int B = static_cast<int>(a.B);
   size_t smem = query_small_smem(a.d_model, a.dtype);
   cudaError_t e = set_max_smem(reinterpret_cast<const void*>(query_small_kernel<T>), smem);
   if (e != cudaSuccess) return e;
-  const bool decode = decode_mode(B, a.d_model, a.dq, a.dtype == 0 ? 4 : 2);
+  const bool decode = decode_mode(B, a.H, a.d_model, a.dq, a.dtype == 0 ? 4 : 2);
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(kSmallWarps * 32, 1, 1);
   cfg.stream = st;
@@ -1361,15 +1672,14 @@ static cudaError_t launch_small_t(const LayerArgs& a, float* q, float* cs, int* 
     const unsigned gq = static_cast<unsigned>((F + kSmallWarps - 1) / kSmallWarps);
     const T* xp = static_cast<const T*>(a.x);
     const T* wp = static_cast<const T*>(a.W_q);
+    cfg.gridDim = dim3(gq, 1, 1);
+    cfg.dynamicSmemBytes = 0;
 #define PKM_QDEC(RV)                                                                     \
-  query_decode_kernel<T, RV><<<gq, kSmallWarps * 32, 0, st>>>(xp, wp, a.bn_mean, a.bn_var, \
-                                                             a.bn_gamma, a.bn_beta, a.bn_eps, \
-                                                             B, a.d_model, F, q)
-    if (rv <= 1) PKM_QDEC(1);
-    else if (rv <= 2) PKM_QDEC(2);
-    else if (rv <= 4) PKM_QDEC(4);
-    else PKM_QDEC(8);
+  cudaLaunchKernelEx(&cfg, query_decode_kernel<T, RV>, xp, wp, a.bn_mean, a.bn_var,        \
+                     a.bn_gamma, a.bn_beta, a.bn_eps, B, a.d_model, F, q, clear)
+    e = rv <= 1 ? PKM_QDEC(1) : rv <= 2 ? PKM_QDEC(2) : rv <= 4 ? PKM_QDEC(4) : PKM_QDEC(8);
 #undef PKM_QDEC
+    if (e != cudaSuccess) return e;
     cfg.gridDim = dim3((a.n + kSChunk - 1) / kSChunk, a.H * 2, 1);
     cfg.dynamicSmemBytes = 0;
     const float* qc = q;
@@ -1378,11 +1688,29 @@ static cudaError_t launch_small_t(const LayerArgs& a, float* q, float* cs, int* 
                                      cs, ci)
                 : cudaLaunchKernelEx(&cfg, score_decode_kernel<T, 2>, qc, kp, B, a.H, a.dq, a.n,
                                      cs, ci);
+  } else if (mma_mode(B, a.H, a.d_model, a.dq, a.dtype == 0 ? 4 : 2)) {
+    const int tiles = (B + kMmaTok - 1) / kMmaTok;
+    const uint16_t* kp = static_cast<const uint16_t*>(a.subkeys);
+    cfg.gridDim = dim3(F / kMmaFeat, tiles, 1);
+    cfg.dynamicSmemBytes = 0;
+    e = cudaLaunchKernelEx(&cfg, query_mma_kernel, static_cast<const uint16_t*>(a.x),
+                           static_cast<const uint16_t*>(a.W_q), a.bn_mean, a.bn_var, a.bn_gamma,
+                           a.bn_beta, a.bn_eps, B, a.d_model, F, q, clear);
+    if (e != cudaSuccess) return e;
+    smem = mma_score_smem(a.dq / 2);
+    e = set_max_smem(reinterpret_cast<const void*>(score_mma_kernel), smem);
+    if (e != cudaSuccess) return e;
+    cfg.gridDim = dim3((a.n + kSChunk - 1) / kSChunk, a.H * 2, tiles);
+    cfg.dynamicSmemBytes = smem;
+    e = cudaLaunchKernelEx(&cfg, score_mma_kernel, static_cast<const float*>(q), kp, B, a.H,
+                           a.dq, a.n, cs, ci);
   } else {
-    dim3 gq((F + kQFeat - 1) / kQFeat, (B + kQTok - 1) / kQTok);
-    query_small_kernel<T><<<gq, kSmallWarps * 32, smem, st>>>(
-        static_cast<const T*>(a.x), static_cast<const T*>(a.W_q), a.bn_mean, a.bn_var,
-        a.bn_gamma, a.bn_beta, a.bn_eps, B, a.d_model, F, q);
+    cfg.gridDim = dim3((F + kQFeat - 1) / kQFeat, (B + kQTok - 1) / kQTok, 1);
+    cfg.dynamicSmemBytes = smem;
+    e = cudaLaunchKernelEx(&cfg, query_small_kernel<T>, static_cast<const T*>(a.x),
+                           static_cast<const T*>(a.W_q), a.bn_mean, a.bn_var, a.bn_gamma,
+                           a.bn_beta, a.bn_eps, B, a.d_model, F, q, clear);
+    if (e != cudaSuccess) return e;
     smem = score_small_smem(a.dq, a.dtype);
     e = set_max_smem(reinterpret_cast<const void*>(score_small_kernel<T>), smem);
     if (e != cudaSuccess) return e;
@@ -1402,9 +1730,11 @@ static cudaError_t launch_small_t(const LayerArgs& a, float* q, float* cs, int* 
 }
 
 cudaError_t launch_forward_small(const LayerArgs& a, float* q, float* chunk_s, int* chunk_i,
-                                 float* out, int* idx, float* w, float* sc, cudaStream_t st) {
-  if (a.dtype == 0) return launch_small_t<float>(a, q, chunk_s, chunk_i, out, idx, w, sc, st);
-  return launch_small_t<uint16_t>(a, q, chunk_s, chunk_i, out, idx, w, sc, st);
+                                 float* out, int* idx, float* w, float* sc, int* clear,
+                                 cudaStream_t st) {
+  if (a.dtype == 0)
+    return launch_small_t<float>(a, q, chunk_s, chunk_i, out, idx, w, sc, clear, st);
+  return launch_small_t<uint16_t>(a, q, chunk_s, chunk_i, out, idx, w, sc, clear, st);
 }
 
 }  // namespace pkm

@@ -1,7 +1,10 @@
-"""GPU parity of the small-batch forward (up to 112 tokens with H <= 4, 96 with more
-heads: pkm_forward picks the small-batch kernels by itself; a pinned form takes up to
-112 tokens for any H <= 8) against the fp64 oracle, through the C ABI, in both forms:
-the single cooperative kernel and the three kernels.
+"""GPU parity of the small-batch forward against the fp64 oracle, through the C ABI, in
+both forms: the single cooperative kernel and the three kernels. pkm_forward picks the
+three kernels by itself up to 384 tokens with H <= 4 and 240 with more heads on bf16
+layers whose query and scores run as tensor-core tiles (112 / 96 otherwise); a pinned
+form takes up to 512 tokens for any H <= 8. Up to 8 tokens both forms run in decode
+mode, above it (bf16) the query network and the per-half scores are warp-level MMA
+tiles of 16 tokens.
 
 Same bar as tests/test_forward_gpu.py: indices bit-exact except fp64 near-ties
 within 1e-5 relative of the k-th score; weights, kept scores and out within
@@ -55,6 +58,16 @@ def test_c1024_small_batches(B, path):
     _check(synth.make_layer(w), w, path)
 
 
+@pytest.mark.parametrize("name,B", [("c1024", 256), ("c1024", 384), ("c512", 376),
+                                    ("wide", 240)])
+def test_larger_batches_default_choice(name, B):
+    """The automatic choice up to its cut-off: the three kernels, MMA tiles over several
+    16-token tiles (a ragged last one at 376), and gathers of more (token, head) CTAs
+    than the GPU holds at once with the default register budget."""
+    w = synth.WORKLOADS[name].with_(B=B)
+    _check(synth.make_layer(w), w)
+
+
 @pytest.mark.parametrize("path", FORMS)
 @pytest.mark.parametrize("name,B", [("c512", 33), ("wide", 4), ("wide", 16), ("wide", 112),
                                     ("tiny", 5)])
@@ -68,8 +81,8 @@ def test_other_shapes(name, B, path):
 @pytest.mark.parametrize("k,n", [(1, 256), (3, 256), (8, 8), (32, 32), (32, 100)])
 def test_k_and_small_codebooks(k, n, B, path):
     """3 tokens take the decode mode (a warp per W_q row or per 8 sub-keys, lanes over
-    the contraction), 9 tokens the token-per-warp kernels; n = 8, 32, 100 leave the
-    last 64-sub-key chunk ragged."""
+    the contraction), 9 tokens the MMA tiles; n = 8, 32, 100 leave the last 64-sub-key
+    chunk ragged (sub-keys past n read as zeros and are never picked)."""
     w = synth.WORKLOADS["c512"].with_(B=B, n=n, k=k)
     _check(synth.make_layer(w), w, path)
 
@@ -84,7 +97,7 @@ def test_odd_half_query_goes_to_large_batch_kernels():
 
 @pytest.mark.parametrize("B", [3, 40])
 def test_fused_and_three_kernel_forms_agree(B):
-    """Same arithmetic in both forms (3 tokens: decode mode; 40: token per warp): picks,
+    """Same arithmetic in both forms (3 tokens: decode mode; 40: MMA tiles): picks,
     weights and scores bit for bit; out up to the order in which the H*k rows are
     added."""
     w = synth.WORKLOADS["c1024"].with_(B=B)

@@ -32,14 +32,19 @@ def _forward(P, w, d, ws=None):
 @pytest.mark.parametrize("name,B,path,stages,launches", [
     ("c512", 1024, "auto", (0, 1, 2), 3),      # tensor-core kernels
     ("c512", 4, "auto", (2,), 3),              # small batch, three kernels (decode mode)
-    ("c512", 16, "auto", (2,), 1),             # small batch, one cooperative kernel
+    ("c512", 16, "auto", (2,), 3),             # small batch, three kernels (MMA tiles)
+    ("c512", 16, "small_fused", (2,), 1),      # small batch, one cooperative kernel
     ("tiny", 64, "simt", (0, 1, 2), 3),        # CUDA-core kernels (fp32)
+    ("tiny", 112, "auto", (2,), 3),            # fp32 small batch: CUDA-core kernels
+    ("tiny", 113, "auto", (0, 1, 2), 3),       # ... up to 112 tokens
     # The automatic cut-off depends on the heads: H = 8 takes the small-batch kernels
-    # up to 96 tokens, the tensor-core kernels above; a pinned form keeps them to 112.
-    ("wide", 96, "auto", (2,), 3),
-    ("wide", 112, "auto", (0, 1, 2), 3),
-    ("wide", 112, "small_split", (2,), 3),
-    ("c1024", 112, "auto", (2,), 3),
+    # up to 240 tokens, the tensor-core kernels above; H = 4 up to 384. A pinned form
+    # takes them to 512.
+    ("wide", 240, "auto", (2,), 3),
+    ("wide", 241, "auto", (0, 1, 2), 3),
+    ("wide", 256, "small_split", (2,), 3),
+    ("c1024", 384, "auto", (2,), 3),
+    ("c1024", 385, "auto", (0, 1, 2), 3),
 ])
 def test_forward_stages(name, B, path, stages, launches):
     P = _P()
