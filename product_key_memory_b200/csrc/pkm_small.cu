@@ -5,19 +5,24 @@
 //
 // The large-batch kernels tile 128 tokens per CTA, so a handful of tokens leaves
 // almost every SM idle and each stage is bound by one SM's bandwidth. Here every
-// stage spreads the layer's parameters over the whole GPU instead:
-//   query_small_kernel   q = BN(x W_q^T): CTA = 16 features x all tokens, its W_q rows
-//                        staged in shared memory, one warp per token (fp32 FMA); up to
-//                        kDecodeB tokens query_decode_kernel / score_decode_kernel
-//                        instead give a warp one W_q row / 8 sub-keys for all tokens
-//   score_small_kernel   CTA = (64 sub-keys, head-half, 16 tokens): the chunk's scores
-//                        and its best 32 per token
-//   gather_small_kernel  CTA = (token, head), the H heads of a token one cluster:
-//                        merge the chunk lists of each half, exact top-k of the
-//                        pruned candidates, softmax, the head's k weighted value rows
-//                        over 8 warps, heads summed over distributed shared memory
-// Same arithmetic as the CUDA-core large-batch path (fp32 q, fp32 dot products, the
-// same selection order and candidate pruning).
+// stage spreads the layer's parameters over the whole GPU instead, in three kernels
+// chained by programmatic dependent launch:
+//   query   q = BN(x W_q^T). Decode mode (a few tokens): query_decode_kernel, a warp
+//           per W_q row for all tokens. bf16 layers above it: query_mma_kernel, CTA =
+//           16 features x 16 tokens as warp-level tensor-core tiles. Otherwise (fp32):
+//           query_small_kernel, CTA = 16 features x 8 tokens, one warp per token.
+//   scores  the per-half scores of 64-sub-key chunks and each token's best 32 of a
+//           chunk: score_decode_kernel (a warp per 8 sub-keys, all tokens),
+//           score_mma_kernel (CTA = 64 sub-keys x 16 tokens, tensor-core tiles),
+//           score_small_kernel (CTA = 64 sub-keys x 16 tokens, a lane per sub-key)
+//   gather  gather_small_kernel, CTA = (token, head), the H heads of a token one
+//           cluster: merge the chunk lists of each half, exact top-k of the pruned
+//           candidates, softmax, the head's k weighted value rows over 8 warps, heads
+//           summed over distributed shared memory
+// forward_small_fused_kernel runs the same three stages as one cooperative launch.
+// fp32 q and fp32 dot products (fp32 accumulation of bf16 products on the tensor
+// cores, q split into two bf16 planes for the scores); the selection order and the
+// candidate pruning of the large-batch path.
 #include <cooperative_groups.h>
 
 #include <algorithm>
