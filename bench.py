@@ -21,6 +21,8 @@ small-batch latency on the 1024^2 layer (small_batch) and the wide layer (wide).
 
     python bench.py --part NAME          # one sub-object alone (for profiling)
     python bench.py --tokens B           # the main workload on its first B tokens
+    python bench.py --part latency --tokens B   # B-token calls through the default
+                                                # choice only (for profiling)
 
 ``--impl reference`` times the fp64 CPU oracle instead (a bounded sample of the
 same workload per step) and prints the same metric with "impl": "reference".
@@ -612,7 +614,7 @@ C1024_LATENCY_B = (1, 4, 8, 16, 32, 64, 96, 128, 192, 256, 384, 448)
 WIDE_LATENCY_B = (64, 128, 192, 240, 256)
 
 
-def latency_table(args, dev, P, wname, d, Bs):
+def latency_table(args, dev, P, wname, d, Bs, paths=("auto", "small_fused", "small_split", "tc")):
     """Forward latency of a few tokens on the layer d (device tensors of workload
     wname), caches warm (one token touches H*k value rows). Each batch size through the
     default choice, each small-batch form forced (the single cooperative kernel
@@ -633,7 +635,7 @@ def latency_table(args, dev, P, wname, d, Bs):
                       d["subkeys"], d["values"], k=w0.k, want_scores=False)
         torch.cuda.synchronize(dev)
     side = torch.cuda.Stream(dev)
-    for path in ("auto", "small_fused", "small_split", "tc"):
+    for path in paths:
         for B in Bs:
             x = d["x"][:B].contiguous()
             out = torch.empty(B, w0.v, device=dev)
@@ -690,6 +692,11 @@ def run_latency(args, dev, P, with_wide=False):
     entries are added where that layer is built (run_c512_and_backward), or here when
     with_wide is set (the latency part run alone)."""
     w0 = synth.WORKLOADS["c1024"]
+    if args.part == "latency" and args.tokens is not None:
+        # One batch size through the default choice only (profiling).
+        L = synth.make_layer(w0.with_(B=args.tokens))
+        d = {k: v.to(dev) for k, v in L.items()}
+        return latency_table(args, dev, P, "c1024", d, (args.tokens,), paths=("auto",))
     L = synth.make_layer(w0.with_(B=max(C1024_LATENCY_B)))
     d = {k: v.to(dev) for k, v in L.items()}
     res = {"workload": "c1024 layer (1024^2 slots, H=4, k=32, v=1024, bf16) and the wide "
