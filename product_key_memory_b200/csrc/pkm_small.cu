@@ -772,11 +772,26 @@ __global__ void __launch_bounds__(kSmallWarps * 32) score_decode_kernel(
 // lists per warp in registers, then a tree over the warps. (b) Exact top-k of the
 // pruned product candidates (sorted 32 per warp, tree-merged), then warp 0: softmax,
 // indices / weights / scores. (c) The k weighted value rows, split over the 8 warps,
-// summed into the CTA's partial output in shared memory. (d) After a cluster
-// barrier, each CTA adds the H partial outputs of its slice of the columns in head
-// order through distributed shared memory and writes them to out[t]; a second
-// barrier keeps every CTA's shared memory alive until the others have read it.
+// added in warp order. (d) Each CTA owns a slice of the columns of out[t]: every CTA
+// stores its head's sums of each slice into the owner's shared memory (distributed
+// shared memory), one cluster barrier, then each owner adds the H rows of its slice in
+// head order and writes them. The cluster barrier is split: arrived at at the start
+// (relaxed), waited for before the first store into another CTA, so its wait only
+// confirms that every CTA of the cluster is running.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.aligned;" ::: "memory");  // release
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");  // acquire
+}
+
+// Floats of the head-sum receive buffer: H slices of ceil(v / H) columns (H <= 8).
+__host__ __device__ inline int gather_part_len(int v) { return (v + 8 + 3) & ~3; }
+
 // MINB: CTAs per SM the register budget is sized for (the launch picks 4 when a grid of
 // (token, head) CTAs would not fit on the GPU at once with the default budget).
 template <typename T, int MAXV, int MINB>
@@ -790,8 +805,8 @@ __global__ void __launch_bounds__(kSmallWarps * 32, MINB) gather_small_kernel(
   extern __shared__ __align__(16) unsigned char gs_raw[];
   const int nchunks = (n + kSChunk - 1) / kSChunk;
   const int list_words = 2 * nchunks * kMaxK;                    // this head's two halves
-  float* part = reinterpret_cast<float*>(gs_raw);                 // [v] this head's output
-  float* red = part + v;                                          // [kSmallWarps][v]
+  float* part = reinterpret_cast<float*>(gs_raw);  // [H][v / H] received head sums
+  float* red = part + gather_part_len(v);           // [kSmallWarps][v]
   float* cls = red;                                               // [2][nchunks][32] (phase a)
   int* cli = reinterpret_cast<int*>(red + list_words);
   const int scratch = max(kSmallWarps * v, 2 * list_words);
@@ -803,7 +818,8 @@ __global__ void __launch_bounds__(kSmallWarps * 32, MINB) gather_small_kernel(
   __shared__ int npairs_s;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t t = blockIdx.x;
-  const int h = blockIdx.y;
+  const int h = blockIdx.y;  // also the CTA's rank in its cluster
+  cluster_arrive_relaxed();
   if (threadIdx.x == 0) npairs_s = build_pairs(k, pairs);
   wait_prior_grid();  // the chunk lists come from the scoring kernel
   // The stream's next kernel may launch now: a later call's first kernel waits for this
@@ -950,32 +966,26 @@ __global__ void __launch_bounds__(kSmallWarps * 32, MINB) gather_small_kernel(
     }
   }
   __syncthreads();
+  // (d) this head's sum of column c goes to row h of the owner's receive buffer.
+  cg::cluster_group cluster = cg::this_cluster();
+  const int slice = (v + H - 1) / H;
+  cluster_wait();  // every CTA of the cluster has started
   for (int c = threadIdx.x; c < v; c += blockDim.x) {
     float sum = 0.f;
 #pragma unroll
     for (int w = 0; w < kSmallWarps; ++w) sum += red[w * v + c];
-    part[c] = sum;
+    const int owner = c / slice;
+    cluster.map_shared_rank(part, owner)[h * slice + (c - owner * slice)] = sum;
   }
-
-  // (d) heads summed in head order, each CTA of the cluster taking one slice of the
-  // columns (all H partial rows of a column read together from the cluster's
-  // shared memory).
-  cg::cluster_group cluster = cg::this_cluster();
-  cluster.sync();
-  const int slice = (v + H - 1) / H;
+  cluster_arrive();  // this CTA's stores are done ...
+  cluster_wait();    // ... and every other CTA's: the slice is complete
   const int c1 = min(v, (h + 1) * slice);
   for (int c = h * slice + threadIdx.x; c < c1; c += blockDim.x) {
-    float pv[8];
-#pragma unroll
-    for (int hh = 0; hh < 8; ++hh)
-      pv[hh] = hh < H ? cluster.map_shared_rank(part, hh)[c] : 0.f;
-    float sum = pv[0];
-#pragma unroll
-    for (int hh = 1; hh < 8; ++hh)
-      if (hh < H) sum += pv[hh];
+    const int j = c - h * slice;
+    float sum = part[j];
+    for (int hh = 1; hh < H; ++hh) sum += part[hh * slice + j];
     out[t * v + c] = sum;
   }
-  cluster.sync();
 }
 
 // ---------------------------------------------------------------------------
@@ -1512,7 +1522,8 @@ static size_t score_small_smem(int dq, int dtype) {
 static size_t gather_small_smem(int n, int v) {
   const size_t list_words = static_cast<size_t>(2) * ((n + kSChunk - 1) / kSChunk) * kMaxK;
   const size_t scratch = std::max(static_cast<size_t>(kSmallWarps) * v, 2 * list_words);
-  return sizeof(float) * (v + scratch) + kMaxPairs * 8 + kMaxK * 8 + sizeof(int) * kMaxPairs;
+  return sizeof(float) * (gather_part_len(v) + scratch) + kMaxPairs * 8 + kMaxK * 8 +
+         sizeof(int) * kMaxPairs;
 }
 
 bool small_mma_shape(int d_model, int dq, int dtype) {
@@ -1562,8 +1573,8 @@ static cudaError_t launch_gather_small_t(const LayerArgs& a, const float* cs, co
                             sc, a.status);
 }
 
-// The default register budget keeps more loads in flight per CTA (c1024: 80 registers,
-// 3 CTAs per SM); when B * H CTAs would not all be resident at once with it, the launch
+// The default register budget keeps more loads in flight per CTA (c1024: 128 registers,
+// 2 CTAs per SM); when B * H CTAs would not all be resident at once with it, the launch
 // takes the 4-CTA-per-SM build (64 registers) instead: one wave rather than a second,
 // nearly empty one (47 vs 53 us per call at 112 tokens on the 1024^2 layer, while at 16
 // and 64 tokens the default build is 6 and 4 us faster).
@@ -1594,8 +1605,9 @@ static cudaError_t launch_gather_small(const LayerArgs& a, const float* cs, cons
     if (a.B * a.H > static_cast<int64_t>(per_sm) * sm_count())
       return launch_gather_small_t<T, MAXV, 4>(a, cs, ci, out, idx, w, sc, st);
     return launch_gather_small_t<T, MAXV, 1>(a, cs, ci, out, idx, w, sc, st);
+  } else {
+    return launch_gather_small_t<T, MAXV, 2>(a, cs, ci, out, idx, w, sc, st);
   }
-  return launch_gather_small_t<T, MAXV, 2>(a, cs, ci, out, idx, w, sc, st);
 }
 
 template <typename T, int MAXV>
