@@ -1574,8 +1574,9 @@ static cudaError_t launch_gather_small_t(const LayerArgs& a, const float* cs, co
 }
 
 // The default register budget keeps more loads in flight per CTA (c1024: 128 registers,
-// 2 CTAs per SM); when B * H CTAs would not all be resident at once with it, the launch
-// takes the 4-CTA-per-SM build (64 registers) instead: one wave rather than a second,
+// 2 CTAs per SM, 71 clusters of 4 at once); when the B clusters would not all be
+// resident at once with it, the launch takes the 4-CTA-per-SM build (64 registers)
+// instead: one wave rather than a second,
 // nearly empty one (47 vs 53 us per call at 112 tokens on the 1024^2 layer, while at 16
 // and 64 tokens the default build is 6 and 4 us faster).
 template <typename T, int MAXV>
@@ -1583,26 +1584,38 @@ static cudaError_t launch_gather_small(const LayerArgs& a, const float* cs, cons
                                        float* out, int* idx, float* w, float* sc,
                                        cudaStream_t st) {
   if constexpr (MAXV < 8) {
-    // Resident CTAs of the default build per SM, looked up once per shared-memory size.
+    // Clusters (the H CTAs of a token) of the default build resident at once, looked up
+    // once per shared-memory size and head count.
     static std::mutex mu;
     static size_t seen_smem = 0;
-    static int seen_per_sm = 0;
+    static int seen_h = 0, seen_clusters = 0;
     const size_t smem = gather_small_smem(a.n, a.v);
-    int per_sm = 0;
+    int clusters = 0;
     {
       std::lock_guard<std::mutex> lock(mu);
-      if (seen_smem != smem) {
+      if (seen_smem != smem || seen_h != a.H) {
         const void* kern = reinterpret_cast<const void*>(gather_small_kernel<T, MAXV, 1>);
         cudaError_t e = set_max_smem(kern, smem);
-        if (e == cudaSuccess)
-          e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&seen_per_sm, kern,
-                                                            kSmallWarps * 32, smem);
+        if (e != cudaSuccess) return e;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(1, a.H, 1);
+        cfg.blockDim = dim3(kSmallWarps * 32, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 1;
+        attr[0].val.clusterDim.y = a.H;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaOccupancyMaxActiveClusters(&seen_clusters, kern, &cfg);
         if (e != cudaSuccess) return e;
         seen_smem = smem;
+        seen_h = a.H;
       }
-      per_sm = seen_per_sm > 0 ? seen_per_sm : 1;
+      clusters = seen_clusters > 0 ? seen_clusters : 1;
     }
-    if (a.B * a.H > static_cast<int64_t>(per_sm) * sm_count())
+    if (a.B > clusters)
       return launch_gather_small_t<T, MAXV, 4>(a, cs, ci, out, idx, w, sc, st);
     return launch_gather_small_t<T, MAXV, 1>(a, cs, ci, out, idx, w, sc, st);
   } else {
