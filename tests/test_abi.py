@@ -58,6 +58,40 @@ def test_workspace_sizes():
     assert P.pkm_workspace_size(_shape(B=0)) > 0
 
 
+def _a256(x):
+    return (x + 255) // 256 * 256
+
+
+def _small_ws(B, H, dq, n, v):
+    """Forward workspace of the small-batch path: status, fp32 q, chunk lists (one list
+    of 32 per 64-sub-key chunk of each half), per-head rows and per-token counts."""
+    L = B * H * 2 * ((n + 63) // 64) * 32
+    return 256 + _a256(B * H * dq * 4) + 2 * _a256(L * 4) + _a256(B * H * v * 4 + B * 4)
+
+
+@pytest.mark.parametrize("name,cut", [("c1024", 384), ("c512", 384), ("wide", 240),
+                                      ("tiny", 112)])
+def test_automatic_small_batch_cut_off(name, cut):
+    """The default choice sends batches up to the cut-off to the small-batch kernels (384
+    tokens with H <= 4 and 240 with H = 8 on bf16 layers with tensor-core tiles, 112
+    with H <= 4 otherwise) and larger ones elsewhere; a pinned small-batch form takes up
+    to 512 tokens. The forward's workspace layout tells the paths apart."""
+    import synth
+    w = synth.WORKLOADS[name]
+    dt = 1 if w.dtype == "bf16" else 0
+
+    def ws(B):
+        return P.pkm_workspace_size(_shape(B=B, d_model=w.d_model, H=w.H, dq=w.dq, n=w.n,
+                                           k=w.k, v=w.v, dtype=dt))
+
+    for B in (1, 9, cut):
+        assert ws(B) == _small_ws(B, w.H, w.dq, w.n, w.v), B
+    assert ws(cut + 1) != _small_ws(cut + 1, w.H, w.dq, w.n, w.v)
+    with P.options(path="small_split"):
+        assert ws(512) == _small_ws(512, w.H, w.dq, w.n, w.v)
+        assert ws(513) != _small_ws(513, w.H, w.dq, w.n, w.v)
+
+
 def test_options_set_get_and_reject():
     assert P.pkm_get_option(P.PKM_OPT_PATH) == P.PKM_PATH_AUTO
     assert P.pkm_get_option(P.PKM_OPT_SUBBATCHES) == 1
