@@ -49,9 +49,22 @@ void init_options() {
   });
 }
 
-Path choose_path(const pkm_shape* s) {
+// The options one call works with, read once when it starts: a concurrent
+// pkm_set_option cannot give a call the workspace layout of one path and the launches
+// of another.
+struct Opts {
+  int path;
+  int subbatches;
+};
+
+Opts current_options() {
   init_options();
-  const int pin = g_opt_path.load(std::memory_order_relaxed);
+  return {g_opt_path.load(std::memory_order_relaxed),
+          g_opt_subbatches.load(std::memory_order_relaxed)};
+}
+
+Path choose_path(const pkm_shape* s, const Opts& o) {
+  const int pin = o.path;
   if (pin == PKM_PATH_SIMT) return Path::kSimt;
   // A pinned small-batch form takes every batch the small-batch kernels support; the
   // automatic choice only those up to the measured crossover for the head count.
@@ -111,9 +124,8 @@ struct ForwardWs {
 
 // Tokens per pipelined sub-batch of the tensor-core path: PKM_OPT_SUBBATCHES (1..4,
 // default 1) sub-batches of at least 2048 tokens, a multiple of the 128-token tile.
-int64_t sub_batch_tokens(int64_t B) {
-  init_options();
-  const int64_t want = g_opt_subbatches.load(std::memory_order_relaxed);
+int64_t sub_batch_tokens(int64_t B, const Opts& o) {
+  const int64_t want = o.subbatches;
   int64_t S = B / 2048;
   if (S > want) S = want;
   if (S < 1) S = 1;
@@ -122,11 +134,11 @@ int64_t sub_batch_tokens(int64_t B) {
   return sub < B ? sub : B;
 }
 
-size_t forward_ws(const pkm_shape* s, ForwardWs* w, char* base) {
+size_t forward_ws(const pkm_shape* s, const Opts& o, ForwardWs* w, char* base) {
   const int64_t F = static_cast<int64_t>(s->H) * s->dq;
-  const Path path = choose_path(s);
+  const Path path = choose_path(s, o);
   const size_t qbytes = path == Path::kTensor
-                            ? static_cast<size_t>(sub_batch_tokens(s->B)) * F * 2 *
+                            ? static_cast<size_t>(sub_batch_tokens(s->B, o)) * F * 2 *
                                   pkm::kScorePlanes
                             : static_cast<size_t>(s->B) * F * 4;
   // The small-batch path keeps each chunk's best 32 before merging them.
@@ -159,11 +171,13 @@ struct TrainWs {
   double* part;
 };
 
-size_t forward_train_ws(const pkm_shape* s, ForwardWs* fw, TrainWs* tw, char* base) {
+size_t forward_train_ws(const pkm_shape* s, const Opts& o, ForwardWs* fw, TrainWs* tw,
+                        char* base) {
   const int64_t F = static_cast<int64_t>(s->H) * s->dq;
-  const size_t accb = static_cast<size_t>(s->B) * F * (choose_path(s) == Path::kTensor ? 6 : 4);
+  const size_t accb =
+      static_cast<size_t>(s->B) * F * (choose_path(s, o) == Path::kTensor ? 6 : 4);
   const int64_t chunks = (s->B + pkm::kStatChunk - 1) / pkm::kStatChunk;
-  size_t off = forward_ws(s, fw, base);
+  size_t off = forward_ws(s, o, fw, base);
   const size_t o_acc = off;  off += align256(accb);
   const size_t o_part = off; off += align256(sizeof(double) * 2 * F * (chunks > 0 ? chunks : 1));
   if (tw && base) {
@@ -419,23 +433,24 @@ int pkm_trace_read(int pass, double* stage_ms, int max_stages, int64_t* calls,
 }
 
 size_t pkm_workspace_size(const pkm_shape* s, int for_backward) {
+  const Opts o = current_options();
   if (for_backward == 4) {
     if (validate_shape(s) != PKM_OK || s->B < 2) return 0;
-    return forward_train_ws(s, nullptr, nullptr, nullptr);
+    return forward_train_ws(s, o, nullptr, nullptr, nullptr);
   }
   if (for_backward == 3) {
     if (validate_shape(s) != PKM_OK || 2 * s->B * s->H * static_cast<int64_t>(s->k) > 0x7fffffffLL)
       return 0;
     LayerArgs a{};
     a.B = s->B; a.H = s->H; a.dq = s->dq; a.n = s->n; a.k = s->k; a.v = s->v;
-    return pkm::backward_full_ws_bytes(a, choose_path(s) == Path::kTensor, nullptr, nullptr);
+    return pkm::backward_full_ws_bytes(a, choose_path(s, o) == Path::kTensor, nullptr, nullptr);
   }
   if (for_backward == 2) {
     if (validate_usage(s) != PKM_OK) return 0;
     return pkm::kStatusBytes + align256(pkm::usage_bitmap_bytes(static_cast<int64_t>(s->n) * s->n));
   }
   if ((for_backward ? validate_common(s) : validate_shape(s)) != PKM_OK) return 0;
-  return for_backward ? backward_ws(s, nullptr, nullptr) : forward_ws(s, nullptr, nullptr);
+  return for_backward ? backward_ws(s, nullptr, nullptr) : forward_ws(s, o, nullptr, nullptr);
 }
 
 }  // extern "C"
@@ -463,7 +478,7 @@ int backward_full_impl(const pkm_shape* s, bool bn_training, const void* x, cons
                         grad_subkeys, grad_values, grad_scores};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return PKM_ERR_UNSUPPORTED;
-  const bool tensor = choose_path(s) == Path::kTensor;
+  const bool tensor = choose_path(s, current_options()) == Path::kTensor;
   LayerArgs a{s->B, s->d_model, s->H, s->dq, s->n, s->k, s->v, s->dtype, s->bn_eps,
               x, W_q, bn_mean, bn_var, bn_gamma, bn_beta, subkeys, values,
               static_cast<int*>(workspace), 0};
@@ -579,8 +594,8 @@ int validate_forward_args(const pkm_shape* s, const void* x, const void* W_q,
 
 // Small-batch path: the single cooperative kernel (only when pinned) rather than the
 // three kernels.
-bool small_fused_chosen(const pkm_shape* s) {
-  return g_opt_path.load(std::memory_order_relaxed) == PKM_PATH_SMALL_FUSED &&
+bool small_fused_chosen(const pkm_shape* s, const Opts& o) {
+  return o.path == PKM_PATH_SMALL_FUSED &&
          pkm::small_fused_supported(s->d_model, s->H, s->dq, s->n, s->v, s->dtype);
 }
 
@@ -590,14 +605,14 @@ bool small_fused_chosen(const pkm_shape* s) {
 // gather; the caller brackets stage 3 (the whole call).
 cudaError_t run_forward(const pkm_shape* s, const LayerArgs& a, const ForwardWs& w, float* out,
                         int32_t* indices, float* weights, float* scores, cudaStream_t st,
-                        Tracer& tr, int* nlaunch, bool clear_status) {
+                        Tracer& tr, int* nlaunch, const Opts& o, bool clear_status) {
   const void* x = a.x;
   cudaError_t e = cudaSuccess;
   int launches = 0;
-  const Path path = choose_path(s);
+  const Path path = choose_path(s, o);
   if (path == Path::kSmall) {
     tr.begin_here(2, st);
-    if (small_fused_chosen(s)) {
+    if (small_fused_chosen(s, o)) {
       e = pkm::launch_forward_small_fused(a, w.q, w.list_s, w.list_i, w.part, out, indices,
                                           weights, scores, st);
       launches = 1;
@@ -617,7 +632,7 @@ cudaError_t run_forward(const pkm_shape* s, const LayerArgs& a, const ForwardWs&
       e = pkm::launch_select_gather(a, w.list_s, w.list_i, out, indices, weights, scores, st);
     tr.end(st);
     launches = 3;
-  } else if (sub_batch_tokens(s->B) >= s->B) {
+  } else if (sub_batch_tokens(s->B, o) >= s->B) {
     // One batch: the three launches in order on the caller's stream.
     tr.begin_here(0, st);
     e = pkm::launch_query_tc(a, w.planes, st);
@@ -635,7 +650,7 @@ cudaError_t run_forward(const pkm_shape* s, const LayerArgs& a, const ForwardWs&
     // by the tensor cores and ALUs). The second stream waits for each sub-batch's
     // lists and the caller's stream waits for the last gather, so the call stays
     // ordered on `stream`.
-    const int64_t sub = sub_batch_tokens(s->B);
+    const int64_t sub = sub_batch_tokens(s->B, o);
     const int nsub = static_cast<int>((s->B + sub - 1) / sub);
     cudaStream_t aux;
     cudaEvent_t ev[5];
@@ -687,7 +702,8 @@ int pkm_forward(const pkm_shape* s, const void* x, const void* W_q, const float*
   int rc = validate_forward_args(s, x, W_q, bn_mean, bn_var, bn_gamma, bn_beta, subkeys, values,
                                  out, indices, weights, scores);
   if (rc != PKM_OK) return rc;
-  const size_t need = forward_ws(s, nullptr, nullptr);
+  const Opts o = current_options();
+  const size_t need = forward_ws(s, o, nullptr, nullptr);
   if (!workspace || workspace_bytes < need ||
       (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return PKM_ERR_WORKSPACE;
@@ -695,20 +711,20 @@ int pkm_forward(const pkm_shape* s, const void* x, const void* W_q, const float*
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   ForwardWs w;
-  forward_ws(s, &w, static_cast<char*>(workspace));
+  forward_ws(s, o, &w, static_cast<char*>(workspace));
   LayerArgs a{s->B, s->d_model, s->H, s->dq, s->n, s->k, s->v, s->dtype, s->bn_eps,
               x, W_q, bn_mean, bn_var, bn_gamma, bn_beta, subkeys, values, w.status, 0};
   // The status word and the small-batch kernel's grid-barrier counter after it. The
   // small-batch three-kernel form clears the status word in its first kernel instead
   // (it does not use the counter): one operation less between back-to-back calls.
-  const bool self_clear = choose_path(s) == Path::kSmall && !small_fused_chosen(s);
+  const bool self_clear = choose_path(s, o) == Path::kSmall && !small_fused_chosen(s, o);
   if (!self_clear && cudaMemsetAsync(w.status, 0, 2 * sizeof(int), st) != cudaSuccess)
     return PKM_ERR_CUDA;
   Tracer tr(0);
   int launches = 0;
   tr.begin(3, st);
   const cudaError_t e =
-      run_forward(s, a, w, out, indices, weights, scores, st, tr, &launches, self_clear);
+      run_forward(s, a, w, out, indices, weights, scores, st, tr, &launches, o, self_clear);
   tr.end_here(st);  // the last stage's end, or a new event after the pipelined join
   tr.finish(e == cudaSuccess, launches);
   return e == cudaSuccess ? PKM_OK : PKM_ERR_CUDA;
@@ -726,7 +742,8 @@ int pkm_forward_train(const pkm_shape* s, const void* x, const void* W_q,
   if (s->B == 1 || !batch_mean || !batch_var || !(momentum >= 0.f && momentum <= 1.f))
     return PKM_ERR_INVALID_ARG;
   if (!aligned16(batch_mean) || !aligned16(batch_var)) return PKM_ERR_UNSUPPORTED;
-  const size_t need = forward_train_ws(s, nullptr, nullptr, nullptr);
+  const Opts o = current_options();
+  const size_t need = forward_train_ws(s, o, nullptr, nullptr, nullptr);
   if (!workspace || workspace_bytes < need ||
       (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return PKM_ERR_WORKSPACE;
@@ -735,7 +752,7 @@ int pkm_forward_train(const pkm_shape* s, const void* x, const void* W_q,
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   ForwardWs w;
   TrainWs tw;
-  forward_train_ws(s, &w, &tw, static_cast<char*>(workspace));
+  forward_train_ws(s, o, &w, &tw, static_cast<char*>(workspace));
   const int F = s->H * s->dq;
   // acc = x W_q^T without BatchNorm, its batch statistics (and the running-statistics
   // update), then the forward normalised by the batch statistics.
@@ -751,7 +768,7 @@ int pkm_forward_train(const pkm_shape* s, const void* x, const void* W_q,
   int launches = 0;
   tr.begin(3, st);
   tr.begin_here(0, st);
-  const bool tensor = choose_path(s) == Path::kTensor;
+  const bool tensor = choose_path(s, o) == Path::kTensor;
   cudaError_t e = tensor ? pkm::launch_query_tc(raw, tw.acc, st)
                          : pkm::launch_query_bn_simt(raw, static_cast<float*>(tw.acc), st);
   if (e == cudaSuccess)
@@ -762,7 +779,7 @@ int pkm_forward_train(const pkm_shape* s, const void* x, const void* W_q,
   tr.end(st);
   launches += 3;
   if (e == cudaSuccess)
-    e = run_forward(s, a, w, out, indices, weights, scores, st, tr, &launches, false);
+    e = run_forward(s, a, w, out, indices, weights, scores, st, tr, &launches, o, false);
   tr.end_here(st);
   tr.finish(e == cudaSuccess, launches);
   return e == cudaSuccess ? PKM_OK : PKM_ERR_CUDA;
