@@ -991,22 +991,24 @@ __global__ void __launch_bounds__(kSmallWarps * 32, MINB) gather_small_kernel(
 // ---------------------------------------------------------------------------
 // The same forward as ONE cooperative launch (one CTA per SM), its phases separated by
 // grid-wide barriers instead of kernel boundaries:
-//   Q  query network: CTA = a group of 16 features for all tokens (W_q rows staged
-//      once); meanwhile the sub-keys of the CTA's first scoring unit are prefetched
-//      into L2, since they do not depend on q
-//   S  scores: CTA = (head-half, 64 sub-keys): scores for every token and each
-//      token's best 32 of the chunk
+//   Q  query network: in decode mode a warp per W_q row; with the tensor-core tiles
+//      CTA = (16 features, 16 tokens) tiles; otherwise CTA = a group of 16 features
+//      for all tokens (W_q rows staged once). Meanwhile the sub-keys of the CTA's
+//      first scoring unit are prefetched into L2, since they do not depend on q
+//   S  scores: CTA = (head-half, 64 sub-keys): scores for every token (the tiles:
+//      the sub-keys held in registers across the 16-token tiles) and each token's best
+//      32 of the chunk
 //   G  gather: CTA = (token, head): the chunk lists merged per half (a tree over the
 //      8 warps), exact top-k of the pruned candidates and softmax, the head's k
 //      weighted value rows over 8 warps (all in flight), added in warp order into the
 //      head's row of a workspace array; the token's last head to finish (a per-token
 //      count) adds the H rows in head order into out
-// With at most kDecodeB tokens, Q and S run in decode mode (above). A barrier is a
-// counter in the workspace (zeroed by the host before the launch): each CTA adds one
-// and waits, bounded by the pipelines' wait limit, until every CTA has; on a timeout
-// the kernel records it in the status word and returns. The arithmetic is
-// that of the three-kernel path above (fp32 q and dot products, the same selection
-// order and candidate pruning; each head's rows in the same order, heads in head order).
+// A barrier is a counter in the workspace (zeroed by the host before the launch): each
+// CTA adds one and waits, bounded by the pipelines' wait limit, until every CTA has; on
+// a timeout the kernel records it in the status word and returns. Q and S use the same
+// device functions and the same mode choice as the three-kernel form above, so picks,
+// weights and scores are equal bit for bit; out adds each head's rows in the same
+// order, heads in head order.
 // ---------------------------------------------------------------------------
 struct FusedArgs {
   const void* x;
