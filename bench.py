@@ -85,6 +85,15 @@ def per_token_bytes(w):
     return w.H * w.k * w.v * esz + w.v * 4 + w.H * 2 * w.k * 8 + w.H * w.k * 12
 
 
+def small_call_bytes(w, B):
+    """Compulsory HBM bytes of one small-batch forward call of B tokens: W_q and the
+    sub-keys read once, x in, the B*H*k value rows, out, indices and weights out."""
+    esz = 2 if w.dtype == "bf16" else 4
+    return (w.H * w.dq * w.d_model * esz + w.H * 2 * w.n * (w.dq // 2) * esz
+            + B * w.d_model * esz + B * w.H * w.k * w.v * esz + B * w.v * 4
+            + B * w.H * w.k * 8)
+
+
 def gemm_flops_per_token(w):
     """Query projection + per-half scoring, as the method defines them."""
     return 2 * w.d_model * w.H * w.dq + 2 * w.H * 2 * w.n * (w.dq // 2)
@@ -705,6 +714,10 @@ def run_latency(args, dev, P, with_wide=False):
            "timing": "plain keys: 10 calls in a CUDA graph replayed 20 times (device time "
                      "per call); '... stream' keys: 200 calls launched one by one"}
     res.update(latency_table(args, dev, P, "c1024", d, C1024_LATENCY_B))
+    # The time those bytes take at the HBM copy peak, next to the measured time.
+    hbm = float(peaks()[0]["hbm_gbs"])
+    res["byte_floor_us"] = {"B=%d" % B: small_call_bytes(w0, B) / (hbm * 1e3)
+                            for B in (1, 64)}
     del d, L
     if with_wide:
         L = synth.make_layer(synth.WORKLOADS["wide"].with_(B=max(WIDE_LATENCY_B)))
