@@ -77,6 +77,16 @@ def test_other_shapes(name, B, path):
 
 
 @pytest.mark.parametrize("path", FORMS)
+@pytest.mark.parametrize("dq,n,B", [(128, 512, 40), (128, 512, 3), (48, 256, 20)])
+def test_query_half_widths(dq, n, B, path):
+    """bf16 layers with narrower query halves: dq/2 = 64 takes the MMA tiles (two
+    32-wide K-blocks per sub-key row; 3 tokens decode mode), dq/2 = 24 (not a multiple
+    of 32) the CUDA-core kernels above decode mode."""
+    w = synth.WORKLOADS["c512"].with_(B=B, dq=dq, n=n)
+    _check(synth.make_layer(w), w, path)
+
+
+@pytest.mark.parametrize("path", FORMS)
 @pytest.mark.parametrize("B", [3, 9])
 @pytest.mark.parametrize("k,n", [(1, 256), (3, 256), (8, 8), (32, 32), (32, 100)])
 def test_k_and_small_codebooks(k, n, B, path):
